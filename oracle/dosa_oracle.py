@@ -1,0 +1,393 @@
+"""Plain fp64 CPU oracle for the DoSA certified indexer Top-K.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The CUDA library never calls it, and it shares no code with the CUDA
+path (no kernels, headers, tables or helpers).
+
+Sources (all web pages on DoSA):
+  [DPC]  "DOSA: Dots Sparse Attention", Daily Paper Cast transcript.
+         Sections: Introduction, Method, Experiments and Results, Related Work.
+  [ZICQ] "arXiv Releases DoSA: Revolutionizing Sparse Attention for Enhanced
+         Indexing Efficiency and Inference Speed", Technical Mechanism Analysis.
+  [PICX] "Xiaohongshu DoSA sparse attention cuts TTFT by up to 48% via score
+         bounds", sections 01-03 of the quoted article.
+
+What the method computes.  The pages state that DoSA keeps the original scoring
+function and returns exactly the Top-K the dense indexer returns ([PICX] 02,
+[ZICQ] point 2 "exact token selection", [DPC] Introduction "rejected tokens
+could not have made it into the Top-K").  So the dense oracle below is the plain
+definition: decode the stored inputs exactly, score every visible key in fp64,
+sort, take K.  The certificate half follows the steps of [DPC] Method in order
+(seed threshold, three bound stages, tile-by-tile refinement); the pages print
+no formula, so every formula here is the plainest construction consistent with
+the wording, and each reading is listed in the design doc.
+
+Parity status of each function (pins live in tests/test_oracle_*.py):
+  decode_bf16, decode_e4m3 ...... pinned (format definitions, hand values, torch)
+  indexer_scores ................ pinned (brute-force loops, integer closed forms)
+  select_topk ................... pinned (repeated argmax, sorted() on tuples)
+  nnls_retained ................. pinned (grid search, KKT conditions)
+  certificate_setup/upper_bound . pinned (UB >= I invariant, closed-form reductions)
+  certified_topk_row ............ pinned (equals dense selection; tau <= K-th)
+  prune rates ................... parity unpinned against the pages (their ~97 %
+                                  is measured on trained indexers); pinned only
+                                  by the ideal-rate upper limit.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+__all__ = [
+    "decode_bf16", "decode_e4m3", "dequantize", "indexer_scores", "select_topk",
+    "dense_topk", "nnls_retained", "Certificate", "certificate_setup", "upper_bound",
+    "soundness_margin", "seed_mask", "certified_topk_row", "certified_topk",
+    "key_mean",
+]
+
+# ----------------------------------------------------------------------------
+# Exact decoding of the stored number formats.
+# ----------------------------------------------------------------------------
+
+
+def decode_bf16(codes: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64, from the format: 1 sign bit, 8 exponent
+    bits (bias 127), 7 fraction bits; exponent 0 is subnormal.  Inf/NaN codes
+    are rejected (the indexer inputs are finite)."""
+    c = np.asarray(codes).astype(np.int64)
+    sign = np.where((c >> 15) & 1, -1.0, 1.0)
+    e = (c >> 7) & 0xFF
+    f = (c & 0x7F).astype(np.float64)
+    if np.any(e == 0xFF):
+        raise ValueError("bf16 input holds Inf or NaN")
+    normal = np.ldexp(1.0 + f / 128.0, (e - 127).astype(np.int64))
+    sub = np.ldexp(f / 128.0, -126)
+    return sign * np.where(e == 0, sub, normal)
+
+
+def _e4m3_table() -> np.ndarray:
+    """The 256 values of OCP FP8 E4M3 (the 'fn' variant: no infinities).
+    1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits.  Exponent 0 is
+    subnormal (m/8 * 2^-6).  Only S.1111.111 is NaN; S.1111.110 = 448 is the
+    largest finite value."""
+    table = np.empty(256, np.float64)
+    for code in range(256):
+        s = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            table[code] = np.nan
+        elif e == 0:
+            table[code] = s * (m / 8.0) * 2.0 ** -6
+        else:
+            table[code] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return table
+
+
+_E4M3 = _e4m3_table()
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """e4m3 bit patterns -> float64 through the table above.  NaN codes are
+    rejected."""
+    v = _E4M3[np.asarray(codes).astype(np.int64)]
+    if np.any(np.isnan(v)):
+        raise ValueError("e4m3 input holds NaN")
+    return v
+
+
+def dequantize(codes: np.ndarray, scale: np.ndarray | None, dtype: str) -> np.ndarray:
+    """Stored value -> real value.  bf16: the value itself.  fp8: one fp32
+    scale per token multiplies the decoded code (the per-token scale of the
+    128K/1M workloads), applied in fp64 over the leading axis."""
+    if dtype == "bf16":
+        return decode_bf16(codes)
+    if dtype == "fp8":
+        v = decode_e4m3(codes)
+        s = np.asarray(scale, np.float64).reshape((-1,) + (1,) * (v.ndim - 1))
+        return v * s
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+# ----------------------------------------------------------------------------
+# Dense indexer: the definition.
+# ----------------------------------------------------------------------------
+
+
+def indexer_scores(q_t: np.ndarray, w_t: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """I(t,s) = sum_h w[t,h] * ReLU(q[t,h] . k[s]) for every row s of ``k``.
+
+    The signed multi-head indexer score that DoSA keeps unchanged ([DPC] Method,
+    problem formulation: one query with several indexer heads, each with its own
+    query vector and weight, scored against shared keys; [PICX] 01: the indexer
+    scores candidates and keeps the K highest).  q_t: [H, d], w_t: [H], k: [n, d],
+    all float64.  Returns [n] float64."""
+    x = k @ q_t.T                        # [n, H]: one dot product per (key, head)
+    return np.maximum(x, 0.0) @ w_t      # ReLU, then the weighted head sum
+
+
+def select_topk(scores: np.ndarray, K: int) -> np.ndarray:
+    """Indices of the K largest scores, ties to the smaller index, returned in
+    ascending index order and padded with -1 when fewer than K keys exist.
+
+    The dense baseline is "dense scoring with Top-K selection" ([DPC]
+    Experiments, baselines).  Tie rule: smaller key index wins."""
+    n = int(scores.shape[0])
+    order = np.lexsort((np.arange(n), -scores))     # -score ascending, then index
+    chosen = np.sort(order[: min(K, n)])
+    out = np.full(K, -1, np.int64)
+    out[: chosen.shape[0]] = chosen
+    return out
+
+
+def dense_topk(q: np.ndarray, w: np.ndarray, k: np.ndarray, positions: np.ndarray,
+               K: int, rows=None) -> np.ndarray:
+    """Dense Top-K for every query row (or the listed ``rows``) of one sequence.
+
+    q: [T, H, d] real values, w: [T, H], k: [S, d] real values, positions: [T]
+    (query row i sees keys 0..positions[i], causal s <= t).  Returns [len(rows), K]."""
+    rows = range(q.shape[0]) if rows is None else rows
+    out = []
+    for t in rows:
+        p = int(positions[t])
+        out.append(select_topk(indexer_scores(q[t], w[t].astype(np.float64), k[: p + 1]), K))
+    return np.stack(out) if out else np.zeros((0, K), np.int64)
+
+
+# ----------------------------------------------------------------------------
+# Certificate ([DPC] Method: three stages; [ZICQ] Technical Mechanism Analysis).
+# ----------------------------------------------------------------------------
+
+
+def nnls_retained(Q_R: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """alpha = argmin_{alpha >= 0} || v - alpha @ Q_R ||  (Q_R: [r, d], v: [d]).
+
+    "Positive-weight heads are retained, while projections minimize their
+    residual norm" ([DPC] Method) with nonnegative coefficients ("nonnegative
+    head projections", [DPC] Conclusion; [ZICQ] point 2).  Solved exactly for
+    small r by trying every support: the NNLS optimum is the unconstrained
+    least-squares solution on its own support, so the best feasible candidate
+    over all supports is the optimum."""
+    r = Q_R.shape[0]
+    best_alpha = np.zeros(r)
+    best_res = float(v @ v)
+    for size in range(1, r + 1):
+        for support in itertools.combinations(range(r), size):
+            B = Q_R[list(support)]                       # [size, d]
+            a, *_ = np.linalg.lstsq(B.T, v, rcond=None)  # unconstrained LS on the support
+            if np.all(a >= 0.0):
+                res_vec = v - a @ B
+                res = float(res_vec @ res_vec)
+                if res < best_res:
+                    best_res = res
+                    best_alpha = np.zeros(r)
+                    best_alpha[list(support)] = a
+    return best_alpha
+
+
+@dataclass
+class Certificate:
+    """Per-query certificate: UB(k) = sum_j omega_j ReLU(q_j.k) + beta ||k||
+    - sum_g ReLU(u_g.k)."""
+    retained: np.ndarray                 # R: indices of the exactly evaluated heads
+    omega: np.ndarray                    # [|R|] folded weights of the retained heads
+    beta: float                          # joint residual coefficient (times ||k||)
+    beta_sum: float                      # the per-head Cauchy-Schwarz sum (for reports)
+    beta_joint: float                    # the joint (spectral) bound (for reports)
+    groups: list = field(default_factory=list)   # negative supports A_g (head indices)
+    u: np.ndarray = None                 # [G, d] aggregated negative directions
+
+
+def certificate_setup(q_t: np.ndarray, w_t: np.ndarray, k_bar: np.ndarray,
+                      r: int, G: int) -> Certificate:
+    """Build the certificate of one query (real-valued q_t [H, d], w_t [H]).
+
+    Stage 1, positive heads ([DPC] Method, "upper-bounding omitted positive
+    heads"; [ZICQ] 2 "nonnegative head projections and joint residual bounds to
+    limit positive contributions"):
+      P = {h : w_h > 0}; R = the r heads of P with the largest w_h ||q_h||
+      (ties to the smaller head).  For each omitted h in O = P \\ R,
+      alpha_h = NNLS projection onto the retained heads, rho_h its residual.
+      ReLU is positively homogeneous and subadditive, and alpha >= 0, so
+        ReLU(q_h.k) <= sum_j alpha_hj ReLU(q_j.k) + |rho_h.k|.
+      The retained heads reuse their computed dot products ([DPC] Method:
+      "retained positive heads reuse computed dot products"):
+        omega_j = w_j + sum_{h in O} w_h alpha_hj.
+      Joint residual bound: sum_h w_h |rho_h.k| <= beta ||k|| with
+        beta = min( sum_h w_h ||rho_h|| ,  sqrt( W_O * lambda_max(M) ) ),
+        W_O = sum_{h in O} w_h,  M = sum_{h in O} w_h rho_h rho_h^T
+      (the second is Cauchy-Schwarz with weights w_h, then the spectral norm:
+      it bounds all residual heads jointly).
+    Stage 2, negative heads ([DPC] Method: "negative heads are aggregated based
+    on support derived from activation patterns"; [ZICQ] 2 "activation-informed
+    aggregation to bound the magnitude subtracted by negative heads"):
+      for a >= 0, sum_{h in A} a_h ReLU(x_h) >= ReLU(sum_{h in A} a_h x_h).
+      N = {h : w_h < 0}.  A_1 = {h in N : q_h.k_bar > 0} (heads active on the
+      mean key), A_2 = N \\ A_1 when G >= 2.  u_g = sum_{h in A_g} |w_h| q_h.
+    Heads with w_h = 0 contribute nothing and are dropped."""
+    H = q_t.shape[0]
+    w = w_t.astype(np.float64)
+    qn = np.linalg.norm(q_t, axis=1)
+    P = [h for h in range(H) if w[h] > 0.0]
+    N = [h for h in range(H) if w[h] < 0.0]
+    # top-r of P by w_h ||q_h||, ties to the smaller head index
+    ranked = sorted(P, key=lambda h: (-(w[h] * qn[h]), h))
+    R = np.array(sorted(ranked[: min(r, len(P))]), np.int64)
+    O = [h for h in P if h not in set(R.tolist())]
+
+    omega = w[R].copy() if R.size else np.zeros(0)
+    rhos = []
+    for h in O:
+        alpha = nnls_retained(q_t[R], q_t[h]) if R.size else np.zeros(0)
+        omega = omega + w[h] * alpha
+        rhos.append(q_t[h] - (alpha @ q_t[R] if R.size else 0.0))
+    if O:
+        rho = np.array(rhos)                              # [|O|, d]
+        wO = w[O]
+        beta_sum = float(np.sum(wO * np.linalg.norm(rho, axis=1)))
+        Ws = np.sqrt(wO)[:, None] * rho
+        lam = float(np.linalg.eigvalsh(Ws @ Ws.T)[-1])    # lambda_max(M) via the Gram matrix
+        beta_joint = math.sqrt(float(wO.sum()) * max(lam, 0.0))
+        beta = min(beta_sum, beta_joint)
+    else:
+        beta_sum = beta_joint = beta = 0.0
+
+    groups = []
+    if G >= 1 and N:
+        act = q_t[N] @ k_bar
+        A1 = [h for h, a in zip(N, act) if a > 0.0]
+        groups.append(np.array(A1, np.int64))
+        if G >= 2:
+            groups.append(np.array([h for h in N if h not in set(A1)], np.int64))
+    d = q_t.shape[1]
+    u = np.zeros((len(groups), d))
+    for g, A in enumerate(groups):
+        if A.size:
+            u[g] = (np.abs(w[A])[:, None] * q_t[A]).sum(axis=0)
+    return Certificate(R, omega, beta, beta_sum, beta_joint, groups, u)
+
+
+def upper_bound(cert: Certificate, q_t: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """Stage 3, the combined bound ([DPC] Method: "a unified score certificate
+    that combines these retained and bounded contributions"):
+      UB(s) = sum_j omega_j ReLU(q_j.k_s) + beta ||k_s|| - sum_g ReLU(u_g.k_s).
+    k: [n, d] real values.  UB(s) >= I(t,s) for every key (tests pin this)."""
+    ub = cert.beta * np.linalg.norm(k, axis=1)
+    if cert.retained.size:
+        ub = ub + np.maximum(k @ q_t[cert.retained].T, 0.0) @ cert.omega
+    for g in range(cert.u.shape[0]):
+        ub = ub - np.maximum(k @ cert.u[g], 0.0)
+    return ub
+
+
+def soundness_margin(q_t: np.ndarray, w_t: np.ndarray, k: np.ndarray,
+                     margin_log2: int) -> np.ndarray:
+    """delta(t,s) = 2^margin_log2 * (sum_h |w_h| ||q_h||) * ||k_s||.
+
+    The pages are silent on rounding.  A GPU evaluates the bound and the score
+    in fp32 with different arithmetic, so a candidate is rejected only when
+    UB + delta < tau.  delta dominates the fp32 error of both sides."""
+    c = float(np.sum(np.abs(w_t.astype(np.float64)) * np.linalg.norm(q_t, axis=1)))
+    return math.ldexp(c, margin_log2) * np.linalg.norm(k, axis=1)
+
+
+def seed_mask(p: int, seed_first: int, seed_last: int) -> np.ndarray:
+    """Seed subset of the visible keys 0..p: the first ``seed_first`` keys and the
+    last ``seed_last`` keys ending at p ([DPC] Method: "choosing a subset of
+    visible keys ... and setting a threshold based on the K-th largest score
+    within this subset")."""
+    s = np.arange(p + 1)
+    return (s < seed_first) | (s > p - seed_last)
+
+
+def key_mean(k: np.ndarray) -> np.ndarray:
+    """Mean key of a sequence: the direction on which head activation is read
+    when choosing the negative support."""
+    return k.mean(axis=0) if k.shape[0] else np.zeros(k.shape[1])
+
+
+def _kth_largest(values: np.ndarray, K: int) -> float:
+    if values.shape[0] < K:
+        return -math.inf
+    return float(np.partition(values, values.shape[0] - K)[values.shape[0] - K])
+
+
+def certified_topk_row(q_t, w_t, k_vis, K, *, k_bar, r=4, G=2, seed_first=64,
+                       seed_last=512, margin_log2=-12, tile=128) -> dict:
+    """One query through the certified pipeline ([DPC] Method, candidate
+    refinement: screening dot products, bound evaluation, pruning and score
+    compaction, repeated for every tile of visible keys).
+
+      1. Exact scores on the seed subset; tau = their K-th largest (-inf while
+         fewer than K exact scores exist).
+      2. The remaining keys, in tiles of ``tile`` keys aligned to absolute key
+         positions, from the diagonal downwards: a key is rejected when
+         UB + delta < tau; every survivor is scored with all heads.  After
+         each tile tau is raised to the K-th largest exact score so far (any
+         such K-th is a lower bound on the true K-th).
+      3. Top-K over the exactly scored keys.
+
+    k_vis: [p+1, d] real values of the visible keys.  Returns the selection and
+    the counts used for the prune rate ([DPC] Experiments: "percentage of
+    query-key pairs removed during certificate screening")."""
+    n = k_vis.shape[0]
+    p = n - 1
+    w64 = w_t.astype(np.float64)
+    cert = certificate_setup(q_t, w64, k_bar, r, G)
+    exact = np.full(n, np.nan)
+    seeds = seed_mask(p, seed_first, seed_last)
+    exact[seeds] = indexer_scores(q_t, w64, k_vis[seeds])
+    tau0 = _kth_largest(exact[seeds], K)
+    tau = tau0
+    ub = upper_bound(cert, q_t, k_vis)
+    delta = soundness_margin(q_t, w64, k_vis, margin_log2)
+    rejected = np.zeros(n, bool)
+    rest = np.nonzero(~seeds)[0]
+    if rest.size:
+        for tile_start in range((int(rest.max()) // tile) * tile, -1, -tile):
+            sel = rest[(rest >= tile_start) & (rest < tile_start + tile)]
+            if sel.size == 0:
+                continue
+            rej = ub[sel] + delta[sel] < tau
+            rejected[sel[rej]] = True
+            keep = sel[~rej]
+            if keep.size:
+                exact[keep] = indexer_scores(q_t, w64, k_vis[keep])
+            tau = max(tau, _kth_largest(exact[~np.isnan(exact)], K))
+    scored = np.nonzero(~np.isnan(exact))[0]
+    vals = exact[scored]
+    order = np.lexsort((scored, -vals))
+    chosen = np.sort(scored[order[: min(K, scored.size)]])
+    idx = np.full(K, -1, np.int64)
+    idx[: chosen.size] = chosen
+    # ideal screening: tau equal to the true K-th score
+    full = indexer_scores(q_t, w64, k_vis)
+    vK = _kth_largest(full, K)
+    ideal_rej = (~seeds) & (ub + delta < vK)
+    return {
+        "idx": idx, "tau0": tau0, "tau_final": tau, "v_K": vK,
+        "visible": n, "seed": int(seeds.sum()), "screened": int((~seeds).sum()),
+        "rejected": int(rejected.sum()), "ideal_rejected": int(ideal_rej.sum()),
+        "cert": cert, "ub": ub, "delta": delta, "scores": full,
+    }
+
+
+def certified_topk(q, w, k, positions, K, rows=None, **kw) -> tuple[np.ndarray, dict]:
+    """certified_topk_row over several rows of one sequence; returns the
+    selections and summed counts (visible, seed, screened, rejected, ideal)."""
+    rows = range(q.shape[0]) if rows is None else rows
+    k_bar = kw.pop("k_bar", None)
+    if k_bar is None:
+        k_bar = key_mean(k)
+    out, tot = [], {"visible": 0, "seed": 0, "screened": 0, "rejected": 0, "ideal_rejected": 0}
+    for t in rows:
+        p = int(positions[t])
+        res = certified_topk_row(q[t], w[t], k[: p + 1], K, k_bar=k_bar, **kw)
+        out.append(res["idx"])
+        for key in tot:
+            tot[key] += res[key]
+    return (np.stack(out) if out else np.zeros((0, K), np.int64)), tot
