@@ -1,0 +1,396 @@
+#!/usr/bin/env python3
+"""Throughput of the DoSA indexer Top-K on B200s (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--path certified|dense]
+
+A step is one pass of the whole indexer (every row of the workload through
+the library's Top-K call) over inputs already resident in HBM.  The headline
+workload is 128K-token causal prefill with fp8 e4m3 inputs, H = 64, d = 128,
+K = 2048.  With N > 1 (torchrun) every rank processes its own independent
+sequence of the same shape (weak scaling, no collective on the data path); the
+step time is the max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_certified_top_b200.workloads import WORKLOADS, generate  # noqa: E402
+
+METRIC = "indexer query·key pairs/sec @128K causal, K=2048 (1 B200); prune %; % roofline"
+UNIT = "pairs/s"
+L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_128k_fp8", choices=sorted(WORKLOADS))
+    ap.add_argument("--path", choices=["certified", "dense"], default="certified")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the oracle CPU baseline sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+CLOCK_FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+                "clocks_event_reasons.active", "clocks_event_reasons.hw_slowdown",
+                "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+def clocks_start(local_rank):
+    path = tempfile.mktemp(prefix="dosa_clocks_", suffix=".csv")
+    try:
+        f = open(path, "w")
+        p = subprocess.Popen(["nvidia-smi", "-i", str(local_rank),
+                              "--query-gpu=" + ",".join(CLOCK_FIELDS),
+                              "--format=csv,noheader,nounits", "-lms", "200"],
+                             stdout=f, stderr=subprocess.DEVNULL)
+        return p, f, path
+    except (OSError, FileNotFoundError):
+        return None
+
+
+def clocks_stop(handle):
+    if handle is None:
+        return None
+    p, f, path = handle
+    p.terminate()
+    try:
+        p.wait(timeout=5)
+    except subprocess.TimeoutExpired:
+        p.kill()
+    f.close()
+    rows = []
+    with open(path) as fh:
+        for line in fh:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(CLOCK_FIELDS):
+                rows.append(parts)
+    os.unlink(path)
+    if not rows:
+        return None
+
+    def num(x):
+        try:
+            return float(x)
+        except ValueError:
+            return float("nan")
+    loaded = [r for r in rows if num(r[4]) >= 50] or rows
+    reasons = set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in loaded:
+        for n, v in zip(names, r[6:10]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(num(r[1]) for r in loaded),
+            "sm_max_mhz": max(num(r[2]) for r in rows),
+            "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
+            "power_w_max": max(num(r[3]) for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# roofline
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str):
+    """Dominant kernel of the step against the tensor-core peak of its dtype."""
+    peaks, src = measured_peaks()
+    kernels = {k: v for k, v in prof.items() if v[0] > 0}
+    if not kernels:
+        return None
+    dom = max(kernels, key=lambda k: kernels[k][1])
+    launches, ms = kernels[dom]
+    flops_per_pair = 2 * wl.H * wl.d
+    # bf16 sustained peak (the kernel runs inside a long step); fp8 = 2x (nominal ratio)
+    peak = peaks["bf16_tflops_sustained"] * (2.0 if dtype == "fp8" else 1.0)
+    traffic = None
+    if dom == "score":
+        work = flops_per_pair * pairs_per_step * steps          # every visible pair, once
+        achieved = work / (ms * 1e-3) / 1e12
+        traffic = _traffic_per_launch("score", wl, pairs_per_step * steps / launches)
+        return {"kernel": "score_tc", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic, "peak_source": f"{src}: bf16_tflops_sustained"
+                + (" x2 (fp8/bf16 nominal ratio)" if dtype == "fp8" else ""),
+                "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
+    return {"kernel": dom, "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
+
+
+def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
+    """DRAM bytes per launch from a committed ncu summary, scaled by pairs, or
+    None when no capture matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(f"{kernel}:{wl.dtype}")
+    if not rec or rec.get("source_sha") != _kernel_source_sha():
+        return None
+    return round(rec["dram_bytes_per_pair"] * pairs_per_launch)
+
+
+def _kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("score_tc.cu", "score_epilogue.cuh", "dosa_device.cuh"):
+        with open(os.path.join(ROOT, "exact_certified_top_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of rows
+
+def oracle_sample(x, wl, budget_s: float):
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle import dense_topk, dequantize
+    from exact_certified_top_b200.workloads import codes_numpy
+    from threadpoolctl import threadpool_info
+    # rows spread evenly over the workload, visited in an interleaved order
+    order = np.linspace(0, wl.T - 1, 64).astype(np.int64)
+    order = np.concatenate([order[::2], order[1::2]])
+    kscale = None if x["k_scale"] is None else x["k_scale"].cpu().numpy()
+    k = dequantize(codes_numpy(x["k"]), kscale, wl.dtype)
+    pos = x["positions"].cpu().numpy()
+    done, pairs = [], 0
+    t0 = time.perf_counter()
+    for t in order:
+        q_t = x["q"][t:t + 1]
+        qs = None if x["q_scale"] is None else x["q_scale"][t:t + 1].cpu().numpy()
+        q = dequantize(codes_numpy(q_t), qs, wl.dtype)
+        w = x["w"][t:t + 1].cpu().numpy().astype(np.float64)
+        dense_topk(q, w, k, pos[t:t + 1], wl.K)
+        done.append(int(t))
+        pairs += int(pos[t]) + 1
+        if time.perf_counter() - t0 > budget_s and len(done) >= 2:
+            break
+    el = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": pairs / el, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{len(done)} rows of {wl.name} spread evenly over positions "
+                      f"(pairs {pairs}), fp64 dense scoring + full sort, {el:.1f} s",
+            "host_cores": os.cpu_count()}
+
+
+# ---------------------------------------------------------------------------
+
+def config_of(wl, path, world):
+    return {"workload": wl.name, "T": wl.T, "S": wl.S, "H": wl.H, "d": wl.d, "K": wl.K,
+            "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, "parallelism": f"rows x{world}",
+            "l2": "flushed between timed steps (256 MiB write, outside the timed windows)",
+            "visible_pairs_per_gpu": wl.visible_pairs}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = generate(wl, device=dev)
+    per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(x, wl, per_step / 4)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample(x, wl, per_step)
+        vals.append(last["value"])
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, "oracle", world),
+            "cpu_baseline": {**last, "value": v},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from exact_certified_top_b200 import binding
+    binding.load()
+    wl = WORKLOADS[args.workload]
+    base_seed = wl.seed
+    from dataclasses import replace
+    wl_r = replace(wl, seed=base_seed + rank)        # independent sequence per rank
+    x = generate(wl_r, device="cuda")
+    idx = binding.Index(wl.dtype, max_K=max(2048, wl.K))
+    certified = args.path == "certified"
+    so = x["seq_offsets"]
+    ws = torch.zeros(idx.workspace_size(wl.T, wl.S, wl.K, certified), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    call_args = (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], so, wl.K)
+
+    def step(o=out, a=call_args):
+        if certified:
+            idx.topk(*a, out=o, workspace=ws)
+        else:
+            idx.dense_topk(*a, out=o, workspace=ws)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    binding.check_device(ws)
+
+    # timed region: per-step CUDA events, L2 flushed between steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = clocks_start(local)
+    binding.profile_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    prof = binding.profile_read()
+    binding.profile_enable(False)
+    clocks = clocks_stop(clk)
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(ms, world)
+    binding.check_device(ws)
+
+    pairs = wl.visible_pairs
+    value = world * pairs / (ms * 1e-3)
+    launches = sum(n for n, _ in prof.values())
+
+    stats = None
+    if certified:
+        _, stats = idx.topk(*call_args, out=out, workspace=ws, stats=True)
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) and v.is_cuda else v)
+                for k, v in x.items()}
+        names = ["q", "q_scale", "w", "k", "k_scale"]
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names if host[n] is not None)
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        d2h = out_host.numel() * out_host.element_size()
+        dev_in = {n: (torch.empty_like(x[n]) if x[n] is not None else None) for n in names}
+
+        def e2e_step():
+            for n in names:
+                if host[n] is not None:
+                    dev_in[n].copy_(host[n], non_blocking=True)
+            a = (dev_in["q"], dev_in["q_scale"], dev_in["w"], dev_in["k"], dev_in["k_scale"], so,
+                 wl.K)
+            step(out, a)
+            out_host.copy_(out, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        n_e2e = max(1, min(args.steps, 3))
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        e2e = {"value": world * pairs / (ems * 1e-3), "unit": UNIT, "ms_per_step": round(ems, 3),
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(x, wl, args.cpu_seconds)
+
+    if rank == 0:
+        roof = roofline(prof, wl, pairs, args.steps, wl.dtype)
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": wl.dtype, "data": "synthetic (seeded low-rank + sink generator)",
+                "config": config_of(wl, args.path, world), "roofline": roof,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+                "kernels": {k: {"launches": n, "ms": round(t, 3)} for k, t in
+                            ((k, v[1]) for k, v in prof.items()) for n in [prof[k][0]] if n},
+                "clocks": clocks}
+        if stats:
+            vis = stats["visible_pairs"]
+            line["prune_pct"] = round(100.0 * stats["rejected_pairs"] / vis, 3) if vis else None
+            line["stats"] = stats
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_init(args)
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+/*
+ * dosa.h -- C ABI of libdosa, the B200 (sm_100a) DoSA certified indexer Top-K.
+ *
+ * The operation.  For a query row t with H indexer heads q[t,h] (head dim d),
+ * signed head weights w[t,h] and keys k[s] shared by all heads, the indexer
+ * score is
+ *     I(t,s) = sum_h w[t,h] * ReLU(q[t,h] . k[s]),     causal: s <= pos(t),
+ * and the result is the K keys with the largest I (ties to the smaller key
+ * index).  Source: "DOSA: Dots Sparse Attention", Daily Paper Cast transcript,
+ * Method section (problem formulation: one query with several indexer heads,
+ * each with its own query vector and weight, scored against shared keys; the
+ * top K keys by score) and Experiments section (the dense baseline is "dense
+ * scoring with Top-K selection", K = 2048).  The certified entry point returns
+ * the same selection while scoring only the keys a certificate cannot reject
+ * (same transcript, Method section: seed threshold, three bound stages,
+ * candidate refinement per key tile; "Xiaohongshu DoSA sparse attention cuts
+ * TTFT by up to 48% via score bounds", section 02: the original scoring
+ * function is kept and every unrejected candidate is scored with all heads).
+ *
+ * Conventions shared by every entry point
+ *  - Device pointers unless stated otherwise; the caller owns every buffer.
+ *    The library allocates no device memory during a call: scratch space is
+ *    the caller's workspace (size from dosa_index_workspace_size).
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = the
+ *    legacy default stream) and is asynchronous unless a `stats` pointer is
+ *    given, in which case the call synchronises `stream` to read counters.
+ *  - Arguments are validated on the host before anything is launched.  A
+ *    device-side bounded wait that expires, or a device bounds check that
+ *    fires, is reported as DOSA_ERR_TIMEOUT / DOSA_ERR_DEVICE_CHECK by the
+ *    call that reads it back (any call given `stats`, or dosa_check_device).
+ *
+ * Layouts
+ *  - q:       [Tq, H, d] row-major codes: bf16 (2 bytes) or OCP FP8 E4M3
+ *             (1 byte).  Base 16-byte aligned.
+ *  - q_scale: [Tq] fp32 per-token scales (E4M3 only; NULL for bf16).  The real
+ *             query is q_scale[t] * decode(q[t,h,:]).
+ *  - w:       [Tq, H] fp32.
+ *  - k:       [S, d] row-major codes, same dtype as q.  Base 16-byte aligned.
+ *  - k_scale: [S] fp32 per-token scales (E4M3 only; NULL for bf16).
+ *  - seq_offsets: HOST array of (B+1) x 3 int64, a packed varlen batch.  Row b
+ *             = {q_row_start[b], k_start[b], q_pos0[b]}; row B = {Tq, S, 0}.
+ *             Sequence b owns query rows [q_row_start[b], q_row_start[b+1]) and
+ *             keys [k_start[b], k_start[b+1]).  Its query row i sits at position
+ *             q_pos0[b] + (i - q_row_start[b]) among its own keys and sees keys
+ *             0..position (causal).  Requires position < number of its keys.
+ *             (Chunked prefill: queries at an offset against a cached key
+ *             prefix -- same transcript, Experiments section, chunks of 4K-32K.)
+ *  - out_idx: [Tq, K] int32.  Per row: the selected key indices, relative to
+ *             the sequence's first key, in ascending order; rows with fewer
+ *             than K visible keys list all of them and pad with -1.
+ */
+#ifndef DOSA_H_
+#define DOSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DOSA_OK = 0,
+  DOSA_ERR_INVALID_ARG = 1,   /* a pointer, size, layout or alignment is wrong */
+  DOSA_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. d != 128)           */
+  DOSA_ERR_WORKSPACE = 3,     /* workspace smaller than dosa_index_workspace_size */
+  DOSA_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, sync, ...) */
+  DOSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired             */
+  DOSA_ERR_DEVICE_CHECK = 6   /* a device-side bounds check fired               */
+} dosa_status;
+
+typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
+
+/* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
+ * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
+ * margin_log2 = -12, screening = 1. */
+typedef struct {
+  int H;            /* indexer heads per query (multiple of 4, <= 64)          */
+  int d;            /* head dimension (128 in this build)                       */
+  dosa_dtype dtype; /* storage type of q and k                                  */
+  int max_K;        /* largest K the handle will be called with (<= 4096)      */
+  int seed_first;   /* seed subset: the first seed_first keys ...               */
+  int seed_last;    /* ... and the last seed_last keys ending at the query      */
+  int r;            /* retained positive heads evaluated exactly (0..4)         */
+  int G;            /* negative-head groups (0 = no negative aggregate, 1, 2)   */
+  int margin_log2;  /* soundness margin 2^margin_log2 * sum|w|||q|| * ||k||     */
+  int screening;    /* 1: reject by certificate; 0: score every key (ablation)  */
+} dosa_index_config;
+
+/* Counters of the last certified call (filled when `stats` is non-NULL). */
+typedef struct {
+  int64_t visible_pairs;   /* sum over rows of (position + 1)                        */
+  int64_t seed_pairs;      /* pairs scored exactly as seeds                          */
+  int64_t screened_pairs;  /* non-seed pairs whose bound was evaluated               */
+  int64_t rejected_pairs;  /* screened pairs rejected (bound + margin < threshold)   */
+  int64_t exact_pairs;     /* pairs scored with all heads (seeds + survivors)        */
+  int64_t candidates;      /* (score, index) pairs written for the final selection   */
+} dosa_stats;
+
+typedef struct dosa_index* dosa_index_t;
+
+/* Fill *cfg with the defaults listed above. */
+void dosa_index_config_default(dosa_index_config* cfg);
+
+/* Validate cfg and create a handle (host memory only; it holds the config and
+ * per-device kernel attributes).  Errors: INVALID_ARG for NULL or out-of-range
+ * fields, UNSUPPORTED for d != 128 or H not a multiple of 4 in [4, 64]. */
+dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out);
+
+/* Free a handle (NULL is accepted). */
+void dosa_index_destroy(dosa_index_t h);
+
+/* Bytes of device workspace a call needs for a batch of Tq query rows, at most
+ * S_max keys in one sequence, and K.  `certified` selects dosa_index_topk (1)
+ * or dosa_index_dense_topk (0).  The dense path's workspace holds one chunk of
+ * fp32 score rows; `chunk_rows` (0 = library choice) sets its height. */
+dosa_status dosa_index_workspace_size(dosa_index_t h, int64_t Tq, int64_t S_max, int K,
+                                      int certified, int64_t chunk_rows, size_t* bytes);
+
+/* Certified Top-K (the DoSA pipeline): key prep, certificate setup, seed
+ * scoring, bound screening, survivor rescoring with all heads, threshold
+ * filtering with packed writeback, radix selection.  Returns exactly the
+ * selection of dosa_index_dense_topk.  Workspace: dosa_index_workspace_size
+ * with certified = 1. */
+dosa_status dosa_index_topk(dosa_index_t h, const void* q, const float* q_scale, const float* w,
+                            const void* k, const float* k_scale, const int64_t* seq_offsets,
+                            int B, int K, int32_t* out_idx, void* workspace, size_t ws_bytes,
+                            void* stream, dosa_stats* stats);
+
+/* Dense Top-K: every visible key is scored with all heads (tensor-core scorer),
+ * score rows are materialised chunk by chunk in the workspace, then a per-row
+ * radix select picks the K largest.  The reference the certified path must
+ * match bit for bit.  Workspace: certified = 0. */
+dosa_status dosa_index_dense_topk(dosa_index_t h, const void* q, const float* q_scale,
+                                  const float* w, const void* k, const float* k_scale,
+                                  const int64_t* seq_offsets, int B, int K, int32_t* out_idx,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Dense scorer alone, for one sequence: scores[i * ld + s] = I(row0 + i, s) for
+ * rows row0..row0+rows-1 of q (positions pos0 + i) and s = 0..position; other
+ * entries are left untouched.  k points at the sequence's first key, S is its
+ * key count.  `scratch` is 16 bytes of zeroed device memory (error word). */
+dosa_status dosa_index_scores(dosa_index_t h, const void* q, const float* q_scale, const float* w,
+                              const void* k, const float* k_scale, int64_t row0, int64_t rows,
+                              int64_t pos0, int64_t S, float* scores, int64_t ld, void* scratch,
+                              void* stream);
+
+/* Plain CUDA-core scorer with the same contract as dosa_index_scores (fp32
+ * FMAs, no tensor cores): a cross-check for the tensor-core path. */
+dosa_status dosa_reference_scores(dosa_index_t h, const void* q, const float* q_scale,
+                                  const float* w, const void* k, const float* k_scale,
+                                  int64_t row0, int64_t rows, int64_t pos0, int64_t S,
+                                  float* scores, int64_t ld, void* stream);
+
+/* Per-row exact Top-K of fp32 score rows (radix select; ties to the smaller
+ * index; -0.0 equals +0.0): row i has n_i = row_len[i] (device int64 array)
+ * scores at scores + i * ld; out[i * K ...] as for out_idx.  NaN scores are
+ * not allowed. */
+dosa_status dosa_topk_rows(const float* scores, int64_t ld, const int64_t* row_len, int64_t rows,
+                           int K, int32_t* out, void* stream);
+
+/* Read back and clear the device error word of the last calls on `stream`
+ * (synchronises it). */
+dosa_status dosa_check_device(void* workspace, void* stream);
+
+/* Kernel kinds reported by the profiling counters. */
+typedef enum {
+  DOSA_KERNEL_SCORE = 0,       /* tensor-core scorer (dense scores)            */
+  DOSA_KERNEL_TOPK = 1,        /* per-row radix select                         */
+  DOSA_KERNEL_REFERENCE = 2,   /* CUDA-core reference scorer                   */
+  DOSA_KERNEL_KEY_PREP = 3,    /* key norms and key mean                       */
+  DOSA_KERNEL_CERT_SETUP = 4,  /* per-query certificate                        */
+  DOSA_KERNEL_CERTIFIED = 5,   /* seed scoring, screening, rescoring, writeback */
+  DOSA_KERNEL_SELECT = 6,      /* selection over the packed candidates         */
+  DOSA_KERNEL_KINDS = 7
+} dosa_kernel;
+
+/* Kernel timing.  While enabled, every kernel a call launches is bracketed by
+ * CUDA events recorded on the call's stream (host-side cost: two event records
+ * per launch; the events are created once and reused).  dosa_profile_read
+ * synchronises on the recorded events and returns, for one kernel kind, the
+ * number of launches and their summed device time in milliseconds since the
+ * last reset.  Enabling or resetting discards earlier records.  Not
+ * thread-safe: profile from one host thread. */
+dosa_status dosa_profile_enable(int on);
+dosa_status dosa_profile_reset(void);
+dosa_status dosa_profile_read(int kind, int64_t* launches, double* ms);
+
+/* Static description of a status code. */
+const char* dosa_status_string(dosa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DOSA_H_ */
