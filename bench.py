@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--path", choices=["certified", "dense"], default="certified")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU baseline sample")
+    ap.add_argument("--tail-rows", type=int, default=0,
+                    help="profile only the last N query rows of the workload (same keys)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -98,7 +100,8 @@ def clocks_start(local_rank):
                               "--format=csv,noheader,nounits", "-lms", "200"],
                              stdout=f, stderr=subprocess.DEVNULL)
         return p, f, path
-    except (OSError, FileNotFoundError):
+    except (OSError, FileNotFoundError) as e:
+        print(f"clock sampling unavailable: {e}", file=sys.stderr)
         return None
 
 
@@ -206,8 +209,12 @@ def oracle_sample(x, wl, budget_s: float):
     from exact_certified_top_b200.workloads import codes_numpy
     from threadpoolctl import threadpool_info
     # rows spread evenly over the workload, visited in an interleaved order
-    order = np.linspace(0, wl.T - 1, 64).astype(np.int64)
-    order = np.concatenate([order[::2], order[1::2]])
+    # bit-reversal order over 1024 evenly spaced rows: any prefix is spread out
+    n_s = min(1024, wl.T)
+    base = np.linspace(0, wl.T - 1, n_s).astype(np.int64)
+    bits = max(1, int(np.ceil(np.log2(n_s))))
+    rev = [int(format(i, f"0{bits}b")[::-1], 2) for i in range(1 << bits)]
+    order = base[[r for r in rev if r < n_s]]
     kscale = None if x["k_scale"] is None else x["k_scale"].cpu().numpy()
     k = dequantize(codes_numpy(x["k"]), kscale, wl.dtype)
     pos = x["positions"].cpu().numpy()
@@ -243,7 +250,7 @@ def config_of(wl, path, world):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     x = generate(wl, device=dev)
     per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
@@ -264,10 +271,19 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def workload_of(args):
+    wl = WORKLOADS[args.workload]
+    if args.tail_rows:
+        from dataclasses import replace
+        n = min(args.tail_rows, wl.T)
+        wl = replace(wl, name=f"{wl.name}[last {n} rows]", T=n, q_pos0=wl.q_pos0 + wl.T - n)
+    return wl
+
+
 def run_ours(args, world, rank, local):
     from exact_certified_top_b200 import binding
     binding.load()
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     base_seed = wl.seed
     from dataclasses import replace
     wl_r = replace(wl, seed=base_seed + rank)        # independent sequence per rank
