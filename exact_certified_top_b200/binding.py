@@ -23,7 +23,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
 # Every function the public header declares (the CPU tests check the export).
 EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy",
            "dosa_index_workspace_size", "dosa_index_topk", "dosa_index_dense_topk",
-           "dosa_index_scores", "dosa_reference_scores", "dosa_topk_rows", "dosa_check_device",
+           "dosa_index_scores", "dosa_reference_scores", "dosa_index_certificate", "dosa_topk_rows", "dosa_check_device",
            "dosa_status_string", "dosa_profile_enable", "dosa_profile_reset",
            "dosa_profile_read")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
@@ -78,6 +78,7 @@ def load(path: str = LIB_PATH):
                                       _P, _P]
     lib.dosa_reference_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P,
                                           _I64, _P]
+    lib.dosa_index_certificate.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]
     lib.dosa_topk_rows.argtypes = [_P, _I64, _P, _I64, _I, _P, _P]
     lib.dosa_check_device.argtypes = [_P, _P]
     lib.dosa_profile_enable.argtypes = [_I]
@@ -180,6 +181,18 @@ class Index:
             ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, K, _ptr(out), _ptr(ws),
             ws.numel(), _stream(), ctypes.byref(st) if stats else None))
         return (out, st.as_dict()) if stats else out
+
+    def certificate(self, q, q_scale, w, k, k_scale, seq_offsets, workspace=None):
+        """Per-query certificate records [Tq, 16] (code domain) and retained heads [Tq, 4]."""
+        so = _seq_offsets(seq_offsets)
+        cert = torch.empty((q.shape[0], 16), dtype=torch.float32, device=q.device)
+        ret = torch.empty((q.shape[0], 4), dtype=torch.int32, device=q.device)
+        ws = self._workspace(q, so, 1, True, workspace)
+        _check("dosa_index_certificate", self._lib.dosa_index_certificate(
+            self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
+            ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, _ptr(cert), _ptr(ret), _ptr(ws),
+            ws.numel(), _stream()))
+        return cert, ret
 
     def scores(self, q, q_scale, w, k, k_scale, row0, rows, pos0, S, out, ld, scratch):
         _check("dosa_index_scores", self._lib.dosa_index_scores(

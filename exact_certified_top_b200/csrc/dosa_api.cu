@@ -6,6 +6,7 @@
 #include <mutex>
 #include <new>
 
+#include "cert_layout.h"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
 
@@ -96,8 +97,90 @@ SeqView make_view(const Handle* h, const void* q, const float* q_scale, const fl
 }
 
 constexpr int64_t kDefaultChunkBytes = (int64_t)4 << 30;   // dense score chunk budget
+constexpr int kRepairRows = 64;                             // overflowed rows per chunk
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Candidate capacity per query row: 16 K (at least 4096), never more than
+// the keys of the longest sequence (a row cannot have more candidates).
+int cand_capacity(int K, int64_t S_max) {
+  int64_t cap = 16 * (int64_t)K;
+  if (cap < 4096) cap = 4096;
+  if (cap > S_max) cap = S_max;
+  if (cap < 1) cap = 1;
+  return (int)cap;
+}
+
+// Workspace of the certified path: a fixed part (header, key norms, key sum,
+// repair area) and Tc rows of per-query state.
+struct CertLayout {
+  size_t key_norm, key_sum, repair_list, repair_count, repair_scores, fixed;
+  size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
+  int cap;
+};
+
+CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
+  CertLayout L;
+  size_t off = kWsHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (size_t)round_up((int64_t)bytes, 256);
+    return at;
+  };
+  L.cap = cand_capacity(K, S_max);
+  L.key_norm = take((size_t)S_max * 4);
+  L.key_sum = take(kHeadDim * 4);
+  L.repair_list = take(kRepairRows * 4);
+  L.repair_count = take(4);
+  L.repair_scores = take((size_t)kRepairRows * S_max * 4);
+  L.fixed = off;
+  L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
+              (size_t)L.cap * 8 + 4 + 4;
+  return L;
+}
+
+// Carve the per-row arrays of a chunk of Tc rows after the fixed part.
+CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int64_t Tc) {
+  CertBuffers b;
+  size_t off = L.fixed;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = ws + off;
+    off += (size_t)round_up((int64_t)bytes, 256);
+    return p;
+  };
+  b.key_norm = reinterpret_cast<float*>(ws + L.key_norm);
+  b.key_sum = reinterpret_cast<float*>(ws + L.key_sum);
+  b.repair_list = reinterpret_cast<int*>(ws + L.repair_list);
+  b.repair_count = reinterpret_cast<int*>(ws + L.repair_count);
+  b.repair_scores = reinterpret_cast<float*>(ws + L.repair_scores);
+  b.repair_cap = kRepairRows;
+  b.cap = L.cap;
+  b.bdir = take((size_t)Tc * kBoundRows * kHeadDim * elem_bytes(h));
+  b.cert = reinterpret_cast<float*>(take((size_t)Tc * kCertFloats * 4));
+  b.retained = reinterpret_cast<int32_t*>(take((size_t)Tc * 16));
+  b.cand = take((size_t)Tc * L.cap * 8);
+  b.cand_count = reinterpret_cast<int*>(take((size_t)Tc * 4));
+  b.tau = reinterpret_cast<float*>(take((size_t)Tc * 4));
+  b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
+  b.err = &reinterpret_cast<WsHeader*>(ws)->error;
+  return b;
+}
+
+// Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
+int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
+  if (ws_bytes <= L.fixed + 6 * 256) return 0;
+  int64_t rows = (int64_t)((ws_bytes - L.fixed - 6 * 256) / L.per_row);
+  return rows / 8 * 8;
+}
+
+int64_t total_visible(const int64_t* so, int B) {
+  int64_t v = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t nq = so[3 * (b + 1)] - so[3 * b], p0 = so[3 * b + 2];
+    v += nq * (2 * p0 + nq + 1) / 2;
+  }
+  return v;
+}
 
 }  // namespace
 
@@ -153,7 +236,20 @@ dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max
   const Handle* h = reinterpret_cast<const Handle*>(hh);
   if (!h || !bytes || Tq < 0 || S_max < 0 || K < 1 || K > h->cfg.max_K || chunk_rows < 0)
     return DOSA_ERR_INVALID_ARG;
-  if (certified) return DOSA_ERR_UNSUPPORTED;
+  if (certified) {
+    const CertLayout L = cert_layout(h, S_max, K);
+    int64_t rows = chunk_rows;
+    if (rows == 0) {
+      rows = kDefaultChunkBytes / (int64_t)L.per_row;
+      rows = rows / 8 * 8;
+      if (rows < 8) rows = 8;
+    }
+    rows = round_up(rows, 8);
+    if (rows > round_up(Tq, 8)) rows = round_up(Tq, 8);
+    if (rows < 8) rows = 8;
+    *bytes = L.fixed + (size_t)rows * L.per_row + 6 * 256;
+    return DOSA_OK;
+  }
   int64_t rows = chunk_rows;
   if (rows == 0) {
     rows = S_max > 0 ? kDefaultChunkBytes / (S_max * 4) : Tq;
@@ -199,13 +295,106 @@ dosa_status dosa_index_dense_topk(dosa_index_t hh, const void* q, const float* q
   return DOSA_OK;
 }
 
+}  // extern "C"
+
+// Runs key prep and certificate setup for one sequence chunk by chunk, calling
+// `body(chunk view, buffers)` after each setup.
+template <typename Body>
+static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const float* q_scale,
+                                       const float* w, const void* k, const float* k_scale,
+                                       const int64_t* seq_offsets, int B, int K, void* workspace,
+                                       size_t ws_bytes, cudaStream_t stream, float* cert_out,
+                                       int32_t* retained_out, Body body) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DOSA_ERR_INVALID_ARG;
+  const int64_t S_max = max_keys(seq_offsets, B);
+  const CertLayout L = cert_layout(h, S_max, K);
+  const int64_t Tc = cert_chunk_rows(L, ws_bytes);
+  if (Tc < 8) return DOSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+  CertBuffers buf = cert_buffers(h, L, ws, Tc);
+  for (int b = 0; b < B; ++b) {
+    const SeqInfo s = seq_info(seq_offsets, b);
+    const SeqView v = make_view(h, q, q_scale, w, k, k_scale, s);
+    if (v.rows == 0) continue;
+    if (launch_key_prep(*h, v.k, v.k_scale, v.S, buf.key_norm, buf.key_sum, stream) !=
+        cudaSuccess)
+      return DOSA_ERR_CUDA;
+    for (int64_t r = 0; r < v.rows; r += Tc) {
+      SeqView c = v;
+      c.row0 = v.row0 + r;
+      c.rows = v.rows - r < Tc ? v.rows - r : Tc;
+      c.pos0 = v.pos0 + r;
+      CertBuffers cb = buf;
+      if (cert_out) cb.cert = cert_out + c.row0 * kCertFloats;
+      if (retained_out) cb.retained = retained_out + c.row0 * 4;
+      if (launch_cert_setup(*h, c, buf.key_sum, cb.bdir, cb.cert, cb.retained, stream) !=
+          cudaSuccess)
+        return DOSA_ERR_CUDA;
+      const dosa_status st = body(c, cb);
+      if (st != DOSA_OK) return st;
+    }
+  }
+  return DOSA_OK;
+}
+
+extern "C" {
+
 dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale, const float* w,
                             const void* k, const float* k_scale, const int64_t* seq_offsets,
                             int B, int K, int32_t* out_idx, void* workspace, size_t ws_bytes,
-                            void* stream, dosa_stats* stats) {
-  (void)hh; (void)q; (void)q_scale; (void)w; (void)k; (void)k_scale; (void)seq_offsets;
-  (void)B; (void)K; (void)out_idx; (void)workspace; (void)ws_bytes; (void)stream; (void)stats;
-  return DOSA_ERR_UNSUPPORTED;
+                            void* stream_, dosa_stats* stats) {
+  const Handle* h = reinterpret_cast<const Handle*>(hh);
+  dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, K, out_idx);
+  if (st != DOSA_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  st = for_each_cert_chunk(
+      h, q, q_scale, w, k, k_scale, seq_offsets, B, K, workspace, ws_bytes, stream, nullptr,
+      nullptr, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {
+        if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
+        if (launch_certified(*h, c, b, K, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+        int32_t* out = out_idx + c.row0 * K;
+        if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+        // rows whose candidate list overflowed: dense rescoring of just those rows
+        if (launch_scores_tc_rows(*h, c, b.repair_list, b.repair_count, b.repair_cap,
+                                  b.repair_scores, c.S, b.err, stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
+        if (launch_topk_list(b.repair_scores, c.S, b.repair_list, b.repair_count, b.repair_cap,
+                             c.pos0 + 1, c.S, K, out, K, stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
+        return DOSA_OK;
+      });
+  if (st != DOSA_OK) return st;
+  if (stats) {
+    WsHeader hdr;
+    if (cudaMemcpyAsync(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+    stats->visible_pairs = total_visible(seq_offsets, B);
+    stats->seed_pairs = (int64_t)hdr.counters[kCntSeedPairs];
+    stats->screened_pairs = (int64_t)hdr.counters[kCntScreened];
+    stats->rejected_pairs = (int64_t)hdr.counters[kCntRejected];
+    stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
+    stats->candidates = (int64_t)hdr.counters[kCntCandidates];
+    if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
+  }
+  return DOSA_OK;
+}
+
+dosa_status dosa_index_certificate(dosa_index_t hh, const void* q, const float* q_scale,
+                                   const float* w, const void* k, const float* k_scale,
+                                   const int64_t* seq_offsets, int B, float* cert_out,
+                                   int32_t* retained_out, void* workspace, size_t ws_bytes,
+                                   void* stream_) {
+  const Handle* h = reinterpret_cast<const Handle*>(hh);
+  if (!cert_out || !retained_out) return DOSA_ERR_INVALID_ARG;
+  dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, 1, retained_out);
+  if (st != DOSA_OK) return st;
+  return for_each_cert_chunk(h, q, q_scale, w, k, k_scale, seq_offsets, B, 1, workspace, ws_bytes,
+                             static_cast<cudaStream_t>(stream_), cert_out, retained_out,
+                             [](const SeqView&, const CertBuffers&) { return DOSA_OK; });
 }
 
 static dosa_status scores_common(dosa_index_t hh, const void* q, const float* q_scale,

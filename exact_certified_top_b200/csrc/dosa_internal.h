@@ -54,10 +54,46 @@ void profile_after(int kind, cudaStream_t stream);
 // Tensor-map encoder from the driver (fetched once through the runtime).
 PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder();
 
+// Device buffers of one certified chunk (all inside the caller's workspace).
+struct CertBuffers {
+  float* key_norm;       // [S] code-domain ||k|| (rounded up)
+  float* key_sum;        // [d] real-domain key sum
+  void* bdir;            // [rows, 8, d] bound rows in the input type
+  float* cert;           // [rows, kCertFloats]
+  int32_t* retained;     // [rows, 4]
+  void* cand;            // [rows, cap] packed (score, key)
+  int* cand_count;       // [rows]; -1 marks a row repaired by the dense pass
+  float* tau;            // [rows] final threshold
+  int* repair_list;      // [repair_cap]
+  int* repair_count;
+  int repair_cap;
+  float* repair_scores;  // [repair_cap, S]
+  int cap;
+  unsigned long long* counters;
+  int* err;
+};
+
 // ---- launches (each returns the cudaError_t of its launch) --------------------
 // Tensor-core scorer writing every visible score of rows [row0, row0+rows).
 cudaError_t launch_scores_tc(const Handle& h, const SeqView& v, float* scores, int64_t ld,
                              int* err, cudaStream_t stream);
+// Same scorer over a device list of rows (row0 + row_list[i] -> output row i).
+cudaError_t launch_scores_tc_rows(const Handle& h, const SeqView& v, const int* row_list,
+                                  const int* row_count, int list_cap, float* scores, int64_t ld,
+                                  int* err, cudaStream_t stream);
+// Certified pipeline pieces.
+cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale, int64_t S,
+                            float* key_norm, float* key_sum, cudaStream_t stream);
+cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
+                              void* bdir, float* cert, int32_t* retained, cudaStream_t stream);
+cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                             cudaStream_t stream);
+cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,
+                          cudaStream_t stream);
+cudaError_t launch_topk_list(const float* scores, int64_t ld, const int* row_list,
+                             const int* row_count, int list_cap, int64_t len0, int64_t max_len,
+                             int K, int32_t* out, int64_t out_ld, cudaStream_t stream);
+size_t certified_smem_bytes(bool fp8);
 // CUDA-core reference scorer, same contract.
 cudaError_t launch_scores_ref(const Handle& h, const SeqView& v, float* scores, int64_t ld,
                               cudaStream_t stream);

@@ -57,22 +57,38 @@ struct ScoreParams {
   int64_t row0, rows, pos0, S;
   int n_items;
   int* err;
+  // Row-list mode (rows repaired after a candidate-list overflow): item i scores
+  // the single row row0 + row_list[i] into output row i; the number of items
+  // is min(*row_count, list_cap), read on the device.
+  const int* row_list;
+  const int* row_count;
+  int list_cap;
 };
 
 struct ItemGeom {
   int64_t t0;     // first query row (absolute)
   int nq;         // valid queries in the tile
   int64_t pos_first;
+  int64_t out0;   // output row of query t0
   int nkt;        // key tiles 0..nkt-1 cover keys 0..pos_last
 };
 
 __device__ __forceinline__ ItemGeom item_geom(const ScoreParams& p, int item) {
   ItemGeom g;
-  const int tile = p.n_items - 1 - item;  // longest rows first
-  g.t0 = p.row0 + (int64_t)tile * kQueryTile;
-  const int64_t left = p.row0 + p.rows - g.t0;
-  g.nq = (int)(left < kQueryTile ? left : kQueryTile);
-  g.pos_first = p.pos0 + (int64_t)tile * kQueryTile;
+  if (p.row_list) {
+    const int64_t r = p.row_list[item];
+    g.t0 = p.row0 + r;
+    g.nq = 1;
+    g.pos_first = p.pos0 + r;
+    g.out0 = item;
+  } else {
+    const int tile = p.n_items - 1 - item;  // longest rows first
+    g.t0 = p.row0 + (int64_t)tile * kQueryTile;
+    const int64_t left = p.row0 + p.rows - g.t0;
+    g.nq = (int)(left < kQueryTile ? left : kQueryTile);
+    g.pos_first = p.pos0 + (int64_t)tile * kQueryTile;
+    g.out0 = g.t0 - p.row0;
+  }
   const int64_t pos_last = g.pos_first + g.nq - 1;
   g.nkt = (int)(pos_last / kKeyTile) + 1;
   return g;
@@ -81,8 +97,13 @@ __device__ __forceinline__ ItemGeom item_geom(const ScoreParams& p, int item) {
 template <bool kFp8>
 __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                    const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
+                    const __grid_constant__ CUtensorMap kmap, ScoreParams p) {
   using C = ScoreCfg<kFp8>;
+  if (p.row_list) {
+    const int n = *p.row_count;
+    p.n_items = n < p.list_cap ? n : p.list_cap;
+    if (p.n_items <= 0) return;
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -240,7 +261,7 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
               const int64_t t = g.t0 + ql;
               float sc = head_reduce64(v, p.w + t * C::kH);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
-              if (s <= g.pos_first + ql) p.scores[(t - p.row0) * p.ld + s] = sc;
+              if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
             }
           }
           tc_fence_before();
@@ -278,7 +299,8 @@ static bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64
 
 template <bool kFp8>
 static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int* err,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const int* row_list = nullptr,
+                               const int* row_count = nullptr, int list_cap = 0) {
   using C = ScoreCfg<kFp8>;
   CUtensorMap qmap, kmap;
   if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
@@ -307,6 +329,10 @@ static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int*
   p.S = v.S;
   p.n_items = (int)((v.rows + kQueryTile - 1) / kQueryTile);
   p.err = err;
+  p.row_list = row_list;
+  p.row_count = row_count;
+  p.list_cap = list_cap;
+  if (row_list) p.n_items = list_cap;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_SCORE, stream);
@@ -320,6 +346,14 @@ cudaError_t launch_scores_tc(const Handle& h, const SeqView& v, float* scores, i
                              int* err, cudaStream_t stream) {
   if (h.cfg.dtype == DOSA_FP8_E4M3) return launch_impl<true>(v, scores, ld, err, stream);
   return launch_impl<false>(v, scores, ld, err, stream);
+}
+
+cudaError_t launch_scores_tc_rows(const Handle& h, const SeqView& v, const int* row_list,
+                                  const int* row_count, int list_cap, float* scores, int64_t ld,
+                                  int* err, cudaStream_t stream) {
+  if (h.cfg.dtype == DOSA_FP8_E4M3)
+    return launch_impl<true>(v, scores, ld, err, stream, row_list, row_count, list_cap);
+  return launch_impl<false>(v, scores, ld, err, stream, row_list, row_count, list_cap);
 }
 
 }  // namespace dosa

@@ -44,16 +44,22 @@ __device__ __forceinline__ int block_exclusive_count(bool flag, int* scratch, in
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(
     const float* __restrict__ scores, int64_t ld, const int64_t* __restrict__ row_len, int64_t len0,
-    int64_t max_len, int K, int32_t* __restrict__ out, int64_t out_ld) {
+    int64_t max_len, int K, int32_t* __restrict__ out, int64_t out_ld,
+    const int* __restrict__ row_list, const int* __restrict__ row_count) {
   __shared__ unsigned hist[256];
   __shared__ int scan_scratch[33];
   __shared__ unsigned s_digit, s_above;
-  const int64_t row = blockIdx.x;
-  int64_t n = row_len ? row_len[row] : len0 + row;
+  // Row-list mode: block i handles scores row i for output row row_list[i].
+  int64_t row = blockIdx.x, orow = blockIdx.x;
+  if (row_list) {
+    if ((int)blockIdx.x >= *row_count) return;
+    orow = row_list[blockIdx.x];
+  }
+  int64_t n = row_len ? row_len[row] : len0 + orow;
   if (n > max_len) n = max_len;
   if (n < 0) n = 0;
   const float* x = scores + row * ld;
-  int32_t* o = out + row * out_ld;
+  int32_t* o = out + orow * out_ld;
   if (n <= K) {
     for (int i = threadIdx.x; i < K; i += blockDim.x) o[i] = i < n ? i : -1;
     return;
@@ -126,7 +132,20 @@ cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int64_t* row
   if (rows <= 0) return cudaSuccess;
   profile_before(DOSA_KERNEL_TOPK, stream);
   topk_rows_kernel<<<(unsigned)rows, kTopkThreads, 0, stream>>>(scores, ld, row_len, len0,
-                                                                 max_len, K, out, out_ld);
+                                                                 max_len, K, out, out_ld, nullptr,
+                                                                 nullptr);
+  const cudaError_t e = cudaGetLastError();
+  profile_after(DOSA_KERNEL_TOPK, stream);
+  return e;
+}
+
+cudaError_t launch_topk_list(const float* scores, int64_t ld, const int* row_list,
+                             const int* row_count, int list_cap, int64_t len0, int64_t max_len,
+                             int K, int32_t* out, int64_t out_ld, cudaStream_t stream) {
+  if (list_cap <= 0) return cudaSuccess;
+  profile_before(DOSA_KERNEL_TOPK, stream);
+  topk_rows_kernel<<<(unsigned)list_cap, kTopkThreads, 0, stream>>>(
+      scores, ld, nullptr, len0, max_len, K, out, out_ld, row_list, row_count);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_TOPK, stream);
   return e;

@@ -127,6 +127,23 @@ dosa_status dosa_index_topk(dosa_index_t h, const void* q, const float* q_scale,
                             int B, int K, int32_t* out_idx, void* workspace, size_t ws_bytes,
                             void* stream, dosa_stats* stats);
 
+/* The per-query certificate the certified path screens with (for inspection
+ * and tests; the Top-K calls compute it internally).  cert_out: [Tq, 16] fp32,
+ * code domain (for E4M3 the real-valued bound is q_scale[t] * k_scale[s] times
+ * the code-domain one): [0..3] folded weights omega of the retained heads,
+ * [4] beta (coefficient of ||k||, including rounding slack and the hi/lo split
+ * error of the negative aggregates), [5] c (the candidate margin is c * ||k||),
+ * [6..9] scales of the negative-aggregate rows (u_1 hi, u_1 lo, u_2 hi, u_2 lo),
+ * [10] the per-head residual sum, [11] the joint (spectral) residual bound,
+ * [12] |A_1|, [13] |A_2|, [14] number of omitted positive heads, [15] unused.
+ * retained_out: [Tq, 4] int32 retained head indices, ascending, -1 padded.
+ * Workspace: as dosa_index_topk (certified = 1, K = 1 is enough). */
+dosa_status dosa_index_certificate(dosa_index_t h, const void* q, const float* q_scale,
+                                   const float* w, const void* k, const float* k_scale,
+                                   const int64_t* seq_offsets, int B, float* cert_out,
+                                   int32_t* retained_out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
 /* Dense Top-K: every visible key is scored with all heads (tensor-core scorer),
  * score rows are materialised chunk by chunk in the workspace, then a per-row
  * radix select picks the K largest.  The reference the certified path must

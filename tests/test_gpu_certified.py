@@ -1,0 +1,170 @@
+"""GPU parity of the certified path (dosa_index_topk): identical selection to
+the GPU's dense path, agreement with the fp64 oracle, certificate quantities
+against the oracle's, the prune-rate invariant, and the overflow repair."""
+import numpy as np
+import pytest
+import torch
+
+from exact_certified_top_b200 import binding
+from exact_certified_top_b200.workloads import codes_numpy, generate, small_case
+from oracle import (certificate_setup, certified_topk_row, dequantize, indexer_scores, key_mean,
+                    select_topk)
+from parity import OracleView, assert_topk_matches, to_numpy
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("causal_1k_bf16", 1003, 1003, 64),
+    ("prefill_128k_fp8", 777, 3000, 300),
+    ("tight_64k_bf16_levels", 517, 2600, 2048),
+    ("chunk_1m_fp8", 203, 5000, 2048),
+]
+
+
+def _inputs(base, T, S, K, **kw):
+    kw.setdefault("q_pos0", S - T)          # rows at the tail: the longest contexts
+    wl = small_case(base, T, S, K=K, **kw)
+    x = generate(wl)
+    xd = {k: (v.cuda() if torch.is_tensor(v) and k != "seq_offsets" else v) for k, v in x.items()}
+    return wl, x, xd
+
+
+def _args(x, K):
+    return (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], x["seq_offsets"], K)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_certified_equals_dense_and_oracle(cuda_lib, case):
+    base, T, S, K = case
+    wl, x, xd = _inputs(base, T, S, K)
+    idx = binding.Index(wl.dtype, max_K=2048)
+    dense = to_numpy(idx.dense_topk(*_args(xd, K)))
+    cert, stats = idx.topk(*_args(xd, K), stats=True)
+    cert = to_numpy(cert)
+    assert np.array_equal(cert, dense), "certified selection differs from the dense selection"
+    ov = OracleView(x, wl.dtype)
+    for t in range(0, wl.T, max(1, wl.T // 120)):
+        assert_topk_matches(cert[t], ov.scores(t), K, t=t, exact=wl.levels > 0)
+    assert stats["visible_pairs"] == wl.visible_pairs
+    assert 0 <= stats["rejected_pairs"] <= stats["screened_pairs"]
+    assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
+
+
+def test_certified_small_workspace_many_chunks(cuda_lib):
+    wl, x, xd = _inputs("causal_1k_bf16", 301, 2500, 100, q_pos0=2199)
+    idx = binding.Index("bf16")
+    ws = torch.zeros(idx.workspace_size(wl.T, wl.S, 100, True, chunk_rows=16), dtype=torch.uint8,
+                     device="cuda")
+    cert = to_numpy(idx.topk(*_args(xd, 100), workspace=ws))
+    binding.check_device(ws)
+    dense = to_numpy(idx.dense_topk(*_args(xd, 100)))
+    assert np.array_equal(cert, dense)
+
+
+def test_certified_varlen_batch(cuda_lib):
+    parts = [small_case("causal_1k_bf16", 130, 2300, seed=1, q_pos0=2170),
+             small_case("causal_1k_bf16", 40, 300, seed=2, q_pos0=260),
+             small_case("causal_1k_bf16", 9, 9, seed=3)]
+    xs = [generate(wl) for wl in parts]
+    q = torch.cat([x["q"] for x in xs]).cuda()
+    w = torch.cat([x["w"] for x in xs]).cuda()
+    k = torch.cat([x["k"] for x in xs]).cuda()
+    so, qr, kr = [], 0, 0
+    for wl in parts:
+        so.append([qr, kr, wl.q_pos0])
+        qr += wl.T
+        kr += wl.S
+    so.append([qr, kr, 0])
+    idx = binding.Index("bf16")
+    cert = to_numpy(idx.topk(q, None, w, k, None, so, 70))
+    dense = to_numpy(idx.dense_topk(q, None, w, k, None, so, 70))
+    assert np.array_equal(cert, dense)
+
+
+def _redundant_heads_case(T=96, S=6000, seed=0, fp8=False):
+    """Heads of a query are near copies of one direction and weights mostly
+    positive: the certificate is tight and most keys are rejected."""
+    g = torch.Generator().manual_seed(seed)
+    d, H = 128, 64
+    base = torch.randn((T, 1, d), generator=g)
+    q = base + 0.02 * torch.randn((T, H, d), generator=g)
+    w = torch.rand((T, H), generator=g) / 8
+    w[:, ::16] *= -0.2
+    k = torch.randn((S, d), generator=g)
+    pos0 = S - T
+    so = [[0, 0, pos0], [T, S, 0]]
+    if fp8:
+        from exact_certified_top_b200.workloads import _e4m3_per_token
+        q8, qs = _e4m3_per_token(q)
+        k8, ks = _e4m3_per_token(k)
+        return dict(q=q8, q_scale=qs, w=w, k=k8, k_scale=ks, seq_offsets=so,
+                    positions=torch.arange(pos0, S)), "fp8"
+    return dict(q=q.to(torch.bfloat16), q_scale=None, w=w, k=k.to(torch.bfloat16), k_scale=None,
+                seq_offsets=so, positions=torch.arange(pos0, S)), "bf16"
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_certified_prunes_and_stays_exact_when_heads_are_redundant(cuda_lib, fp8):
+    x, dtype = _redundant_heads_case(fp8=fp8)
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 64
+    idx = binding.Index(dtype)
+    cert, stats = idx.topk(*_args(xd, K), stats=True)
+    dense = idx.dense_topk(*_args(xd, K))
+    assert torch.equal(cert, dense)
+    prune = stats["rejected_pairs"] / stats["visible_pairs"]
+    assert prune > 0.5, stats
+    # the schedule's threshold is <= the true K-th and the GPU bound is >= the
+    # oracle's, so the GPU rejects no more than the oracle's ideal screening
+    ov = OracleView(x, dtype)
+    kb = key_mean(ov.k)
+    ideal = 0
+    for t in range(0, x["q"].shape[0]):
+        p = int(ov.positions[t])
+        res = certified_topk_row(ov.q[t], ov.w[t], ov.k[: p + 1], K, k_bar=kb, r=4, G=2,
+                                 margin_log2=-12)
+        ideal += res["ideal_rejected"]
+        assert np.array_equal(res["idx"], to_numpy(cert[t]).astype(np.int64))
+    assert stats["rejected_pairs"] <= ideal * 1.002 + 16, (stats, ideal)
+
+
+def test_certificate_matches_oracle(cuda_lib):
+    for fp8 in (False, True):
+        x, dtype = _redundant_heads_case(T=24, S=700, seed=3, fp8=fp8)
+        # make heads less redundant so the residual bounds are non-trivial
+        xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+        idx = binding.Index(dtype)
+        cert, ret = idx.certificate(xd["q"], xd["q_scale"], xd["w"], xd["k"], xd["k_scale"],
+                                    x["seq_offsets"])
+        cert, ret = to_numpy(cert), to_numpy(ret)
+        ov = OracleView(x, dtype)
+        kb = key_mean(ov.k)
+        for t in range(x["q"].shape[0]):
+            sq = 1.0 if x["q_scale"] is None else float(x["q_scale"][t])
+            c = certificate_setup(ov.q[t], ov.w[t], kb, 4, 2)
+            assert ret[t][ret[t] >= 0].tolist() == c.retained.tolist()
+            np.testing.assert_allclose(cert[t, 0:len(c.retained)], c.omega, rtol=2e-4, atol=1e-6)
+            # GPU beta (code domain) scaled to the real domain is an upper bound
+            # of the oracle's residual bound, and not far above it
+            assert cert[t, 4] * sq >= c.beta * (1 - 1e-5)
+            assert cert[t, 10] * sq == pytest.approx(c.beta_sum, rel=1e-3)
+            assert cert[t, 11] * sq >= c.beta_joint * (1 - 1e-5)
+            assert cert[t, 12] + cert[t, 13] == sum(g.size for g in c.groups)
+
+
+def test_repair_pass_when_candidates_overflow(cuda_lib):
+    """All keys identical: every score ties, every key becomes a candidate and
+    the candidate list overflows; the rows are rescored densely and the
+    selection (ties to the smaller index) is still exact."""
+    T, S, K = 40, 5200, 64
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn((T, 64, 128), generator=g).to(torch.bfloat16)
+    w = torch.randn((T, 64), generator=g) / 8
+    k = torch.randn((1, 128), generator=g).expand(S, 128).contiguous().to(torch.bfloat16)
+    so = [[0, 0, S - T], [T, S, 0]]
+    idx = binding.Index("bf16")
+    qd, wd, kd = q.cuda(), w.cuda(), k.cuda()
+    cert = to_numpy(idx.topk(qd, None, wd, kd, None, so, K))
+    dense = to_numpy(idx.dense_topk(qd, None, wd, kd, None, so, K))
+    assert np.array_equal(cert, dense)
+    assert np.array_equal(cert, np.tile(np.arange(K, dtype=np.int32), (T, 1)))
