@@ -23,7 +23,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
 # Every function the public header declares (the CPU tests check the export).
 EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy",
            "dosa_index_workspace_size", "dosa_index_topk", "dosa_index_dense_topk",
-           "dosa_index_scores", "dosa_reference_scores", "dosa_index_certificate", "dosa_topk_rows", "dosa_check_device",
+           "dosa_index_scores", "dosa_reference_scores", "dosa_index_certificate",
+           "dosa_index_dense_topk_static", "dosa_topk_rows", "dosa_check_device",
            "dosa_status_string", "dosa_profile_enable", "dosa_profile_reset",
            "dosa_profile_read")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
@@ -78,6 +79,7 @@ def load(path: str = LIB_PATH):
                                       _P, _P]
     lib.dosa_reference_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P,
                                           _I64, _P]
+    lib.dosa_index_dense_topk_static.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P]
     lib.dosa_index_certificate.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]
     lib.dosa_topk_rows.argtypes = [_P, _I64, _P, _I64, _I, _P, _P]
     lib.dosa_check_device.argtypes = [_P, _P]

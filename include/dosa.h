@@ -153,6 +153,25 @@ dosa_status dosa_index_dense_topk(dosa_index_t h, const void* q, const float* q_
                                   const int64_t* seq_offsets, int B, int K, int32_t* out_idx,
                                   void* workspace, size_t ws_bytes, void* stream);
 
+/* Dense Top-K that allocates nothing and takes no workspace.  For callers
+ * that cannot allocate device memory themselves -- for example code running
+ * inside a host framework whose memory pool must not be bypassed, or a
+ * latency-critical path where an allocation could block or fail.  The paper
+ * has no counterpart; it is a deployment convenience.  Scratch space is a
+ * fixed 16 MiB array compiled into the library (every GPU that loads the
+ * library holds it until the process exits).  The first call on each device
+ * looks up that array's device address; make the first call on a device
+ * before any stream capture.  All calls share the array and it keeps the last
+ * call's contents (the call clears the part that must start at zero), so calls
+ * whose work overlaps on the GPU race on it: serialise them.  Sizes: returns
+ * DOSA_ERR_WORKSPACE when 256 + 32 * S_max bytes exceed 16 MiB (S_max = the
+ * largest key count of a sequence, so up to 524280 keys), before any CUDA
+ * call.  Otherwise as dosa_index_dense_topk, with identical results. */
+dosa_status dosa_index_dense_topk_static(dosa_index_t h, const void* q, const float* q_scale,
+                                         const float* w, const void* k, const float* k_scale,
+                                         const int64_t* seq_offsets, int B, int K,
+                                         int32_t* out_idx, void* stream);
+
 /* Dense scorer alone, for one sequence: scores[i * ld + s] = I(row0 + i, s) for
  * rows row0..row0+rows-1 of q (positions pos0 + i) and s = 0..position; other
  * entries are left untouched.  k points at the sequence's first key, S is its
