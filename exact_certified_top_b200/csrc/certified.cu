@@ -36,6 +36,14 @@
 namespace dosa {
 
 constexpr int kBins = 256;
+// Adaptive screening: decided once per work item, after at least this many
+// screened pairs; screening stops when fewer than 1 in kAdaptiveRejectRatio
+// screened pairs were rejected.
+constexpr unsigned long long kAdaptiveMinScreened = 4096;
+constexpr unsigned long long kAdaptiveRejectRatio = 32;
+// Epilogue warps meet (threshold refresh, adaptive decision) every this many
+// key tiles and at the last tile of a work item.
+constexpr int kCkptTiles = 4;
 
 struct QState {
   float tau;
@@ -72,8 +80,9 @@ struct CertCfg {
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 64 + kEpiWarps * 32;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kAccCol = 0;       // two 128-column exact accumulators
-  static constexpr uint32_t kBndCol = 256;     // two 64-column bound accumulators
+  static constexpr int kAccBufs = 3;
+  static constexpr uint32_t kAccCol = 0;       // three 128-column exact accumulators
+  static constexpr uint32_t kBndCol = 384;     // two 64-column bound accumulators
   static constexpr uint32_t kStateBytes = sizeof(QState) * kQT;
   static constexpr uint32_t kMiscBytes = 1024;  // barriers, masks, flags
   static constexpr uint32_t kSmemBytes =
@@ -210,21 +219,26 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
   uint64_t* q_empty = bars + 1;
   uint64_t* bnd_full = bars + 2;     // [2]
   uint64_t* bnd_empty = bars + 4;    // [2]
-  uint64_t* acc_full = bars + 6;     // [2]
-  uint64_t* acc_empty = bars + 8;    // [2]
+  uint64_t* acc_full = bars + 6;     // [3]
+  uint64_t* acc_empty = bars + 9;    // [3]
   // mask_ready is double-buffered by tile parity: with one barrier, a tile
   // without survivors lets the epilogue complete the next tile's phase before
   // the MMA thread polls for this one, and a parity wait would then block.
-  uint64_t* mask_ready = bars + 10;  // [2]
-  uint64_t* tile_done = bars + 12;
-  uint64_t* item_ready = bars + 13;
-  uint64_t* done_bar = bars + 14;
-  uint64_t* k_full = bars + 15;                    // [kKeyStages]
+  uint64_t* mask_ready = bars + 12;  // [2]
+  uint64_t* tile_done = bars + 14;
+  uint64_t* item_ready = bars + 15;
+  uint64_t* done_bar = bars + 16;
+  uint64_t* k_full = bars + 17;                    // [kKeyStages]
   uint64_t* k_empty = k_full + C::kKeyStages;      // [kKeyStages]
-  uint32_t* masks = reinterpret_cast<uint32_t*>(k_empty + C::kKeyStages);  // [2][8][4]
-  uint32_t* gflag = masks + 2 * 8 * 4;                                      // [2][8]
-  uint32_t* s_tmem = gflag + 2 * 8;
+  // Survivor masks and query-pair flags of a screened tile, three slots: a
+  // slot is rewritten (bound evaluation of tile b+3) only after every warp has
+  // passed the bound evaluation of tile b+2, which follows its exact stage of b.
+  uint32_t* masks = reinterpret_cast<uint32_t*>(k_empty + C::kKeyStages);  // [3][8][4]
+  uint32_t* gflag = masks + 3 * 8 * 4;                                      // [3][8]
+  uint32_t* s_tmem = gflag + 3 * 8;
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* stop_word = reinterpret_cast<int*>(s_tmem + 2);             // first unscreened tile
+  unsigned long long* snap = reinterpret_cast<unsigned long long*>(s_tmem + 4);  // [2][8][2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -235,6 +249,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bnd_full[i], 1);
       mbar_init(&bnd_empty[i], C::kEpiWarps);
+    }
+    for (int i = 0; i < C::kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], C::kEpiWarps);
     }
@@ -248,6 +264,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       mbar_init(&k_empty[i], 1);
     }
     *s_abort = 0;
+    *stop_word = 0x7FFFFFFF;
     fence_barrier_init();
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&bmap);
@@ -304,9 +321,16 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
+      // Order per item: bound(0); then for each tile t: bound(t+1), [wait for
+      // tile t's survivor masks], exact(t).  The epilogue screens one tile
+      // ahead, so tile t's exact MMAs run while tile t+1's bounds are
+      // evaluated.  Screened tiles form a prefix of the processing order: all
+      // of them (screening = 1), none (0), or those before the item's stop
+      // tile (2, adaptive), which the epilogue publishes in *stop_word before
+      // its mask arrival for the tile that precedes this thread's last use.
       constexpr uint32_t idesc_b = make_idesc<kFp8>(kKeyTile, C::kBRows);
       constexpr uint32_t idesc_e = make_idesc<kFp8>(kKeyTile, C::kGroupN);
-      uint32_t kc = 0, bt = 0, u = 0;
+      uint32_t kc = 0, nb = 0, u = 0;
       int it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
@@ -314,63 +338,91 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
         tc_fence_after();
         const uint32_t b_bound = smem_u32(sB);
-        for (int ti = 0; ti <= g.n_tiles && ok; ++ti) {
-          if (ti < g.n_tiles) {
-            const uint32_t c = kc + ti, s_ = c % C::kKeyStages;
-            if (!mbar_wait(&k_full[s_], (c / C::kKeyStages) & 1, s_abort, p.err) ||
-                !mbar_wait(&bnd_empty[(bt + ti) & 1], (((bt + ti) >> 1) & 1) ^ 1, s_abort,
-                           p.err)) {
+        // (a decision never stops before tile 4, so tiles 0-3 need no read)
+        auto screened = [&](int t) -> bool {
+          if (p.screening == 0) return false;
+          if (p.screening == 1) return true;
+          return t < 4 || t < *reinterpret_cast<volatile int*>(stop_word);
+        };
+        auto issue_bound = [&](int t) -> bool {
+          const uint32_t c = kc + t, s_ = c % C::kKeyStages, b = nb + t;
+          if (!mbar_wait(&k_full[s_], (c / C::kKeyStages) & 1, s_abort, p.err) ||
+              !mbar_wait(&bnd_empty[b & 1], ((b >> 1) & 1) ^ 1, s_abort, p.err))
+            return false;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
+          const uint32_t d = tmem_base + C::kBndCol + (b & 1) * C::kBRows;
+#pragma unroll
+          for (int step = 0; step < C::kKSteps; ++step) {
+            const uint32_t sub = step >> 2, off = (step & 3) * 32;
+            tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
+                         smem_desc_sw128(b_bound + sub * C::kBSubBytes + off), idesc_b,
+                         step > 0 ? 1u : 0u);
+          }
+          tc_commit(&bnd_full[b & 1]);
+          return true;
+        };
+        bool scr_cur = screened(0);
+        if (scr_cur && !issue_bound(0)) break;
+        int n_scr = scr_cur ? 1 : 0;
+        for (int ti = 0; ti < g.n_tiles && ok; ++ti) {
+          bool scr_next = false;
+          if (ti + 1 < g.n_tiles) {
+            scr_next = scr_cur && screened(ti + 1);
+            if (scr_next) {
+              if (!issue_bound(ti + 1)) {
+                ok = false;
+                break;
+              }
+              ++n_scr;
+            }
+          }
+          // exact MMAs of tile ti
+          const uint32_t c = kc + ti, s_ = c % C::kKeyStages;
+          uint32_t groups;
+          if (scr_cur) {
+            const uint32_t b = nb + ti;
+            if (!mbar_wait(&mask_ready[b & 1], (b >> 1) & 1, s_abort, p.err)) {
+              ok = false;
+              break;
+            }
+            groups = 0;
+            for (int w = 0; w < C::kEpiWarps; ++w)
+              groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(b % 3) * 8 + w];
+          } else {
+            if (!mbar_wait(&k_full[s_], (c / C::kKeyStages) & 1, s_abort, p.err)) {
+              ok = false;
+              break;
+            }
+            groups = (1u << ((g.nq + 1) / 2)) - 1u;   // every pair with a valid query
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
+          for (int grp = 0; grp < C::kGroups && ok; ++grp) {
+            if (!(groups >> grp & 1)) continue;
+            const uint32_t ab = u % C::kAccBufs;
+            if (!mbar_wait(&acc_empty[ab], ((u / C::kAccBufs) & 1) ^ 1, s_abort, p.err)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
-            const uint32_t d = tmem_base + C::kBndCol + ((bt + ti) & 1) * C::kBRows;
+            const uint32_t b_base = smem_u32(sQ + grp * C::kGroupN * 128);
+            const uint32_t d = tmem_base + C::kAccCol + ab * C::kGroupN;
 #pragma unroll
             for (int step = 0; step < C::kKSteps; ++step) {
               const uint32_t sub = step >> 2, off = (step & 3) * 32;
               tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
-                           smem_desc_sw128(b_bound + sub * C::kBSubBytes + off), idesc_b,
+                           smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc_e,
                            step > 0 ? 1u : 0u);
             }
-            tc_commit(&bnd_full[(bt + ti) & 1]);
+            tc_commit(&acc_full[ab]);
+            ++u;
           }
-          if (ti > 0) {
-            // exact MMAs of the previous tile, for the query pairs with survivors
-            const uint32_t c = kc + ti - 1, s_ = c % C::kKeyStages;
-            const uint32_t m = bt + ti - 1;
-            if (!mbar_wait(&mask_ready[m & 1], (m >> 1) & 1, s_abort, p.err)) {
-              ok = false;
-              break;
-            }
-            uint32_t groups = 0;
-            for (int w = 0; w < C::kEpiWarps; ++w)
-              groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(m & 1) * 8 + w];
-            const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
-            for (int grp = 0; grp < C::kGroups && ok; ++grp) {
-              if (!(groups >> grp & 1)) continue;
-              if (!mbar_wait(&acc_empty[u & 1], ((u >> 1) & 1) ^ 1, s_abort, p.err)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t b_base = smem_u32(sQ + grp * C::kGroupN * 128);
-              const uint32_t d = tmem_base + C::kAccCol + (u & 1) * C::kGroupN;
-#pragma unroll
-              for (int step = 0; step < C::kKSteps; ++step) {
-                const uint32_t sub = step >> 2, off = (step & 3) * 32;
-                tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
-                             smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc_e,
-                             step > 0 ? 1u : 0u);
-              }
-              tc_commit(&acc_full[u & 1]);
-              ++u;
-            }
-            tc_commit(&k_empty[s_]);
-          }
+          tc_commit(&k_empty[s_]);
+          scr_cur = scr_next;
         }
         kc += g.n_tiles;
-        bt += g.n_tiles;
+        nb += n_scr;
         tc_commit(q_empty);
       }
       tc_commit(done_bar);
@@ -378,11 +430,13 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
+    // Order per item: bound(0); then for each tile t: bound(t+1), exact(t),
+    // tile barrier, threshold refresh by each query's owner warp.
     const int ew = warp - 2;                 // owner of query slot ew
     const int quad = warp & 3;
     const int half = ew >> 2;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint32_t bt = 0, u = 0;
+    uint32_t nb = 0, u = 0, nbar = 0;
     int it = 0;
     unsigned long long n_seed = 0, n_screened = 0, n_rejected = 0, n_exact = 0, n_cand = 0;
     bool ok = true;
@@ -410,6 +464,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           s.beta = valid ? cf[kCertBeta] : 0.f;
           s.margin = valid ? cf[kCertMargin] : 0.f;
           s.sq = (kFp8 && valid) ? __ldg(p.q_scale + g.t0 + ew) : 1.f;
+          if (ew == 0) *reinterpret_cast<volatile int*>(stop_word) = 0x7FFFFFFF;
         }
         for (int b = lane; b < kBins; b += 32) s.hist[b] = 0;
         __syncwarp();
@@ -417,22 +472,28 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         if (lane == 0) mbar_arrive(item_ready);
         if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
       }
-      for (int ti = 0; ti < g.n_tiles && ok; ++ti) {
-        const uint32_t m = bt + ti;
-        const int j = tile_at(ti, g.n_tiles);
-        const int64_t s = (int64_t)j * kKeyTile + quad * 32 + lane;
+      int stop = 0x7FFFFFFF;                 // first unscreened tile (adaptive mode)
+      bool decided = p.screening != 2;
+      unsigned long long it_scr = 0, it_rej = 0;   // this warp's screened/rejected, this item
+      auto screened = [&](int t) -> bool {
+        return p.screening == 1 || (p.screening == 2 && t < stop);
+      };
+      // key of this lane in tile ti
+      auto key_of = [&](int ti) -> int64_t {
+        return (int64_t)tile_at(ti, g.n_tiles) * kKeyTile + quad * 32 + lane;
+      };
+      // ---- bound evaluation of tile t (a screened tile) ----
+      auto bound_eval = [&](int t) -> bool {
+        const uint32_t b = nb + t;
+        const int64_t s = key_of(t);
         const bool key_ok = s < p.S;
         const float nk = key_ok ? __ldg(p.key_norm + s) : 0.f;
         float sk = 1.f;
         if constexpr (kFp8) sk = key_ok ? __ldg(p.k_scale + s) : 0.f;
-        // ---- bound evaluation ----
-        if (!mbar_wait(&bnd_full[m & 1], (m >> 1) & 1, s_abort, p.err)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&bnd_full[b & 1], (b >> 1) & 1, s_abort, p.err)) return false;
         tc_fence_after();
         float v[32];
-        tmem_ld32(tmem_base + lane_off + C::kBndCol + (m & 1) * C::kBRows + half * 32, v);
+        tmem_ld32(tmem_base + lane_off + C::kBndCol + (b & 1) * C::kBRows + half * 32, v);
         uint32_t gbits = 0;
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
@@ -441,7 +502,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
           const bool vis = phase != 0 && key_ok && s <= q.pos;
           const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
-          const bool screen = vis && !seed && phase == 2 && p.screening;
+          const bool screen = vis && !seed && phase == 2;
           bool rej = false;
           if (screen) {
             const float* x = v + qq * 8;
@@ -459,43 +520,82 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           const bool surv = vis && !rej;
           const uint32_t mk = __ballot_sync(0xFFFFFFFFu, surv);
-          const uint32_t scr = __ballot_sync(0xFFFFFFFFu, screen);
-          const uint32_t rjm = __ballot_sync(0xFFFFFFFFu, rej);
-          const uint32_t sdm = __ballot_sync(0xFFFFFFFFu, vis && seed);
-          n_screened += __popc(scr);
-          n_rejected += __popc(rjm);
-          n_seed += __popc(sdm);
-          if (lane == 0) masks[((m & 1) * 8 + ql) * 4 + quad] = mk;
+          const uint32_t scr = __popc(__ballot_sync(0xFFFFFFFFu, screen));
+          const uint32_t rjm = __popc(__ballot_sync(0xFFFFFFFFu, rej));
+          n_seed += __popc(__ballot_sync(0xFFFFFFFFu, vis && seed));
+          n_screened += scr;
+          n_rejected += rjm;
+          it_scr += scr;
+          it_rej += rjm;
+          if (lane == 0) masks[((b % 3) * 8 + ql) * 4 + quad] = mk;
           if (mk) gbits |= 1u << (ql >> 1);
         }
-        if (lane == 0) gflag[(m & 1) * 8 + ew] = gbits;
+        if (lane == 0) gflag[(b % 3) * 8 + ew] = gbits;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bnd_empty[m & 1]);
-          mbar_arrive(&mask_ready[m & 1]);
+          mbar_arrive(&bnd_empty[b & 1]);
+          mbar_arrive(&mask_ready[b & 1]);
         }
-        if (!mbar_wait(&mask_ready[m & 1], (m >> 1) & 1, s_abort, p.err)) {
-          ok = false;
-          break;
+        return mbar_wait(&mask_ready[b & 1], (b >> 1) & 1, s_abort, p.err);
+      };
+      bool scr_cur = screened(0);
+      int n_scr = scr_cur ? 1 : 0;
+      if (scr_cur && !bound_eval(0)) break;
+      for (int ti = 0; ti < g.n_tiles && ok; ++ti) {
+        bool scr_next = false;
+        if (ti + 1 < g.n_tiles) {
+          scr_next = scr_cur && screened(ti + 1);
+          if (scr_next) {
+            if (!bound_eval(ti + 1)) {
+              ok = false;
+              break;
+            }
+            ++n_scr;
+          }
         }
-        uint32_t groups = 0;
-        for (int w = 0; w < C::kEpiWarps; ++w)
-          groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(m & 1) * 8 + w];
-        // ---- exact scoring of survivors, filter, packed writeback ----
+        // ---- exact scoring of tile ti's survivors, filter, packed writeback ----
+        const int64_t s = key_of(ti);
+        const bool key_ok = s < p.S;
+        float sk = 1.f;
+        if constexpr (kFp8) sk = key_ok ? __ldg(p.k_scale + s) : 0.f;
+        uint32_t groups;
+        const uint32_t b = nb + ti;
+        if (scr_cur) {
+          groups = 0;
+          for (int w = 0; w < C::kEpiWarps; ++w)
+            groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(b % 3) * 8 + w];
+        } else {
+          groups = (1u << ((g.nq + 1) / 2)) - 1u;
+        }
         for (int grp = 0; grp < C::kGroups; ++grp) {
           if (!(groups >> grp & 1)) continue;
-          if (!mbar_wait(&acc_full[u & 1], (u >> 1) & 1, s_abort, p.err)) {
+          const uint32_t ab = u % C::kAccBufs;
+          if (!mbar_wait(&acc_full[ab], (u / C::kAccBufs) & 1, s_abort, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int ql = grp * 2 + half;
           QState& q = st[ql];
-          const uint32_t mk = reinterpret_cast<volatile uint32_t*>(masks)[((m & 1) * 8 + ql) * 4 + quad];
+          uint32_t mk;
+          if (scr_cur) {
+            mk = reinterpret_cast<volatile uint32_t*>(masks)[((b % 3) * 8 + ql) * 4 + quad];
+          } else {
+            const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
+            mk = __ballot_sync(0xFFFFFFFFu, phase != 0 && key_ok && s <= q.pos);
+            if (p.screening == 2) {
+              // pairs no longer screened still count as seeds when they are
+              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
+              n_seed += __popc(mk & __ballot_sync(0xFFFFFFFFu, seed));
+            } else {
+              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
+              n_seed += __popc(mk & __ballot_sync(0xFFFFFFFFu, seed));
+            }
+          }
           if (mk) {
             float x[64];
-            tmem_ld64(tmem_base + lane_off + C::kAccCol + (u & 1) * C::kGroupN + half * 64, x);
+            tmem_ld64(tmem_base + lane_off + C::kAccCol + ab * C::kGroupN + half * 64, x);
             const bool mine = (mk >> lane) & 1;
             float sc = 0.f;
             if (mine) {
@@ -529,59 +629,97 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[u & 1]);
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
           ++u;
         }
         if (!ok) break;
-        // ---- tile boundary: refresh the owner's threshold ----
-        __threadfence_block();
-        if (lane == 0) mbar_arrive(tile_done);
-        if (!mbar_wait(tile_done, m & 1, s_abort, p.err)) {
-          ok = false;
-          break;
-        }
-        if (ti + 1 < g.n_tiles && ew < g.nq) {
-          QState& q = st[ew];
-          const int phase = q.phase;
-          const int cnt = *reinterpret_cast<volatile int*>(&q.count);
-          if (phase == 1 && cnt >= p.K && cnt <= p.cap) {
-            // warm-up complete: bin the candidates so far over [min, max]
-            const Cand* cl = p.cand + q.row * (int64_t)p.cap;
-            float mn = INFINITY, mx = -INFINITY;
-            for (int i = lane; i < cnt; i += 32) {
-              const float x = cl[i].score;
-              mn = fminf(mn, x);
-              mx = fmaxf(mx, x);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-              mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-            }
-            float w = (mx - mn) / (float)kBins;
-            if (!(w > 0.f) || !isfinite(w)) w = fmaxf(fabsf(mn), 1e-30f) * 0x1p-8f;
-            if (lane == 0) {
-              q.lo = mn;
-              q.w = w;
-              q.inv_w = 1.f / w;
-            }
-            __syncwarp();
-            for (int i = lane; i < cnt; i += 32) atomicAdd(&q.hist[bin_of(q, cl[i].score)], 1u);
-            __syncwarp();
-            const float tn = hist_threshold(q, p.K, lane);
-            if (lane == 0) {
-              q.tau = fmaxf(q.tau, tn);
-              __threadfence_block();
-              *reinterpret_cast<volatile int*>(&q.phase) = 2;
-            }
-          } else if (phase == 2) {
-            const float tn = hist_threshold(q, p.K, lane);
-            if (lane == 0 && tn > q.tau) *reinterpret_cast<volatile float*>(&q.tau) = tn;
+        // ---- checkpoint (every kCkptTiles tiles, and at the item's last tile) ----
+        // All epilogue warps meet; each owner then refreshes its query's
+        // threshold.  Between checkpoints the warps are coupled only through
+        // the accumulator and mask barriers.
+        const bool ckpt = ((ti + 1) % kCkptTiles) == 0 || ti + 1 == g.n_tiles;
+        if (ckpt) {
+          // The owner's own count, read before it arrives: every slot below it
+          // was reserved in a tile <= ti and written before its writer arrived,
+          // and none of those writers saw the screening phase, so the warm-up
+          // scan below neither misses a written entry nor counts one twice.
+          int snap_cnt = 0;
+          if (lane == 0 && ew < g.nq) snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
+          snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
+          if (lane == 0) {
+            snap[(nbar & 1) * 16 + ew * 2 + 0] = it_scr;
+            snap[(nbar & 1) * 16 + ew * 2 + 1] = it_rej;
           }
-          __syncwarp();
+          __threadfence_block();
+          if (lane == 0) mbar_arrive(tile_done);
+          if (!mbar_wait(tile_done, nbar & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t slot = nbar & 1;
+          ++nbar;
+          // adaptive screening: every warp reads the same snapshot and takes
+          // the same decision; screening ends at tile ti + 4 (the MMA thread
+          // learns it from *stop_word before it would issue that tile's bound)
+          if (!decided) {
+            unsigned long long tot_s = 0, tot_r = 0;
+            for (int w = 0; w < C::kEpiWarps; ++w) {
+              tot_s += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2];
+              tot_r += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2 + 1];
+            }
+            if (tot_s >= kAdaptiveMinScreened) {
+              decided = true;
+              if (tot_r * kAdaptiveRejectRatio < tot_s) {
+                stop = ti + 4;
+                if (ew == 0 && lane == 0) *reinterpret_cast<volatile int*>(stop_word) = stop;
+              }
+            }
+          }
+          // the owner refreshes its query's threshold
+          if (ti + 1 < g.n_tiles && ew < g.nq) {
+            QState& q = st[ew];
+            const int phase = q.phase;
+            const int cnt = snap_cnt;
+            if (phase == 1 && cnt >= p.K && cnt <= p.cap) {
+              // warm-up complete: bin the candidates so far over [min, max]
+              const Cand* cl = p.cand + q.row * (int64_t)p.cap;
+              float mn = INFINITY, mx = -INFINITY;
+              for (int i = lane; i < cnt; i += 32) {
+                const float x = cl[i].score;
+                mn = fminf(mn, x);
+                mx = fmaxf(mx, x);
+              }
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+              }
+              float w = (mx - mn) / (float)kBins;
+              if (!(w > 0.f) || !isfinite(w)) w = fmaxf(fabsf(mn), 1e-30f) * 0x1p-8f;
+              if (lane == 0) {
+                q.lo = mn;
+                q.w = w;
+                q.inv_w = 1.f / w;
+              }
+              __syncwarp();
+              for (int i = lane; i < cnt; i += 32) atomicAdd(&q.hist[bin_of(q, cl[i].score)], 1u);
+              __syncwarp();
+              const float tn = hist_threshold(q, p.K, lane);
+              if (lane == 0) {
+                q.tau = fmaxf(q.tau, tn);
+                __threadfence_block();
+                *reinterpret_cast<volatile int*>(&q.phase) = 2;
+              }
+            } else if (phase == 2) {
+              const float tn = hist_threshold(q, p.K, lane);
+              if (lane == 0 && tn > q.tau) *reinterpret_cast<volatile float*>(&q.tau) = tn;
+            }
+            __syncwarp();
+          }
         }
+        scr_cur = scr_next;
       }
-      bt += g.n_tiles;
+      nb += n_scr;
       // ---- item end: the owner publishes its query ----
       if (ok && ew < g.nq && lane == 0) {
         QState& q = st[ew];

@@ -210,7 +210,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->r = 4;
   cfg->G = 2;
   cfg->margin_log2 = -12;
-  cfg->screening = 1;
+  cfg->screening = 2;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -219,7 +219,8 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   if (cfg->dtype != DOSA_BF16 && cfg->dtype != DOSA_FP8_E4M3) return DOSA_ERR_INVALID_ARG;
   if (cfg->max_K < 1 || cfg->max_K > 4096) return DOSA_ERR_INVALID_ARG;
   if (cfg->seed_first < 0 || cfg->seed_last < 0 || cfg->r < 0 || cfg->r > 4 || cfg->G < 0 ||
-      cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24)
+      cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
+      cfg->screening > 2)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || cfg->H != 64) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/dosa.h"
+#include "dosa.h"
 
 namespace dosa {
 

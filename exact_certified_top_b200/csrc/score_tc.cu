@@ -252,14 +252,15 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
             break;
           }
           tc_fence_after();
-#pragma unroll 1
+          // both of this warp's queries in one TMEM load (128 columns)
+          float v[128];
+          tmem_ld128(tmem_base + lane_off + buf * C::kGroupRows + half * 128, v);
+#pragma unroll
           for (int qi = 0; qi < 2; ++qi) {
             const int ql = grp * C::kQPerGroup + half * 2 + qi;
-            float v[64];
-            tmem_ld64(tmem_base + lane_off + buf * C::kGroupRows + (half * 2 + qi) * 64, v);
             if (ql < g.nq) {
               const int64_t t = g.t0 + ql;
-              float sc = head_reduce64(v, p.w + t * C::kH);
+              float sc = head_reduce64(v + qi * 64, p.w + t * C::kH);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
               if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
             }

@@ -5,10 +5,14 @@
 //
 // Every candidate was written with a score >= the row's threshold at the
 // time, and the row's final threshold tau is <= its K-th score, so the Top-K
-// are exactly the K best of the candidates with score >= tau.  Those are
-// gathered into shared memory, the K-th score is found by 4 radix passes over
-// order-preserving keys, ties at the K-th score go to the smallest key
-// indices, and the K indices are written in ascending order.
+// are exactly the K best candidates with score >= tau.  Those are gathered
+// into shared memory (when they fit; otherwise the passes read the whole list
+// from global memory), the K-th score is found by 4 radix passes over
+// order-preserving keys, and when more entries tie with it than are needed, a
+// second radix select over the complemented key indices of the tied entries
+// finds the smallest indices.  The K indices are sorted ascending in shared
+// memory and written.  Every step is a parallel pass; nothing is serial in the
+// number of ties.
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
 
@@ -43,19 +47,39 @@ __device__ void block_bitonic_sort(uint32_t* a, int n_pow2) {
   }
 }
 
-// Radix select over n keys read through `get(i)`: returns the key of the K-th
-// largest and writes how many elements equal to it must be taken.
+// Warp-aggregated slot reservation: one atomic per warp; returns this lane's
+// slot (meaningful only for active lanes).
+__device__ __forceinline__ uint32_t agg_slot(uint32_t* counter, bool active) {
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, active);
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0;
+  const int leader = m ? __ffs(m) - 1 : 0;
+  if (m && lane == leader) base = atomicAdd(counter, __popc(m));
+  base = __shfl_sync(0xFFFFFFFFu, base, leader);
+  return base + __popc(m & ((1u << lane) - 1u));
+}
+
+// Radix select over n elements: `get(i, &key)` returns false to skip element i.
+// Returns the key of the K-th largest selected element; *take = how many
+// elements equal to it belong to the K largest.
 template <typename Get>
-__device__ uint32_t radix_kth(Get get, int n, int K, uint32_t* hist, uint32_t* s_digit,
+__device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32_t* s_digit,
                               uint32_t* s_above, uint32_t* take) {
-  uint32_t prefix = 0, mask = 0, remaining = (uint32_t)K;
+  uint32_t prefix = 0, mask = 0, remaining = K;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t u = get(i);
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    const int nn = (n + 31) & ~31;             // whole warps for the aggregated adds
+    for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+      uint32_t u = 0;
+      const bool in = i < n && get(i, &u) && (u & mask) == prefix;
+      const uint32_t bin = (u >> shift) & 255u;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+      if (in) {
+        const uint32_t peers = __match_any_sync(m, bin);
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+      }
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -99,11 +123,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const CandView* __restrict__ cand, int cap, const int* __restrict__ cand_count,
     const float* __restrict__ tau, int64_t pos0, int K, int32_t* __restrict__ out) {
   extern __shared__ uint32_t sel_smem[];
-  uint32_t* lkey = sel_smem;                  // [kSelList]
-  int32_t* lidx = reinterpret_cast<int32_t*>(lkey + kSelList);   // [kSelList]
-  uint32_t* outv = reinterpret_cast<uint32_t*>(lidx + kSelList); // [kSelOut]
+  uint32_t* lkey = sel_smem;                                        // [kSelList]
+  int32_t* lidx = reinterpret_cast<int32_t*>(lkey + kSelList);     // [kSelList]
+  uint32_t* outv = reinterpret_cast<uint32_t*>(lidx + kSelList);   // [kSelOut]
   __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_digit, s_above, s_take, s_n, s_nout, s_nties;
+  __shared__ uint32_t s_digit, s_above, s_take, s_n, s_nout;
   const int64_t row = blockIdx.x;
   const int64_t nvis = pos0 + row + 1;
   int32_t* o = out + row * K;
@@ -116,101 +140,60 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     return;
   }
   const float th = tau[row];
-  if (threadIdx.x == 0) s_n = 0;
+  if (threadIdx.x == 0) {
+    s_n = 0;
+    s_nout = 0;
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-    const CandView c = cl[i];
-    if (c.score >= th) {
-      const uint32_t slot = atomicAdd(&s_n, 1u);
-      if (slot < (uint32_t)kSelList) {
-        lkey[slot] = ordered_key(c.score);
-        lidx[slot] = c.key;
-      }
+  const int cnt_w = (cnt + 31) & ~31;
+  for (int i = threadIdx.x; i < cnt_w; i += blockDim.x) {
+    CandView c;
+    c.score = -INFINITY;
+    c.key = 0;
+    if (i < cnt) c = cl[i];
+    const bool in = i < cnt && c.score >= th;
+    const uint32_t slot = agg_slot(&s_n, in);
+    if (in && slot < (uint32_t)kSelList) {
+      lkey[slot] = ordered_key(c.score);
+      lidx[slot] = c.key;
     }
   }
   __syncthreads();
   const int n = (int)s_n;
   const bool in_smem = n <= kSelList;
-  auto key_at = [&](int i) -> uint32_t {
-    return in_smem ? lkey[i] : ordered_key(cl[i].score);
-  };
-  auto idx_at = [&](int i) -> int32_t { return in_smem ? lidx[i] : cl[i].key; };
   const int m = in_smem ? n : cnt;            // the global path scans every candidate
-  const uint32_t kth = radix_kth([&](int i) { return key_at(i); }, m, K, hist, &s_digit,
-                                 &s_above, &s_take);
+  auto key_at = [&](int i) -> uint32_t { return in_smem ? lkey[i] : ordered_key(cl[i].score); };
+  auto idx_at = [&](int i) -> uint32_t { return (uint32_t)(in_smem ? lidx[i] : cl[i].key); };
+  const uint32_t kth = radix_kth(
+      [&](int i, uint32_t* u) {
+        *u = key_at(i);
+        return true;
+      },
+      m, (uint32_t)K, hist, &s_digit, &s_above, &s_take);
   const uint32_t take = s_take;
-  // gather: keys above the K-th go straight to the output list; ties are
-  // collected (ascending index order is decided by sorting them)
-  if (threadIdx.x == 0) {
-    s_nout = 0;
-    s_nties = 0;
+  // Among entries equal to the K-th key, keep those with the `take` smallest
+  // indices: the take-th largest complemented index is the cut.
+  const uint32_t cut = ~radix_kth(
+      [&](int i, uint32_t* u) {
+        if (key_at(i) != kth) return false;
+        *u = ~idx_at(i);
+        return true;
+      },
+      m, take, hist, &s_digit, &s_above, &s_take);
+  // gather the K winners (distinct indices: exactly K of them), sort, write
+  const int mw = (m + 31) & ~31;
+  for (int i = threadIdx.x; i < mw; i += blockDim.x) {
+    bool in = false;
+    uint32_t id = 0;
+    if (i < m) {
+      const uint32_t u = key_at(i);
+      id = idx_at(i);
+      in = u > kth || (u == kth && id <= cut);
+    }
+    const uint32_t slot = agg_slot(&s_nout, in);
+    if (in && slot < (uint32_t)kSelOut) outv[slot] = id;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < m; i += blockDim.x) {
-    const uint32_t u = key_at(i);
-    if (u > kth) {
-      const uint32_t p = atomicAdd(&s_nout, 1u);
-      outv[p] = (uint32_t)idx_at(i);
-    }
-  }
-  __syncthreads();
-  const uint32_t n_above = s_nout;            // == K - take
-  // ties: reuse the tail of the output buffer region as scratch when they fit
-  uint32_t* ties = outv + n_above;
-  const uint32_t tie_room = kSelOut - n_above;
-  for (int i = threadIdx.x; i < m; i += blockDim.x) {
-    if (key_at(i) == kth) {
-      const uint32_t p = atomicAdd(&s_nties, 1u);
-      if (p < tie_room) ties[p] = (uint32_t)idx_at(i);
-    }
-  }
-  __syncthreads();
-  const uint32_t n_ties = s_nties;
-  if (n_ties <= tie_room) {
-    // sort the ties, keep the `take` smallest indices
-    uint32_t pw = 1;
-    while (pw < n_ties) pw <<= 1;
-    if (pw > tie_room) {
-      // not enough room to pad: fall back to repeated minimum extraction
-      for (uint32_t r = 0; r < take; ++r) {
-        __shared__ uint32_t best;
-        if (threadIdx.x == 0) best = 0xFFFFFFFFu;
-        __syncthreads();
-        for (uint32_t i = threadIdx.x + r; i < n_ties; i += blockDim.x) atomicMin(&best, ties[i]);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-          for (uint32_t i = r; i < n_ties; ++i)
-            if (ties[i] == best) {
-              ties[i] = ties[r];
-              ties[r] = best;
-              break;
-            }
-        }
-        __syncthreads();
-      }
-    } else {
-      for (uint32_t i = n_ties + threadIdx.x; i < pw; i += blockDim.x) ties[i] = 0xFFFFFFFFu;
-      __syncthreads();
-      block_bitonic_sort(ties, (int)pw);
-    }
-  } else {
-    // more ties than room: take the `take` smallest tie indices by repeated
-    // selection over the candidates (rare; many exactly equal scores)
-    uint32_t floor_idx = 0;
-    for (uint32_t r = 0; r < take; ++r) {
-      __shared__ uint32_t best;
-      if (threadIdx.x == 0) best = 0xFFFFFFFFu;
-      __syncthreads();
-      for (int i = threadIdx.x; i < m; i += blockDim.x)
-        if (key_at(i) == kth && (uint32_t)idx_at(i) >= floor_idx) atomicMin(&best, (uint32_t)idx_at(i));
-      __syncthreads();
-      if (threadIdx.x == 0) ties[r] = best;
-      floor_idx = best + 1;
-      __syncthreads();
-    }
-  }
-  __syncthreads();
-  // the K selected indices: n_above + take == K; pad to a power of two and sort
   uint32_t pw = 1;
   while (pw < (uint32_t)K) pw <<= 1;
   for (uint32_t i = K + threadIdx.x; i < pw; i += blockDim.x) outv[i] = 0xFFFFFFFFu;

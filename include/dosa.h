@@ -73,7 +73,7 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
- * margin_log2 = -12, screening = 1. */
+ * margin_log2 = -12, screening = 2. */
 typedef struct {
   int H;            /* indexer heads per query (multiple of 4, <= 64)          */
   int d;            /* head dimension (128 in this build)                       */
@@ -84,7 +84,10 @@ typedef struct {
   int r;            /* retained positive heads evaluated exactly (0..4)         */
   int G;            /* negative-head groups (0 = no negative aggregate, 1, 2)   */
   int margin_log2;  /* soundness margin 2^margin_log2 * sum|w|||q|| * ||k||     */
-  int screening;    /* 1: reject by certificate; 0: score every key (ablation)  */
+  int screening;    /* 1: screen every key tile with the certificate; 2: adaptive
+                       (per tile of 8 queries, stop screening once 4096 screened
+                       pairs show under 1/32 rejected); 0: never (ablation).
+                       The selection is exact in every mode.                    */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */

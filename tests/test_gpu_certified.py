@@ -33,11 +33,12 @@ def _args(x, K):
     return (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], x["seq_offsets"], K)
 
 
+@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
-def test_certified_equals_dense_and_oracle(cuda_lib, case):
+def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     base, T, S, K = case
     wl, x, xd = _inputs(base, T, S, K)
-    idx = binding.Index(wl.dtype, max_K=2048)
+    idx = binding.Index(wl.dtype, max_K=2048, screening=screening)
     dense = to_numpy(idx.dense_topk(*_args(xd, K)))
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     cert = to_numpy(cert)
@@ -48,6 +49,8 @@ def test_certified_equals_dense_and_oracle(cuda_lib, case):
     assert stats["visible_pairs"] == wl.visible_pairs
     assert 0 <= stats["rejected_pairs"] <= stats["screened_pairs"]
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
+    if screening == 0:
+        assert stats["screened_pairs"] == 0
 
 
 def test_certified_small_workspace_many_chunks(cuda_lib):
@@ -103,12 +106,13 @@ def _redundant_heads_case(T=96, S=6000, seed=0, fp8=False):
                 seq_offsets=so, positions=torch.arange(pos0, S)), "bf16"
 
 
+@pytest.mark.parametrize("screening", [2, 1])
 @pytest.mark.parametrize("fp8", [False, True])
-def test_certified_prunes_and_stays_exact_when_heads_are_redundant(cuda_lib, fp8):
+def test_certified_prunes_and_stays_exact_when_heads_are_redundant(cuda_lib, fp8, screening):
     x, dtype = _redundant_heads_case(fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
-    idx = binding.Index(dtype)
+    idx = binding.Index(dtype, screening=screening)
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     dense = idx.dense_topk(*_args(xd, K))
     assert torch.equal(cert, dense)
