@@ -28,7 +28,7 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_status_string", "dosa_profile_enable", "dosa_profile_reset",
            "dosa_profile_read")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
-           "certified": 5, "select": 6}
+           "certified": 5, "select": 6, "filter": 7}
 
 
 class DosaError(RuntimeError):

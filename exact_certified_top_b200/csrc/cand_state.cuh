@@ -1,0 +1,234 @@
+// Per-query candidate state shared by the certified scorer and the filter
+// scorer: the running threshold tau, the candidate count, and the 256-bin
+// score histogram that keeps tau a sound lower bound on the K-th largest exact
+// score seen so far ("DOSA: Dots Sparse Attention", Daily Paper Cast
+// transcript, Method section: a threshold from the K-th largest exact score of
+// a subset of visible keys, refined tile by tile).
+//
+// tau is -inf during warm-up (fewer than K exact scores).  Once K candidates
+// exist, their scores are binned over [min, max]; from then on tau is the
+// rounded-down lower edge of the highest bin whose suffix count reaches K.
+// Every counted candidate in those bins has a score >= that edge, so at least
+// K exact scores are >= tau.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "dosa_device.cuh"
+
+namespace dosa {
+
+constexpr int kBins = 256;
+
+// Shared-memory state of one query of a work item.
+struct QState {
+  float tau;
+  int phase;          // 0 = unused slot, 1 = warm-up, 2 = screening/filtering
+  int count;          // candidates reserved (may exceed the capacity)
+  int overflow;
+  float lo, inv_w, w;
+  float omega[4];
+  float beta, margin;
+  float scale[4];
+  float sq;
+  long long pos;      // position of the query among the sequence's keys
+  long long row;      // chunk-local row
+  unsigned hist[kBins];
+};
+
+// The part of QState that survives from one kernel to the next (global memory,
+// one record per chunk-local query row).
+struct QStateG {
+  float tau;
+  int phase;
+  int count;
+  int overflow;
+  float lo, inv_w, w;
+  int pad;
+  unsigned hist[kBins];
+};
+
+struct Cand {
+  float score;
+  int key;
+};
+
+// Sound lower edge of bin i: every score binned at >= i is >= the result.
+__device__ __forceinline__ float bin_edge(const QState& s, int i) {
+  const float iw = (float)i * s.w;
+  return fmaf((float)i, s.w, s.lo) - (fabsf(s.lo) + iw) * 0x1p-20f;
+}
+
+__device__ __forceinline__ int bin_of(const QState& s, float score) {
+  float b = floorf((score - s.lo) * s.inv_w);
+  b = fminf(fmaxf(b, 0.f), (float)(kBins - 1));
+  return (int)b;
+}
+
+// Owner warp: highest bin whose suffix count reaches K -> its sound edge
+// (or -inf when fewer than K are counted).
+__device__ __forceinline__ float hist_threshold(const QState& s, int K, int lane) {
+  unsigned c[8], local = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = *reinterpret_cast<const volatile unsigned*>(&s.hist[lane * 8 + j]);
+    local += c[j];
+  }
+  unsigned suf = local;   // sum over lanes >= this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned n = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+    if (lane + o < 32) suf += n;
+  }
+  const unsigned above = suf - local;
+  int best = -1;
+  if (above < (unsigned)K && suf >= (unsigned)K) {
+    unsigned acc = above;
+    for (int j = 7; j >= 0; --j) {
+      acc += c[j];
+      if (acc >= (unsigned)K) {
+        best = lane * 8 + j;
+        break;
+      }
+    }
+  }
+  const unsigned who = __ballot_sync(0xFFFFFFFFu, best >= 0);
+  if (!who) return -INFINITY;
+  best = __shfl_sync(0xFFFFFFFFu, best, __ffs(who) - 1);
+  return bin_edge(s, best);
+}
+
+// Owner warp, at a checkpoint: finish warm-up (bin the first `cnt`
+// candidates, whose writes are all complete) or refresh tau from the
+// histogram.  `cnt` is the query's count read before the checkpoint barrier.
+__device__ __forceinline__ void refresh_threshold(QState& q, const Cand* cl, int cnt, int K,
+                                                  int cap, int lane) {
+  const int phase = q.phase;
+  if (phase == 1 && cnt >= K && cnt <= cap) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int i = lane; i < cnt; i += 32) {
+      const float x = cl[i].score;
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    }
+    float w = (mx - mn) / (float)kBins;
+    if (!(w > 0.f) || !isfinite(w)) w = fmaxf(fabsf(mn), 1e-30f) * 0x1p-8f;
+    if (lane == 0) {
+      q.lo = mn;
+      q.w = w;
+      q.inv_w = 1.f / w;
+    }
+    __syncwarp();
+    for (int i = lane; i < cnt; i += 32) atomicAdd(&q.hist[bin_of(q, cl[i].score)], 1u);
+    __syncwarp();
+    const float tn = hist_threshold(q, K, lane);
+    if (lane == 0) {
+      q.tau = fmaxf(q.tau, tn);
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(&q.phase) = 2;
+    }
+  } else if (phase == 2) {
+    const float tn = hist_threshold(q, K, lane);
+    if (lane == 0 && tn > q.tau) *reinterpret_cast<volatile float*>(&q.tau) = tn;
+  }
+  __syncwarp();
+}
+
+// Append the warp's candidates (lanes with app set) to query q's list.
+// Returns the number appended.
+__device__ __forceinline__ unsigned append_candidates(QState& q, Cand* list, int cap, bool app,
+                                                      float sc, int key, int lane) {
+  const unsigned am = __ballot_sync(0xFFFFFFFFu, app);
+  if (!am) return 0;
+  int base = 0;
+  if (lane == 0) base = atomicAdd(&q.count, __popc(am));
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  const int slot = base + __popc(am & ((1u << lane) - 1u));
+  const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
+  if (app) {
+    if (slot < cap) {
+      Cand cd;
+      cd.score = sc;
+      cd.key = key;
+      list[slot] = cd;
+      if (phase == 2) atomicAdd(&q.hist[bin_of(q, sc)], 1u);
+    } else {
+      q.overflow = 1;
+    }
+  }
+  return __popc(am);
+}
+
+// Owner warp: copy the carried part of a query's state between shared and
+// global memory.
+__device__ __forceinline__ void state_save(const QState& q, QStateG* g, int lane) {
+  if (lane == 0) {
+    g->tau = q.tau;
+    g->phase = q.phase;
+    g->count = q.count;
+    g->overflow = q.overflow;
+    g->lo = q.lo;
+    g->inv_w = q.inv_w;
+    g->w = q.w;
+  }
+  for (int b = lane; b < kBins; b += 32) g->hist[b] = q.hist[b];
+}
+
+__device__ __forceinline__ void state_load(QState& q, const QStateG* g, int lane) {
+  if (lane == 0) {
+    q.tau = g->tau;
+    q.phase = g->phase;
+    q.count = g->count;
+    q.overflow = g->overflow;
+    q.lo = g->lo;
+    q.inv_w = g->inv_w;
+    q.w = g->w;
+  }
+  for (int b = lane; b < kBins; b += 32) q.hist[b] = g->hist[b];
+}
+
+// Owner warp: a fresh state (warm-up) for a valid query slot, or an unused one.
+__device__ __forceinline__ void state_fresh(QState& q, bool valid, int lane) {
+  if (lane == 0) {
+    q.tau = -INFINITY;
+    q.phase = valid ? 1 : 0;
+    q.count = 0;
+    q.overflow = 0;
+    q.lo = 0.f;
+    q.inv_w = 0.f;
+    q.w = 0.f;
+  }
+  for (int b = lane; b < kBins; b += 32) q.hist[b] = 0;
+}
+
+// Where a finished query's result goes.
+struct PublishOut {
+  int* cand_count;     // [rows]: candidates, or -1 when the list overflowed
+  float* tau;          // [rows]: final threshold
+  int* repair_list;    // rows whose list overflowed (rescored densely)
+  int* repair_count;
+  int repair_cap;
+  int cap;
+  int* err;
+};
+
+// Owner lane 0: publish a finished query.
+__device__ __forceinline__ void publish_query(const QState& q, const PublishOut& o) {
+  const int cnt = *reinterpret_cast<const volatile int*>(&q.count);
+  const bool over = q.overflow || cnt > o.cap;
+  o.cand_count[q.row] = over ? -1 : cnt;
+  o.tau[q.row] = q.tau;
+  if (over) {
+    const int r = atomicAdd(o.repair_count, 1);
+    if (r < o.repair_cap) o.repair_list[r] = (int)q.row;
+    else record_error(o.err, kDevBounds);
+  }
+}
+
+}  // namespace dosa

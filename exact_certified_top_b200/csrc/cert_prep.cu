@@ -26,6 +26,7 @@
 //   2^-18 of that scale).  The candidate margin is
 //   c = 2^margin_log2 * sum_h |w_h| ||q_h||, rounded up.
 #include <cuda_bf16.h>
+#include <utility>
 #include <cuda_fp8.h>
 
 #include "cert_layout.h"
@@ -81,67 +82,86 @@ __global__ void __launch_bounds__(256) key_prep_kernel(const void* k, const floa
 
 // ---- certificate setup ------------------------------------------------------------
 constexpr int kSetupThreads = 256;
-constexpr int kSetupSmem = (64 * (kHeadDim + 1) + 60 * 61) * 4;
+constexpr int kSetupSmem = (64 * (kHeadDim + 1) + 64 * 65) * 4;
 constexpr int kPowerIters = 12;
 
-// Solve the r x r symmetric positive definite system G a = b (Cholesky, fp64).
-// Returns false when G is not numerically positive definite.
-__device__ bool chol_solve(const double* G, const double* b, int n, double* a) {
-  double L[4][4] = {};
+__host__ __device__ constexpr int popc4(int m) { return (m & 1) + ((m >> 1) & 1) + ((m >> 2) & 1) + ((m >> 3) & 1); }
+__host__ __device__ constexpr int nth_bit(int m, int k) {
+  for (int j = 0; j < 4; ++j)
+    if ((m >> j) & 1) {
+      if (k == 0) return j;
+      --k;
+    }
+  return 0;
+}
+
+// Least squares restricted to the retained heads in MASK (Cholesky in fp64,
+// every index a compile-time constant so the arrays stay in registers).  If
+// the solution is strictly positive and its residual is the smallest so far,
+// it becomes the NNLS candidate.  NNLS optimum = the unconstrained LS solution
+// on its own support, so the best feasible support over all supports is it.
+template <int MASK>
+__device__ __forceinline__ void try_support(const double (&G)[4][4], const double (&b)[4],
+                                            double qq, int r, double& best, double (&alpha)[4]) {
+  constexpr int n = popc4(MASK);
+  constexpr int i0 = nth_bit(MASK, 0), i1 = nth_bit(MASK, 1), i2 = nth_bit(MASK, 2),
+                i3 = nth_bit(MASK, 3);
+  constexpr int idx[4] = {i0, i1, i2, i3};
+  if ((MASK >> r) != 0) return;       // uses a head beyond the retained count
+  double L[4][4];
+#pragma unroll
   for (int i = 0; i < n; ++i) {
+#pragma unroll
     for (int j = 0; j <= i; ++j) {
-      double s = G[i * 4 + j];
-      for (int k = 0; k < j; ++k) s -= L[i][k] * L[j][k];
+      double v = G[idx[i]][idx[j]];
+#pragma unroll
+      for (int k = 0; k < j; ++k) v -= L[i][k] * L[j][k];
       if (i == j) {
-        if (!(s > 1e-12 * (G[i * 4 + i] + 1e-300))) return false;
-        L[i][i] = sqrt(s);
+        if (!(v > 1e-12 * (G[idx[i]][idx[i]] + 1e-300))) return;
+        L[i][i] = sqrt(v);
       } else {
-        L[i][j] = s / L[j][j];
+        L[i][j] = v / L[j][j];
       }
     }
   }
-  double y[4];
+  double y[4], a[4];
+#pragma unroll
   for (int i = 0; i < n; ++i) {
-    double s = b[i];
-    for (int k = 0; k < i; ++k) s -= L[i][k] * y[k];
-    y[i] = s / L[i][i];
+    double v = b[idx[i]];
+#pragma unroll
+    for (int k = 0; k < i; ++k) v -= L[i][k] * y[k];
+    y[i] = v / L[i][i];
   }
+#pragma unroll
   for (int i = n - 1; i >= 0; --i) {
-    double s = y[i];
-    for (int k = i + 1; k < n; ++k) s -= L[k][i] * a[k];
-    a[i] = s / L[i][i];
+    double v = y[i];
+#pragma unroll
+    for (int k = i + 1; k < n; ++k) v -= L[k][i] * a[k];
+    a[i] = v / L[i][i];
   }
-  return true;
+  double ab = 0.0;
+#pragma unroll
+  for (int i = 0; i < n; ++i) {
+    if (!(a[i] > 0.0)) return;
+    ab += a[i] * b[idx[i]];
+  }
+  // residual^2 = qq - a.b at the least-squares point
+  const double res = qq - ab;
+  if (res < best) {
+    best = res;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) alpha[j] = 0.0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) alpha[idx[i]] = a[i];
+  }
 }
 
-// NNLS over supports of the r retained heads.  Gram: r x r (row stride 4),
-// bh: r, qq = ||q_h||^2.  Writes alpha (>= 0, zeros off the support).
-__device__ void nnls_enum(const double* Gram, const double* bh, double qq, int r, double* alpha) {
-  double best = qq;
-  for (int j = 0; j < 4; ++j) alpha[j] = 0.0;
-  for (int mask = 1; mask < (1 << r); ++mask) {
-    int idx[4], n = 0;
-    for (int j = 0; j < r; ++j)
-      if (mask >> j & 1) idx[n++] = j;
-    double G[16], b[4], a[4];
-    for (int i = 0; i < n; ++i) {
-      b[i] = bh[idx[i]];
-      for (int j = 0; j < n; ++j) G[i * 4 + j] = Gram[idx[i] * 4 + idx[j]];
-    }
-    if (!chol_solve(G, b, n, a)) continue;
-    bool feasible = true;
-    for (int i = 0; i < n; ++i) feasible &= a[i] > 0.0;
-    if (!feasible) continue;
-    // residual^2 = qq - 2 a.b + a^T G a = qq - a.b at the least-squares point
-    double ab = 0.0;
-    for (int i = 0; i < n; ++i) ab += a[i] * b[i];
-    const double res = qq - ab;
-    if (res < best) {
-      best = res;
-      for (int j = 0; j < 4; ++j) alpha[j] = 0.0;
-      for (int i = 0; i < n; ++i) alpha[idx[i]] = a[i];
-    }
-  }
+template <int... Ms>
+__device__ __forceinline__ void try_supports(std::integer_sequence<int, Ms...>,
+                                             const double (&G)[4][4], const double (&b)[4],
+                                             double qq, int r, double& best,
+                                             double (&alpha)[4]) {
+  (try_support<Ms + 1>(G, b, qq, r, best, alpha), ...);
 }
 
 template <bool kFp8>
@@ -165,6 +185,17 @@ __device__ __forceinline__ float roundtrip(float x) {
   }
 }
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
 struct SetupParams {
   const void* q;          // [rows, 64, d] codes (absolute rows)
   const float* w;         // [rows, 64]
@@ -184,15 +215,17 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   extern __shared__ float setup_dyn[];
   // code-domain heads, then residuals in place (padded rows); weighted residual Gram
   float(*qs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(setup_dyn);
-  float(*gt)[61] = reinterpret_cast<float(*)[61]>(setup_dyn + H * (D + 1));
+  float(*gt)[65] = reinterpret_cast<float(*)[65]>(setup_dyn + H * (D + 1));
   __shared__ float wv[H], qn[H], act[H], rn[H];
   __shared__ float kbar[D];
-  __shared__ float vec[2][60];
+  __shared__ float vec[64];
   __shared__ double gram_r[16];
   __shared__ double alpha_s[H][4];
   __shared__ int R[4], O[64], A1[64], A2[64];
   __shared__ int nR, nO, nA1, nA2;
-  __shared__ float red[kSetupThreads / 32];
+  __shared__ float red[8];
+  __shared__ float uv[2][D], rv[2][D];
+  __shared__ float s_lam;
   const int64_t i = blockIdx.x;
   const int64_t t = p.row0 + i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,67 +242,83 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
       ss = fmaf(qs[h][e], qs[h][e], ss);
       ka = fmaf(qs[h][e], kbar[e], ka);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-      ka += __shfl_xor_sync(0xFFFFFFFFu, ka, o);
-    }
+    ss = warp_sum(ss);
+    ka = warp_sum(ka);
     if (lane == 0) {
       qn[h] = sqrtf(ss);
       act[h] = ka;
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    // retained heads: top-r positive heads by w_h ||q_h||, ties to the smaller head
-    int n = 0;
-    bool taken[64] = {};
+  if (warp == 0) {
+    // retained heads: the r positive heads with the largest w_h ||q_h||, ties
+    // to the smaller head; lane l holds heads l and l + 32
+    const int ha = lane, hb = lane + 32;
+    bool ta = false, tb = false;
     for (int k = 0; k < p.r; ++k) {
-      int best = -1;
-      for (int h = 0; h < H; ++h) {
-        if (wv[h] > 0.f && !taken[h] &&
-            (best < 0 || wv[h] * qn[h] > wv[best] * qn[best]))
-          best = h;
+      const float va = (wv[ha] > 0.f && !ta) ? wv[ha] * qn[ha] : -1.f;
+      const float vb = (wv[hb] > 0.f && !tb) ? wv[hb] * qn[hb] : -1.f;
+      float bv = va >= vb ? va : vb;                 // prefer the smaller head on a tie
+      int bh = va >= vb ? ha : hb;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oh = __shfl_xor_sync(0xFFFFFFFFu, bh, o);
+        if (ov > bv || (ov == bv && oh < bh)) {
+          bv = ov;
+          bh = oh;
+        }
       }
-      if (best < 0) break;
-      taken[best] = true;
-      ++n;
+      if (bv < 0.f) break;                           // no positive head left
+      ta |= bh == ha;
+      tb |= bh == hb;
     }
-    nR = 0;
-    for (int h = 0; h < H; ++h)
-      if (taken[h]) R[nR++] = h;     // ascending head order
-    nO = nA1 = nA2 = 0;
-    for (int h = 0; h < H; ++h) {
-      if (wv[h] > 0.f && !taken[h]) O[nO++] = h;
-      if (wv[h] < 0.f) {
-        if (p.G >= 1 && act[h] > 0.f) A1[nA1++] = h;
-        else if (p.G >= 2) A2[nA2++] = h;
-      }
-    }
+    // lists in ascending head order via ballots (heads 0..31 then 32..63)
+    const bool pa = wv[ha] > 0.f, pb = wv[hb] > 0.f, na = wv[ha] < 0.f, nb = wv[hb] < 0.f;
+    const unsigned below = (1u << lane) - 1u;
+    auto compact = [&](bool ca, bool cb, int* list, int* count) {
+      const unsigned ma = __ballot_sync(0xFFFFFFFFu, ca), mb = __ballot_sync(0xFFFFFFFFu, cb);
+      if (ca) list[__popc(ma & below)] = ha;
+      if (cb) list[__popc(ma) + __popc(mb & below)] = hb;
+      if (lane == 0) *count = __popc(ma) + __popc(mb);
+    };
+    compact(ta, tb, R, &nR);
+    compact(pa && !ta, pb && !tb, O, &nO);
+    compact(na && p.G >= 1 && act[ha] > 0.f, nb && p.G >= 1 && act[hb] > 0.f, A1, &nA1);
+    compact(na && p.G >= 2 && !(act[ha] > 0.f), nb && p.G >= 2 && !(act[hb] > 0.f), A2, &nA2);
   }
   __syncthreads();
   const int r = nR, no = nO;
-  // Gram of the retained heads (fp64 from fp32 products summed in fp64)
+  // Gram of the retained heads (fp64 sums of fp32 products)
   if (threadIdx.x < 16) {
     const int a = threadIdx.x >> 2, b = threadIdx.x & 3;
-    double s = 0.0;
+    double v = 0.0;
     if (a < r && b < r)
-      for (int e = 0; e < D; ++e) s += (double)qs[R[a]][e] * (double)qs[R[b]][e];
-    gram_r[threadIdx.x] = s;
+      for (int e = 0; e < D; ++e) v += (double)qs[R[a]][e] * (double)qs[R[b]][e];
+    gram_r[threadIdx.x] = v;
   }
   __syncthreads();
   // NNLS for every omitted positive head: one thread per head
   if (threadIdx.x < no) {
     const int h = O[threadIdx.x];
-    double bh[4] = {0, 0, 0, 0}, qq = 0.0;
+    double G[4][4], bh[4] = {0, 0, 0, 0}, qq = 0.0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) G[a][b] = gram_r[a * 4 + b];
+    const int R0 = R[0], R1 = r > 1 ? R[1] : R[0], R2 = r > 2 ? R[2] : R[0], R3 = r > 3 ? R[3] : R[0];
     for (int e = 0; e < D; ++e) {
       const double x = qs[h][e];
       qq += x * x;
-      for (int j = 0; j < r; ++j) bh[j] += (double)qs[R[j]][e] * x;
+      bh[0] += (double)qs[R0][e] * x;
+      bh[1] += (double)qs[R1][e] * x;
+      bh[2] += (double)qs[R2][e] * x;
+      bh[3] += (double)qs[R3][e] * x;
     }
-    double a[4];
-    nnls_enum(gram_r, bh, qq, r, a);
-    for (int j = 0; j < 4; ++j) alpha_s[h][j] = a[j];
+    double best = qq, alpha[4] = {0.0, 0.0, 0.0, 0.0};
+    if (r > 0) try_supports(std::make_integer_sequence<int, 15>{}, G, bh, qq, r, best, alpha);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) alpha_s[h][j] = alpha[j];
   }
   __syncthreads();
   // residuals in place of the omitted heads (retained rows are not modified)
@@ -284,61 +333,110 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     const int h = O[k];
     float ss = 0.f;
     for (int e = lane; e < D; e += 32) ss = fmaf(qs[h][e], qs[h][e], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    ss = warp_sum(ss);
     if (lane == 0) rn[h] = sqrtf(ss);
   }
-  // weighted residual Gram |[sqrt(w w') rho . rho']|
+  // weighted residual Gram |[sqrt(w w') rho . rho']| (upper triangle by warps)
   for (int e = warp; e < no * no; e += NW) {
     const int a = e / no, b = e % no;
     if (b < a) continue;
     const int ha = O[a], hb = O[b];
-    float s = 0.f;
-    for (int c = lane; c < D; c += 32) s = fmaf(qs[ha][c], qs[hb][c], s);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    float v = 0.f;
+    for (int c = lane; c < D; c += 32) v = fmaf(qs[ha][c], qs[hb][c], v);
+    v = warp_sum(v);
     if (lane == 0) {
-      const float g = fabsf(sqrtf(wv[ha] * wv[hb]) * s);
+      const float g = fabsf(sqrtf(wv[ha] * wv[hb]) * v);
       gt[a][b] = g;
       gt[b][a] = g;
     }
   }
   __syncthreads();
-  // power iterations on |Gram| from the all-ones vector, then the
-  // Collatz-Wielandt bound max_i (|Gram| v)_i / v_i
-  if (threadIdx.x < 60) vec[0][threadIdx.x] = 1.f;
+  // power iterations on |Gram| from the all-ones vector (warp 0; lane l owns
+  // rows l and l + 32), then the Collatz-Wielandt bound max_a (|Gram| v)_a / v_a
+  if (warp == 0) {
+    const int a0 = lane, a1 = lane + 32;
+    if (a0 < no) vec[a0] = 1.f;
+    if (a1 < no) vec[a1] = 1.f;
+    __syncwarp();
+    float s0 = 0.f, s1 = 0.f;
+    for (int it = 0; it <= kPowerIters; ++it) {
+      s0 = 0.f;
+      s1 = 0.f;
+      for (int b = 0; b < no; ++b) {
+        const float vb = vec[b];
+        if (a0 < no) s0 = fmaf(gt[a0][b], vb, s0);
+        if (a1 < no) s1 = fmaf(gt[a1][b], vb, s1);
+      }
+      if (it == kPowerIters) break;
+      const float m = warp_max(fmaxf(s0, s1));
+      __syncwarp();
+      if (a0 < no) vec[a0] = m > 0.f ? s0 / m : 1.f;
+      if (a1 < no) vec[a1] = m > 0.f ? s1 / m : 1.f;
+      __syncwarp();
+    }
+    float lam = 0.f;
+    if (a0 < no) lam = s0 / fmaxf(vec[a0], 1e-30f);
+    if (a1 < no) lam = fmaxf(lam, s1 / fmaxf(vec[a1], 1e-30f));
+    lam = warp_max(lam);
+    if (lane == 0) s_lam = lam;
+  }
+  // negative aggregates: thread c < D owns element c of u_1 and u_2
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float u1 = 0.f, u2 = 0.f;
+    for (int k = 0; k < nA1; ++k) u1 = fmaf(fabsf(wv[A1[k]]), qs[A1[k]][c], u1);
+    for (int k = 0; k < nA2; ++k) u2 = fmaf(fabsf(wv[A2[k]]), qs[A2[k]][c], u2);
+    uv[0][c] = u1;
+    uv[1][c] = u2;
+  }
   __syncthreads();
-  int cur = 0;
-  for (int it = 0; it < kPowerIters; ++it) {
-    if (threadIdx.x < no) {
-      float s = 0.f;
-      for (int b = 0; b < no; ++b) s = fmaf(gt[threadIdx.x][b], vec[cur][b], s);
-      vec[cur ^ 1][threadIdx.x] = s;
+  float beta_add = 0.f;   // split errors of the aggregates (thread 0)
+  const size_t esz = kFp8 ? 1 : 2;
+  uint8_t* rows_out = static_cast<uint8_t*>(p.bdir) + (size_t)i * 8 * D * esz;
+  float s_hi[2], s_lo[2];
+  for (int g = 0; g < 2; ++g) {
+    // hi part: scale then round; lo part: the remainder, scaled and rounded
+    float m = threadIdx.x < D ? fabsf(uv[g][threadIdx.x]) : 0.f;
+    m = warp_max(m);
+    if (lane == 0 && warp < 4) red[warp] = m;
+    __syncthreads();
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    s_hi[g] = kFp8 ? (m > 0.f ? m / 448.f : 0.f) : 1.f;
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      const float x = s_hi[g] > 0.f ? uv[g][c] / s_hi[g] : 0.f;
+      store_code<kFp8>(rows_out, (4 + 2 * g) * D + c, x);
+      rv[g][c] = uv[g][c] - s_hi[g] * roundtrip<kFp8>(x);
     }
     __syncthreads();
-    // normalise by the max entry
-    float m = 0.f;
-    for (int b = 0; b < no; ++b) m = fmaxf(m, vec[cur ^ 1][b]);
+    float m2 = threadIdx.x < D ? fabsf(rv[g][threadIdx.x]) : 0.f;
+    m2 = warp_max(m2);
+    if (lane == 0 && warp < 4) red[4 + warp] = m2;
     __syncthreads();
-    if (threadIdx.x < no) vec[cur ^ 1][threadIdx.x] = m > 0.f ? vec[cur ^ 1][threadIdx.x] / m : 1.f;
+    m2 = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+    s_lo[g] = kFp8 ? (m2 > 0.f ? m2 / 448.f : 0.f) : 1.f;
+    float e2 = 0.f;
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      const float x = s_lo[g] > 0.f ? rv[g][c] / s_lo[g] : 0.f;
+      store_code<kFp8>(rows_out, (5 + 2 * g) * D + c, x);
+      const float err = rv[g][c] - s_lo[g] * roundtrip<kFp8>(x);
+      e2 = err * err;
+    }
+    e2 = warp_sum(e2);
     __syncthreads();
-    cur ^= 1;
+    if (lane == 0 && warp < 4) red[warp] = e2;
+    __syncthreads();
+    if (threadIdx.x == 0) beta_add += sqrtf(red[0] + red[1] + red[2] + red[3]) * (1.f + 0x1p-10f);
+    __syncthreads();
   }
-  float lam_part = 0.f;
-  if (threadIdx.x < no) {
-    float s = 0.f;
-    for (int b = 0; b < no; ++b) s = fmaf(gt[threadIdx.x][b], vec[cur][b], s);
-    const float v = fmaxf(vec[cur][threadIdx.x], 1e-30f);
-    lam_part = s / v;
+  // bound rows 0..3: the retained heads' own codes
+  const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (size_t)t * H * D * esz;
+  for (int e = threadIdx.x; e < 4 * D * (int)esz; e += blockDim.x) {
+    const int j = e / (D * esz), b = e % (D * esz);
+    rows_out[e] = j < r ? qrow[(size_t)R[j] * D * esz + b] : 0;
   }
-  // block max of lam_part
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lam_part = fmaxf(lam_part, __shfl_xor_sync(0xFFFFFFFFu, lam_part, o));
-  if (lane == 0) red[warp] = lam_part;
-  __syncthreads();
   if (threadIdx.x == 0) {
-    float lam = 0.f;
-    for (int w = 0; w < NW; ++w) lam = fmaxf(lam, red[w]);
     float wO = 0.f, bsum = 0.f, z2 = 0.f, scale = 0.f;
     for (int k = 0; k < no; ++k) {
       const int h = O[k];
@@ -348,11 +446,11 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     }
     for (int h = 0; h < H; ++h) scale = fmaf(fabsf(wv[h]), qn[h], scale);
     // lambda bound: CW value with rounding headroom plus the Gram entry errors
-    const float lam_b = lam * (1.f + 0x1p-16f) + 0x1p-16f * z2;
+    const float lam_b = s_lam * (1.f + 0x1p-16f) + 0x1p-16f * z2;
     const float bjoint = sqrtf(wO * lam_b) * (1.f + 0x1p-20f);
     const float bs = bsum * (1.f + 0x1p-20f);
     float beta = no > 0 ? fminf(bs, bjoint) : 0.f;
-    beta += 0x1p-16f * scale;
+    beta += 0x1p-16f * scale + beta_add;
     float* cf = p.cert + i * kCertFloats;
     for (int j = 0; j < 4; ++j) {
       float om = 0.f;
@@ -364,71 +462,17 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
       cf[kCertOmega + j] = om;
       p.retained[i * 4 + j] = j < r ? R[j] : -1;
     }
-    cf[kCertBeta] = beta;   // the split errors of u_g are added below
+    cf[kCertBeta] = beta;
     cf[kCertMargin] = ldexpf(scale, p.margin_log2) * (1.f + 0x1p-20f);
+    cf[kCertScale + 0] = s_hi[0];
+    cf[kCertScale + 1] = s_lo[0];
+    cf[kCertScale + 2] = s_hi[1];
+    cf[kCertScale + 3] = s_lo[1];
     cf[kCertBetaSum] = bs;
     cf[kCertBetaJoint] = bjoint;
     cf[kCertNA1] = (float)nA1;
     cf[kCertNA2] = (float)nA2;
     cf[kCertNO] = (float)no;
-  }
-  __syncthreads();
-  // bound rows 0..3: the retained heads' own codes; 4..7: u_1 hi/lo, u_2 hi/lo
-  const size_t esz = kFp8 ? 1 : 2;
-  uint8_t* rows_out = static_cast<uint8_t*>(p.bdir) + (size_t)i * 8 * D * esz;
-  const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (size_t)t * H * D * esz;
-  for (int e = threadIdx.x; e < 4 * D * (int)esz; e += blockDim.x) {
-    const int j = e / (D * esz), b = e % (D * esz);
-    rows_out[e] = j < r ? qrow[(size_t)R[j] * D * esz + b] : 0;
-  }
-  // negative aggregates: thread c < D owns element c of u_1 and u_2
-  __shared__ float uv[2][D], rv[2][D], red2[2][4];
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
-    float u1 = 0.f, u2 = 0.f;
-    for (int k = 0; k < nA1; ++k) u1 = fmaf(fabsf(wv[A1[k]]), qs[A1[k]][c], u1);
-    for (int k = 0; k < nA2; ++k) u2 = fmaf(fabsf(wv[A2[k]]), qs[A2[k]][c], u2);
-    uv[0][c] = u1;
-    uv[1][c] = u2;
-  }
-  __syncthreads();
-  for (int g = 0; g < 2; ++g) {
-    // hi part: scale then round; lo part: the remainder, scaled and rounded
-    float m = 0.f;
-    for (int c = 0; c < D; ++c) m = fmaxf(m, fabsf(uv[g][c]));
-    const float s_hi = kFp8 ? (m > 0.f ? m / 448.f : 0.f) : 1.f;
-    if (threadIdx.x < D) {
-      const int c = threadIdx.x;
-      const float x = s_hi > 0.f ? uv[g][c] / s_hi : 0.f;
-      const float hi = roundtrip<kFp8>(x);
-      store_code<kFp8>(rows_out, (4 + 2 * g) * D + c, x);
-      rv[g][c] = uv[g][c] - s_hi * hi;
-    }
-    __syncthreads();
-    float m2 = 0.f;
-    for (int c = 0; c < D; ++c) m2 = fmaxf(m2, fabsf(rv[g][c]));
-    const float s_lo = kFp8 ? (m2 > 0.f ? m2 / 448.f : 0.f) : 1.f;
-    float e2 = 0.f;
-    if (threadIdx.x < D) {
-      const int c = threadIdx.x;
-      const float x = s_lo > 0.f ? rv[g][c] / s_lo : 0.f;
-      const float lo = roundtrip<kFp8>(x);
-      store_code<kFp8>(rows_out, (5 + 2 * g) * D + c, x);
-      const float err = rv[g][c] - s_lo * lo;
-      e2 = err * err;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) e2 += __shfl_xor_sync(0xFFFFFFFFu, e2, o);
-    if (lane == 0 && warp < 4) red2[g][warp] = e2;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const float err = sqrtf(red2[g][0] + red2[g][1] + red2[g][2] + red2[g][3]);
-      float* cf = p.cert + i * kCertFloats;
-      cf[kCertScale + 2 * g] = s_hi;
-      cf[kCertScale + 2 * g + 1] = s_lo;
-      cf[kCertBeta] += err * (1.f + 0x1p-10f);
-    }
-    __syncthreads();
   }
 }
 

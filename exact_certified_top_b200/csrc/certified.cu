@@ -7,58 +7,43 @@
 // compacted into shared streams so key loads are not repeated, full-score
 // computation fused with threshold filtering and packed writeback).
 //
-// Work item = 8 consecutive query rows.  Resident in shared memory: their
-// 8 x 64 head rows and their 8 x 8 bound rows (4 retained heads, u_1 hi/lo,
-// u_2 hi/lo, from cert_setup).  For each key tile of 128 keys (tile 0 first,
-// which holds the first seed keys, then from the diagonal downwards):
+// Work item = 8 consecutive query rows (work_items.cuh).  Resident in shared
+// memory: their 8 x 64 head rows and their 8 x 8 bound rows (4 retained heads,
+// u_1 hi/lo, u_2 hi/lo, from cert_setup).  For each key tile of 128 keys of
+// the item's range, in processing order:
 //   1. bound MMA   D_b[128 keys x 64] = keys x bound rows            (N = 64)
 //   2. bound epilogue: UB(t,s) per (key, query); a key survives when it is a
 //      seed, when the query is still warming up (fewer than K exact scores),
-//      or when UB + margin >= tau_t.  Survivor masks go to shared memory.
+//      or when (UB + margin) * scales >= tau_t.  Masks go to shared memory.
 //   3. exact MMA for each pair of queries with at least one survivor
 //      D_e[128 keys x 128] = keys x (2 queries x 64 heads)           (N = 128)
-//   4. exact epilogue on survivors only: the same head reduction as the
+//   4. exact epilogue on survivors only: the head reduction shared with the
 //      dense scorer (bit-identical scores); scores >= tau_t are appended as
-//      packed (score, key) pairs to the query's candidate list.
-//   5. tile barrier; the warp that owns each query refreshes tau_t.
-// tau_t is a lower bound on the K-th largest exact score so far: during
-// warm-up it is -inf; once K candidates exist the owner bins them into a
-// 256-bin histogram over [min, max] and from then on tau_t is the (rounded
-// down) lower edge of the highest bin whose suffix count reaches K.  Every
-// candidate counted there has a score >= that edge, so at least K exact scores
-// are >= tau_t: rejecting UB + margin < tau_t never drops a Top-K key, and a
-// key tied with the K-th score is never rejected.
+//      packed (score, key) pairs (cand_state.cuh keeps tau_t sound).
+// The epilogue screens one tile ahead of the exact MMAs (bound(t+1) before
+// exact(t)), so screening overlaps the tensor core.  Every 4 tiles, and at the
+// end of a range, the epilogue warps meet and each query's owner warp
+// refreshes its threshold.
+//
+// One kernel, two uses per chunk.  The probe pass screens the first
+// `probe_tiles` tiles of every item and decides from the item's own counts
+// whether screening pays there: an item that rejected fewer than 1 in 32
+// screened pairs hands its state over to the filter scorer (filter.cu), which
+// finishes it without bounds; any other unfinished item is finished by the
+// continue pass of this kernel, which screens every remaining tile.
+#include "cand_state.cuh"
 #include "cert_layout.h"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
 #include "score_epilogue.cuh"
+#include "work_items.cuh"
 
 namespace dosa {
 
-constexpr int kBins = 256;
-// Adaptive screening: decided once per work item, after at least this many
-// screened pairs; screening stops when fewer than 1 in kAdaptiveRejectRatio
-// screened pairs were rejected.
-constexpr unsigned long long kAdaptiveMinScreened = 4096;
-constexpr unsigned long long kAdaptiveRejectRatio = 32;
-// Epilogue warps meet (threshold refresh, adaptive decision) every this many
-// key tiles and at the last tile of a work item.
-constexpr int kCkptTiles = 4;
-
-struct QState {
-  float tau;
-  int phase;          // 0 = unused slot, 1 = warm-up, 2 = screening
-  int count;          // candidates reserved (may exceed the capacity)
-  int overflow;
-  float lo, inv_w, w;
-  float omega[4];
-  float beta, margin;
-  float scale[4];
-  float sq;
-  long long pos;      // position of the query among the sequence's keys
-  long long row;      // chunk-local row
-  unsigned hist[kBins];
-};
+// Items whose probe screened at least this many pairs and rejected fewer than
+// 1 in kRejectRatio of them are handed to the filter scorer.
+constexpr unsigned long long kMinScreened = 4096;
+constexpr unsigned long long kRejectRatio = 32;
 
 template <bool kFp8>
 struct CertCfg {
@@ -66,7 +51,7 @@ struct CertCfg {
   static constexpr int kKSteps = kFp8 ? 4 : 8;
   static constexpr int kKeyStages = kFp8 ? 4 : 2;
   static constexpr int kH = 64;
-  static constexpr int kQT = 8;
+  static constexpr int kQT = kItemQueries;
   static constexpr int kQRows = kQT * kH;
   static constexpr int kBRows = kQT * kBoundRows;      // 64
   static constexpr int kGroupN = 2 * kH;               // 128 columns = 2 queries
@@ -89,11 +74,6 @@ struct CertCfg {
       1024 + kQBytes + kBBytes + kKeyStages * kKeyStageBytes + kStateBytes + kMiscBytes;
 };
 
-struct Cand {
-  float score;
-  int key;
-};
-
 struct CertParams {
   const float* w;          // [rows_total, 64] absolute rows
   const float* q_scale;    // absolute rows (fp8)
@@ -101,15 +81,15 @@ struct CertParams {
   const float* key_norm;   // [S] code-domain ||k||, rounded up
   const float* cert;       // [chunk rows, kCertFloats]
   Cand* cand;              // [chunk rows, cap]
-  int* cand_count;         // [chunk rows]
-  float* tau_out;          // [chunk rows]
-  int* repair_list;        // [repair_cap] chunk-local rows whose list overflowed
-  int* repair_count;
-  int repair_cap;
+  QStateG* qstate;         // [chunk rows] state carried between passes
+  int* item_flag;          // [n_items] decision of the probe pass
+  PublishOut out;
   unsigned long long* counters;
   int* err;
   int64_t row0, rows, pos0, S;   // chunk: absolute first row, rows, first position
-  int n_items, K, cap, seed_first, seed_last, screening;
+  int n_items, K, cap, seed_first, seed_last;
+  int probe_tiles;         // tiles screened by the probe pass
+  int continue_pass;       // 0: probe pass, 1: continue pass
 };
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -127,77 +107,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "r"(taddr));
 }
 
-struct Geom {
-  int64_t t0;        // absolute first row
-  int64_t local0;    // chunk-local first row
-  int nq;
-  int64_t pos_first;
-  int n_tiles;       // key tiles 0..n_tiles-1
+// Steps [begin, end) of an item this launch processes (empty: skip the item).
+struct Range {
+  int begin, end;
 };
 
-__device__ __forceinline__ Geom cert_geom(const CertParams& p, int item) {
-  Geom g;
-  const int tile = p.n_items - 1 - item;       // longest rows first
-  g.local0 = (int64_t)tile * 8;
-  g.t0 = p.row0 + g.local0;
-  const int64_t left = p.rows - g.local0;
-  g.nq = (int)(left < 8 ? left : 8);
-  g.pos_first = p.pos0 + g.local0;
-  g.n_tiles = (int)((g.pos_first + g.nq - 1) / kKeyTile) + 1;
-  return g;
-}
-
-// Processing order of key tiles: tile 0 (the first seed keys), then from the
-// diagonal tile downwards.
-__device__ __forceinline__ int tile_at(int ti, int n_tiles) {
-  return ti == 0 ? 0 : n_tiles - ti;
-}
-
-// Sound lower edge of bin i: every score binned at >= i is >= the result.
-__device__ __forceinline__ float bin_edge(const QState& s, int i) {
-  const float iw = (float)i * s.w;
-  return fmaf((float)i, s.w, s.lo) - (fabsf(s.lo) + iw) * 0x1p-20f;
-}
-
-__device__ __forceinline__ int bin_of(const QState& s, float score) {
-  float b = floorf((score - s.lo) * s.inv_w);
-  b = fminf(fmaxf(b, 0.f), (float)(kBins - 1));
-  return (int)b;
-}
-
-// Owner warp: highest bin whose suffix count reaches K -> its sound edge
-// (or -inf when fewer than K are counted).
-__device__ float hist_threshold(const QState& s, int K, int lane) {
-  unsigned c[8], local = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    c[j] = *reinterpret_cast<const volatile unsigned*>(&s.hist[lane * 8 + j]);
-    local += c[j];
+__device__ __forceinline__ Range item_range(const CertParams& p, const Geom& g, int item) {
+  Range r;
+  if (!p.continue_pass) {
+    r.begin = 0;
+    r.end = g.n_tiles < p.probe_tiles ? g.n_tiles : p.probe_tiles;
+  } else {
+    const bool go = p.item_flag[item] == kItemScreen;
+    r.begin = go ? p.probe_tiles : 0;
+    r.end = go ? g.n_tiles : 0;
   }
-  unsigned suf = local;   // sum over lanes >= this one
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned n = __shfl_down_sync(0xFFFFFFFFu, suf, o);
-    if (lane + o < 32) suf += n;
-  }
-  const unsigned above = suf - local;
-  int best = -1;
-  if (above < (unsigned)K && suf >= (unsigned)K) {
-    unsigned acc = above;
-    for (int j = 7; j >= 0; --j) {
-      acc += c[j];
-      if (acc >= (unsigned)K) {
-        best = lane * 8 + j;
-        break;
-      }
-    }
-  }
-  // exactly one lane can hold the answer
-  const unsigned who = __ballot_sync(0xFFFFFFFFu, best >= 0);
-  if (!who) return -INFINITY;
-  const int src = __ffs(who) - 1;
-  best = __shfl_sync(0xFFFFFFFFu, best, src);
-  return bin_edge(s, best);
+  return r;
 }
 
 template <bool kFp8>
@@ -230,14 +155,13 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
   uint64_t* done_bar = bars + 16;
   uint64_t* k_full = bars + 17;                    // [kKeyStages]
   uint64_t* k_empty = k_full + C::kKeyStages;      // [kKeyStages]
-  // Survivor masks and query-pair flags of a screened tile, three slots: a
-  // slot is rewritten (bound evaluation of tile b+3) only after every warp has
-  // passed the bound evaluation of tile b+2, which follows its exact stage of b.
+  // Survivor masks and query-pair flags of a tile, three slots: a slot is
+  // rewritten (bound evaluation of tile b+3) only after every warp has passed
+  // the bound evaluation of tile b+2, which follows its exact stage of b.
   uint32_t* masks = reinterpret_cast<uint32_t*>(k_empty + C::kKeyStages);  // [3][8][4]
   uint32_t* gflag = masks + 3 * 8 * 4;                                      // [3][8]
   uint32_t* s_tmem = gflag + 3 * 8;
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* stop_word = reinterpret_cast<int*>(s_tmem + 2);             // first unscreened tile
   unsigned long long* snap = reinterpret_cast<unsigned long long*>(s_tmem + 4);  // [2][8][2]
 
   const int warp = threadIdx.x >> 5;
@@ -249,13 +173,12 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bnd_full[i], 1);
       mbar_init(&bnd_empty[i], C::kEpiWarps);
+      mbar_init(&mask_ready[i], C::kEpiWarps);
     }
     for (int i = 0; i < C::kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], C::kEpiWarps);
     }
-    mbar_init(&mask_ready[0], C::kEpiWarps);
-    mbar_init(&mask_ready[1], C::kEpiWarps);
     mbar_init(tile_done, C::kEpiWarps);
     mbar_init(item_ready, C::kEpiWarps);
     mbar_init(done_bar, 1);
@@ -264,7 +187,6 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       mbar_init(&k_empty[i], 1);
     }
     *s_abort = 0;
-    *stop_word = 0x7FFFFFFF;
     fence_barrier_init();
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&bmap);
@@ -286,8 +208,10 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       int it = 0;
       bool ok = true;
       uint32_t inflight_q = 0xFFFFFFFFu;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-        const Geom g = cert_geom(p, item);
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const Range rg = item_range(p, g, item);
+        if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
         mbar_arrive_expect_tx(q_full, C::kQBytes + C::kBBytes);
         for (int sub = 0; sub < C::kSub; ++sub) {
@@ -298,7 +222,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
                       (int32_t)(g.local0 * kBoundRows));
         }
         inflight_q = it & 1;
-        for (int ti = 0; ti < g.n_tiles; ++ti, ++kc) {
+        ++it;
+        for (int ti = rg.begin; ti < rg.end; ++ti, ++kc) {
           const int s_ = kc % C::kKeyStages;
           const uint32_t rnd = kc / C::kKeyStages;
           if (!mbar_wait(&k_empty[s_], (rnd & 1) ^ 1, s_abort, p.err)) {
@@ -321,37 +246,31 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      // Order per item: bound(0); then for each tile t: bound(t+1), [wait for
-      // tile t's survivor masks], exact(t).  The epilogue screens one tile
-      // ahead, so tile t's exact MMAs run while tile t+1's bounds are
-      // evaluated.  Screened tiles form a prefix of the processing order: all
-      // of them (screening = 1), none (0), or those before the item's stop
-      // tile (2, adaptive), which the epilogue publishes in *stop_word before
-      // its mask arrival for the tile that precedes this thread's last use.
+      // Per item: bound(first); then for each step i: bound(i+1), [wait for
+      // step i's survivor masks], exact MMAs of step i.
       constexpr uint32_t idesc_b = make_idesc<kFp8>(kKeyTile, C::kBRows);
       constexpr uint32_t idesc_e = make_idesc<kFp8>(kKeyTile, C::kGroupN);
-      uint32_t kc = 0, nb = 0, u = 0;
+      uint32_t kc = 0, u = 0;
       int it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-        const Geom g = cert_geom(p, item);
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const Range rg = item_range(p, g, item);
+        if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
+        ++it;
         tc_fence_after();
         const uint32_t b_bound = smem_u32(sB);
-        // (a decision never stops before tile 4, so tiles 0-3 need no read)
-        auto screened = [&](int t) -> bool {
-          if (p.screening == 0) return false;
-          if (p.screening == 1) return true;
-          return t < 4 || t < *reinterpret_cast<volatile int*>(stop_word);
-        };
-        auto issue_bound = [&](int t) -> bool {
-          const uint32_t c = kc + t, s_ = c % C::kKeyStages, b = nb + t;
+        const int n = rg.end - rg.begin;
+        // bound tiles use the same running index as key stages (kc)
+        auto issue_bound = [&](int i) -> bool {
+          const uint32_t c = kc + i, s_ = c % C::kKeyStages;
           if (!mbar_wait(&k_full[s_], (c / C::kKeyStages) & 1, s_abort, p.err) ||
-              !mbar_wait(&bnd_empty[b & 1], ((b >> 1) & 1) ^ 1, s_abort, p.err))
+              !mbar_wait(&bnd_empty[c & 1], ((c >> 1) & 1) ^ 1, s_abort, p.err))
             return false;
           tc_fence_after();
           const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
-          const uint32_t d = tmem_base + C::kBndCol + (b & 1) * C::kBRows;
+          const uint32_t d = tmem_base + C::kBndCol + (c & 1) * C::kBRows;
 #pragma unroll
           for (int step = 0; step < C::kKSteps; ++step) {
             const uint32_t sub = step >> 2, off = (step & 3) * 32;
@@ -359,43 +278,23 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
                          smem_desc_sw128(b_bound + sub * C::kBSubBytes + off), idesc_b,
                          step > 0 ? 1u : 0u);
           }
-          tc_commit(&bnd_full[b & 1]);
+          tc_commit(&bnd_full[c & 1]);
           return true;
         };
-        bool scr_cur = screened(0);
-        if (scr_cur && !issue_bound(0)) break;
-        int n_scr = scr_cur ? 1 : 0;
-        for (int ti = 0; ti < g.n_tiles && ok; ++ti) {
-          bool scr_next = false;
-          if (ti + 1 < g.n_tiles) {
-            scr_next = scr_cur && screened(ti + 1);
-            if (scr_next) {
-              if (!issue_bound(ti + 1)) {
-                ok = false;
-                break;
-              }
-              ++n_scr;
-            }
+        if (!issue_bound(0)) break;
+        for (int i = 0; i < n && ok; ++i) {
+          if (i + 1 < n && !issue_bound(i + 1)) {
+            ok = false;
+            break;
           }
-          // exact MMAs of tile ti
-          const uint32_t c = kc + ti, s_ = c % C::kKeyStages;
-          uint32_t groups;
-          if (scr_cur) {
-            const uint32_t b = nb + ti;
-            if (!mbar_wait(&mask_ready[b & 1], (b >> 1) & 1, s_abort, p.err)) {
-              ok = false;
-              break;
-            }
-            groups = 0;
-            for (int w = 0; w < C::kEpiWarps; ++w)
-              groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(b % 3) * 8 + w];
-          } else {
-            if (!mbar_wait(&k_full[s_], (c / C::kKeyStages) & 1, s_abort, p.err)) {
-              ok = false;
-              break;
-            }
-            groups = (1u << ((g.nq + 1) / 2)) - 1u;   // every pair with a valid query
+          const uint32_t c = kc + i, s_ = c % C::kKeyStages;
+          if (!mbar_wait(&mask_ready[c & 1], (c >> 1) & 1, s_abort, p.err)) {
+            ok = false;
+            break;
           }
+          uint32_t groups = 0;
+          for (int w = 0; w < C::kEpiWarps; ++w)
+            groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(c % 3) * 8 + w];
           tc_fence_after();
           const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
           for (int grp = 0; grp < C::kGroups && ok; ++grp) {
@@ -419,10 +318,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             ++u;
           }
           tc_commit(&k_empty[s_]);
-          scr_cur = scr_next;
         }
-        kc += g.n_tiles;
-        nb += n_scr;
+        kc += n;
         tc_commit(q_empty);
       }
       tc_commit(done_bar);
@@ -430,33 +327,30 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
-    // Order per item: bound(0); then for each tile t: bound(t+1), exact(t),
-    // tile barrier, threshold refresh by each query's owner warp.
+    // Per item: bound(first); then for each step i: bound(i+1), exact(i), and
+    // at checkpoints the threshold refresh by each query's owner warp.
     const int ew = warp - 2;                 // owner of query slot ew
     const int quad = warp & 3;
     const int half = ew >> 2;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint32_t nb = 0, u = 0, nbar = 0;
+    uint32_t kc = 0, u = 0, nbar = 0;
     int it = 0;
     unsigned long long n_seed = 0, n_screened = 0, n_rejected = 0, n_exact = 0, n_cand = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-      const Geom g = cert_geom(p, item);
-      // owner: load this item's state of query slot ew
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+      const Range rg = item_range(p, g, item);
+      if (rg.end <= rg.begin) continue;
+      const int n = rg.end - rg.begin;
+      // owner: this item's state of query slot ew (fresh, or carried over)
       {
         QState& s = st[ew];
+        const bool valid = ew < g.nq;
+        const int64_t row = g.local0 + ew;
         if (lane == 0) {
-          const bool valid = ew < g.nq;
-          s.tau = -INFINITY;
-          s.phase = valid ? 1 : 0;
-          s.count = 0;
-          s.overflow = 0;
-          s.lo = 0.f;
-          s.inv_w = 0.f;
-          s.w = 0.f;
-          s.row = g.local0 + ew;
+          s.row = row;
           s.pos = valid ? g.pos_first + ew : -1;
-          const float* cf = p.cert + (valid ? s.row : 0) * kCertFloats;
+          const float* cf = p.cert + (valid ? row : 0) * kCertFloats;
           for (int j = 0; j < 4; ++j) {
             s.omega[j] = valid ? cf[kCertOmega + j] : 0.f;
             s.scale[j] = valid ? cf[kCertScale + j] : 0.f;
@@ -464,36 +358,31 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           s.beta = valid ? cf[kCertBeta] : 0.f;
           s.margin = valid ? cf[kCertMargin] : 0.f;
           s.sq = (kFp8 && valid) ? __ldg(p.q_scale + g.t0 + ew) : 1.f;
-          if (ew == 0) *reinterpret_cast<volatile int*>(stop_word) = 0x7FFFFFFF;
         }
-        for (int b = lane; b < kBins; b += 32) s.hist[b] = 0;
+        if (valid && rg.begin > 0) state_load(s, p.qstate + row, lane);
+        else state_fresh(s, valid, lane);
         __syncwarp();
         __threadfence_block();
         if (lane == 0) mbar_arrive(item_ready);
         if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
+        ++it;
       }
-      int stop = 0x7FFFFFFF;                 // first unscreened tile (adaptive mode)
-      bool decided = p.screening != 2;
-      unsigned long long it_scr = 0, it_rej = 0;   // this warp's screened/rejected, this item
-      auto screened = [&](int t) -> bool {
-        return p.screening == 1 || (p.screening == 2 && t < stop);
+      unsigned long long it_scr = 0, it_rej = 0;   // this warp's counts, this item
+      auto key_of = [&](int i) -> int64_t {
+        return (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
       };
-      // key of this lane in tile ti
-      auto key_of = [&](int ti) -> int64_t {
-        return (int64_t)tile_at(ti, g.n_tiles) * kKeyTile + quad * 32 + lane;
-      };
-      // ---- bound evaluation of tile t (a screened tile) ----
-      auto bound_eval = [&](int t) -> bool {
-        const uint32_t b = nb + t;
-        const int64_t s = key_of(t);
+      // ---- bound evaluation of step i ----
+      auto bound_eval = [&](int i) -> bool {
+        const uint32_t c = kc + i;
+        const int64_t s = key_of(i);
         const bool key_ok = s < p.S;
         const float nk = key_ok ? __ldg(p.key_norm + s) : 0.f;
         float sk = 1.f;
         if constexpr (kFp8) sk = key_ok ? __ldg(p.k_scale + s) : 0.f;
-        if (!mbar_wait(&bnd_full[b & 1], (b >> 1) & 1, s_abort, p.err)) return false;
+        if (!mbar_wait(&bnd_full[c & 1], (c >> 1) & 1, s_abort, p.err)) return false;
         tc_fence_after();
         float v[32];
-        tmem_ld32(tmem_base + lane_off + C::kBndCol + (b & 1) * C::kBRows + half * 32, v);
+        tmem_ld32(tmem_base + lane_off + C::kBndCol + (c & 1) * C::kBRows + half * 32, v);
         uint32_t gbits = 0;
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
@@ -527,47 +416,33 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           n_rejected += rjm;
           it_scr += scr;
           it_rej += rjm;
-          if (lane == 0) masks[((b % 3) * 8 + ql) * 4 + quad] = mk;
+          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = mk;
           if (mk) gbits |= 1u << (ql >> 1);
         }
-        if (lane == 0) gflag[(b % 3) * 8 + ew] = gbits;
+        if (lane == 0) gflag[(c % 3) * 8 + ew] = gbits;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bnd_empty[b & 1]);
-          mbar_arrive(&mask_ready[b & 1]);
+          mbar_arrive(&bnd_empty[c & 1]);
+          mbar_arrive(&mask_ready[c & 1]);
         }
-        return mbar_wait(&mask_ready[b & 1], (b >> 1) & 1, s_abort, p.err);
+        return mbar_wait(&mask_ready[c & 1], (c >> 1) & 1, s_abort, p.err);
       };
-      bool scr_cur = screened(0);
-      int n_scr = scr_cur ? 1 : 0;
-      if (scr_cur && !bound_eval(0)) break;
-      for (int ti = 0; ti < g.n_tiles && ok; ++ti) {
-        bool scr_next = false;
-        if (ti + 1 < g.n_tiles) {
-          scr_next = scr_cur && screened(ti + 1);
-          if (scr_next) {
-            if (!bound_eval(ti + 1)) {
-              ok = false;
-              break;
-            }
-            ++n_scr;
-          }
+      if (!bound_eval(0)) break;
+      for (int i = 0; i < n && ok; ++i) {
+        if (i + 1 < n && !bound_eval(i + 1)) {
+          ok = false;
+          break;
         }
-        // ---- exact scoring of tile ti's survivors, filter, packed writeback ----
-        const int64_t s = key_of(ti);
+        // ---- exact scoring of step i's survivors, filter, packed writeback ----
+        const int64_t s = key_of(i);
         const bool key_ok = s < p.S;
         float sk = 1.f;
         if constexpr (kFp8) sk = key_ok ? __ldg(p.k_scale + s) : 0.f;
-        uint32_t groups;
-        const uint32_t b = nb + ti;
-        if (scr_cur) {
-          groups = 0;
-          for (int w = 0; w < C::kEpiWarps; ++w)
-            groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(b % 3) * 8 + w];
-        } else {
-          groups = (1u << ((g.nq + 1) / 2)) - 1u;
-        }
+        const uint32_t c = kc + i;
+        uint32_t groups = 0;
+        for (int w = 0; w < C::kEpiWarps; ++w)
+          groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(c % 3) * 8 + w];
         for (int grp = 0; grp < C::kGroups; ++grp) {
           if (!(groups >> grp & 1)) continue;
           const uint32_t ab = u % C::kAccBufs;
@@ -578,21 +453,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           tc_fence_after();
           const int ql = grp * 2 + half;
           QState& q = st[ql];
-          uint32_t mk;
-          if (scr_cur) {
-            mk = reinterpret_cast<volatile uint32_t*>(masks)[((b % 3) * 8 + ql) * 4 + quad];
-          } else {
-            const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
-            mk = __ballot_sync(0xFFFFFFFFu, phase != 0 && key_ok && s <= q.pos);
-            if (p.screening == 2) {
-              // pairs no longer screened still count as seeds when they are
-              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
-              n_seed += __popc(mk & __ballot_sync(0xFFFFFFFFu, seed));
-            } else {
-              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
-              n_seed += __popc(mk & __ballot_sync(0xFFFFFFFFu, seed));
-            }
-          }
+          const uint32_t mk =
+              reinterpret_cast<volatile uint32_t*>(masks)[((c % 3) * 8 + ql) * 4 + quad];
           if (mk) {
             float x[64];
             tmem_ld64(tmem_base + lane_off + C::kAccCol + ab * C::kGroupN + half * 64, x);
@@ -605,27 +467,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             }
             n_exact += __popc(mk);
             const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-            const bool app = mine && sc >= tau;
-            const uint32_t am = __ballot_sync(0xFFFFFFFFu, app);
-            if (am) {
-              int base = 0;
-              if (lane == 0) base = atomicAdd(&q.count, __popc(am));
-              base = __shfl_sync(0xFFFFFFFFu, base, 0);
-              const int slot = base + __popc(am & ((1u << lane) - 1u));
-              const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
-              if (app) {
-                if (slot < p.cap) {
-                  Cand cd;
-                  cd.score = sc;
-                  cd.key = (int)s;
-                  p.cand[q.row * (int64_t)p.cap + slot] = cd;
-                  if (phase == 2) atomicAdd(&q.hist[bin_of(q, sc)], 1u);
-                } else {
-                  q.overflow = 1;
-                }
-              }
-              n_cand += __popc(am);
-            }
+            n_cand += append_candidates(q, p.cand + q.row * (int64_t)p.cap, p.cap,
+                                        mine && sc >= tau, sc, (int)s, lane);
           }
           tc_fence_before();
           __syncwarp();
@@ -633,16 +476,13 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           ++u;
         }
         if (!ok) break;
-        // ---- checkpoint (every kCkptTiles tiles, and at the item's last tile) ----
-        // All epilogue warps meet; each owner then refreshes its query's
-        // threshold.  Between checkpoints the warps are coupled only through
-        // the accumulator and mask barriers.
-        const bool ckpt = ((ti + 1) % kCkptTiles) == 0 || ti + 1 == g.n_tiles;
-        if (ckpt) {
+        // ---- checkpoint: every kCkptTiles steps and at the range's last ----
+        const bool last = i + 1 == n;
+        if (((i + 1) % kCkptTiles) == 0 || last) {
           // The owner's own count, read before it arrives: every slot below it
-          // was reserved in a tile <= ti and written before its writer arrived,
+          // was reserved in a step <= i and written before its writer arrived,
           // and none of those writers saw the screening phase, so the warm-up
-          // scan below neither misses a written entry nor counts one twice.
+          // scan neither misses a written entry nor counts one twice.
           int snap_cnt = 0;
           if (lane == 0 && ew < g.nq) snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
           snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
@@ -658,81 +498,29 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           const uint32_t slot = nbar & 1;
           ++nbar;
-          // adaptive screening: every warp reads the same snapshot and takes
-          // the same decision; screening ends at tile ti + 4 (the MMA thread
-          // learns it from *stop_word before it would issue that tile's bound)
-          if (!decided) {
+          if (ew < g.nq)
+            refresh_threshold(st[ew], p.cand + st[ew].row * (int64_t)p.cap, snap_cnt, p.K, p.cap,
+                              lane);
+          if (last && !p.continue_pass && rg.end < g.n_tiles && ew == 0 && lane == 0) {
+            // the probe's decision, from the counts every warp left at this barrier
             unsigned long long tot_s = 0, tot_r = 0;
             for (int w = 0; w < C::kEpiWarps; ++w) {
               tot_s += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2];
               tot_r += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2 + 1];
             }
-            if (tot_s >= kAdaptiveMinScreened) {
-              decided = true;
-              if (tot_r * kAdaptiveRejectRatio < tot_s) {
-                stop = ti + 4;
-                if (ew == 0 && lane == 0) *reinterpret_cast<volatile int*>(stop_word) = stop;
-              }
-            }
-          }
-          // the owner refreshes its query's threshold
-          if (ti + 1 < g.n_tiles && ew < g.nq) {
-            QState& q = st[ew];
-            const int phase = q.phase;
-            const int cnt = snap_cnt;
-            if (phase == 1 && cnt >= p.K && cnt <= p.cap) {
-              // warm-up complete: bin the candidates so far over [min, max]
-              const Cand* cl = p.cand + q.row * (int64_t)p.cap;
-              float mn = INFINITY, mx = -INFINITY;
-              for (int i = lane; i < cnt; i += 32) {
-                const float x = cl[i].score;
-                mn = fminf(mn, x);
-                mx = fmaxf(mx, x);
-              }
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-              }
-              float w = (mx - mn) / (float)kBins;
-              if (!(w > 0.f) || !isfinite(w)) w = fmaxf(fabsf(mn), 1e-30f) * 0x1p-8f;
-              if (lane == 0) {
-                q.lo = mn;
-                q.w = w;
-                q.inv_w = 1.f / w;
-              }
-              __syncwarp();
-              for (int i = lane; i < cnt; i += 32) atomicAdd(&q.hist[bin_of(q, cl[i].score)], 1u);
-              __syncwarp();
-              const float tn = hist_threshold(q, p.K, lane);
-              if (lane == 0) {
-                q.tau = fmaxf(q.tau, tn);
-                __threadfence_block();
-                *reinterpret_cast<volatile int*>(&q.phase) = 2;
-              }
-            } else if (phase == 2) {
-              const float tn = hist_threshold(q, p.K, lane);
-              if (lane == 0 && tn > q.tau) *reinterpret_cast<volatile float*>(&q.tau) = tn;
-            }
-            __syncwarp();
+            const bool pays = tot_s < kMinScreened || tot_r * kRejectRatio >= tot_s;
+            p.item_flag[item] = pays ? kItemScreen : kItemFilter;
           }
         }
-        scr_cur = scr_next;
       }
-      nb += n_scr;
-      // ---- item end: the owner publishes its query ----
-      if (ok && ew < g.nq && lane == 0) {
-        QState& q = st[ew];
-        const int cnt = *reinterpret_cast<volatile int*>(&q.count);
-        const bool over = q.overflow || cnt > p.cap;
-        p.cand_count[q.row] = over ? -1 : cnt;
-        p.tau_out[q.row] = q.tau;
-        if (over) {
-          const int r = atomicAdd(p.repair_count, 1);
-          if (r < p.repair_cap) p.repair_list[r] = (int)q.row;
-          else record_error(p.err, kDevBounds);
-        }
+      kc += n;
+      // ---- range end: carry the query's state over, or publish it ----
+      if (ok && ew < g.nq) {
+        if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
+        else if (lane == 0) publish_query(st[ew], p.out);
       }
+      if (ok && !p.continue_pass && rg.end >= g.n_tiles && ew == 0 && lane == 0)
+        p.item_flag[item] = kItemDone;
     }
     if (lane == 0) {
       atomicAdd(&p.counters[kCntSeedPairs], n_seed);
@@ -753,28 +541,15 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
 
 // ---- host side ---------------------------------------------------------------------
 
-static bool encode_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
-                       uint32_t box_rows) {
-  auto enc = get_tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * (fp8 ? 1 : 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)(fp8 ? 128 : 64), box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool kFp8>
 static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
-                                    int K, cudaStream_t stream) {
+                                    int K, int probe_tiles, int continue_pass,
+                                    cudaStream_t stream) {
   using C = CertCfg<kFp8>;
   CUtensorMap qmap, bmap, kmap;
-  if (!encode_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
-      !encode_map(&bmap, b.bdir, kFp8, (uint64_t)v.rows * kBoundRows, C::kBRows) ||
-      !encode_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
+  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+      !encode_rows_map(&bmap, b.bdir, kFp8, (uint64_t)v.rows * kBoundRows, C::kBRows) ||
+      !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -794,23 +569,28 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.key_norm = b.key_norm;
   p.cert = b.cert;
   p.cand = reinterpret_cast<Cand*>(b.cand);
-  p.cand_count = b.cand_count;
-  p.tau_out = b.tau;
-  p.repair_list = b.repair_list;
-  p.repair_count = b.repair_count;
-  p.repair_cap = b.repair_cap;
+  p.qstate = reinterpret_cast<QStateG*>(b.qstate);
+  p.item_flag = b.item_flag;
+  p.out.cand_count = b.cand_count;
+  p.out.tau = b.tau;
+  p.out.repair_list = b.repair_list;
+  p.out.repair_count = b.repair_count;
+  p.out.repair_cap = b.repair_cap;
+  p.out.cap = b.cap;
+  p.out.err = b.err;
   p.counters = b.counters;
   p.err = b.err;
   p.row0 = v.row0;
   p.rows = v.rows;
   p.pos0 = v.pos0;
   p.S = v.S;
-  p.n_items = (int)((v.rows + 7) / 8);
+  p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
   p.K = K;
   p.cap = b.cap;
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
-  p.screening = h.cfg.screening;
+  p.probe_tiles = probe_tiles;
+  p.continue_pass = continue_pass;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
@@ -821,9 +601,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
 }
 
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             cudaStream_t stream) {
-  if (h.cfg.dtype == DOSA_FP8_E4M3) return launch_cert_impl<true>(h, v, b, K, stream);
-  return launch_cert_impl<false>(h, v, b, K, stream);
+                             int probe_tiles, int continue_pass, cudaStream_t stream) {
+  if (h.cfg.dtype == DOSA_FP8_E4M3)
+    return launch_cert_impl<true>(h, v, b, K, probe_tiles, continue_pass, stream);
+  return launch_cert_impl<false>(h, v, b, K, probe_tiles, continue_pass, stream);
 }
 
 size_t certified_smem_bytes(bool fp8) {

@@ -134,8 +134,9 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.repair_count = take(4);
   L.repair_scores = take((size_t)kRepairRows * S_max * 4);
   L.fixed = off;
+  // bound rows, record, retained, list, count, tau, carried state, item flag
   L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
-              (size_t)L.cap * 8 + 4 + 4;
+              (size_t)L.cap * 8 + 4 + 4 + qstate_bytes() + 1;
   return L;
 }
 
@@ -161,16 +162,30 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.cand = take((size_t)Tc * L.cap * 8);
   b.cand_count = reinterpret_cast<int*>(take((size_t)Tc * 4));
   b.tau = reinterpret_cast<float*>(take((size_t)Tc * 4));
+  b.qstate = take((size_t)Tc * qstate_bytes());
+  b.item_flag = reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4));
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
   b.err = &reinterpret_cast<WsHeader*>(ws)->error;
   return b;
 }
 
+// Padding the per-row arrays of a chunk may need (each starts 256-aligned),
+// plus the item-flag array's extra entry.
+constexpr size_t kCertPad = 8 * 256 + 4;
+
 // Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
 int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
-  if (ws_bytes <= L.fixed + 6 * 256) return 0;
-  int64_t rows = (int64_t)((ws_bytes - L.fixed - 6 * 256) / L.per_row);
+  if (ws_bytes <= L.fixed + kCertPad) return 0;
+  int64_t rows = (int64_t)((ws_bytes - L.fixed - kCertPad) / L.per_row);
   return rows / 8 * 8;
+}
+
+// Key tiles the probe pass screens per work item: enough for the warm-up (K
+// exact scores besides the seed tiles) plus 8 screened tiles, rounded up to
+// the threshold checkpoint interval.
+int probe_tiles(const Handle* h, int K) {
+  const int warm = (K + h->cfg.seed_first + h->cfg.seed_last + kKeyTile - 1) / kKeyTile + 1;
+  return (warm + 8 + 3) / 4 * 4;
 }
 
 int64_t total_visible(const int64_t* so, int B) {
@@ -248,7 +263,7 @@ dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max
     rows = round_up(rows, 8);
     if (rows > round_up(Tq, 8)) rows = round_up(Tq, 8);
     if (rows < 8) rows = 8;
-    *bytes = L.fixed + (size_t)rows * L.per_row + 6 * 256;
+    *bytes = L.fixed + (size_t)rows * L.per_row + kCertPad;
     return DOSA_OK;
   }
   int64_t rows = chunk_rows;
@@ -354,7 +369,17 @@ dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale
       nullptr, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {
         if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
           return DOSA_ERR_CUDA;
-        if (launch_certified(*h, c, b, K, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+        // screening 1: the probe pass covers every key tile; 2: probe, then the
+        // filter scorer and the continue pass finish what the probe flagged;
+        // 0: the filter scorer alone
+        const int mode = h->cfg.screening;
+        const int P = mode == 1 ? 0x3FFFFFFF : probe_tiles(h, K);
+        if (mode != 0 && launch_certified(*h, c, b, K, P, 0, stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
+        if (mode != 1 && launch_filter(*h, c, b, K, P, mode == 0, stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
+        if (mode == 2 && launch_certified(*h, c, b, K, P, 1, stream) != cudaSuccess)
+          return DOSA_ERR_CUDA;
         int32_t* out = out_idx + c.row0 * K;
         if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
         // rows whose candidate list overflowed: dense rescoring of just those rows

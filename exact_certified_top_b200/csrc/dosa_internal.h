@@ -53,6 +53,10 @@ void profile_after(int kind, cudaStream_t stream);
 
 // Tensor-map encoder from the driver (fetched once through the runtime).
 PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder();
+// 2-D map over `rows` rows of d = 128 elements (bf16 or fp8 codes), 128-byte
+// swizzle, boxes of one 128-byte row segment x box_rows rows (score_tc.cu).
+bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
+                     uint32_t box_rows);
 
 // Device buffers of one certified chunk (all inside the caller's workspace).
 struct CertBuffers {
@@ -64,6 +68,8 @@ struct CertBuffers {
   void* cand;            // [rows, cap] packed (score, key)
   int* cand_count;       // [rows]; -1 marks a row repaired by the dense pass
   float* tau;            // [rows] final threshold
+  void* qstate;          // [rows] candidate state carried from the probe pass
+  int* item_flag;        // [rows / 8] what the probe pass decided per work item
   int* repair_list;      // [repair_cap]
   int* repair_count;
   int repair_cap;
@@ -86,8 +92,17 @@ cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale
                             float* key_norm, float* key_sum, cudaStream_t stream);
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
                               void* bdir, float* cert, int32_t* retained, cudaStream_t stream);
+// Probe pass (continue_pass = 0): steps [0, probe_tiles) of every item with
+// screening, flags each unfinished item.  Continue pass: the remaining steps of
+// the items flagged for screening.
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             cudaStream_t stream);
+                             int probe_tiles, int continue_pass, cudaStream_t stream);
+// Filter scorer: the items the probe pass handed over (from step begin_step),
+// or every item from step 0 (all_items = 1).
+cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                          int begin_step, int all_items, cudaStream_t stream);
+// Bytes of carried candidate state per query row.
+size_t qstate_bytes();
 cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,
                           cudaStream_t stream);
 cudaError_t launch_topk_list(const float* scores, int64_t ld, const int* row_list,

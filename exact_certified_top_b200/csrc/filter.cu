@@ -1,0 +1,392 @@
+// Filter scorer of the certified indexer for sm_100a: exact scores of every
+// visible pair of a work item, filtered against the running threshold and
+// written back packed ("DOSA: Dots Sparse Attention", Daily Paper Cast
+// transcript, Method section: full-score computation fused with threshold
+// filtering and packed writeback; GPU kernel design: fixed-width query tiles on
+// dense tensor-core matrix operations).
+//
+// Same tile machinery as the dense scorer (score_tc.cu): A = 128 keys x d,
+// B = 4 queries x 64 heads (N = 256), two 256-column TMEM accumulators, one
+// persistent CTA per SM with a TMA producer warp, an MMA warp and 8 epilogue
+// warps.  The epilogue differs: instead of storing every score it keeps the
+// candidate state of the item's 8 queries in shared memory (cand_state.cuh)
+// and appends only scores >= tau_t, refreshing tau_t every 4 key tiles.
+//
+// It finishes the items that the certified kernel's probe pass handed over
+// (screening rejected too little there to pay for its bound evaluation),
+// resuming their state, or with screening switched off it runs every item
+// from its first key tile.
+#include "cand_state.cuh"
+#include "dosa_device.cuh"
+#include "dosa_internal.h"
+#include "score_epilogue.cuh"
+#include "work_items.cuh"
+
+namespace dosa {
+
+template <bool kFp8>
+struct FilterCfg {
+  static constexpr int kSub = kFp8 ? 1 : 2;
+  static constexpr int kKSteps = kFp8 ? 4 : 8;
+  static constexpr int kKeyStages = kFp8 ? 4 : 2;
+  static constexpr int kH = 64;
+  static constexpr int kQT = kItemQueries;
+  static constexpr int kQRows = kQT * kH;
+  static constexpr int kGroupRows = 256;               // MMA N: 4 queries
+  static constexpr int kGroups = kQRows / kGroupRows;
+  static constexpr int kQPerGroup = kGroupRows / kH;
+  static constexpr uint32_t kKeySubBytes = kKeyTile * 128;
+  static constexpr uint32_t kKeyStageBytes = kKeySubBytes * kSub;
+  static constexpr uint32_t kQSubBytes = kQRows * 128;
+  static constexpr uint32_t kQBytes = kQSubBytes * kSub;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 64 + kEpiWarps * 32;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kStateBytes = sizeof(QState) * kQT;
+  static constexpr uint32_t kSmemBytes =
+      1024 + kQBytes + kKeyStages * kKeyStageBytes + kStateBytes + 256;
+};
+
+struct FilterParams {
+  const float* w;          // [rows_total, 64] absolute rows
+  const float* q_scale;    // absolute rows (fp8)
+  const float* k_scale;    // sequence base (fp8)
+  Cand* cand;              // [chunk rows, cap]
+  QStateG* qstate;         // [chunk rows] state handed over by the probe pass
+  const int* item_flag;    // [n_items]
+  PublishOut out;
+  unsigned long long* counters;
+  int* err;
+  int64_t row0, rows, pos0, S;
+  int n_items, K, cap, seed_first, seed_last;
+  int begin_step;          // first step of a handed-over item
+  int all_items;           // 1: every item from step 0 with a fresh state
+};
+
+struct FRange {
+  int begin, end;
+};
+
+__device__ __forceinline__ FRange filter_range(const FilterParams& p, const Geom& g, int item) {
+  FRange r;
+  if (p.all_items) {
+    r.begin = 0;
+    r.end = g.n_tiles;
+  } else {
+    const bool go = p.item_flag[item] == kItemFilter;
+    r.begin = go ? p.begin_step : 0;
+    r.end = go ? g.n_tiles : 0;
+  }
+  return r;
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
+    filter_kernel(const __grid_constant__ CUtensorMap qmap,
+                  const __grid_constant__ CUtensorMap kmap, const FilterParams p) {
+  using C = FilterCfg<kFp8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + C::kQBytes;
+  QState* st = reinterpret_cast<QState*>(sK + C::kKeyStages * C::kKeyStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(st + C::kQT);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* acc_full = bars + 2;     // [2]
+  uint64_t* acc_empty = bars + 4;    // [2]
+  uint64_t* tile_done = bars + 6;
+  uint64_t* item_ready = bars + 7;
+  uint64_t* done_bar = bars + 8;
+  uint64_t* k_full = bars + 9;                   // [kKeyStages]
+  uint64_t* k_empty = k_full + C::kKeyStages;    // [kKeyStages]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(k_empty + C::kKeyStages);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::kEpiWarps);
+    }
+    mbar_init(tile_done, C::kEpiWarps);
+    mbar_init(item_ready, C::kEpiWarps);
+    mbar_init(done_bar, 1);
+    for (int i = 0; i < C::kKeyStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t kc = 0;
+      int it = 0;
+      bool ok = true;
+      uint32_t inflight_q = 0xFFFFFFFFu;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const FRange rg = filter_range(p, g, item);
+        if (rg.end <= rg.begin) continue;
+        if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        for (int sub = 0; sub < C::kSub; ++sub)
+          for (int b = 0; b < C::kQRows / 256; ++b)
+            tma_load_2d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64,
+                        (int32_t)(g.t0 * C::kH + b * 256));
+        inflight_q = it & 1;
+        ++it;
+        for (int ti = rg.begin; ti < rg.end; ++ti, ++kc) {
+          const int s_ = kc % C::kKeyStages;
+          const uint32_t rnd = kc / C::kKeyStages;
+          if (!mbar_wait(&k_empty[s_], (rnd & 1) ^ 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[s_], C::kKeyStageBytes);
+          const int j = tile_at(ti, g.n_tiles);
+          for (int sub = 0; sub < C::kSub; ++sub)
+            tma_load_2d(sK + s_ * C::kKeyStageBytes + sub * C::kKeySubBytes, &kmap, &k_full[s_],
+                        sub * 64, j * kKeyTile);
+        }
+      }
+      if (*s_abort) {
+        if (inflight_q != 0xFFFFFFFFu) mbar_wait_drain(q_full, inflight_q);
+        for (uint32_t c = (kc > (uint32_t)C::kKeyStages ? kc - C::kKeyStages : 0); c < kc; ++c)
+          mbar_wait_drain(&k_full[c % C::kKeyStages], (c / C::kKeyStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = make_idesc<kFp8>(kKeyTile, C::kGroupRows);
+      uint32_t kc = 0, u = 0;
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const FRange rg = filter_range(p, g, item);
+        if (rg.end <= rg.begin) continue;
+        if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
+        ++it;
+        tc_fence_after();
+        for (int ti = rg.begin; ti < rg.end && ok; ++ti, ++kc) {
+          const int s_ = kc % C::kKeyStages;
+          if (!mbar_wait(&k_full[s_], (kc / C::kKeyStages) & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
+          for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
+            const uint32_t buf = u & 1;
+            if (!mbar_wait(&acc_empty[buf], ((u >> 1) & 1) ^ 1, s_abort, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t b_base = smem_u32(sQ + grp * C::kGroupRows * 128);
+            const uint32_t d = tmem_base + buf * C::kGroupRows;
+#pragma unroll
+            for (int step = 0; step < C::kKSteps; ++step) {
+              const uint32_t sub = step >> 2, off = (step & 3) * 32;
+              tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
+                           smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc,
+                           step > 0 ? 1u : 0u);
+            }
+            tc_commit(&acc_full[buf]);
+          }
+          tc_commit(&k_empty[s_]);
+        }
+        tc_commit(q_empty);
+      }
+      tc_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int ew = warp - 2;                 // owner of query slot ew
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may read
+    const int half = ew >> 2;                // which two queries of each MMA tile
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint32_t u = 0, nbar = 0;
+    int it = 0;
+    unsigned long long n_seed = 0, n_exact = 0, n_cand = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+      const FRange rg = filter_range(p, g, item);
+      if (rg.end <= rg.begin) continue;
+      const int n = rg.end - rg.begin;
+      {
+        QState& s = st[ew];
+        const bool valid = ew < g.nq;
+        const int64_t row = g.local0 + ew;
+        if (lane == 0) {
+          s.row = row;
+          s.pos = valid ? g.pos_first + ew : -1;
+        }
+        if (valid && rg.begin > 0) state_load(s, p.qstate + row, lane);
+        else state_fresh(s, valid, lane);
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) mbar_arrive(item_ready);
+        if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
+        ++it;
+      }
+      for (int i = 0; i < n && ok; ++i) {
+        const int64_t s = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        float sk = 1.f;
+        if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
+        for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
+          const uint32_t buf = u & 1;
+          if (!mbar_wait(&acc_full[buf], (u >> 1) & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int qi = 0; qi < 2; ++qi) {
+            const int ql = grp * C::kQPerGroup + half * 2 + qi;
+            float x[64];
+            tmem_ld64(tmem_base + lane_off + buf * C::kGroupRows + (half * 2 + qi) * 64, x);
+            if (ql < g.nq) {
+              QState& q = st[ql];
+              const int64_t t = g.t0 + ql;
+              float sc = head_reduce64(x, p.w + t * C::kH);
+              if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
+              const bool vis = s <= q.pos;
+              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
+              n_exact += __popc(__ballot_sync(0xFFFFFFFFu, vis));
+              n_seed += __popc(__ballot_sync(0xFFFFFFFFu, vis && seed));
+              const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
+              n_cand += append_candidates(q, p.cand + q.row * (int64_t)p.cap, p.cap,
+                                          vis && sc >= tau, sc, (int)s, lane);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        if (!ok) break;
+        // ---- checkpoint: every kCkptTiles steps and at the item's last ----
+        if (((i + 1) % kCkptTiles) == 0 || i + 1 == n) {
+          // The owner's count read before it arrives: every slot below it was
+          // written before its writer arrived (see certified.cu).
+          int snap_cnt = 0;
+          if (lane == 0 && ew < g.nq) snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
+          snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
+          __threadfence_block();
+          if (lane == 0) mbar_arrive(tile_done);
+          if (!mbar_wait(tile_done, nbar & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          ++nbar;
+          if (ew < g.nq)
+            refresh_threshold(st[ew], p.cand + st[ew].row * (int64_t)p.cap, snap_cnt, p.K, p.cap,
+                              lane);
+        }
+      }
+      if (ok && ew < g.nq && lane == 0) publish_query(st[ew], p.out);
+    }
+    if (lane == 0) {
+      atomicAdd(&p.counters[kCntSeedPairs], n_seed);
+      atomicAdd(&p.counters[kCntExact], n_exact);
+      atomicAdd(&p.counters[kCntCandidates], n_cand);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---- host side ---------------------------------------------------------------------
+
+template <bool kFp8>
+static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
+                                      int K, int begin_step, int all_items, cudaStream_t stream) {
+  using C = FilterCfg<kFp8>;
+  CUtensorMap qmap, kmap;
+  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+      !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(filter_kernel<kFp8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  FilterParams p;
+  p.w = v.w;
+  p.q_scale = v.q_scale;
+  p.k_scale = v.k_scale;
+  p.cand = reinterpret_cast<Cand*>(b.cand);
+  p.qstate = reinterpret_cast<QStateG*>(b.qstate);
+  p.item_flag = b.item_flag;
+  p.out.cand_count = b.cand_count;
+  p.out.tau = b.tau;
+  p.out.repair_list = b.repair_list;
+  p.out.repair_count = b.repair_count;
+  p.out.repair_cap = b.repair_cap;
+  p.out.cap = b.cap;
+  p.out.err = b.err;
+  p.counters = b.counters;
+  p.err = b.err;
+  p.row0 = v.row0;
+  p.rows = v.rows;
+  p.pos0 = v.pos0;
+  p.S = v.S;
+  p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
+  p.K = K;
+  p.cap = b.cap;
+  p.seed_first = h.cfg.seed_first;
+  p.seed_last = h.cfg.seed_last;
+  p.begin_step = begin_step;
+  p.all_items = all_items;
+  if (p.n_items == 0) return cudaSuccess;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  profile_before(DOSA_KERNEL_FILTER, stream);
+  filter_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  const cudaError_t e = cudaGetLastError();
+  profile_after(DOSA_KERNEL_FILTER, stream);
+  return e;
+}
+
+size_t qstate_bytes() { return sizeof(QStateG); }
+
+cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                          int begin_step, int all_items, cudaStream_t stream) {
+  if (h.cfg.dtype == DOSA_FP8_E4M3)
+    return launch_filter_impl<true>(h, v, b, K, begin_step, all_items, stream);
+  return launch_filter_impl<false>(h, v, b, K, begin_step, all_items, stream);
+}
+
+}  // namespace dosa

@@ -252,15 +252,16 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
             break;
           }
           tc_fence_after();
-          // both of this warp's queries in one TMEM load (128 columns)
-          float v[128];
-          tmem_ld128(tmem_base + lane_off + buf * C::kGroupRows + half * 128, v);
-#pragma unroll
+          // the warp's two queries one after the other (measured faster on B200
+          // than one 128-column load or an overlapped second load)
+#pragma unroll 1
           for (int qi = 0; qi < 2; ++qi) {
             const int ql = grp * C::kQPerGroup + half * 2 + qi;
+            float v[64];
+            tmem_ld64(tmem_base + lane_off + buf * C::kGroupRows + (half * 2 + qi) * 64, v);
             if (ql < g.nq) {
               const int64_t t = g.t0 + ql;
-              float sc = head_reduce64(v + qi * 64, p.w + t * C::kH);
+              float sc = head_reduce64(v, p.w + t * C::kH);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
               if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
             }
@@ -283,8 +284,8 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
 
 // ---- host side ------------------------------------------------------------------
 
-static bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
-                            uint32_t box_rows) {
+bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
+                     uint32_t box_rows) {
   auto enc = get_tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};

@@ -1,0 +1,47 @@
+// Work items of the certified and filter scorers: tiles of 8 consecutive
+// query rows of a chunk, longest rows first, and the processing order of the
+// key tiles each item sees (tile 0, which holds the first seed keys, then from
+// the diagonal tile downwards).
+#pragma once
+
+#include <stdint.h>
+
+#include "dosa_internal.h"
+
+namespace dosa {
+
+constexpr int kItemQueries = 8;
+// The epilogue warps meet (threshold refresh) every this many key tiles of an
+// item and at the end of the item's range.
+constexpr int kCkptTiles = 4;
+
+struct Geom {
+  int64_t t0;        // absolute first row
+  int64_t local0;    // chunk-local first row
+  int nq;            // valid queries in the item
+  int64_t pos_first; // position of the first query
+  int n_tiles;       // key tiles 0..n_tiles-1 hold every visible key
+};
+
+__device__ __forceinline__ Geom item_geometry(int64_t row0, int64_t rows, int64_t pos0, int n_items,
+                                              int item) {
+  Geom g;
+  const int tile = n_items - 1 - item;        // longest rows first
+  g.local0 = (int64_t)tile * kItemQueries;
+  g.t0 = row0 + g.local0;
+  const int64_t left = rows - g.local0;
+  g.nq = (int)(left < kItemQueries ? left : kItemQueries);
+  g.pos_first = pos0 + g.local0;
+  g.n_tiles = (int)((g.pos_first + g.nq - 1) / kKeyTile) + 1;
+  return g;
+}
+
+// Key tile processed at step ti of an item with n_tiles tiles.
+__device__ __forceinline__ int tile_at(int ti, int n_tiles) {
+  return ti == 0 ? 0 : n_tiles - ti;
+}
+
+// What the probe pass decided for an item (certified workspace flags).
+enum ItemFlag : int { kItemDone = 0, kItemFilter = 1, kItemScreen = 2 };
+
+}  // namespace dosa

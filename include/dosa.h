@@ -85,9 +85,12 @@ typedef struct {
   int G;            /* negative-head groups (0 = no negative aggregate, 1, 2)   */
   int margin_log2;  /* soundness margin 2^margin_log2 * sum|w|||q|| * ||k||     */
   int screening;    /* 1: screen every key tile with the certificate; 2: adaptive
-                       (per tile of 8 queries, stop screening once 4096 screened
-                       pairs show under 1/32 rejected); 0: never (ablation).
-                       The selection is exact in every mode.                    */
+                       (every tile of 8 queries is screened over its first key
+                       tiles; where that rejected under 1/32 of 4096 or more
+                       screened pairs, the rest of its keys is scored exactly
+                       without bounds, else screening goes on to the end);
+                       0: never (ablation).  The selection is exact in every
+                       mode.                                                    */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */
@@ -211,7 +214,8 @@ typedef enum {
   DOSA_KERNEL_CERT_SETUP = 4,  /* per-query certificate                        */
   DOSA_KERNEL_CERTIFIED = 5,   /* seed scoring, screening, rescoring, writeback */
   DOSA_KERNEL_SELECT = 6,      /* selection over the packed candidates         */
-  DOSA_KERNEL_KINDS = 7
+  DOSA_KERNEL_FILTER = 7,      /* exact scoring + threshold filter, no bounds  */
+  DOSA_KERNEL_KINDS = 8
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

@@ -156,7 +156,44 @@ def test_certificate_matches_oracle(cuda_lib):
             assert cert[t, 12] + cert[t, 13] == sum(g.size for g in c.groups)
 
 
-def test_repair_pass_when_candidates_overflow(cuda_lib):
+@pytest.mark.parametrize("fp8", [False, True])
+def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
+    """Work items of 8 queries alternate between redundant heads (screening
+    rejects most keys: the probe lets screening continue) and independent
+    random heads (screening rejects almost nothing: the probe hands the item to
+    the filter scorer).  Both finishers run in one call; the selection stays
+    identical to the dense path and to the oracle."""
+    x, dtype = _redundant_heads_case(T=160, S=7000, seed=11, fp8=fp8)
+    g = torch.Generator().manual_seed(12)
+    rand_rows = torch.cat([torch.arange(i, i + 8) for i in range(8, 160, 16)])
+    if fp8:
+        from exact_certified_top_b200.workloads import _e4m3_per_token
+        q8, qs = _e4m3_per_token(torch.randn((len(rand_rows), 64, 128), generator=g))
+        x["q"][rand_rows] = q8
+        x["q_scale"][rand_rows] = qs
+    else:
+        x["q"][rand_rows] = torch.randn((len(rand_rows), 64, 128), generator=g).to(torch.bfloat16)
+    x["w"][rand_rows] = torch.randn((len(rand_rows), 64), generator=g) / 8
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 128
+    idx = binding.Index(dtype, screening=2)
+    cert, stats = idx.topk(*_args(xd, K), stats=True)
+    dense = idx.dense_topk(*_args(xd, K))
+    assert torch.equal(cert, dense)
+    assert stats["exact_pairs"] + stats["rejected_pairs"] == stats["visible_pairs"]
+    # about half the rows prune most of their keys, the other half hardly any
+    prune = stats["rejected_pairs"] / stats["visible_pairs"]
+    assert 0.2 < prune < 0.6, stats
+    # the filtered half is not screened past its probe tiles
+    assert stats["screened_pairs"] < 0.75 * stats["visible_pairs"], stats
+    ov = OracleView(x, dtype)
+    cert = to_numpy(cert)
+    for t in range(0, 160, 7):
+        assert_topk_matches(cert[t], ov.scores(t), K, t=t, exact=False)
+
+
+@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
+def test_repair_pass_when_candidates_overflow(cuda_lib, screening):
     """All keys identical: every score ties, every key becomes a candidate and
     the candidate list overflows; the rows are rescored densely and the
     selection (ties to the smaller index) is still exact."""
@@ -166,7 +203,7 @@ def test_repair_pass_when_candidates_overflow(cuda_lib):
     w = torch.randn((T, 64), generator=g) / 8
     k = torch.randn((1, 128), generator=g).expand(S, 128).contiguous().to(torch.bfloat16)
     so = [[0, 0, S - T], [T, S, 0]]
-    idx = binding.Index("bf16")
+    idx = binding.Index("bf16", screening=screening)
     qd, wd, kd = q.cuda(), w.cuda(), k.cuda()
     cert = to_numpy(idx.topk(qd, None, wd, kd, None, so, K))
     dense = to_numpy(idx.dense_topk(qd, None, wd, kd, None, so, K))
