@@ -39,7 +39,7 @@ struct FilterCfg {
   static constexpr uint32_t kKeyStageBytes = kKeySubBytes * kSub;
   static constexpr uint32_t kQSubBytes = kQRows * 128;
   static constexpr uint32_t kQBytes = kQSubBytes * kSub;
-  static constexpr int kEpiWarps = 8;
+  static constexpr int kEpiWarps = 16;                 // 4 per TMEM lane quadrant
   static constexpr int kThreads = 64 + kEpiWarps * 32;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kStateBytes = sizeof(QState) * kQT;
@@ -223,9 +223,14 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
-    const int ew = warp - 2;                 // owner of query slot ew
-    const int quad = warp & 3;               // TMEM lane quadrant this warp may read
-    const int half = ew >> 2;                // which two queries of each MMA tile
+    // 16 warps: warp (2 + ew) reads TMEM lane quadrant (warp & 3), i.e. 32
+    // keys, and query (ew >> 2) of each 4-query MMA tile.  Warps 0-7 of the
+    // epilogue also own query slot ew (state set-up, threshold refresh,
+    // publication).
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int sub = ew >> 2;
+    const bool owner = ew < C::kQT;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     uint32_t u = 0, nbar = 0;
     int it = 0;
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       const FRange rg = filter_range(p, g, item);
       if (rg.end <= rg.begin) continue;
       const int n = rg.end - rg.begin;
-      {
+      if (owner) {
         QState& s = st[ew];
         const bool valid = ew < g.nq;
         const int64_t row = g.local0 + ew;
@@ -248,12 +253,13 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
         else state_fresh(s, valid, lane);
         __syncwarp();
         __threadfence_block();
-        if (lane == 0) mbar_arrive(item_ready);
-        if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
-        ++it;
       }
+      if (lane == 0) mbar_arrive(item_ready);
+      if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
+      ++it;
       for (int i = 0; i < n && ok; ++i) {
-        const int64_t s = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        const int64_t base = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32;
+        const int64_t s = base + lane;
         float sk = 1.f;
         if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
         for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
@@ -263,28 +269,38 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             break;
           }
           tc_fence_after();
-#pragma unroll 1
-          for (int qi = 0; qi < 2; ++qi) {
-            const int ql = grp * C::kQPerGroup + half * 2 + qi;
-            float x[64];
-            tmem_ld64(tmem_base + lane_off + buf * C::kGroupRows + (half * 2 + qi) * 64, x);
-            if (ql < g.nq) {
-              QState& q = st[ql];
-              const int64_t t = g.t0 + ql;
-              float sc = head_reduce64(x, p.w + t * C::kH);
-              if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
-              const bool vis = s <= q.pos;
-              const bool seed = s < p.seed_first || s > q.pos - p.seed_last;
-              n_exact += __popc(__ballot_sync(0xFFFFFFFFu, vis));
-              n_seed += __popc(__ballot_sync(0xFFFFFFFFu, vis && seed));
-              const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-              n_cand += append_candidates(q, p.cand + q.row * (int64_t)p.cap, p.cap,
-                                          vis && sc >= tau, sc, (int)s, lane);
-            }
-          }
+          const int ql = grp * C::kQPerGroup + sub;
+          // 32 heads at a time (the register budget of 18 warps is 96 per thread)
+          const uint32_t col = tmem_base + lane_off + buf * C::kGroupRows + sub * 64;
+          const float* wq = p.w + (g.t0 + (ql < g.nq ? ql : g.nq - 1)) * C::kH;
+          float x[32];
+          HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
+          tmem_ld32_async(col, x);
+          tmem_wait_ld(x);
+          head_accumulate32(acc, x, wq);
+          tmem_ld32_async(col + 32, x);
+          tmem_wait_ld(x);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          head_accumulate32(acc, x, wq + 32);
+          if (ql < g.nq) {
+            QState& q = st[ql];
+            const int64_t t = g.t0 + ql;
+            const int64_t pos = g.pos_first + ql;
+            float sc = head_total(acc);
+            if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
+            // visible and seed pairs of these 32 keys, from the intervals
+            const int64_t e = base + 31 < pos ? base + 31 : pos;
+            const int64_t nvis = e >= base ? e - base + 1 : 0;
+            const int64_t lo = base > p.seed_first ? base : (int64_t)p.seed_first;
+            const int64_t hi = e < pos - p.seed_last ? e : pos - p.seed_last;
+            n_exact += nvis;
+            n_seed += nvis - (hi >= lo ? hi - lo + 1 : 0);
+            const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
+            n_cand += append_candidates(q, p.cand + (g.local0 + ql) * (int64_t)p.cap, p.cap,
+                                        s <= pos && sc >= tau, sc, (int)s, lane);
+          }
         }
         if (!ok) break;
         // ---- checkpoint: every kCkptTiles steps and at the item's last ----
@@ -292,7 +308,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           // The owner's count read before it arrives: every slot below it was
           // written before its writer arrived (see certified.cu).
           int snap_cnt = 0;
-          if (lane == 0 && ew < g.nq) snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
+          if (lane == 0 && owner && ew < g.nq)
+            snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
           snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
           __threadfence_block();
           if (lane == 0) mbar_arrive(tile_done);
@@ -301,12 +318,12 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             break;
           }
           ++nbar;
-          if (ew < g.nq)
+          if (owner && ew < g.nq)
             refresh_threshold(st[ew], p.cand + st[ew].row * (int64_t)p.cap, snap_cnt, p.K, p.cap,
                               lane);
         }
       }
-      if (ok && ew < g.nq && lane == 0) publish_query(st[ew], p.out);
+      if (ok && owner && ew < g.nq && lane == 0) publish_query(st[ew], p.out);
     }
     if (lane == 0) {
       atomicAdd(&p.counters[kCntSeedPairs], n_seed);

@@ -11,7 +11,7 @@
 // memory while every key tile it can see streams through a ring of stages.
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM owner and MMA issuer (one elected thread)
-//   warps 2-9   epilogue: TMEM -> registers, w * ReLU, head sum, store
+//   warps 2-17  epilogue: TMEM -> registers, w * ReLU, head sum, store
 // MMA tile: A = 128 keys x d (K-major), B = 256 head rows (4 queries x 64
 // heads) x d (K-major), D = 128 x 256 fp32 in TMEM.  Two D buffers (512 TMEM
 // columns) let the epilogue of one tile overlap the MMA of the next.  TMEM lane
@@ -41,7 +41,7 @@ struct ScoreCfg {
   static constexpr uint32_t kKeyStageBytes = kKeySubBytes * kSub;
   static constexpr uint32_t kQSubBytes = kQRows * 128;
   static constexpr uint32_t kQBytes = kQSubBytes * kSub;
-  static constexpr int kEpiWarps = 8;
+  static constexpr int kEpiWarps = 16;                 // 4 per TMEM lane quadrant
   static constexpr int kThreads = 64 + kEpiWarps * 32;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSmemBytes =
@@ -233,9 +233,11 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
+    // 16 warps: warp (2 + ew) reads TMEM lane quadrant (warp & 3), i.e. 32
+    // keys, and query (ew >> 2) of each 4-query MMA tile.
     const int ew = warp - 2;
-    const int quad = warp & 3;           // TMEM lane quadrant this warp may read
-    const int half = ew >> 2;            // which two queries of each MMA tile
+    const int quad = warp & 3;
+    const int sub = ew >> 2;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     uint32_t u = 0;
     bool ok = true;
@@ -252,23 +254,27 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
             break;
           }
           tc_fence_after();
-          // the warp's two queries one after the other (measured faster on B200
-          // than one 128-column load or an overlapped second load)
-#pragma unroll 1
-          for (int qi = 0; qi < 2; ++qi) {
-            const int ql = grp * C::kQPerGroup + half * 2 + qi;
-            float v[64];
-            tmem_ld64(tmem_base + lane_off + buf * C::kGroupRows + (half * 2 + qi) * 64, v);
-            if (ql < g.nq) {
-              const int64_t t = g.t0 + ql;
-              float sc = head_reduce64(v, p.w + t * C::kH);
-              if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
-              if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
-            }
-          }
+          const int ql = grp * C::kQPerGroup + sub;
+          // 32 heads at a time (the register budget of 18 warps is 96 per thread)
+          const uint32_t col = tmem_base + lane_off + buf * C::kGroupRows + sub * 64;
+          const float* wq = p.w + (g.t0 + (ql < g.nq ? ql : g.nq - 1)) * C::kH;
+          float v[32];
+          HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
+          tmem_ld32_async(col, v);
+          tmem_wait_ld(v);
+          head_accumulate32(acc, v, wq);
+          tmem_ld32_async(col + 32, v);
+          tmem_wait_ld(v);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          head_accumulate32(acc, v, wq + 32);
+          if (ql < g.nq) {
+            const int64_t t = g.t0 + ql;
+            float sc = head_total(acc);
+            if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
+            if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
+          }
         }
       }
     }
