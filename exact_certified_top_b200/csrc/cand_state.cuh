@@ -1,5 +1,5 @@
 // Per-query candidate state shared by the certified scorer and the filter
-// scorer: the running threshold tau, the candidate count, and the 256-bin
+// scorer: the running threshold tau, the candidate lists, and the 256-bin
 // score histogram that keeps tau a sound lower bound on the K-th largest exact
 // score seen so far ("DOSA: Dots Sparse Attention", Daily Paper Cast
 // transcript, Method section: a threshold from the K-th largest exact score of
@@ -10,6 +10,13 @@
 // rounded-down lower edge of the highest bin whose suffix count reaches K.
 // Every counted candidate in those bins has a score >= that edge, so at least
 // K exact scores are >= tau.
+//
+// Candidate lists are split into kSegs segments per query, one per TMEM lane
+// quadrant: key s of a tile is scored by a warp of quadrant (s mod 128) / 32
+// in every kernel, and for a given query exactly one warp of each quadrant
+// does so.  That warp is the only writer of its segment and keeps the
+// segment's count in a register; counts are published to shared memory at the
+// threshold checkpoints, where all epilogue warps meet.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -20,14 +27,15 @@
 namespace dosa {
 
 constexpr int kBins = 256;
+constexpr int kSegs = 4;
 
 // Shared-memory state of one query of a work item.
 struct QState {
   float tau;
   int phase;          // 0 = unused slot, 1 = warm-up, 2 = screening/filtering
-  int count;          // candidates reserved (may exceed the capacity)
-  int overflow;
+  int overflow;       // a segment ran out of room
   float lo, inv_w, w;
+  int seg[kSegs];     // candidates per segment, as of the last checkpoint
   float omega[4];
   float beta, margin;
   float scale[4];
@@ -42,10 +50,10 @@ struct QState {
 struct QStateG {
   float tau;
   int phase;
-  int count;
   int overflow;
   float lo, inv_w, w;
-  int pad;
+  int seg[kSegs];
+  int pad[2];
   unsigned hist[kBins];
 };
 
@@ -99,19 +107,31 @@ __device__ __forceinline__ float hist_threshold(const QState& s, int K, int lane
   return bin_edge(s, best);
 }
 
-// Owner warp, at a checkpoint: finish warm-up (bin the first `cnt`
-// candidates, whose writes are all complete) or refresh tau from the
-// histogram.  `cnt` is the query's count read before the checkpoint barrier.
-__device__ __forceinline__ void refresh_threshold(QState& q, const Cand* cl, int cnt, int K,
-                                                  int cap, int lane) {
+// Owner warp, after a checkpoint barrier: finish warm-up (bin every candidate
+// so far: the segment counts published at this barrier cover only entries
+// whose writes are complete, and their writers saw the warm-up phase, so
+// none of them is in the histogram yet) or refresh tau from the histogram.
+// Segment j of the query's list starts at list + j * seg_cap.
+__device__ __forceinline__ void refresh_threshold(QState& q, const Cand* list, int seg_cap, int K,
+                                                  int lane) {
   const int phase = q.phase;
-  if (phase == 1 && cnt >= K && cnt <= cap) {
-    float mn = INFINITY, mx = -INFINITY;
-    for (int i = lane; i < cnt; i += 32) {
-      const float x = cl[i].score;
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+  if (phase == 1) {
+    int cnt[kSegs], total = 0;
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j) {
+      const int c = q.seg[j];
+      cnt[j] = c < seg_cap ? c : seg_cap;
+      total += cnt[j];
     }
+    if (total < K || *reinterpret_cast<const volatile int*>(&q.overflow)) return;
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j)
+      for (int i = lane; i < cnt[j]; i += 32) {
+        const float x = list[j * seg_cap + i].score;
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+      }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
@@ -125,7 +145,10 @@ __device__ __forceinline__ void refresh_threshold(QState& q, const Cand* cl, int
       q.inv_w = 1.f / w;
     }
     __syncwarp();
-    for (int i = lane; i < cnt; i += 32) atomicAdd(&q.hist[bin_of(q, cl[i].score)], 1u);
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j)
+      for (int i = lane; i < cnt[j]; i += 32)
+        atomicAdd(&q.hist[bin_of(q, list[j * seg_cap + i].score)], 1u);
     __syncwarp();
     const float tn = hist_threshold(q, K, lane);
     if (lane == 0) {
@@ -140,24 +163,23 @@ __device__ __forceinline__ void refresh_threshold(QState& q, const Cand* cl, int
   __syncwarp();
 }
 
-// Append the warp's candidates (lanes with app set) to query q's list.
-// Returns the number appended.
-__device__ __forceinline__ unsigned append_candidates(QState& q, Cand* list, int cap, bool app,
-                                                      float sc, int key, int lane) {
+// Append the warp's candidates (lanes with app set) to the warp's segment of
+// query q, whose count the warp holds in `cnt`.  Returns the number appended.
+// No atomic on the count: the warp is the segment's only writer.
+__device__ __forceinline__ unsigned append_candidates(QState& q, Cand* seg, int seg_cap, int& cnt,
+                                                      bool app, float sc, int key, int lane) {
   const unsigned am = __ballot_sync(0xFFFFFFFFu, app);
   if (!am) return 0;
-  int base = 0;
-  if (lane == 0) base = atomicAdd(&q.count, __popc(am));
-  base = __shfl_sync(0xFFFFFFFFu, base, 0);
-  const int slot = base + __popc(am & ((1u << lane) - 1u));
-  const int phase = *reinterpret_cast<const volatile int*>(&q.phase);
+  const int slot = cnt + __popc(am & ((1u << lane) - 1u));
+  cnt += __popc(am);
   if (app) {
-    if (slot < cap) {
+    if (slot < seg_cap) {
       Cand cd;
       cd.score = sc;
       cd.key = key;
-      list[slot] = cd;
-      if (phase == 2) atomicAdd(&q.hist[bin_of(q, sc)], 1u);
+      seg[slot] = cd;
+      if (*reinterpret_cast<const volatile int*>(&q.phase) == 2)
+        atomicAdd(&q.hist[bin_of(q, sc)], 1u);
     } else {
       q.overflow = 1;
     }
@@ -171,11 +193,12 @@ __device__ __forceinline__ void state_save(const QState& q, QStateG* g, int lane
   if (lane == 0) {
     g->tau = q.tau;
     g->phase = q.phase;
-    g->count = q.count;
     g->overflow = q.overflow;
     g->lo = q.lo;
     g->inv_w = q.inv_w;
     g->w = q.w;
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j) g->seg[j] = q.seg[j];
   }
   for (int b = lane; b < kBins; b += 32) g->hist[b] = q.hist[b];
 }
@@ -184,11 +207,12 @@ __device__ __forceinline__ void state_load(QState& q, const QStateG* g, int lane
   if (lane == 0) {
     q.tau = g->tau;
     q.phase = g->phase;
-    q.count = g->count;
     q.overflow = g->overflow;
     q.lo = g->lo;
     q.inv_w = g->inv_w;
     q.w = g->w;
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j) q.seg[j] = g->seg[j];
   }
   for (int b = lane; b < kBins; b += 32) q.hist[b] = g->hist[b];
 }
@@ -198,37 +222,46 @@ __device__ __forceinline__ void state_fresh(QState& q, bool valid, int lane) {
   if (lane == 0) {
     q.tau = -INFINITY;
     q.phase = valid ? 1 : 0;
-    q.count = 0;
     q.overflow = 0;
     q.lo = 0.f;
     q.inv_w = 0.f;
     q.w = 0.f;
+#pragma unroll
+    for (int j = 0; j < kSegs; ++j) q.seg[j] = 0;
   }
   for (int b = lane; b < kBins; b += 32) q.hist[b] = 0;
 }
 
 // Where a finished query's result goes.
 struct PublishOut {
-  int* cand_count;     // [rows]: candidates, or -1 when the list overflowed
+  int* cand_count;     // [rows][kSegs]: per-segment counts; all -1 on overflow
   float* tau;          // [rows]: final threshold
   int* repair_list;    // rows whose list overflowed (rescored densely)
   int* repair_count;
   int repair_cap;
-  int cap;
   int* err;
 };
 
-// Owner lane 0: publish a finished query.
+// Owner lane 0: publish a finished query (segment counts as of the last
+// checkpoint, which every range ends with).
 __device__ __forceinline__ void publish_query(const QState& q, const PublishOut& o) {
-  const int cnt = *reinterpret_cast<const volatile int*>(&q.count);
-  const bool over = q.overflow || cnt > o.cap;
-  o.cand_count[q.row] = over ? -1 : cnt;
+  const bool over = *reinterpret_cast<const volatile int*>(&q.overflow) != 0;
+  int* cc = o.cand_count + q.row * kSegs;
+#pragma unroll
+  for (int j = 0; j < kSegs; ++j) cc[j] = over ? -1 : q.seg[j];
   o.tau[q.row] = q.tau;
   if (over) {
     const int r = atomicAdd(o.repair_count, 1);
     if (r < o.repair_cap) o.repair_list[r] = (int)q.row;
     else record_error(o.err, kDevBounds);
   }
+}
+
+// Integers in [a, b] that also lie in [c, d].
+__device__ __forceinline__ long long overlap_count(long long a, long long b, long long c,
+                                                  long long d) {
+  const long long lo = a > c ? a : c, hi = b < d ? b : d;
+  return hi >= lo ? hi - lo + 1 : 0;
 }
 
 }  // namespace dosa

@@ -26,7 +26,6 @@
 //   2^-18 of that scale).  The candidate margin is
 //   c = 2^margin_log2 * sum_h |w_h| ||q_h||, rounded up.
 #include <cuda_bf16.h>
-#include <utility>
 #include <cuda_fp8.h>
 
 #include "cert_layout.h"
@@ -81,87 +80,69 @@ __global__ void __launch_bounds__(256) key_prep_kernel(const void* k, const floa
 }
 
 // ---- certificate setup ------------------------------------------------------------
+// One CTA of 256 threads per query.  Every phase spreads its work over all
+// warps: dot products are split 8 ways (fp64 partial sums for the NNLS
+// inputs), the NNLS tries its supports on 16 lanes per omitted head at once,
+// and the power iteration runs in warp 0 while warps 4-7 aggregate the
+// negative heads.
 constexpr int kSetupThreads = 256;
-constexpr int kSetupSmem = (64 * (kHeadDim + 1) + 64 * 65) * 4;
+constexpr int kQPad = kHeadDim + 1;
+constexpr int kSetupSmem = (64 * kQPad + 64 * 65) * 4;
 constexpr int kPowerIters = 12;
 
-__host__ __device__ constexpr int popc4(int m) { return (m & 1) + ((m >> 1) & 1) + ((m >> 2) & 1) + ((m >> 3) & 1); }
-__host__ __device__ constexpr int nth_bit(int m, int k) {
-  for (int j = 0; j < 4; ++j)
-    if ((m >> j) & 1) {
-      if (k == 0) return j;
-      --k;
-    }
-  return 0;
-}
-
-// Least squares restricted to the retained heads in MASK (Cholesky in fp64,
-// every index a compile-time constant so the arrays stay in registers).  If
-// the solution is strictly positive and its residual is the smallest so far,
-// it becomes the NNLS candidate.  NNLS optimum = the unconstrained LS solution
-// on its own support, so the best feasible support over all supports is it.
-template <int MASK>
-__device__ __forceinline__ void try_support(const double (&G)[4][4], const double (&b)[4],
-                                            double qq, int r, double& best, double (&alpha)[4]) {
-  constexpr int n = popc4(MASK);
-  constexpr int i0 = nth_bit(MASK, 0), i1 = nth_bit(MASK, 1), i2 = nth_bit(MASK, 2),
-                i3 = nth_bit(MASK, 3);
-  constexpr int idx[4] = {i0, i1, i2, i3};
-  if ((MASK >> r) != 0) return;       // uses a head beyond the retained count
-  double L[4][4];
+// Least squares on the support `mask` (bits over the 4 retained slots) of
+// G a = b, in fp64: inactive slots get an identity row and column and a zero
+// right-hand side, so their coefficient is exactly 0 and the active block is
+// solved as if alone (Cholesky, one reciprocal per pivot).  False when a pivot
+// shows the support (numerically) rank deficient.
+__device__ __forceinline__ bool ls_support(const double (&G)[4][4], const double (&b)[4],
+                                           int mask, double (&a)[4]) {
+  double M[4][4], rhs[4];
 #pragma unroll
-  for (int i = 0; i < n; ++i) {
+  for (int i = 0; i < 4; ++i) {
+    const bool ai = (mask >> i) & 1;
+    rhs[i] = ai ? b[i] : 0.0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool aj = (mask >> j) & 1;
+      M[i][j] = (ai && aj) ? G[i][j] : (i == j ? 1.0 : 0.0);
+    }
+  }
+  double L[4][4], inv[4];
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
 #pragma unroll
     for (int j = 0; j <= i; ++j) {
-      double v = G[idx[i]][idx[j]];
+      double v = M[i][j];
 #pragma unroll
       for (int k = 0; k < j; ++k) v -= L[i][k] * L[j][k];
       if (i == j) {
-        if (!(v > 1e-12 * (G[idx[i]][idx[i]] + 1e-300))) return;
-        L[i][i] = sqrt(v);
+        ok = ok && (v > 1e-12 * (M[i][i] + 1e-300));
+        const double d = sqrt(v > 0.0 ? v : 1.0);
+        L[i][i] = d;
+        inv[i] = 1.0 / d;
       } else {
-        L[i][j] = v / L[j][j];
+        L[i][j] = v * inv[j];
       }
     }
   }
-  double y[4], a[4];
+  double y[4];
 #pragma unroll
-  for (int i = 0; i < n; ++i) {
-    double v = b[idx[i]];
+  for (int i = 0; i < 4; ++i) {
+    double v = rhs[i];
 #pragma unroll
     for (int k = 0; k < i; ++k) v -= L[i][k] * y[k];
-    y[i] = v / L[i][i];
+    y[i] = v * inv[i];
   }
 #pragma unroll
-  for (int i = n - 1; i >= 0; --i) {
+  for (int i = 3; i >= 0; --i) {
     double v = y[i];
 #pragma unroll
-    for (int k = i + 1; k < n; ++k) v -= L[k][i] * a[k];
-    a[i] = v / L[i][i];
+    for (int k = i + 1; k < 4; ++k) v -= L[k][i] * a[k];
+    a[i] = v * inv[i];
   }
-  double ab = 0.0;
-#pragma unroll
-  for (int i = 0; i < n; ++i) {
-    if (!(a[i] > 0.0)) return;
-    ab += a[i] * b[idx[i]];
-  }
-  // residual^2 = qq - a.b at the least-squares point
-  const double res = qq - ab;
-  if (res < best) {
-    best = res;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) alpha[j] = 0.0;
-#pragma unroll
-    for (int i = 0; i < n; ++i) alpha[idx[i]] = a[i];
-  }
-}
-
-template <int... Ms>
-__device__ __forceinline__ void try_supports(std::integer_sequence<int, Ms...>,
-                                             const double (&G)[4][4], const double (&b)[4],
-                                             double qq, int r, double& best,
-                                             double (&alpha)[4]) {
-  (try_support<Ms + 1>(G, b, qq, r, best, alpha), ...);
+  return ok;
 }
 
 template <bool kFp8>
@@ -196,6 +177,30 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Decode 16 consecutive input codes starting at element e into dst[0..15].
+template <bool kFp8>
+__device__ __forceinline__ void decode16(const void* q, int64_t e, float* dst) {
+  if constexpr (kFp8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(q) + e);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      __nv_fp8_e4m3 c;
+      c.__x = (uint8_t)(w[i >> 2] >> (8 * (i & 3)));
+      dst[i] = float(c);
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(q) + e);
+    const uint4 v0 = p[0], v1 = p[1];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t bits = (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
+      dst[i] = __uint_as_float(bits);
+    }
+  }
+}
+
 struct SetupParams {
   const void* q;          // [rows, 64, d] codes (absolute rows)
   const float* w;         // [rows, 64]
@@ -209,17 +214,22 @@ struct SetupParams {
   int32_t* retained;      // [rows, 4]
 };
 
+// upper-triangle pairs of the 4 retained slots
+__constant__ int8_t kPairA[10] = {0, 0, 0, 0, 1, 1, 1, 2, 2, 3};
+__constant__ int8_t kPairB[10] = {0, 1, 2, 3, 1, 2, 3, 2, 3, 3};
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupParams p) {
   constexpr int H = 64, D = kHeadDim;
   extern __shared__ float setup_dyn[];
   // code-domain heads, then residuals in place (padded rows); weighted residual Gram
-  float(*qs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(setup_dyn);
-  float(*gt)[65] = reinterpret_cast<float(*)[65]>(setup_dyn + H * (D + 1));
+  float(*qs)[kQPad] = reinterpret_cast<float(*)[kQPad]>(setup_dyn);
+  float(*gt)[65] = reinterpret_cast<float(*)[65]>(setup_dyn + H * kQPad);
   __shared__ float wv[H], qn[H], act[H], rn[H];
   __shared__ float kbar[D];
   __shared__ float vec[64];
-  __shared__ double gram_r[16];
+  __shared__ double Gr[4][4];
+  __shared__ double Bm[H][4], QQ[H];
   __shared__ double alpha_s[H][4];
   __shared__ int R[4], O[64], A1[64], A2[64];
   __shared__ int nR, nO, nA1, nA2;
@@ -229,30 +239,43 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   const int64_t i = blockIdx.x;
   const int64_t t = p.row0 + i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NW = kSetupThreads / 32;
 
-  for (int e = threadIdx.x; e < H * D; e += blockDim.x)
-    qs[e / D][e % D] = decode_code<kFp8>(p.q, t * H * D + e);
+  // ---- A: decode q (16 codes per load), weights, mean key ----
+  for (int e = threadIdx.x * 16; e < H * D; e += blockDim.x * 16) {
+    float v[16];
+    decode16<kFp8>(p.q, t * H * D + e, v);
+    const int h = e / D, c = e % D;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) qs[h][c + k] = v[k];
+  }
   if (threadIdx.x < H) wv[threadIdx.x] = p.w[t * H + threadIdx.x];
   if (threadIdx.x < D) kbar[threadIdx.x] = p.key_sum[threadIdx.x] * p.inv_nkeys;
   __syncthreads();
-  for (int h = warp; h < H; h += NW) {
+  // ---- B: ||q_h|| and q_h . k_mean, 4 threads per head ----
+  {
+    const int h = threadIdx.x >> 2, part = threadIdx.x & 3;
     float ss = 0.f, ka = 0.f;
-    for (int e = lane; e < D; e += 32) {
-      ss = fmaf(qs[h][e], qs[h][e], ss);
-      ka = fmaf(qs[h][e], kbar[e], ka);
+#pragma unroll 8
+    for (int k = 0; k < D / 4; ++k) {
+      const int c = part + 4 * k;
+      const float x = qs[h][c];
+      ss = fmaf(x, x, ss);
+      ka = fmaf(x, kbar[c], ka);
     }
-    ss = warp_sum(ss);
-    ka = warp_sum(ka);
-    if (lane == 0) {
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
+    ka += __shfl_xor_sync(0xFFFFFFFFu, ka, 1);
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 2);
+    ka += __shfl_xor_sync(0xFFFFFFFFu, ka, 2);
+    if (part == 0) {
       qn[h] = sqrtf(ss);
       act[h] = ka;
     }
   }
   __syncthreads();
+  // ---- C: retained heads and head lists (warp 0) ----
   if (warp == 0) {
-    // retained heads: the r positive heads with the largest w_h ||q_h||, ties
-    // to the smaller head; lane l holds heads l and l + 32
+    // the r positive heads with the largest w_h ||q_h||, ties to the smaller
+    // head; lane l holds heads l and l + 32
     const int ha = lane, hb = lane + 32;
     bool ta = false, tb = false;
     for (int k = 0; k < p.r; ++k) {
@@ -289,39 +312,104 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   }
   __syncthreads();
   const int r = nR, no = nO;
-  // Gram of the retained heads (fp64 sums of fp32 products)
-  if (threadIdx.x < 16) {
-    const int a = threadIdx.x >> 2, b = threadIdx.x & 3;
-    double v = 0.0;
-    if (a < r && b < r)
-      for (int e = 0; e < D; ++e) v += (double)qs[R[a]][e] * (double)qs[R[b]][e];
-    gram_r[threadIdx.x] = v;
+  // ---- D: NNLS inputs in fp64 (exact products of fp32 values): q_h . q_Rj
+  // and ||q_h||^2 for every omitted head, and the retained heads' Gram.
+  // Eight threads per dot product. ----
+  {
+    const int nd = no * 5 + 10;
+    const int part = threadIdx.x & 7;
+    for (int base = 0; base < nd; base += kSetupThreads / 8) {
+      const int task = base + (threadIdx.x >> 3);
+      int ha = -1, hb = -1;
+      if (task < no * 5) {
+        const int k = task / 5, j = task % 5;
+        ha = O[k];
+        hb = j == 4 ? ha : (j < r ? R[j] : -1);
+      } else if (task < nd) {
+        const int a = kPairA[task - no * 5], b = kPairB[task - no * 5];
+        if (a < r && b < r) {
+          ha = R[a];
+          hb = R[b];
+        }
+      }
+      double v = 0.0;
+      if (ha >= 0 && hb >= 0) {
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) {
+          const int c = part + 8 * k;
+          v = fma((double)qs[ha][c], (double)qs[hb][c], v);
+        }
+      }
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+      if (part == 0 && task < nd) {
+        if (task < no * 5) {
+          const int k = task / 5, j = task % 5;
+          if (j == 4) QQ[k] = v;
+          else Bm[k][j] = v;
+        } else {
+          const int a = kPairA[task - no * 5], b = kPairB[task - no * 5];
+          Gr[a][b] = v;
+          Gr[b][a] = v;
+        }
+      }
+    }
   }
   __syncthreads();
-  // NNLS for every omitted positive head: one thread per head
-  if (threadIdx.x < no) {
-    const int h = O[threadIdx.x];
-    double G[4][4], bh[4] = {0, 0, 0, 0}, qq = 0.0;
+  // ---- E: NNLS for every omitted head, one support per lane (16 lanes per
+  // head: support masks 0..15 over the retained slots), best feasible
+  // support by a half-warp reduction.  The empty support (alpha = 0) is
+  // always feasible with residual ||q_h||^2. ----
+  {
+    const int m = lane & 15;
+    double G[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) G[a][b] = gram_r[a * 4 + b];
-    const int R0 = R[0], R1 = r > 1 ? R[1] : R[0], R2 = r > 2 ? R[2] : R[0], R3 = r > 3 ? R[3] : R[0];
-    for (int e = 0; e < D; ++e) {
-      const double x = qs[h][e];
-      qq += x * x;
-      bh[0] += (double)qs[R0][e] * x;
-      bh[1] += (double)qs[R1][e] * x;
-      bh[2] += (double)qs[R2][e] * x;
-      bh[3] += (double)qs[R3][e] * x;
-    }
-    double best = qq, alpha[4] = {0.0, 0.0, 0.0, 0.0};
-    if (r > 0) try_supports(std::make_integer_sequence<int, 15>{}, G, bh, qq, r, best, alpha);
+      for (int b = 0; b < 4; ++b) G[a][b] = Gr[a][b];
+    for (int base = 0; base < no; base += kSetupThreads / 16) {
+      const int k = base + (threadIdx.x >> 4);
+      double res = INFINITY, a[4] = {0.0, 0.0, 0.0, 0.0};
+      if (k < no && (m >> r) == 0) {
+        const double qq = QQ[k];
+        if (m == 0) {
+          res = qq;
+        } else {
+          double b[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) alpha_s[h][j] = alpha[j];
+          for (int j = 0; j < 4; ++j) b[j] = Bm[k][j];
+          bool ok = ls_support(G, b, m, a);
+          double ab = 0.0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if ((m >> j) & 1) ok = ok && a[j] > 0.0;
+            ab += a[j] * b[j];
+          }
+          if (ok) res = qq - ab;   // residual^2 at the least-squares point
+        }
+      }
+      // min residual over the 16 lanes, ties to the smaller mask
+      double best = res;
+      int who = m;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int ow = __shfl_xor_sync(0xFFFFFFFFu, who, o);
+        if (ob < best || (ob == best && ow < who)) {
+          best = ob;
+          who = ow;
+        }
+      }
+      if (k < no && who == m) {
+        const int h = O[k];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) alpha_s[h][j] = m == 0 ? 0.0 : a[j];
+      }
+    }
   }
   __syncthreads();
-  // residuals in place of the omitted heads (retained rows are not modified)
+  // ---- F: residuals in place of the omitted heads ----
   for (int e = threadIdx.x; e < no * D; e += blockDim.x) {
     const int h = O[e / D], c = e % D;
     float x = qs[h][c];
@@ -329,44 +417,64 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     qs[h][c] = x;
   }
   __syncthreads();
-  for (int k = warp; k < no; k += NW) {
-    const int h = O[k];
-    float ss = 0.f;
-    for (int e = lane; e < D; e += 32) ss = fmaf(qs[h][e], qs[h][e], ss);
-    ss = warp_sum(ss);
-    if (lane == 0) rn[h] = sqrtf(ss);
-  }
-  // weighted residual Gram |[sqrt(w w') rho . rho']| (upper triangle by warps)
-  for (int e = warp; e < no * no; e += NW) {
-    const int a = e / no, b = e % no;
-    if (b < a) continue;
-    const int ha = O[a], hb = O[b];
-    float v = 0.f;
-    for (int c = lane; c < D; c += 32) v = fmaf(qs[ha][c], qs[hb][c], v);
-    v = warp_sum(v);
-    if (lane == 0) {
-      const float g = fabsf(sqrtf(wv[ha] * wv[hb]) * v);
-      gt[a][b] = g;
-      gt[b][a] = g;
+  // ---- G: weighted residual Gram |[sqrt(w w') rho . rho']| and ||rho_h||,
+  // one pair (a >= b) per 8 threads ----
+  {
+    const int np = no * (no + 1) / 2;
+    const int part = threadIdx.x & 7;
+    for (int base = 0; base < np; base += kSetupThreads / 8) {
+      const int task = base + (threadIdx.x >> 3);
+      int a = 0, b = 0;
+      if (task < np) {
+        a = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
+        while (a * (a + 1) / 2 > task) --a;
+        while ((a + 1) * (a + 2) / 2 <= task) ++a;
+        b = task - a * (a + 1) / 2;
+      }
+      const int ha = O[a], hb = O[b];
+      float v = 0.f;
+      if (task < np) {
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) {
+          const int c = part + 8 * k;
+          v = fmaf(qs[ha][c], qs[hb][c], v);
+        }
+      }
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+      v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+      if (part == 0 && task < np) {
+        const float g = fabsf(sqrtf(wv[ha] * wv[hb]) * v);
+        gt[a][b] = g;
+        gt[b][a] = g;
+        if (a == b) rn[ha] = sqrtf(v);
+      }
     }
   }
   __syncthreads();
-  // power iterations on |Gram| from the all-ones vector (warp 0; lane l owns
-  // rows l and l + 32), then the Collatz-Wielandt bound max_a (|Gram| v)_a / v_a
   if (warp == 0) {
+    // ---- H: power iterations on |Gram| from the all-ones vector (lane l
+    // owns rows l and l + 32), then the Collatz-Wielandt bound
+    // max_a (|Gram| v)_a / v_a ----
     const int a0 = lane, a1 = lane + 32;
     if (a0 < no) vec[a0] = 1.f;
     if (a1 < no) vec[a1] = 1.f;
     __syncwarp();
     float s0 = 0.f, s1 = 0.f;
     for (int it = 0; it <= kPowerIters; ++it) {
-      s0 = 0.f;
-      s1 = 0.f;
-      for (int b = 0; b < no; ++b) {
-        const float vb = vec[b];
-        if (a0 < no) s0 = fmaf(gt[a0][b], vb, s0);
-        if (a1 < no) s1 = fmaf(gt[a1][b], vb, s1);
+      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int b = 0; b < no; b += 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (b + j < no) {
+            const float vb = vec[b + j];
+            if (a0 < no) p0[j] = fmaf(gt[a0][b + j], vb, p0[j]);
+            if (a1 < no) p1[j] = fmaf(gt[a1][b + j], vb, p1[j]);
+          }
+        }
       }
+      s0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
+      s1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
       if (it == kPowerIters) break;
       const float m = warp_max(fmaxf(s0, s1));
       __syncwarp();
@@ -379,10 +487,9 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     if (a1 < no) lam = fmaxf(lam, s1 / fmaxf(vec[a1], 1e-30f));
     lam = warp_max(lam);
     if (lane == 0) s_lam = lam;
-  }
-  // negative aggregates: thread c < D owns element c of u_1 and u_2
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
+  } else if (warp >= 4) {
+    // ---- I: negative aggregates, thread c owns element c of u_1 and u_2 ----
+    const int c = threadIdx.x - 128;
     float u1 = 0.f, u2 = 0.f;
     for (int k = 0; k < nA1; ++k) u1 = fmaf(fabsf(wv[A1[k]]), qs[A1[k]][c], u1);
     for (int k = 0; k < nA2; ++k) u2 = fmaf(fabsf(wv[A2[k]]), qs[A2[k]][c], u2);
@@ -390,7 +497,9 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     uv[1][c] = u2;
   }
   __syncthreads();
-  float beta_add = 0.f;   // split errors of the aggregates (thread 0)
+  // ---- J: each aggregate as a hi row and a lo row in the input type, with
+  // fp32 scales; the split error is added to beta ----
+  float beta_add = 0.f;   // (thread 0)
   const size_t esz = kFp8 ? 1 : 2;
   uint8_t* rows_out = static_cast<uint8_t*>(p.bdir) + (size_t)i * 8 * D * esz;
   float s_hi[2], s_lo[2];
@@ -436,43 +545,51 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     const int j = e / (D * esz), b = e % (D * esz);
     rows_out[e] = j < r ? qrow[(size_t)R[j] * D * esz + b] : 0;
   }
-  if (threadIdx.x == 0) {
+  float* cf = p.cert + i * kCertFloats;
+  if (warp == 1 && lane < 4) {
+    // omega_j = w_j + sum_h w_h alpha_hj (fp64)
+    const int j = lane;
+    float om = 0.f;
+    if (j < r) {
+      double o = wv[R[j]];
+      for (int k = 0; k < no; ++k) o += (double)wv[O[k]] * alpha_s[O[k]][j];
+      om = (float)o;
+    }
+    cf[kCertOmega + j] = om;
+    p.retained[i * 4 + j] = j < r ? R[j] : -1;
+  }
+  if (warp == 0) {
     float wO = 0.f, bsum = 0.f, z2 = 0.f, scale = 0.f;
-    for (int k = 0; k < no; ++k) {
+    for (int k = lane; k < no; k += 32) {
       const int h = O[k];
       wO += wv[h];
       bsum = fmaf(wv[h], rn[h], bsum);
       z2 = fmaf(wv[h], rn[h] * rn[h], z2);
     }
-    for (int h = 0; h < H; ++h) scale = fmaf(fabsf(wv[h]), qn[h], scale);
-    // lambda bound: CW value with rounding headroom plus the Gram entry errors
-    const float lam_b = s_lam * (1.f + 0x1p-16f) + 0x1p-16f * z2;
-    const float bjoint = sqrtf(wO * lam_b) * (1.f + 0x1p-20f);
-    const float bs = bsum * (1.f + 0x1p-20f);
-    float beta = no > 0 ? fminf(bs, bjoint) : 0.f;
-    beta += 0x1p-16f * scale + beta_add;
-    float* cf = p.cert + i * kCertFloats;
-    for (int j = 0; j < 4; ++j) {
-      float om = 0.f;
-      if (j < r) {
-        double o = wv[R[j]];
-        for (int k = 0; k < no; ++k) o += (double)wv[O[k]] * alpha_s[O[k]][j];
-        om = (float)o;
-      }
-      cf[kCertOmega + j] = om;
-      p.retained[i * 4 + j] = j < r ? R[j] : -1;
+    for (int h = lane; h < H; h += 32) scale = fmaf(fabsf(wv[h]), qn[h], scale);
+    wO = warp_sum(wO);
+    bsum = warp_sum(bsum);
+    z2 = warp_sum(z2);
+    scale = warp_sum(scale);
+    if (lane == 0) {
+      // lambda bound: CW value with rounding headroom plus the Gram entry errors
+      const float lam_b = s_lam * (1.f + 0x1p-16f) + 0x1p-16f * z2;
+      const float bjoint = sqrtf(wO * lam_b) * (1.f + 0x1p-20f);
+      const float bs = bsum * (1.f + 0x1p-20f);
+      float beta = no > 0 ? fminf(bs, bjoint) : 0.f;
+      beta += 0x1p-16f * scale + beta_add;
+      cf[kCertBeta] = beta;
+      cf[kCertMargin] = ldexpf(scale, p.margin_log2) * (1.f + 0x1p-20f);
+      cf[kCertScale + 0] = s_hi[0];
+      cf[kCertScale + 1] = s_lo[0];
+      cf[kCertScale + 2] = s_hi[1];
+      cf[kCertScale + 3] = s_lo[1];
+      cf[kCertBetaSum] = bs;
+      cf[kCertBetaJoint] = bjoint;
+      cf[kCertNA1] = (float)nA1;
+      cf[kCertNA2] = (float)nA2;
+      cf[kCertNO] = (float)no;
     }
-    cf[kCertBeta] = beta;
-    cf[kCertMargin] = ldexpf(scale, p.margin_log2) * (1.f + 0x1p-20f);
-    cf[kCertScale + 0] = s_hi[0];
-    cf[kCertScale + 1] = s_lo[0];
-    cf[kCertScale + 2] = s_hi[1];
-    cf[kCertScale + 3] = s_lo[1];
-    cf[kCertBetaSum] = bs;
-    cf[kCertBetaJoint] = bjoint;
-    cf[kCertNA1] = (float)nA1;
-    cf[kCertNA2] = (float)nA2;
-    cf[kCertNO] = (float)no;
   }
 }
 

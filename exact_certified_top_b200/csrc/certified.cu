@@ -80,14 +80,14 @@ struct CertParams {
   const float* k_scale;    // sequence base (fp8)
   const float* key_norm;   // [S] code-domain ||k||, rounded up
   const float* cert;       // [chunk rows, kCertFloats]
-  Cand* cand;              // [chunk rows, cap]
+  Cand* cand;              // [chunk rows][kSegs][seg_cap]
   QStateG* qstate;         // [chunk rows] state carried between passes
   int* item_flag;          // [n_items] decision of the probe pass
   PublishOut out;
   unsigned long long* counters;
   int* err;
   int64_t row0, rows, pos0, S;   // chunk: absolute first row, rows, first position
-  int n_items, K, cap, seed_first, seed_last;
+  int n_items, K, seg_cap, seed_first, seed_last;
   int probe_tiles;         // tiles screened by the probe pass
   int continue_pass;       // 0: probe pass, 1: continue pass
 };
@@ -367,6 +367,11 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
         ++it;
       }
+      // this warp's segment counts of its queries grp * 2 + half (grp = 0..3)
+      int cnt[C::kGroups];
+#pragma unroll
+      for (int grp = 0; grp < C::kGroups; ++grp)
+        cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * 2 + half].seg[quad]);
       unsigned long long it_scr = 0, it_rej = 0;   // this warp's counts, this item
       auto key_of = [&](int i) -> int64_t {
         return (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
@@ -443,12 +448,13 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         uint32_t groups = 0;
         for (int w = 0; w < C::kEpiWarps; ++w)
           groups |= reinterpret_cast<volatile uint32_t*>(gflag)[(c % 3) * 8 + w];
+#pragma unroll
         for (int grp = 0; grp < C::kGroups; ++grp) {
-          if (!(groups >> grp & 1)) continue;
+          if (!(groups >> grp & 1) || !ok) continue;
           const uint32_t ab = u % C::kAccBufs;
           if (!mbar_wait(&acc_full[ab], (u / C::kAccBufs) & 1, s_abort, p.err)) {
             ok = false;
-            break;
+            continue;
           }
           tc_fence_after();
           const int ql = grp * 2 + half;
@@ -467,8 +473,9 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             }
             n_exact += __popc(mk);
             const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-            n_cand += append_candidates(q, p.cand + q.row * (int64_t)p.cap, p.cap,
-                                        mine && sc >= tau, sc, (int)s, lane);
+            n_cand += append_candidates(
+                q, p.cand + (q.row * kSegs + quad) * (int64_t)p.seg_cap, p.seg_cap, cnt[grp],
+                mine && sc >= tau, sc, (int)s, lane);
           }
           tc_fence_before();
           __syncwarp();
@@ -479,14 +486,12 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         // ---- checkpoint: every kCkptTiles steps and at the range's last ----
         const bool last = i + 1 == n;
         if (((i + 1) % kCkptTiles) == 0 || last) {
-          // The owner's own count, read before it arrives: every slot below it
-          // was reserved in a step <= i and written before its writer arrived,
-          // and none of those writers saw the screening phase, so the warm-up
-          // scan neither misses a written entry nor counts one twice.
-          int snap_cnt = 0;
-          if (lane == 0 && ew < g.nq) snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
-          snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
+          // Publish this warp's segment counts: every entry below them is
+          // written, so the owner's warm-up scan after the barrier neither
+          // misses a written entry nor counts one twice.
           if (lane == 0) {
+#pragma unroll
+            for (int grp = 0; grp < C::kGroups; ++grp) st[grp * 2 + half].seg[quad] = cnt[grp];
             snap[(nbar & 1) * 16 + ew * 2 + 0] = it_scr;
             snap[(nbar & 1) * 16 + ew * 2 + 1] = it_rej;
           }
@@ -499,8 +504,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           const uint32_t slot = nbar & 1;
           ++nbar;
           if (ew < g.nq)
-            refresh_threshold(st[ew], p.cand + st[ew].row * (int64_t)p.cap, snap_cnt, p.K, p.cap,
-                              lane);
+            refresh_threshold(st[ew], p.cand + st[ew].row * kSegs * (int64_t)p.seg_cap, p.seg_cap,
+                              p.K, lane);
           if (last && !p.continue_pass && rg.end < g.n_tiles && ew == 0 && lane == 0) {
             // the probe's decision, from the counts every warp left at this barrier
             unsigned long long tot_s = 0, tot_r = 0;
@@ -576,7 +581,6 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
-  p.out.cap = b.cap;
   p.out.err = b.err;
   p.counters = b.counters;
   p.err = b.err;
@@ -586,7 +590,7 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.S = v.S;
   p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
   p.K = K;
-  p.cap = b.cap;
+  p.seg_cap = b.seg_cap;
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
   p.probe_tiles = probe_tiles;

@@ -1,6 +1,7 @@
 // C-ABI layer of libdosa: argument validation, workspace layout, launch
 // orchestration.  No device memory is allocated here; every kernel runs on the
 // caller's stream.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -101,12 +102,22 @@ constexpr int kRepairRows = 64;                             // overflowed rows p
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
-// Candidate capacity per query row: 16 K (at least 4096), never more than
-// the keys of the longest sequence (a row cannot have more candidates).
-int cand_capacity(int K, int64_t S_max) {
-  int64_t cap = 16 * (int64_t)K;
-  if (cap < 4096) cap = 4096;
-  if (cap > S_max) cap = S_max;
+// Candidate capacity per query row and segment.  A row's list has 4
+// segments, one per 32-key quarter of every key tile.  A row with n keys
+// appends about K (1 + ln(n / K)) candidates (a key is appended when it
+// enters the running Top-K, with probability about K / its rank in the
+// processing order), and the histogram threshold's coarseness adds up to
+// about as much again on inputs with a few very large scores.  A segment
+// holds 0.65 K (1 + ln(S_max / K)) entries (at least 1024, rounded up to 64),
+// and never more than the keys it can see: 32 per key tile.  A row that
+// overflows is rescored densely.
+int seg_capacity(int K, int64_t S_max) {
+  const double ratio = S_max > K ? (double)S_max / K : 1.0;
+  int64_t cap = (int64_t)ceil(0.65 * K * (1.0 + log(ratio)));
+  cap = (cap + 63) / 64 * 64;
+  if (cap < 1024) cap = 1024;
+  const int64_t most = (S_max + kKeyTile - 1) / kKeyTile * 32;
+  if (cap > most) cap = most;
   if (cap < 1) cap = 1;
   return (int)cap;
 }
@@ -116,7 +127,7 @@ int cand_capacity(int K, int64_t S_max) {
 struct CertLayout {
   size_t key_norm, key_sum, repair_list, repair_count, repair_scores, fixed;
   size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
-  int cap;
+  int seg_cap;
 };
 
 CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
@@ -127,7 +138,7 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
     off += (size_t)round_up((int64_t)bytes, 256);
     return at;
   };
-  L.cap = cand_capacity(K, S_max);
+  L.seg_cap = seg_capacity(K, S_max);
   L.key_norm = take((size_t)S_max * 4);
   L.key_sum = take(kHeadDim * 4);
   L.repair_list = take(kRepairRows * 4);
@@ -136,7 +147,7 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.fixed = off;
   // bound rows, record, retained, list, count, tau, carried state, item flag
   L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
-              (size_t)L.cap * 8 + 4 + 4 + qstate_bytes() + 1;
+              (size_t)L.seg_cap * 4 * 8 + 4 * 4 + 4 + qstate_bytes() + 1;
   return L;
 }
 
@@ -155,12 +166,12 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.repair_count = reinterpret_cast<int*>(ws + L.repair_count);
   b.repair_scores = reinterpret_cast<float*>(ws + L.repair_scores);
   b.repair_cap = kRepairRows;
-  b.cap = L.cap;
+  b.seg_cap = L.seg_cap;
   b.bdir = take((size_t)Tc * kBoundRows * kHeadDim * elem_bytes(h));
   b.cert = reinterpret_cast<float*>(take((size_t)Tc * kCertFloats * 4));
   b.retained = reinterpret_cast<int32_t*>(take((size_t)Tc * 16));
-  b.cand = take((size_t)Tc * L.cap * 8);
-  b.cand_count = reinterpret_cast<int*>(take((size_t)Tc * 4));
+  b.cand = take((size_t)Tc * 4 * L.seg_cap * 8);
+  b.cand_count = reinterpret_cast<int*>(take((size_t)Tc * 4 * 4));
   b.tau = reinterpret_cast<float*>(take((size_t)Tc * 4));
   b.qstate = take((size_t)Tc * qstate_bytes());
   b.item_flag = reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4));

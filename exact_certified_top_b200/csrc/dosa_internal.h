@@ -65,8 +65,8 @@ struct CertBuffers {
   void* bdir;            // [rows, 8, d] bound rows in the input type
   float* cert;           // [rows, kCertFloats]
   int32_t* retained;     // [rows, 4]
-  void* cand;            // [rows, cap] packed (score, key)
-  int* cand_count;       // [rows]; -1 marks a row repaired by the dense pass
+  void* cand;            // [rows][4][seg_cap] packed (score, key), 4 segments per row
+  int* cand_count;       // [rows][4] per-segment counts; -1 marks a row repaired densely
   float* tau;            // [rows] final threshold
   void* qstate;          // [rows] candidate state carried from the probe pass
   int* item_flag;        // [rows / 8] what the probe pass decided per work item
@@ -74,7 +74,7 @@ struct CertBuffers {
   int* repair_count;
   int repair_cap;
   float* repair_scores;  // [repair_cap, S]
-  int cap;
+  int seg_cap;           // entries per candidate segment
   unsigned long long* counters;
   int* err;
 };

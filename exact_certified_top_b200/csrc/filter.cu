@@ -51,14 +51,14 @@ struct FilterParams {
   const float* w;          // [rows_total, 64] absolute rows
   const float* q_scale;    // absolute rows (fp8)
   const float* k_scale;    // sequence base (fp8)
-  Cand* cand;              // [chunk rows, cap]
+  Cand* cand;              // [chunk rows][kSegs][seg_cap]
   QStateG* qstate;         // [chunk rows] state handed over by the probe pass
   const int* item_flag;    // [n_items]
   PublishOut out;
   unsigned long long* counters;
   int* err;
   int64_t row0, rows, pos0, S;
-  int n_items, K, cap, seed_first, seed_last;
+  int n_items, K, seg_cap, seed_first, seed_last;
   int begin_step;          // first step of a handed-over item
   int all_items;           // 1: every item from step 0 with a fresh state
 };
@@ -253,21 +253,49 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
         else state_fresh(s, valid, lane);
         __syncwarp();
         __threadfence_block();
+        if (valid && lane == 0) {
+          // Visible and seed pairs of this query in the item's range: step 0
+          // is key tile 0, steps ti >= 1 are key tiles n_tiles - ti.
+          const int64_t pos = g.pos_first + ew;
+          const int64_t nonseed_lo = p.seed_first, nonseed_hi = pos - p.seed_last;
+          long long vis = 0, nonseed = 0;
+          if (rg.begin == 0) {
+            vis += overlap_count(0, kKeyTile - 1, 0, pos);
+            nonseed += overlap_count(0, (kKeyTile - 1 < pos ? kKeyTile - 1 : pos), nonseed_lo,
+                                     nonseed_hi);
+          }
+          const int t_first = rg.begin > 1 ? rg.begin : 1;
+          if (t_first < rg.end) {
+            const int64_t k_lo = (int64_t)(g.n_tiles - (rg.end - 1)) * kKeyTile;
+            const int64_t k_hi = (int64_t)(g.n_tiles - t_first) * kKeyTile + kKeyTile - 1;
+            vis += overlap_count(k_lo, k_hi, 0, pos);
+            nonseed += overlap_count(k_lo, (k_hi < pos ? k_hi : pos), nonseed_lo, nonseed_hi);
+          }
+          n_exact += vis;
+          n_seed += vis - nonseed;
+        }
       }
       if (lane == 0) mbar_arrive(item_ready);
       if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
       ++it;
+      // this warp's segment counts of its queries grp * 4 + sub (grp = 0, 1)
+      int cnt[C::kGroups];
+#pragma unroll
+      for (int grp = 0; grp < C::kGroups; ++grp)
+        cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * C::kQPerGroup + sub].seg[quad]);
       for (int i = 0; i < n && ok; ++i) {
-        const int64_t base = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32;
-        const int64_t s = base + lane;
+        const int64_t s = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
         float sk = 1.f;
         if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
-        for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
+#pragma unroll
+        for (int grp = 0; grp < C::kGroups; ++grp) {
+          if (!ok) continue;
           const uint32_t buf = u & 1;
           if (!mbar_wait(&acc_full[buf], (u >> 1) & 1, s_abort, p.err)) {
             ok = false;
-            break;
+            continue;
           }
+          ++u;
           tc_fence_after();
           const int ql = grp * C::kQPerGroup + sub;
           // 32 heads at a time (the register budget of 18 warps is 96 per thread)
@@ -287,30 +315,23 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           if (ql < g.nq) {
             QState& q = st[ql];
             const int64_t t = g.t0 + ql;
-            const int64_t pos = g.pos_first + ql;
             float sc = head_total(acc);
             if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
-            // visible and seed pairs of these 32 keys, from the intervals
-            const int64_t e = base + 31 < pos ? base + 31 : pos;
-            const int64_t nvis = e >= base ? e - base + 1 : 0;
-            const int64_t lo = base > p.seed_first ? base : (int64_t)p.seed_first;
-            const int64_t hi = e < pos - p.seed_last ? e : pos - p.seed_last;
-            n_exact += nvis;
-            n_seed += nvis - (hi >= lo ? hi - lo + 1 : 0);
             const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-            n_cand += append_candidates(q, p.cand + (g.local0 + ql) * (int64_t)p.cap, p.cap,
-                                        s <= pos && sc >= tau, sc, (int)s, lane);
+            n_cand += append_candidates(
+                q, p.cand + ((g.local0 + ql) * kSegs + quad) * (int64_t)p.seg_cap, p.seg_cap,
+                cnt[grp], s <= g.pos_first + ql && sc >= tau, sc, (int)s, lane);
           }
         }
         if (!ok) break;
         // ---- checkpoint: every kCkptTiles steps and at the item's last ----
         if (((i + 1) % kCkptTiles) == 0 || i + 1 == n) {
-          // The owner's count read before it arrives: every slot below it was
-          // written before its writer arrived (see certified.cu).
-          int snap_cnt = 0;
-          if (lane == 0 && owner && ew < g.nq)
-            snap_cnt = *reinterpret_cast<volatile int*>(&st[ew].count);
-          snap_cnt = __shfl_sync(0xFFFFFFFFu, snap_cnt, 0);
+          // publish this warp's segment counts (see certified.cu)
+          if (lane == 0) {
+#pragma unroll
+            for (int grp = 0; grp < C::kGroups; ++grp)
+              st[grp * C::kQPerGroup + sub].seg[quad] = cnt[grp];
+          }
           __threadfence_block();
           if (lane == 0) mbar_arrive(tile_done);
           if (!mbar_wait(tile_done, nbar & 1, s_abort, p.err)) {
@@ -319,8 +340,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           }
           ++nbar;
           if (owner && ew < g.nq)
-            refresh_threshold(st[ew], p.cand + st[ew].row * (int64_t)p.cap, snap_cnt, p.K, p.cap,
-                              lane);
+            refresh_threshold(st[ew], p.cand + st[ew].row * kSegs * (int64_t)p.seg_cap, p.seg_cap,
+                              p.K, lane);
         }
       }
       if (ok && owner && ew < g.nq && lane == 0) publish_query(st[ew], p.out);
@@ -373,7 +394,6 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
-  p.out.cap = b.cap;
   p.out.err = b.err;
   p.counters = b.counters;
   p.err = b.err;
@@ -383,7 +403,7 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.S = v.S;
   p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
   p.K = K;
-  p.cap = b.cap;
+  p.seg_cap = b.seg_cap;
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
   p.begin_step = begin_step;

@@ -10,17 +10,20 @@
 // from global memory), the K-th score is found by 4 radix passes over
 // order-preserving keys, and when more entries tie with it than are needed, a
 // second radix select over the complemented key indices of the tied entries
-// finds the smallest indices.  The K indices are sorted ascending in shared
-// memory and written.  Every step is a parallel pass; nothing is serial in the
-// number of ties.
+// finds the smallest indices (skipped when every tied entry is needed).  The
+// K indices are put in ascending order through a bitmap over the row's keys
+// (one bit per key, then a block-wide prefix count), or by a bitonic sort for
+// rows longer than the bitmap.  Every step is a parallel pass; nothing is
+// serial in the number of ties.
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
 
 namespace dosa {
 
 constexpr int kSelThreads = 512;
-constexpr int kSelList = 6144;        // candidates >= tau held in shared memory
+constexpr int kSelList = 4096;        // candidates >= tau held in shared memory
 constexpr int kSelOut = 4096;         // >= max K, power of two
+constexpr int kBitmapWords = 8192;    // rows of up to 262,144 keys use the bitmap
 
 struct CandView {
   float score;
@@ -64,7 +67,7 @@ __device__ __forceinline__ uint32_t agg_slot(uint32_t* counter, bool active) {
 // elements equal to it belong to the K largest.
 template <typename Get>
 __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32_t* s_digit,
-                              uint32_t* s_above, uint32_t* take) {
+                              uint32_t* s_above, uint32_t* s_eq, uint32_t* take, uint32_t* eq) {
   uint32_t prefix = 0, mask = 0, remaining = K;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
@@ -104,6 +107,7 @@ __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32
           if (acc < remaining && remaining <= acc + c[j]) {
             *s_digit = 255 - 8 * lane - j;
             *s_above = acc;
+            *s_eq = c[j];
           }
           acc += c[j];
         }
@@ -116,24 +120,60 @@ __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32
     __syncthreads();
   }
   *take = remaining;
+  *eq = *s_eq;          // elements whose key equals the result (last digit's bin)
   return prefix;
 }
 
+// Exclusive prefix sum of v over the CTA in thread order (scratch: 32 words).
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    const uint32_t t = lane < nw ? scratch[lane] : 0u;
+    uint32_t ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += n;
+    }
+    if (lane < nw) scratch[lane] = ti - t;
+  }
+  __syncthreads();
+  return scratch[warp] + incl - v;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
-    const CandView* __restrict__ cand, int cap, const int* __restrict__ cand_count,
+    const CandView* __restrict__ cand, int seg_cap, const int* __restrict__ cand_count,
     const float* __restrict__ tau, int64_t pos0, int K, int32_t* __restrict__ out) {
   extern __shared__ uint32_t sel_smem[];
   uint32_t* lkey = sel_smem;                                        // [kSelList]
   int32_t* lidx = reinterpret_cast<int32_t*>(lkey + kSelList);     // [kSelList]
-  uint32_t* outv = reinterpret_cast<uint32_t*>(lidx + kSelList);   // [kSelOut]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(lidx + kSelList);     // [kBitmapWords] or sort area
   __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_digit, s_above, s_take, s_n, s_nout;
+  __shared__ uint32_t scan[32];
+  __shared__ uint32_t s_digit, s_above, s_eq, s_n, s_nout;
   const int64_t row = blockIdx.x;
   const int64_t nvis = pos0 + row + 1;
   int32_t* o = out + row * K;
-  const int cnt = cand_count[row];
-  if (cnt < 0) return;                        // overflowed: written by the repair pass
-  const CandView* cl = cand + row * (int64_t)cap;
+  // the row's list: kSegs segments of seg_cap entries, counts c0..c3
+  const int4 cc = *reinterpret_cast<const int4*>(cand_count + row * 4);
+  if (cc.x < 0) return;                       // overflowed: written by the repair pass
+  const CandView* cl = cand + row * 4 * (int64_t)seg_cap;
+  const int e1 = cc.x, e2 = e1 + cc.y, e3 = e2 + cc.z, cnt = e3 + cc.w;
+  // i-th entry of the concatenated segments
+  auto entry = [&](int i) -> const CandView& {
+    const int j = (i >= e1) + (i >= e2) + (i >= e3);
+    const int off = i - (j == 0 ? 0 : j == 1 ? e1 : j == 2 ? e2 : e3);
+    return cl[j * (int64_t)seg_cap + off];
+  };
   if (nvis <= K) {
     // every visible key is a candidate; the answer is all of them
     for (int i = threadIdx.x; i < K; i += blockDim.x) o[i] = i < nvis ? i : -1;
@@ -150,7 +190,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     CandView c;
     c.score = -INFINITY;
     c.key = 0;
-    if (i < cnt) c = cl[i];
+    if (i < cnt) c = entry(i);
     const bool in = i < cnt && c.score >= th;
     const uint32_t slot = agg_slot(&s_n, in);
     if (in && slot < (uint32_t)kSelList) {
@@ -162,34 +202,66 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int n = (int)s_n;
   const bool in_smem = n <= kSelList;
   const int m = in_smem ? n : cnt;            // the global path scans every candidate
-  auto key_at = [&](int i) -> uint32_t { return in_smem ? lkey[i] : ordered_key(cl[i].score); };
-  auto idx_at = [&](int i) -> uint32_t { return (uint32_t)(in_smem ? lidx[i] : cl[i].key); };
+  auto key_at = [&](int i) -> uint32_t { return in_smem ? lkey[i] : ordered_key(entry(i).score); };
+  auto idx_at = [&](int i) -> uint32_t { return (uint32_t)(in_smem ? lidx[i] : entry(i).key); };
+  uint32_t take = 0, eq = 0;
   const uint32_t kth = radix_kth(
       [&](int i, uint32_t* u) {
         *u = key_at(i);
         return true;
       },
-      m, (uint32_t)K, hist, &s_digit, &s_above, &s_take);
-  const uint32_t take = s_take;
+      m, (uint32_t)K, hist, &s_digit, &s_above, &s_eq, &take, &eq);
   // Among entries equal to the K-th key, keep those with the `take` smallest
-  // indices: the take-th largest complemented index is the cut.
-  const uint32_t cut = ~radix_kth(
-      [&](int i, uint32_t* u) {
-        if (key_at(i) != kth) return false;
-        *u = ~idx_at(i);
-        return true;
-      },
-      m, take, hist, &s_digit, &s_above, &s_take);
-  // gather the K winners (distinct indices: exactly K of them), sort, write
+  // indices: the take-th largest complemented index is the cut.  When all of
+  // them are needed there is nothing to cut.
+  uint32_t cut = 0xFFFFFFFFu;
+  if (take < eq) {
+    uint32_t t2, e2;
+    cut = ~radix_kth(
+        [&](int i, uint32_t* u) {
+          if (key_at(i) != kth) return false;
+          *u = ~idx_at(i);
+          return true;
+        },
+        m, take, hist, &s_digit, &s_above, &s_eq, &t2, &e2);
+  }
+  auto winner = [&](int i, uint32_t* id) -> bool {
+    const uint32_t u = key_at(i);
+    *id = idx_at(i);
+    return u > kth || (u == kth && *id <= cut);
+  };
+  if (nvis <= (int64_t)kBitmapWords * 32) {
+    // ascending order through a bitmap over the row's keys
+    const int nwords = (int)((nvis + 31) >> 5);
+    for (int w = threadIdx.x; w < nwords; w += blockDim.x) bm[w] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+      uint32_t id;
+      if (winner(i, &id) && id < (uint32_t)nvis) atomicOr(&bm[id >> 5], 1u << (id & 31));
+    }
+    __syncthreads();
+    const int per = (nwords + blockDim.x - 1) / blockDim.x;
+    const int w0 = threadIdx.x * per, w1 = min(w0 + per, nwords);
+    uint32_t c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
+    uint32_t at = block_exclusive_sum(c, scan);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (at < (uint32_t)K) o[at] = (int32_t)(w * 32 + b);
+        ++at;
+      }
+    }
+    return;
+  }
+  // long rows: gather the K winners (distinct indices: exactly K), sort, write
+  uint32_t* outv = bm;
   const int mw = (m + 31) & ~31;
   for (int i = threadIdx.x; i < mw; i += blockDim.x) {
-    bool in = false;
     uint32_t id = 0;
-    if (i < m) {
-      const uint32_t u = key_at(i);
-      id = idx_at(i);
-      in = u > kth || (u == kth && id <= cut);
-    }
+    const bool in = i < m && winner(i, &id);
     const uint32_t slot = agg_slot(&s_nout, in);
     if (in && slot < (uint32_t)kSelOut) outv[slot] = id;
   }
@@ -202,7 +274,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   for (int i = threadIdx.x; i < K; i += blockDim.x) o[i] = (int32_t)outv[i];
 }
 
-constexpr int kSelSmem = (2 * kSelList + kSelOut) * 4;
+constexpr int kSelSmem = (2 * kSelList + (kBitmapWords > kSelOut ? kBitmapWords : kSelOut)) * 4;
 
 cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,
                           cudaStream_t stream) {
@@ -216,7 +288,7 @@ cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int 
   }
   profile_before(DOSA_KERNEL_SELECT, stream);
   select_kernel<<<(unsigned)rows, kSelThreads, kSelSmem, stream>>>(
-      reinterpret_cast<const CandView*>(b.cand), b.cap, b.cand_count, b.tau, pos0, K, out);
+      reinterpret_cast<const CandView*>(b.cand), b.seg_cap, b.cand_count, b.tau, pos0, K, out);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_SELECT, stream);
   return e;
