@@ -25,12 +25,13 @@
 // end of a range, the epilogue warps meet and each query's owner warp
 // refreshes its threshold.
 //
-// One kernel, two uses per chunk.  The probe pass screens the first
-// `probe_tiles` tiles of every item and decides from the item's own counts
-// whether screening pays there: an item that rejected fewer than 1 in 32
-// screened pairs hands its state over to the filter scorer (filter.cu), which
-// finishes it without bounds; any other unfinished item is finished by the
-// continue pass of this kernel, which screens every remaining tile.
+// A launch processes a range of steps of every item (work_items.cuh).  With
+// adaptive screening, the filter scorer (filter.cu) scores the warm-up tiles,
+// where nothing can be rejected yet; this kernel then probes the next 8 tiles
+// of each item with screening and decides from the item's own counts whether
+// screening pays there: an item that rejected fewer than 1 in 32 screened
+// pairs is finished by the filter scorer without bounds, any other by this
+// kernel, screening every remaining tile.
 #include "cand_state.cuh"
 #include "cert_layout.h"
 #include "dosa_device.cuh"
@@ -88,8 +89,8 @@ struct CertParams {
   int* err;
   int64_t row0, rows, pos0, S;   // chunk: absolute first row, rows, first position
   int n_items, K, seg_cap, seed_first, seed_last;
-  int probe_tiles;         // tiles screened by the probe pass
-  int continue_pass;       // 0: probe pass, 1: continue pass
+  StepRange steps;         // what this launch processes
+  int decide;              // 1: flag every item whose range ends before its last step
 };
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -105,24 +106,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-}
-
-// Steps [begin, end) of an item this launch processes (empty: skip the item).
-struct Range {
-  int begin, end;
-};
-
-__device__ __forceinline__ Range item_range(const CertParams& p, const Geom& g, int item) {
-  Range r;
-  if (!p.continue_pass) {
-    r.begin = 0;
-    r.end = g.n_tiles < p.probe_tiles ? g.n_tiles : p.probe_tiles;
-  } else {
-    const bool go = p.item_flag[item] == kItemScreen;
-    r.begin = go ? p.probe_tiles : 0;
-    r.end = go ? g.n_tiles : 0;
-  }
-  return r;
 }
 
 template <bool kFp8>
@@ -210,7 +193,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       uint32_t inflight_q = 0xFFFFFFFFu;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-        const Range rg = item_range(p, g, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
         if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
         mbar_arrive_expect_tx(q_full, C::kQBytes + C::kBBytes);
@@ -255,7 +238,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-        const Range rg = item_range(p, g, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
         if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
         ++it;
@@ -339,7 +322,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-      const Range rg = item_range(p, g, item);
+      const Range rg = item_steps(p.steps, p.item_flag, g, item);
       if (rg.end <= rg.begin) continue;
       const int n = rg.end - rg.begin;
       // owner: this item's state of query slot ew (fresh, or carried over)
@@ -506,7 +489,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           if (ew < g.nq)
             refresh_threshold(st[ew], p.cand + st[ew].row * kSegs * (int64_t)p.seg_cap, p.seg_cap,
                               p.K, lane);
-          if (last && !p.continue_pass && rg.end < g.n_tiles && ew == 0 && lane == 0) {
+          if (last && p.decide && rg.end < g.n_tiles && ew == 0 && lane == 0) {
             // the probe's decision, from the counts every warp left at this barrier
             unsigned long long tot_s = 0, tot_r = 0;
             for (int w = 0; w < C::kEpiWarps; ++w) {
@@ -524,8 +507,6 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
         else if (lane == 0) publish_query(st[ew], p.out);
       }
-      if (ok && !p.continue_pass && rg.end >= g.n_tiles && ew == 0 && lane == 0)
-        p.item_flag[item] = kItemDone;
     }
     if (lane == 0) {
       atomicAdd(&p.counters[kCntSeedPairs], n_seed);
@@ -548,7 +529,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
 
 template <bool kFp8>
 static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
-                                    int K, int probe_tiles, int continue_pass,
+                                    int K, StepRange steps, int decide,
                                     cudaStream_t stream) {
   using C = CertCfg<kFp8>;
   CUtensorMap qmap, bmap, kmap;
@@ -593,8 +574,8 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.seg_cap = b.seg_cap;
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
-  p.probe_tiles = probe_tiles;
-  p.continue_pass = continue_pass;
+  p.steps = steps;
+  p.decide = decide;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
@@ -605,10 +586,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
 }
 
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             int probe_tiles, int continue_pass, cudaStream_t stream) {
+                             StepRange steps, int decide, cudaStream_t stream) {
   if (h.cfg.dtype == DOSA_FP8_E4M3)
-    return launch_cert_impl<true>(h, v, b, K, probe_tiles, continue_pass, stream);
-  return launch_cert_impl<false>(h, v, b, K, probe_tiles, continue_pass, stream);
+    return launch_cert_impl<true>(h, v, b, K, steps, decide, stream);
+  return launch_cert_impl<false>(h, v, b, K, steps, decide, stream);
 }
 
 size_t certified_smem_bytes(bool fp8) {

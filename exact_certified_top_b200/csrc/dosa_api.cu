@@ -10,6 +10,7 @@
 #include "cert_layout.h"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
+#include "work_items.cuh"
 
 namespace dosa {
 
@@ -191,13 +192,11 @@ int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
   return rows / 8 * 8;
 }
 
-// Key tiles the probe pass screens per work item: enough for the warm-up (K
-// exact scores besides the seed tiles) plus 8 screened tiles, rounded up to
-// the threshold checkpoint interval.
-int probe_tiles(const Handle* h, int K) {
-  const int warm = (K + h->cfg.seed_first + h->cfg.seed_last + kKeyTile - 1) / kKeyTile + 1;
-  return (warm + 8 + 3) / 4 * 4;
-}
+// Steps of the warm-up (enough key tiles for K exact scores, whichever tile
+// is partial), rounded up to the threshold checkpoint interval, and the
+// steps the probe screens after it.
+int warmup_steps(int K) { return ((K + kKeyTile - 1) / kKeyTile + 1 + 3) / 4 * 4; }
+constexpr int kProbeSteps = 8;
 
 int64_t total_visible(const int64_t* so, int B) {
   int64_t v = 0;
@@ -380,17 +379,26 @@ dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale
       nullptr, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {
         if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
           return DOSA_ERR_CUDA;
-        // screening 1: the probe pass covers every key tile; 2: probe, then the
-        // filter scorer and the continue pass finish what the probe flagged;
-        // 0: the filter scorer alone
+        // screening 0: the filter scorer alone; 1: the certified scorer alone;
+        // 2: warm-up by the filter scorer, a probe of kProbeSteps screened
+        // steps, then each item finished by the scorer its probe chose
+        constexpr int kAll = 0x3FFFFFFF;
         const int mode = h->cfg.screening;
-        const int P = mode == 1 ? 0x3FFFFFFF : probe_tiles(h, K);
-        if (mode != 0 && launch_certified(*h, c, b, K, P, 0, stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
-        if (mode != 1 && launch_filter(*h, c, b, K, P, mode == 0, stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
-        if (mode == 2 && launch_certified(*h, c, b, K, P, 1, stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
+        if (mode == 0) {
+          if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
+            return DOSA_ERR_CUDA;
+        } else if (mode == 1) {
+          if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
+            return DOSA_ERR_CUDA;
+        } else {
+          const int W = warmup_steps(K), P = W + kProbeSteps;
+          if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
+              launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
+              launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
+              launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream) !=
+                  cudaSuccess)
+            return DOSA_ERR_CUDA;
+        }
         int32_t* out = out_idx + c.row0 * K;
         if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
         // rows whose candidate list overflowed: dense rescoring of just those rows

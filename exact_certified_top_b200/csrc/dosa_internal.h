@@ -92,15 +92,21 @@ cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale
                             float* key_norm, float* key_sum, cudaStream_t stream);
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
                               void* bdir, float* cert, int32_t* retained, cudaStream_t stream);
-// Probe pass (continue_pass = 0): steps [0, probe_tiles) of every item with
-// screening, flags each unfinished item.  Continue pass: the remaining steps of
-// the items flagged for screening.
+// The steps of every work item one launch processes: [begin, min(end,
+// n_tiles)) for the items whose probe flag equals want_flag (every item when
+// want_flag < 0).  Step 0 is key tile 0, step i >= 1 is key tile n_tiles - i.
+// A range that starts after step 0 resumes the state the previous launch
+// saved; a range that ends before the item's last step saves it again.
+struct StepRange {
+  int begin, end, want_flag;
+};
+// Certified scorer over a range of steps; decide = 1 flags each item whose
+// range ends before its last step (filter or keep screening).
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             int probe_tiles, int continue_pass, cudaStream_t stream);
-// Filter scorer: the items the probe pass handed over (from step begin_step),
-// or every item from step 0 (all_items = 1).
+                             StepRange steps, int decide, cudaStream_t stream);
+// Filter scorer (exact scores, threshold filter, no bounds) over a range.
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                          int begin_step, int all_items, cudaStream_t stream);
+                          StepRange steps, cudaStream_t stream);
 // Bytes of carried candidate state per query row.
 size_t qstate_bytes();
 cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,

@@ -12,10 +12,10 @@
 // candidate state of the item's 8 queries in shared memory (cand_state.cuh)
 // and appends only scores >= tau_t, refreshing tau_t every 4 key tiles.
 //
-// It finishes the items that the certified kernel's probe pass handed over
-// (screening rejected too little there to pay for its bound evaluation),
-// resuming their state, or with screening switched off it runs every item
-// from its first key tile.
+// A launch processes a range of steps of every item (work_items.cuh): the
+// warm-up tiles before screening starts, the rest of the items that the
+// certified kernel's probe found screening does not pay for (resuming their
+// state), or every tile when screening is switched off.
 #include "cand_state.cuh"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
@@ -53,32 +53,14 @@ struct FilterParams {
   const float* k_scale;    // sequence base (fp8)
   Cand* cand;              // [chunk rows][kSegs][seg_cap]
   QStateG* qstate;         // [chunk rows] state handed over by the probe pass
-  const int* item_flag;    // [n_items]
+  const int* item_flag;    // [n_items] decisions of the probe pass
   PublishOut out;
   unsigned long long* counters;
   int* err;
   int64_t row0, rows, pos0, S;
   int n_items, K, seg_cap, seed_first, seed_last;
-  int begin_step;          // first step of a handed-over item
-  int all_items;           // 1: every item from step 0 with a fresh state
+  StepRange steps;         // what this launch processes
 };
-
-struct FRange {
-  int begin, end;
-};
-
-__device__ __forceinline__ FRange filter_range(const FilterParams& p, const Geom& g, int item) {
-  FRange r;
-  if (p.all_items) {
-    r.begin = 0;
-    r.end = g.n_tiles;
-  } else {
-    const bool go = p.item_flag[item] == kItemFilter;
-    r.begin = go ? p.begin_step : 0;
-    r.end = go ? g.n_tiles : 0;
-  }
-  return r;
-}
 
 template <bool kFp8>
 __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
@@ -144,7 +126,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       uint32_t inflight_q = 0xFFFFFFFFu;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-        const FRange rg = filter_range(p, g, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
         if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
         mbar_arrive_expect_tx(q_full, C::kQBytes);
@@ -183,7 +165,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-        const FRange rg = filter_range(p, g, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
         if (rg.end <= rg.begin) continue;
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
         ++it;
@@ -238,7 +220,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
-      const FRange rg = filter_range(p, g, item);
+      const Range rg = item_steps(p.steps, p.item_flag, g, item);
       if (rg.end <= rg.begin) continue;
       const int n = rg.end - rg.begin;
       if (owner) {
@@ -344,7 +326,10 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
                               p.K, lane);
         }
       }
-      if (ok && owner && ew < g.nq && lane == 0) publish_query(st[ew], p.out);
+      if (ok && owner && ew < g.nq) {
+        if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
+        else if (lane == 0) publish_query(st[ew], p.out);
+      }
     }
     if (lane == 0) {
       atomicAdd(&p.counters[kCntSeedPairs], n_seed);
@@ -365,7 +350,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
 
 template <bool kFp8>
 static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
-                                      int K, int begin_step, int all_items, cudaStream_t stream) {
+                                      int K, StepRange steps, cudaStream_t stream) {
   using C = FilterCfg<kFp8>;
   CUtensorMap qmap, kmap;
   if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
@@ -406,8 +391,7 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.seg_cap = b.seg_cap;
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
-  p.begin_step = begin_step;
-  p.all_items = all_items;
+  p.steps = steps;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_FILTER, stream);
@@ -420,10 +404,10 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
 size_t qstate_bytes() { return sizeof(QStateG); }
 
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                          int begin_step, int all_items, cudaStream_t stream) {
+                          StepRange steps, cudaStream_t stream) {
   if (h.cfg.dtype == DOSA_FP8_E4M3)
-    return launch_filter_impl<true>(h, v, b, K, begin_step, all_items, stream);
-  return launch_filter_impl<false>(h, v, b, K, begin_step, all_items, stream);
+    return launch_filter_impl<true>(h, v, b, K, steps, stream);
+  return launch_filter_impl<false>(h, v, b, K, steps, stream);
 }
 
 }  // namespace dosa

@@ -42,6 +42,19 @@ __device__ __forceinline__ int tile_at(int ti, int n_tiles) {
 }
 
 // What the probe pass decided for an item (certified workspace flags).
-enum ItemFlag : int { kItemDone = 0, kItemFilter = 1, kItemScreen = 2 };
+enum ItemFlag : int { kItemFilter = 1, kItemScreen = 2 };
+
+struct Range {
+  int begin, end;   // empty when end <= begin
+};
+
+__device__ __forceinline__ Range item_steps(const StepRange& sr, const int* item_flag,
+                                            const Geom& g, int item) {
+  Range r;
+  r.begin = sr.begin;
+  r.end = g.n_tiles < sr.end ? g.n_tiles : sr.end;
+  if (sr.want_flag >= 0 && r.begin < r.end && item_flag[item] != sr.want_flag) r.end = r.begin;
+  return r;
+}
 
 }  // namespace dosa
