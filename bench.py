@@ -171,9 +171,10 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
     """Dominant kernel of the step against the tensor-core peak of its dtype.
 
     Algorithmic work: the dense scorer does 2*H*d flops per visible pair; the
-    certified kernel does 2*H*d per exactly scored pair plus 2*d*8 per
-    screened pair (the bound GEMM's dot products), counted by the call's own
-    counters (one untimed call of the same workload)."""
+    filter scorer 2*H*d per pair it scores; the certified kernel 2*H*d per
+    exactly scored pair plus 2*d*8 per screened pair (the bound GEMM's dot
+    products).  Pair counts come from the call's own counters (one untimed
+    call of the same workload)."""
     peaks, src = measured_peaks()
     kernels = {k: v for k, v in prof.items() if v[0] > 0}
     if not kernels:
@@ -188,8 +189,12 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
     if dom == "score":
         work = flops_per_pair * pairs_per_step * steps          # every visible pair, once
         name = "score_tc"
+    elif dom == "filter" and stats:
+        work = flops_per_pair * stats["filtered_pairs"] * steps
+        name = "filter_kernel"
     elif dom == "certified" and stats:
-        work = (flops_per_pair * stats["exact_pairs"] + 2 * wl.d * 8 * stats["screened_pairs"]) * steps
+        exact = stats["exact_pairs"] - stats.get("filtered_pairs", 0)
+        work = (flops_per_pair * exact + 2 * wl.d * 8 * stats["screened_pairs"]) * steps
         name = "certified_kernel"
     else:
         return {"kernel": dom, "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
@@ -217,7 +222,8 @@ def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
 def _kernel_source_sha():
     import hashlib
     h = hashlib.sha256()
-    for name in ("score_tc.cu", "certified.cu", "score_epilogue.cuh", "dosa_device.cuh"):
+    for name in ("score_tc.cu", "certified.cu", "filter.cu", "cand_state.cuh", "work_items.cuh",
+                 "score_epilogue.cuh", "dosa_device.cuh"):
         with open(os.path.join(ROOT, "exact_certified_top_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

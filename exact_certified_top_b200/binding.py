@@ -47,7 +47,8 @@ class Config(ctypes.Structure):
 class Stats(ctypes.Structure):
     _fields_ = [("visible_pairs", ctypes.c_int64), ("seed_pairs", ctypes.c_int64),
                 ("screened_pairs", ctypes.c_int64), ("rejected_pairs", ctypes.c_int64),
-                ("exact_pairs", ctypes.c_int64), ("candidates", ctypes.c_int64)]
+                ("exact_pairs", ctypes.c_int64), ("candidates", ctypes.c_int64),
+                ("filtered_pairs", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: int(getattr(self, name)) for name, _ in self._fields_}

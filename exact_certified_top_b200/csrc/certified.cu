@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             float sc = 0.f;
             if (mine) {
               const int64_t t = g.t0 + ql;
-              sc = head_reduce64(x, p.w + t * C::kH);
+              sc = head_reduce64_packed(x, p.w + t * C::kH);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
             }
             n_exact += __popc(mk);

@@ -423,6 +423,7 @@ dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale
     stats->rejected_pairs = (int64_t)hdr.counters[kCntRejected];
     stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
     stats->candidates = (int64_t)hdr.counters[kCntCandidates];
+    stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
     if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
   }
   return DOSA_OK;

@@ -27,6 +27,7 @@ enum CounterId : int {
   kCntExact = 3,
   kCntCandidates = 4,
   kCntOverflow = 5,
+  kCntFiltered = 6,
 };
 constexpr size_t kWsHeaderBytes = 256;
 

@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           const uint32_t col = tmem_base + lane_off + buf * C::kGroupRows + sub * 64;
           const float* wq = p.w + (g.t0 + (ql < g.nq ? ql : g.nq - 1)) * C::kH;
           float x[32];
-          HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
+          HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           tmem_ld32_async(col, x);
           tmem_wait_ld(x);
           head_accumulate32(acc, x, wq);
@@ -335,6 +335,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       atomicAdd(&p.counters[kCntSeedPairs], n_seed);
       atomicAdd(&p.counters[kCntExact], n_exact);
       atomicAdd(&p.counters[kCntCandidates], n_cand);
+      atomicAdd(&p.counters[kCntFiltered], n_exact);
     }
   }
 

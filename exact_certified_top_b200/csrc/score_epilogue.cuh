@@ -43,4 +43,41 @@ __device__ __forceinline__ float head_reduce64(const float* x, const float* __re
   return head_total(a);
 }
 
+// The same reduction with two heads per packed FMA (fma.rn.f32x2).  y = x + |x|
+// is exactly 2 ReLU(x), and doubling commutes with round-to-nearest (no
+// overflow or subnormals at these magnitudes), so each chain holds exactly
+// twice the chain of head_accumulate32 after every step and the halved total
+// is bit-identical to head_total.  Fewer instructions, and no max on the ALU
+// pipe: measured faster in the filter and certified scorers, slower in the
+// dense scorer, which keeps the form above.
+struct HeadAcc2 {
+  float2 c01, c23;   // chains 0,1 and 2,3
+};
+
+__device__ __forceinline__ void head_accumulate32(HeadAcc2& a, const float* x,
+                                                  const float* __restrict__ w) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 ww = __ldg(w4 + i);
+    const float y0 = x[4 * i + 0] + fabsf(x[4 * i + 0]);
+    const float y1 = x[4 * i + 1] + fabsf(x[4 * i + 1]);
+    const float y2 = x[4 * i + 2] + fabsf(x[4 * i + 2]);
+    const float y3 = x[4 * i + 3] + fabsf(x[4 * i + 3]);
+    a.c01 = __ffma2_rn(make_float2(ww.x, ww.y), make_float2(y0, y1), a.c01);
+    a.c23 = __ffma2_rn(make_float2(ww.z, ww.w), make_float2(y2, y3), a.c23);
+  }
+}
+
+__device__ __forceinline__ float head_total(const HeadAcc2& a) {
+  return 0.5f * ((a.c01.x + a.c01.y) + (a.c23.x + a.c23.y));
+}
+
+__device__ __forceinline__ float head_reduce64_packed(const float* x, const float* __restrict__ w) {
+  HeadAcc2 a = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  head_accumulate32(a, x, w);
+  head_accumulate32(a, x + 32, w + 32);
+  return head_total(a);
+}
+
 }  // namespace dosa

@@ -185,17 +185,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     s_nout = 0;
   }
   __syncthreads();
-  const int cnt_w = (cnt + 31) & ~31;
-  for (int i = threadIdx.x; i < cnt_w; i += blockDim.x) {
-    CandView c;
-    c.score = -INFINITY;
-    c.key = 0;
-    if (i < cnt) c = entry(i);
-    const bool in = i < cnt && c.score >= th;
-    const uint32_t slot = agg_slot(&s_n, in);
-    if (in && slot < (uint32_t)kSelList) {
-      lkey[slot] = ordered_key(c.score);
-      lidx[slot] = c.key;
+  // gather the candidates >= tau, segment by segment, four per thread per
+  // pass (two 16-byte loads; segments start 512-byte aligned)
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    const int cj = j == 0 ? cc.x : j == 1 ? cc.y : j == 2 ? cc.z : cc.w;
+    const CandView* sp = cl + j * (int64_t)seg_cap;
+    for (int b0 = 0; b0 < cj; b0 += blockDim.x * 4) {
+      const int b = b0 + threadIdx.x * 4;
+      CandView c[4];
+      if (b + 3 < cj) {
+        const int4 v0 = *reinterpret_cast<const int4*>(sp + b);
+        const int4 v1 = *reinterpret_cast<const int4*>(sp + b + 2);
+        c[0] = CandView{__int_as_float(v0.x), v0.y};
+        c[1] = CandView{__int_as_float(v0.z), v0.w};
+        c[2] = CandView{__int_as_float(v1.x), v1.y};
+        c[3] = CandView{__int_as_float(v1.z), v1.w};
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[e] = b + e < cj ? sp[b + e] : CandView{-INFINITY, 0};
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool in = b + e < cj && c[e].score >= th;
+        const uint32_t slot = agg_slot(&s_n, in);
+        if (in && slot < (uint32_t)kSelList) {
+          lkey[slot] = ordered_key(c[e].score);
+          lidx[slot] = c[e].key;
+        }
+      }
     }
   }
   __syncthreads();

@@ -101,6 +101,7 @@ typedef struct {
   int64_t rejected_pairs;  /* screened pairs rejected (bound + margin < threshold)   */
   int64_t exact_pairs;     /* pairs scored with all heads (seeds + survivors)        */
   int64_t candidates;      /* (score, index) pairs written for the final selection   */
+  int64_t filtered_pairs;  /* exact pairs scored by the filter scorer (no bounds)    */
 } dosa_stats;
 
 typedef struct dosa_index* dosa_index_t;

@@ -49,8 +49,12 @@ def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     assert stats["visible_pairs"] == wl.visible_pairs
     assert 0 <= stats["rejected_pairs"] <= stats["screened_pairs"]
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
+    assert 0 <= stats["filtered_pairs"] <= stats["exact_pairs"]
     if screening == 0:
         assert stats["screened_pairs"] == 0
+        assert stats["filtered_pairs"] == wl.visible_pairs
+    if screening == 1:
+        assert stats["filtered_pairs"] == 0
 
 
 def test_certified_small_workspace_many_chunks(cuda_lib):
