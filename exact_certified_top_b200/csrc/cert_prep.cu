@@ -225,12 +225,16 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   // code-domain heads, then residuals in place (padded rows); weighted residual Gram
   float(*qs)[kQPad] = reinterpret_cast<float(*)[kQPad]>(setup_dyn);
   float(*gt)[65] = reinterpret_cast<float(*)[65]>(setup_dyn + H * kQPad);
+  // The NNLS inputs and coefficients live in the Gram's space: they are dead
+  // (omega already written) before the Gram is computed.
+  double(*Bm)[4] = reinterpret_cast<double(*)[4]>(setup_dyn + H * kQPad);
+  double* QQ = reinterpret_cast<double*>(Bm + H);
+  double(*alpha_s)[4] = reinterpret_cast<double(*)[4]>(QQ + H);
+  static_assert(H * 4 * 8 * 2 + H * 8 <= H * 65 * 4, "NNLS arrays fit in the Gram's space");
   __shared__ float wv[H], qn[H], act[H], rn[H];
   __shared__ float kbar[D];
   __shared__ float vec[64];
   __shared__ double Gr[4][4];
-  __shared__ double Bm[H][4], QQ[H];
-  __shared__ double alpha_s[H][4];
   __shared__ int R[4], O[64], A1[64], A2[64];
   __shared__ int nR, nO, nA1, nA2;
   __shared__ float red[8];
@@ -409,7 +413,21 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     }
   }
   __syncthreads();
-  // ---- F: residuals in place of the omitted heads ----
+  float* cf = p.cert + i * kCertFloats;
+  if (warp == 1 && lane < 4) {
+    // omega_j = w_j + sum_h w_h alpha_hj (fp64)
+    const int j = lane;
+    float om = 0.f;
+    if (j < r) {
+      double o = wv[R[j]];
+      for (int k = 0; k < no; ++k) o += (double)wv[O[k]] * alpha_s[O[k]][j];
+      om = (float)o;
+    }
+    cf[kCertOmega + j] = om;
+    p.retained[i * 4 + j] = j < r ? R[j] : -1;
+  }
+  // ---- F: residuals in place of the omitted heads (the coefficients are
+  // read before the barrier that precedes the Gram, which reuses their space) ----
   for (int e = threadIdx.x; e < no * D; e += blockDim.x) {
     const int h = O[e / D], c = e % D;
     float x = qs[h][c];
@@ -452,49 +470,58 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    // ---- H: power iterations on |Gram| from the all-ones vector (lane l
-    // owns rows l and l + 32), then the Collatz-Wielandt bound
-    // max_a (|Gram| v)_a / v_a ----
-    const int a0 = lane, a1 = lane + 32;
-    if (a0 < no) vec[a0] = 1.f;
-    if (a1 < no) vec[a1] = 1.f;
-    __syncwarp();
-    float s0 = 0.f, s1 = 0.f;
+  // ---- H: power iterations on |Gram| from the all-ones vector, then the
+  // Collatz-Wielandt bound max_a (|Gram| v)_a / v_a.  Four threads per row
+  // (columns q * 16 + k), block-wide maximum through shared memory. ----
+  {
+    const int a = threadIdx.x >> 2, q = threadIdx.x & 3;
+    const bool row = a < no;
+    if (threadIdx.x < 64) vec[threadIdx.x] = 1.f;
+    __syncthreads();
+    float sa = 0.f, lam = 0.f;
     for (int it = 0; it <= kPowerIters; ++it) {
-      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int b = 0; b < no; b += 4) {
+      float p0 = 0.f, p1 = 0.f;
+      if (row) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (b + j < no) {
-            const float vb = vec[b + j];
-            if (a0 < no) p0[j] = fmaf(gt[a0][b + j], vb, p0[j]);
-            if (a1 < no) p1[j] = fmaf(gt[a1][b + j], vb, p1[j]);
-          }
+        for (int k = 0; k < 16; k += 2) {
+          const int b0 = q * 16 + k, b1 = b0 + 1;
+          if (b0 < no) p0 = fmaf(gt[a][b0], vec[b0], p0);
+          if (b1 < no) p1 = fmaf(gt[a][b1], vec[b1], p1);
         }
       }
-      s0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
-      s1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
+      sa = p0 + p1;
+      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
+      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 2);
       if (it == kPowerIters) break;
-      const float m = warp_max(fmaxf(s0, s1));
-      __syncwarp();
-      if (a0 < no) vec[a0] = m > 0.f ? s0 / m : 1.f;
-      if (a1 < no) vec[a1] = m > 0.f ? s1 / m : 1.f;
-      __syncwarp();
+      const float m = warp_max(row ? sa : 0.f);
+      if (lane == 0) red[warp] = m;
+      __syncthreads();
+      const float mm = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
+                             fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+      if (row && q == 0) vec[a] = mm > 0.f ? sa / mm : 1.f;
+      __syncthreads();
     }
-    float lam = 0.f;
-    if (a0 < no) lam = s0 / fmaxf(vec[a0], 1e-30f);
-    if (a1 < no) lam = fmaxf(lam, s1 / fmaxf(vec[a1], 1e-30f));
+    lam = row ? sa / fmaxf(vec[a], 1e-30f) : 0.f;
     lam = warp_max(lam);
-    if (lane == 0) s_lam = lam;
-  } else if (warp >= 4) {
-    // ---- I: negative aggregates, thread c owns element c of u_1 and u_2 ----
-    const int c = threadIdx.x - 128;
-    float u1 = 0.f, u2 = 0.f;
-    for (int k = 0; k < nA1; ++k) u1 = fmaf(fabsf(wv[A1[k]]), qs[A1[k]][c], u1);
-    for (int k = 0; k < nA2; ++k) u2 = fmaf(fabsf(wv[A2[k]]), qs[A2[k]][c], u2);
-    uv[0][c] = u1;
-    uv[1][c] = u2;
+    __syncthreads();
+    if (lane == 0) red[warp] = lam;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      s_lam = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
+                    fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+  }
+  // ---- I: negative aggregates, thread c < 128 owns element c of u_1, thread
+  // 128 + c element c of u_2 ----
+  {
+    const int c = threadIdx.x & (D - 1);
+    const int* list = threadIdx.x < D ? A1 : A2;
+    const int cnt = threadIdx.x < D ? nA1 : nA2;
+    float u = 0.f;
+    for (int k = 0; k < cnt; ++k) {
+      const int h = list[k];
+      u = fmaf(fabsf(wv[h]), qs[h][c], u);
+    }
+    uv[threadIdx.x < D ? 0 : 1][c] = u;
   }
   __syncthreads();
   // ---- J: each aggregate as a hi row and a lo row in the input type, with
@@ -544,19 +571,6 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   for (int e = threadIdx.x; e < 4 * D * (int)esz; e += blockDim.x) {
     const int j = e / (D * esz), b = e % (D * esz);
     rows_out[e] = j < r ? qrow[(size_t)R[j] * D * esz + b] : 0;
-  }
-  float* cf = p.cert + i * kCertFloats;
-  if (warp == 1 && lane < 4) {
-    // omega_j = w_j + sum_h w_h alpha_hj (fp64)
-    const int j = lane;
-    float om = 0.f;
-    if (j < r) {
-      double o = wv[R[j]];
-      for (int k = 0; k < no; ++k) o += (double)wv[O[k]] * alpha_s[O[k]][j];
-      om = (float)o;
-    }
-    cf[kCertOmega + j] = om;
-    p.retained[i * 4 + j] = j < r ? R[j] : -1;
   }
   if (warp == 0) {
     float wO = 0.f, bsum = 0.f, z2 = 0.f, scale = 0.f;
