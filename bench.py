@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--path", choices=["certified", "dense"], default="certified")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU baseline sample")
+    ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
+                    help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
     ap.add_argument("--tail-rows", type=int, default=0,
                     help="profile only the last N query rows of the workload (same keys)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -269,9 +271,11 @@ def oracle_sample(x, wl, budget_s: float):
 
 # ---------------------------------------------------------------------------
 
-def config_of(wl, path, world):
+def config_of(wl, path, world, screening=None):
+    extra = {"screening": screening} if screening is not None else {}
     return {"workload": wl.name, "T": wl.T, "S": wl.S, "H": wl.H, "d": wl.d, "K": wl.K,
-            "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, "parallelism": f"rows x{world}",
+            "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, **extra,
+            "parallelism": f"rows x{world}",
             "l2": "flushed between timed steps (256 MiB write, outside the timed windows)",
             "visible_pairs_per_gpu": wl.visible_pairs}
 
@@ -314,7 +318,7 @@ def run_ours(args, world, rank, local):
     binding.load()
     wl = workload_of(args)
     x = generate(rank_workload(wl, rank), device="cuda")
-    idx = binding.Index(wl.dtype, max_K=max(2048, wl.K))
+    idx = binding.Index(wl.dtype, max_K=max(2048, wl.K), screening=args.screening)
     certified = args.path == "certified"
     so = x["seq_offsets"]
     ws = torch.zeros(idx.workspace_size(wl.T, wl.S, wl.K, certified), dtype=torch.uint8,
@@ -407,7 +411,9 @@ def run_ours(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": wl.dtype, "data": "synthetic (seeded low-rank + sink generator)",
-                "config": config_of(wl, args.path, world), "roofline": roof,
+                "config": config_of(wl, args.path, world,
+                                    args.screening if args.path == "certified" else None),
+                "roofline": roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "kernels": {k: {"launches": n, "ms": round(t, 3)} for k, t in
                             ((k, v[1]) for k, v in prof.items()) for n in [prof[k][0]] if n},

@@ -260,13 +260,25 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       if (lane == 0) mbar_arrive(item_ready);
       if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
       ++it;
-      // this warp's segment counts of its queries grp * 4 + sub (grp = 0, 1)
-      int cnt[C::kGroups];
-#pragma unroll
-      for (int grp = 0; grp < C::kGroups; ++grp)
-        cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * C::kQPerGroup + sub].seg[quad]);
+      // Per item: this warp's queries sub (MMA tile 0) and 4 + sub (tile 1),
+      // their positions, weight rows, scales, list segments and counts.
+      const int qa = sub, qb = C::kQPerGroup + sub;
+      const bool va = qa < g.nq, vb = qb < g.nq;
+      const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
+      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * C::kH;
+      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * C::kH;
+      float qsa = 1.f, qsb = 1.f;
+      if constexpr (kFp8) {
+        qsa = __ldg(p.q_scale + g.t0 + (va ? qa : 0));
+        qsb = __ldg(p.q_scale + g.t0 + (vb ? qb : 0));
+      }
+      Cand* la = p.cand + ((g.local0 + qa) * kSegs + quad) * (int64_t)p.seg_cap;
+      Cand* lb = p.cand + ((g.local0 + qb) * kSegs + quad) * (int64_t)p.seg_cap;
+      int cnt_a = *reinterpret_cast<volatile int*>(&st[qa].seg[quad]);
+      int cnt_b = *reinterpret_cast<volatile int*>(&st[qb].seg[quad]);
+      const uint32_t col0 = tmem_base + lane_off + sub * 64;
       for (int i = 0; i < n && ok; ++i) {
-        const int64_t s = (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        const int s = tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
         float sk = 1.f;
         if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
 #pragma unroll
@@ -279,10 +291,9 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           }
           ++u;
           tc_fence_after();
-          const int ql = grp * C::kQPerGroup + sub;
           // 32 heads at a time (the register budget of 18 warps is 96 per thread)
-          const uint32_t col = tmem_base + lane_off + buf * C::kGroupRows + sub * 64;
-          const float* wq = p.w + (g.t0 + (ql < g.nq ? ql : g.nq - 1)) * C::kH;
+          const uint32_t col = col0 + buf * C::kGroupRows;
+          const float* wq = grp ? wb : wa;
           float x[32];
           HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           tmem_ld32_async(col, x);
@@ -294,15 +305,14 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
           head_accumulate32(acc, x, wq + 32);
-          if (ql < g.nq) {
-            QState& q = st[ql];
-            const int64_t t = g.t0 + ql;
+          if (grp ? vb : va) {
+            QState& q = st[grp ? qb : qa];
             float sc = head_total(acc);
-            if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
+            if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
             const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-            n_cand += append_candidates(
-                q, p.cand + ((g.local0 + ql) * kSegs + quad) * (int64_t)p.seg_cap, p.seg_cap,
-                cnt[grp], s <= g.pos_first + ql && sc >= tau, sc, (int)s, lane);
+            int& cnt = grp ? cnt_b : cnt_a;
+            n_cand += append_candidates(q, grp ? lb : la, p.seg_cap, cnt,
+                                        s <= (grp ? pos_b : pos_a) && sc >= tau, sc, s, lane);
           }
         }
         if (!ok) break;
@@ -310,9 +320,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
         if (((i + 1) % kCkptTiles) == 0 || i + 1 == n) {
           // publish this warp's segment counts (see certified.cu)
           if (lane == 0) {
-#pragma unroll
-            for (int grp = 0; grp < C::kGroups; ++grp)
-              st[grp * C::kQPerGroup + sub].seg[quad] = cnt[grp];
+            st[qa].seg[quad] = cnt_a;
+            st[qb].seg[quad] = cnt_b;
           }
           __threadfence_block();
           if (lane == 0) mbar_arrive(tile_done);

@@ -243,21 +243,37 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const ItemGeom g = item_geom(p, item);
+      // this warp's queries sub (MMA tile 0) and 4 + sub (MMA tile 1)
+      const int qa = sub, qb = C::kQPerGroup + sub;
+      const bool va = qa < g.nq, vb = qb < g.nq;
+      const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
+      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * C::kH;
+      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * C::kH;
+      float qsa = 1.f, qsb = 1.f;
+      if constexpr (kFp8) {
+        qsa = __ldg(p.q_scale + g.t0 + (va ? qa : 0));
+        qsb = __ldg(p.q_scale + g.t0 + (vb ? qb : 0));
+      }
+      float* ra = p.scores + (g.out0 + (va ? qa : 0)) * p.ld;
+      float* rb = p.scores + (g.out0 + (vb ? qb : 0)) * p.ld;
+      const uint32_t col0 = tmem_base + lane_off + sub * 64;
       for (int j = 0; j < g.nkt && ok; ++j) {
-        const int64_t s = (int64_t)j * kKeyTile + quad * 32 + lane;
+        const int s = j * kKeyTile + quad * 32 + lane;
         float sk = 1.0f;
         if constexpr (kFp8) sk = (s < p.S) ? __ldg(p.k_scale + s) : 0.0f;
-        for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
+#pragma unroll
+        for (int grp = 0; grp < C::kGroups; ++grp) {
+          if (!ok) continue;
           const uint32_t buf = u & 1;
           if (!mbar_wait(&acc_full[buf], (u >> 1) & 1, s_abort, p.err)) {
             ok = false;
-            break;
+            continue;
           }
+          ++u;
           tc_fence_after();
-          const int ql = grp * C::kQPerGroup + sub;
           // 32 heads at a time (the register budget of 18 warps is 96 per thread)
-          const uint32_t col = tmem_base + lane_off + buf * C::kGroupRows + sub * 64;
-          const float* wq = p.w + (g.t0 + (ql < g.nq ? ql : g.nq - 1)) * C::kH;
+          const uint32_t col = col0 + buf * C::kGroupRows;
+          const float* wq = grp ? wb : wa;
           float v[32];
           HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
           tmem_ld32_async(col, v);
@@ -269,11 +285,10 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
           head_accumulate32(acc, v, wq + 32);
-          if (ql < g.nq) {
-            const int64_t t = g.t0 + ql;
+          if (grp ? vb : va) {
             float sc = head_total(acc);
-            if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
-            if (s <= g.pos_first + ql) p.scores[(g.out0 + ql) * p.ld + s] = sc;
+            if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
+            if (s <= (grp ? pos_b : pos_a)) (grp ? rb : ra)[s] = sc;
           }
         }
       }
