@@ -43,11 +43,11 @@ __device__ __forceinline__ float head_reduce64(const float* x, const float* __re
   return head_total(a);
 }
 
-// The same reduction with two heads per packed FMA (fma.rn.f32x2).  y = x + |x|
-// is exactly 2 ReLU(x), and doubling commutes with round-to-nearest (no
-// overflow or subnormals at these magnitudes), so each chain holds exactly
-// twice the chain of head_accumulate32 after every step and the halved total
-// is bit-identical to head_total.  Fewer instructions, and no max on the ALU
+// The same reduction with two heads per packed add and FMA (add.rn.f32x2,
+// fma.rn.f32x2).  y = x + |x| is exactly 2 ReLU(x), and doubling commutes with
+// round-to-nearest (no overflow or subnormals at these magnitudes), so each
+// chain holds exactly twice the chain of head_accumulate32 after every step
+// and the halved total is bit-identical to head_total.  Fewer instructions, and no max on the ALU
 // pipe: measured faster in the filter and certified scorers, slower in the
 // dense scorer, which keeps the form above.
 struct HeadAcc2 {
@@ -60,12 +60,12 @@ __device__ __forceinline__ void head_accumulate32(HeadAcc2& a, const float* x,
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 ww = __ldg(w4 + i);
-    const float y0 = x[4 * i + 0] + fabsf(x[4 * i + 0]);
-    const float y1 = x[4 * i + 1] + fabsf(x[4 * i + 1]);
-    const float y2 = x[4 * i + 2] + fabsf(x[4 * i + 2]);
-    const float y3 = x[4 * i + 3] + fabsf(x[4 * i + 3]);
-    a.c01 = __ffma2_rn(make_float2(ww.x, ww.y), make_float2(y0, y1), a.c01);
-    a.c23 = __ffma2_rn(make_float2(ww.z, ww.w), make_float2(y2, y3), a.c23);
+    const float2 y01 = __fadd2_rn(make_float2(x[4 * i + 0], x[4 * i + 1]),
+                                  make_float2(fabsf(x[4 * i + 0]), fabsf(x[4 * i + 1])));
+    const float2 y23 = __fadd2_rn(make_float2(x[4 * i + 2], x[4 * i + 3]),
+                                  make_float2(fabsf(x[4 * i + 2]), fabsf(x[4 * i + 3])));
+    a.c01 = __ffma2_rn(make_float2(ww.x, ww.y), y01, a.c01);
+    a.c23 = __ffma2_rn(make_float2(ww.z, ww.w), y23, a.c23);
   }
 }
 
