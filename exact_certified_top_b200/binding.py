@@ -26,7 +26,7 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_index_scores", "dosa_reference_scores", "dosa_index_certificate",
            "dosa_index_dense_topk_static", "dosa_topk_rows", "dosa_check_device",
            "dosa_status_string", "dosa_profile_enable", "dosa_profile_reset",
-           "dosa_profile_read")
+           "dosa_profile_read", "dosa_index_topk_host", "dosa_index_host_workspace_size")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
            "certified": 5, "select": 6, "filter": 7}
 
@@ -76,6 +76,9 @@ def load(path: str = LIB_PATH):
     common = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P]
     lib.dosa_index_topk.argtypes = common + [ctypes.POINTER(Stats)]
     lib.dosa_index_dense_topk.argtypes = common
+    lib.dosa_index_topk_host.argtypes = common + [ctypes.POINTER(Stats)]
+    lib.dosa_index_host_workspace_size.argtypes = [_P, _I64, _I64, _I64, _I, _I64,
+                                                   ctypes.POINTER(_SZ)]
     lib.dosa_index_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64,
                                       _P, _P]
     lib.dosa_reference_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P,
@@ -183,6 +186,32 @@ class Index:
             self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
             ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, K, _ptr(out), _ptr(ws),
             ws.numel(), _stream(), ctypes.byref(st) if stats else None))
+        return (out, st.as_dict()) if stats else out
+
+    def host_workspace_size(self, Tq: int, S_total: int, S_max: int, K: int,
+                            chunk_rows: int = 0) -> int:
+        n = ctypes.c_size_t()
+        _check("dosa_index_host_workspace_size",
+               self._lib.dosa_index_host_workspace_size(self._h, Tq, S_total, S_max, K,
+                                                        chunk_rows, ctypes.byref(n)))
+        return int(n.value)
+
+    def topk_host(self, q, q_scale, w, k, k_scale, seq_offsets, K, out=None, workspace=None,
+                  stats: bool = False):
+        """Certified Top-K with host (CPU, ideally pinned) inputs and output; the
+        workspace is a CUDA tensor (host_workspace_size bytes)."""
+        so = _seq_offsets(seq_offsets)
+        if out is None:
+            out = torch.empty((q.shape[0], K), dtype=torch.int32, pin_memory=True)
+        if workspace is None:
+            S_max = int((so[1:, 1] - so[:-1, 1]).max())
+            n = self.host_workspace_size(q.shape[0], int(so[-1, 1]), S_max, K)
+            workspace = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        st = Stats()
+        _check("dosa_index_topk_host", self._lib.dosa_index_topk_host(
+            self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
+            ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, K, _ptr(out), _ptr(workspace),
+            workspace.numel(), _stream(), ctypes.byref(st) if stats else None))
         return (out, st.as_dict()) if stats else out
 
     def certificate(self, q, q_scale, w, k, k_scale, seq_offsets, workspace=None):

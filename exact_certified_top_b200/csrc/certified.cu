@@ -27,7 +27,7 @@
 //
 // A launch processes a range of steps of every item (work_items.cuh).  With
 // adaptive screening, the filter scorer (filter.cu) scores the warm-up tiles,
-// where nothing can be rejected yet; this kernel then probes the next 8 tiles
+// where nothing can be rejected yet; this kernel then probes the next 4 tiles
 // of each item with screening and decides from the item's own counts whether
 // screening pays there: an item that rejected fewer than 1 in 32 screened
 // pairs is finished by the filter scorer without bounds, any other by this
@@ -43,7 +43,7 @@ namespace dosa {
 
 // Items whose probe screened at least this many pairs and rejected fewer than
 // 1 in kRejectRatio of them are handed to the filter scorer.
-constexpr unsigned long long kMinScreened = 4096;
+constexpr unsigned long long kMinScreened = 2048;
 constexpr unsigned long long kRejectRatio = 32;
 
 template <bool kFp8>

@@ -6,6 +6,8 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
+#include <algorithm>
 
 #include "cert_layout.h"
 #include "dosa_device.cuh"
@@ -99,6 +101,7 @@ SeqView make_view(const Handle* h, const void* q, const float* q_scale, const fl
 }
 
 constexpr int64_t kDefaultChunkBytes = (int64_t)4 << 30;   // dense score chunk budget
+constexpr int64_t kDefaultCertChunkBytes = (int64_t)8 << 30;   // certified per-row arrays
 constexpr int kRepairRows = 64;                             // overflowed rows per chunk
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -107,14 +110,15 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 // segments, one per 32-key quarter of every key tile.  A row with n keys
 // appends about K (1 + ln(n / K)) candidates (a key is appended when it
 // enters the running Top-K, with probability about K / its rank in the
-// processing order), and the histogram threshold's coarseness adds up to
-// about as much again on inputs with a few very large scores.  A segment
-// holds 0.65 K (1 + ln(S_max / K)) entries (at least 1024, rounded up to 64),
+// processing order).  The histogram threshold's coarseness adds more on rows
+// where a few very large scores stretch its range: measured tails reach 1.75x
+// the mean at 128K keys and more at 1M.  A segment holds 0.9 K (1 + ln(S_max /
+// K)) entries (3.6x the mean per segment; at least 1024, rounded up to 64),
 // and never more than the keys it can see: 32 per key tile.  A row that
 // overflows is rescored densely.
 int seg_capacity(int K, int64_t S_max) {
   const double ratio = S_max > K ? (double)S_max / K : 1.0;
-  int64_t cap = (int64_t)ceil(0.65 * K * (1.0 + log(ratio)));
+  int64_t cap = (int64_t)ceil(0.9 * K * (1.0 + log(ratio)));
   cap = (cap + 63) / 64 * 64;
   if (cap < 1024) cap = 1024;
   const int64_t most = (S_max + kKeyTile - 1) / kKeyTile * 32;
@@ -196,7 +200,7 @@ int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
 // is partial), rounded up to the threshold checkpoint interval, and the
 // steps the probe screens after it.
 int warmup_steps(int K) { return ((K + kKeyTile - 1) / kKeyTile + 1 + 3) / 4 * 4; }
-constexpr int kProbeSteps = 8;
+constexpr int kProbeSteps = 4;
 
 int64_t total_visible(const int64_t* so, int B) {
   int64_t v = 0;
@@ -255,7 +259,21 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   return DOSA_OK;
 }
 
-void dosa_index_destroy(dosa_index_t h) { delete reinterpret_cast<Handle*>(h); }
+void dosa_index_destroy(dosa_index_t hh) {
+  Handle* h = reinterpret_cast<Handle*>(hh);
+  if (!h) return;
+  if (h->copy_stream) {
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(h->copy_device);
+    cudaStreamDestroy(h->copy_stream);
+    for (cudaEvent_t e : {h->ev_loaded[0], h->ev_loaded[1], h->ev_done[0], h->ev_done[1],
+                          h->ev_keys, h->ev_out})
+      if (e) cudaEventDestroy(e);
+    cudaSetDevice(cur);
+  }
+  delete h;
+}
 
 dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max, int K,
                                       int certified, int64_t chunk_rows, size_t* bytes) {
@@ -266,7 +284,7 @@ dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max
     const CertLayout L = cert_layout(h, S_max, K);
     int64_t rows = chunk_rows;
     if (rows == 0) {
-      rows = kDefaultChunkBytes / (int64_t)L.per_row;
+      rows = kDefaultCertChunkBytes / (int64_t)L.per_row;
       rows = rows / 8 * 8;
       if (rows < 8) rows = 8;
     }
@@ -364,6 +382,139 @@ static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const flo
   return DOSA_OK;
 }
 
+// The certified Top-K of one chunk of rows whose certificate is set up:
+// scoring passes, selection, repair of overflowed rows.  out: row 0 of the
+// chunk's indices.
+static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffers& b, int K,
+                              int32_t* out, cudaStream_t stream) {
+  if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  // screening 0: the filter scorer alone; 1: the certified scorer alone;
+  // 2: warm-up by the filter scorer, a probe of kProbeSteps screened steps,
+  // then each item finished by the scorer its probe chose
+  constexpr int kAll = 0x3FFFFFFF;
+  const int mode = h->cfg.screening;
+  if (mode == 0) {
+    if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+  } else if (mode == 1) {
+    if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+  } else {
+    const int W = warmup_steps(K), P = W + kProbeSteps;
+    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
+        launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
+        launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
+        launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+  }
+  if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+  // rows whose candidate list overflowed: dense rescoring of just those rows
+  if (launch_scores_tc_rows(*h, c, b.repair_list, b.repair_count, b.repair_cap, b.repair_scores,
+                            c.S, b.err, stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  if (launch_topk_list(b.repair_scores, c.S, b.repair_list, b.repair_count, b.repair_cap,
+                       c.pos0 + 1, c.S, K, out, K, stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  return DOSA_OK;
+}
+
+// Counters of the workspace header into *stats (synchronises the stream).
+static dosa_status read_stats(const void* workspace, const int64_t* seq_offsets, int B,
+                              cudaStream_t stream, dosa_stats* stats) {
+  WsHeader hdr;
+  if (cudaMemcpyAsync(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  stats->visible_pairs = total_visible(seq_offsets, B);
+  stats->seed_pairs = (int64_t)hdr.counters[kCntSeedPairs];
+  stats->screened_pairs = (int64_t)hdr.counters[kCntScreened];
+  stats->rejected_pairs = (int64_t)hdr.counters[kCntRejected];
+  stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
+  stats->candidates = (int64_t)hdr.counters[kCntCandidates];
+  stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
+  if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
+  return DOSA_OK;
+}
+
+// ---- host-staged certified calls ---------------------------------------------------
+
+namespace {
+
+// Device workspace of a host-staged call: the certified workspace for Tc rows,
+// the keys (and key scales) of every sequence, and two staging slots of Tc
+// query rows (q, q_scale, w in; indices out).
+struct HostLayout {
+  CertLayout L;
+  int64_t Tc;
+  size_t keys, kscale, slot[2], slot_q, slot_qs, slot_w, slot_out, total;
+};
+
+constexpr int64_t kHostChunkRows = 16384;
+
+HostLayout host_layout(const Handle* h, int64_t Tq, int64_t S_total, int64_t S_max, int K,
+                       int64_t chunk_rows) {
+  HostLayout H;
+  H.L = cert_layout(h, S_max, K);
+  int64_t rows = chunk_rows > 0 ? chunk_rows : kHostChunkRows;
+  rows = round_up(rows, 8);
+  if (rows > round_up(Tq, 8)) rows = round_up(Tq, 8);
+  if (rows < 8) rows = 8;
+  H.Tc = rows;
+  const size_t esz = elem_bytes(h);
+  const bool fp8 = h->cfg.dtype == DOSA_FP8_E4M3;
+  size_t off = (size_t)round_up((int64_t)(H.L.fixed + (size_t)rows * H.L.per_row + kCertPad), 256);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (size_t)round_up((int64_t)bytes, 256);
+    return at;
+  };
+  H.keys = take((size_t)S_total * kHeadDim * esz);
+  H.kscale = take(fp8 ? (size_t)S_total * 4 : 0);
+  size_t so = 0;
+  auto take_slot = [&](size_t bytes) {
+    const size_t at = so;
+    so += (size_t)round_up((int64_t)bytes, 256);
+    return at;
+  };
+  H.slot_q = take_slot((size_t)rows * 64 * kHeadDim * esz);
+  H.slot_qs = take_slot(fp8 ? (size_t)rows * 4 : 0);
+  H.slot_w = take_slot((size_t)rows * 64 * 4);
+  H.slot_out = take_slot((size_t)rows * K * 4);
+  H.slot[0] = take(so);
+  H.slot[1] = take(so);
+  H.total = off;
+  return H;
+}
+
+// The handle's copy stream and events on the current device (created on
+// first use, recreated when the device changes).
+dosa_status ensure_copy_stream(Handle* h) {
+  std::lock_guard<std::mutex> lock(h->copy_mutex);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DOSA_ERR_CUDA;
+  if (h->copy_stream && h->copy_device == dev) return DOSA_OK;
+  if (h->copy_stream) {
+    cudaSetDevice(h->copy_device);
+    cudaStreamDestroy(h->copy_stream);
+    for (cudaEvent_t* e : {&h->ev_loaded[0], &h->ev_loaded[1], &h->ev_done[0], &h->ev_done[1],
+                           &h->ev_keys, &h->ev_out})
+      if (*e) cudaEventDestroy(*e), *e = nullptr;
+    h->copy_stream = nullptr;
+    cudaSetDevice(dev);
+  }
+  if (cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  for (cudaEvent_t* e : {&h->ev_loaded[0], &h->ev_loaded[1], &h->ev_done[0], &h->ev_done[1],
+                         &h->ev_keys, &h->ev_out})
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return DOSA_ERR_CUDA;
+  h->copy_device = dev;
+  return DOSA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale, const float* w,
@@ -377,55 +528,134 @@ dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale
   st = for_each_cert_chunk(
       h, q, q_scale, w, k, k_scale, seq_offsets, B, K, workspace, ws_bytes, stream, nullptr,
       nullptr, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {
-        if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
-        // screening 0: the filter scorer alone; 1: the certified scorer alone;
-        // 2: warm-up by the filter scorer, a probe of kProbeSteps screened
-        // steps, then each item finished by the scorer its probe chose
-        constexpr int kAll = 0x3FFFFFFF;
-        const int mode = h->cfg.screening;
-        if (mode == 0) {
-          if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
-            return DOSA_ERR_CUDA;
-        } else if (mode == 1) {
-          if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
-            return DOSA_ERR_CUDA;
-        } else {
-          const int W = warmup_steps(K), P = W + kProbeSteps;
-          if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
-              launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
-              launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
-              launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream) !=
-                  cudaSuccess)
-            return DOSA_ERR_CUDA;
-        }
-        int32_t* out = out_idx + c.row0 * K;
-        if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
-        // rows whose candidate list overflowed: dense rescoring of just those rows
-        if (launch_scores_tc_rows(*h, c, b.repair_list, b.repair_count, b.repair_cap,
-                                  b.repair_scores, c.S, b.err, stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
-        if (launch_topk_list(b.repair_scores, c.S, b.repair_list, b.repair_count, b.repair_cap,
-                             c.pos0 + 1, c.S, K, out, K, stream) != cudaSuccess)
-          return DOSA_ERR_CUDA;
-        return DOSA_OK;
+        return cert_chunk(h, c, b, K, out_idx + c.row0 * K, stream);
       });
   if (st != DOSA_OK) return st;
-  if (stats) {
-    WsHeader hdr;
-    if (cudaMemcpyAsync(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, stream) !=
-            cudaSuccess ||
-        cudaStreamSynchronize(stream) != cudaSuccess)
-      return DOSA_ERR_CUDA;
-    stats->visible_pairs = total_visible(seq_offsets, B);
-    stats->seed_pairs = (int64_t)hdr.counters[kCntSeedPairs];
-    stats->screened_pairs = (int64_t)hdr.counters[kCntScreened];
-    stats->rejected_pairs = (int64_t)hdr.counters[kCntRejected];
-    stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
-    stats->candidates = (int64_t)hdr.counters[kCntCandidates];
-    stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
-    if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
+  if (stats) return read_stats(workspace, seq_offsets, B, stream, stats);
+  return DOSA_OK;
+}
+
+dosa_status dosa_index_host_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_total,
+                                           int64_t S_max, int K, int64_t chunk_rows,
+                                           size_t* bytes) {
+  const Handle* h = reinterpret_cast<const Handle*>(hh);
+  if (!h || !bytes || Tq < 0 || S_total < 0 || S_max < 0 || S_max > S_total || K < 1 ||
+      K > h->cfg.max_K || chunk_rows < 0)
+    return DOSA_ERR_INVALID_ARG;
+  *bytes = host_layout(h, Tq, S_total, S_max, K, chunk_rows).total;
+  return DOSA_OK;
+}
+
+dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_scale,
+                                 const float* w, const void* k, const float* k_scale,
+                                 const int64_t* seq_offsets, int B, int K, int32_t* out_idx,
+                                 void* workspace, size_t ws_bytes, void* stream_,
+                                 dosa_stats* stats) {
+  Handle* h = reinterpret_cast<Handle*>(hh);
+  dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, K, out_idx);
+  if (st != DOSA_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DOSA_ERR_INVALID_ARG;
+  const int64_t Tq = seq_offsets[3 * B], S_total = seq_offsets[3 * B + 1];
+  const int64_t S_max = max_keys(seq_offsets, B);
+  // the most rows per staging slot (up to the default) that fit the workspace
+  HostLayout H = host_layout(h, Tq, S_total, S_max, K, 0);
+  if (ws_bytes < H.total) {
+    int64_t lo = 8, hi = H.Tc;            // largest multiple of 8 in [lo, hi) that fits
+    if (host_layout(h, Tq, S_total, S_max, K, lo).total > ws_bytes) return DOSA_ERR_WORKSPACE;
+    while (hi - lo > 8) {
+      const int64_t mid = (lo + hi) / 2 / 8 * 8;
+      if (host_layout(h, Tq, S_total, S_max, K, mid).total <= ws_bytes) lo = mid;
+      else hi = mid;
+    }
+    H = host_layout(h, Tq, S_total, S_max, K, lo);
   }
+  st = ensure_copy_stream(h);
+  if (st != DOSA_OK) return st;
+  cudaStream_t main = static_cast<cudaStream_t>(stream_), cpy = h->copy_stream;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool fp8 = h->cfg.dtype == DOSA_FP8_E4M3;
+  const size_t esz = elem_bytes(h), qrow = (size_t)64 * kHeadDim * esz;
+  const CertBuffers buf = cert_buffers(h, H.L, ws, H.Tc);
+  uint8_t* dk = ws + H.keys;
+  float* dks = fp8 ? reinterpret_cast<float*>(ws + H.kscale) : nullptr;
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // keys first (on the caller's stream, ordered after its earlier work); the
+  // copy stream starts after that point, so it never overwrites a slot that
+  // an earlier call on this stream still reads
+  if (!ok(cudaMemsetAsync(ws, 0, kWsHeaderBytes, main)) ||
+      !ok(cudaMemcpyAsync(dk, k, (size_t)S_total * kHeadDim * esz, cudaMemcpyHostToDevice, main)) ||
+      (fp8 && !ok(cudaMemcpyAsync(dks, k_scale, (size_t)S_total * 4, cudaMemcpyHostToDevice,
+                                  main))) ||
+      !ok(cudaEventRecord(h->ev_keys, main)) || !ok(cudaStreamWaitEvent(cpy, h->ev_keys, 0)))
+    return DOSA_ERR_CUDA;
+  struct Chunk {
+    int b;
+    int64_t r0, rows;
+  };
+  std::vector<Chunk> chunks;
+  for (int b = 0; b < B; ++b) {
+    const SeqInfo si = seq_info(seq_offsets, b);
+    for (int64_t r = 0; r < si.q_end - si.q_start; r += H.Tc)
+      chunks.push_back({b, r, std::min<int64_t>(H.Tc, si.q_end - si.q_start - r)});
+  }
+  const uint8_t* qh = static_cast<const uint8_t*>(q);
+  // stage chunk ci's query rows into slot ci % 2 (after the compute that last
+  // read that slot)
+  auto load = [&](size_t ci) -> bool {
+    const Chunk& ch = chunks[ci];
+    const int slot = (int)(ci & 1);
+    const int64_t t0 = seq_info(seq_offsets, ch.b).q_start + ch.r0;
+    uint8_t* sb = ws + H.slot[slot];
+    return ok(cudaStreamWaitEvent(cpy, h->ev_done[slot], 0)) &&
+           ok(cudaMemcpyAsync(sb + H.slot_q, qh + (size_t)t0 * qrow, (size_t)ch.rows * qrow,
+                              cudaMemcpyHostToDevice, cpy)) &&
+           (!fp8 || ok(cudaMemcpyAsync(sb + H.slot_qs, q_scale + t0, (size_t)ch.rows * 4,
+                                       cudaMemcpyHostToDevice, cpy))) &&
+           ok(cudaMemcpyAsync(sb + H.slot_w, w + t0 * 64, (size_t)ch.rows * 64 * 4,
+                              cudaMemcpyHostToDevice, cpy)) &&
+           ok(cudaEventRecord(h->ev_loaded[slot], cpy));
+  };
+  if (!chunks.empty() && !load(0)) return DOSA_ERR_CUDA;
+  int prev_b = -1;
+  for (size_t ci = 0; ci < chunks.size(); ++ci) {
+    if (ci + 1 < chunks.size() && !load(ci + 1)) return DOSA_ERR_CUDA;
+    const Chunk& ch = chunks[ci];
+    const int slot = (int)(ci & 1);
+    const SeqInfo si = seq_info(seq_offsets, ch.b);
+    uint8_t* sb = ws + H.slot[slot];
+    SeqView c;
+    c.q = sb + H.slot_q;
+    c.q_scale = fp8 ? reinterpret_cast<const float*>(sb + H.slot_qs) : nullptr;
+    c.w = reinterpret_cast<const float*>(sb + H.slot_w);
+    c.k = dk + (size_t)si.k_start * kHeadDim * esz;
+    c.k_scale = fp8 ? dks + si.k_start : nullptr;
+    c.row0 = 0;
+    c.rows = ch.rows;
+    c.pos0 = si.q_pos0 + ch.r0;
+    c.S = si.k_end - si.k_start;
+    int32_t* dout = reinterpret_cast<int32_t*>(sb + H.slot_out);
+    if (ch.b != prev_b) {
+      if (launch_key_prep(*h, c.k, c.k_scale, c.S, buf.key_norm, buf.key_sum, main) !=
+          cudaSuccess)
+        return DOSA_ERR_CUDA;
+      prev_b = ch.b;
+    }
+    if (!ok(cudaStreamWaitEvent(main, h->ev_loaded[slot], 0)) ||
+        launch_cert_setup(*h, c, buf.key_sum, buf.bdir, buf.cert, buf.retained, main) !=
+            cudaSuccess)
+      return DOSA_ERR_CUDA;
+    st = cert_chunk(h, c, buf, K, dout, main);
+    if (st != DOSA_OK) return st;
+    if (!ok(cudaEventRecord(h->ev_done[slot], main)) ||
+        !ok(cudaStreamWaitEvent(cpy, h->ev_done[slot], 0)) ||
+        !ok(cudaMemcpyAsync(out_idx + (si.q_start + ch.r0) * K, dout, (size_t)ch.rows * K * 4,
+                            cudaMemcpyDeviceToHost, cpy)))
+      return DOSA_ERR_CUDA;
+  }
+  // the caller's stream completes after the last copy out
+  if (!ok(cudaEventRecord(h->ev_out, cpy)) || !ok(cudaStreamWaitEvent(main, h->ev_out, 0)))
+    return DOSA_ERR_CUDA;
+  if (stats) return read_stats(workspace, seq_offsets, B, main, stats);
   return DOSA_OK;
 }
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "dosa.h"
 
 namespace dosa {
@@ -46,6 +48,14 @@ struct SeqView {
 
 struct Handle {
   dosa_index_config cfg;
+  // Host-staged calls: a copy stream and staging events, created on first use
+  // on the device current at that time (per device).
+  int copy_device = -1;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_loaded[2] = {nullptr, nullptr};
+  cudaEvent_t ev_done[2] = {nullptr, nullptr};
+  cudaEvent_t ev_keys = nullptr, ev_out = nullptr;
+  std::mutex copy_mutex;
 };
 
 // Kernel timing hooks (profile.cu): bracket one launch with events when enabled.

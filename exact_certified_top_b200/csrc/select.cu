@@ -64,15 +64,16 @@ __device__ __forceinline__ uint32_t agg_slot(uint32_t* counter, bool active) {
 
 // Radix select over n elements: `get(i, &key)` returns false to skip element i.
 // Returns the key of the K-th largest selected element; *take = how many
-// elements equal to it belong to the K largest.
+// elements equal to it belong to the K largest, *eq = how many equal it.
+// hist: 2 x 256 words, both zero on entry and left zero on return; each pass
+// counts into one while the other is being cleared, two barriers per pass.
 template <typename Get>
-__device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32_t* s_digit,
-                              uint32_t* s_above, uint32_t* s_eq, uint32_t* take, uint32_t* eq) {
-  uint32_t prefix = 0, mask = 0, remaining = K;
+__device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32_t* s_res,
+                              uint32_t* take, uint32_t* eq) {
+  uint32_t prefix = 0, mask = 0, remaining = K, eq_count = 0;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
-    __syncthreads();
+    uint32_t* h = hist + (pass & 1) * 256;
     const int nn = (n + 31) & ~31;             // whole warps for the aggregated adds
     for (int i = threadIdx.x; i < nn; i += blockDim.x) {
       uint32_t u = 0;
@@ -81,7 +82,7 @@ __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32
       const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
       if (in) {
         const uint32_t peers = __match_any_sync(m, bin);
-        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
       }
     }
     __syncthreads();
@@ -90,7 +91,7 @@ __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c[j] = hist[255 - 8 * lane - j];
+        c[j] = h[255 - 8 * lane - j];
         sum += c[j];
       }
       uint32_t incl = sum;
@@ -105,22 +106,30 @@ __device__ uint32_t radix_kth(Get get, int n, uint32_t K, uint32_t* hist, uint32
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (acc < remaining && remaining <= acc + c[j]) {
-            *s_digit = 255 - 8 * lane - j;
-            *s_above = acc;
-            *s_eq = c[j];
+            s_res[(pass & 1) * 4 + 0] = 255 - 8 * lane - j;
+            s_res[(pass & 1) * 4 + 1] = acc;
+            s_res[(pass & 1) * 4 + 2] = c[j];
           }
           acc += c[j];
         }
       }
+    } else if (threadIdx.x < 64) {
+      // clear the other histogram for the next pass (and on return)
+      uint32_t* o = hist + ((pass + 1) & 1) * 256;
+      for (int j = threadIdx.x - 32; j < 256; j += 32) o[j] = 0u;
     }
     __syncthreads();
-    prefix |= *s_digit << shift;
+    const uint32_t* r = s_res + (pass & 1) * 4;
+    prefix |= r[0] << shift;
     mask |= 255u << shift;
-    remaining -= *s_above;
-    __syncthreads();
+    remaining -= r[1];
+    eq_count = r[2];
   }
+  // the last pass's histogram is still counted: clear it (the caller
+  // synchronises before the next use)
+  for (int j = threadIdx.x; j < 256; j += blockDim.x) hist[256 + j] = 0u;
   *take = remaining;
-  *eq = *s_eq;          // elements whose key equals the result (last digit's bin)
+  *eq = eq_count;       // elements whose key equals the result (last digit's bin)
   return prefix;
 }
 
@@ -157,9 +166,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   uint32_t* lkey = sel_smem;                                        // [kSelList]
   int32_t* lidx = reinterpret_cast<int32_t*>(lkey + kSelList);     // [kSelList]
   uint32_t* bm = reinterpret_cast<uint32_t*>(lidx + kSelList);     // [kBitmapWords] or sort area
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[2 * 256];
   __shared__ uint32_t scan[32];
-  __shared__ uint32_t s_digit, s_above, s_eq, s_n, s_nout;
+  __shared__ uint32_t s_res[8];
+  __shared__ uint32_t s_n, s_nout;
   const int64_t row = blockIdx.x;
   const int64_t nvis = pos0 + row + 1;
   int32_t* o = out + row * K;
@@ -184,30 +194,39 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     s_n = 0;
     s_nout = 0;
   }
+  for (int j = threadIdx.x; j < 2 * 256; j += blockDim.x) hist[j] = 0u;
   __syncthreads();
-  // gather the candidates >= tau, segment by segment, four per thread per
-  // pass (two 16-byte loads; segments start 512-byte aligned)
+  // gather the candidates >= tau, segment by segment, eight per thread per
+  // pass: four 16-byte loads issued before any is used (segments start
+  // 512-byte aligned)
 #pragma unroll 1
   for (int j = 0; j < 4; ++j) {
     const int cj = j == 0 ? cc.x : j == 1 ? cc.y : j == 2 ? cc.z : cc.w;
     const CandView* sp = cl + j * (int64_t)seg_cap;
-    for (int b0 = 0; b0 < cj; b0 += blockDim.x * 4) {
+    for (int b0 = 0; b0 < cj; b0 += blockDim.x * 8) {
       const int b = b0 + threadIdx.x * 4;
-      CandView c[4];
-      if (b + 3 < cj) {
-        const int4 v0 = *reinterpret_cast<const int4*>(sp + b);
-        const int4 v1 = *reinterpret_cast<const int4*>(sp + b + 2);
-        c[0] = CandView{__int_as_float(v0.x), v0.y};
-        c[1] = CandView{__int_as_float(v0.z), v0.w};
-        c[2] = CandView{__int_as_float(v1.x), v1.y};
-        c[3] = CandView{__int_as_float(v1.z), v1.w};
-      } else {
+      const int bh = b + blockDim.x * 4;
+      CandView c[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] = b + e < cj ? sp[b + e] : CandView{-INFINITY, 0};
+      for (int hh = 0; hh < 2; ++hh) {
+        const int bb = hh ? bh : b;
+        if (bb + 3 < cj) {
+          const int4 v0 = *reinterpret_cast<const int4*>(sp + bb);
+          const int4 v1 = *reinterpret_cast<const int4*>(sp + bb + 2);
+          c[hh * 4 + 0] = CandView{__int_as_float(v0.x), v0.y};
+          c[hh * 4 + 1] = CandView{__int_as_float(v0.z), v0.w};
+          c[hh * 4 + 2] = CandView{__int_as_float(v1.x), v1.y};
+          c[hh * 4 + 3] = CandView{__int_as_float(v1.z), v1.w};
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            c[hh * 4 + e] = bb + e < cj ? sp[bb + e] : CandView{-INFINITY, 0};
+        }
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool in = b + e < cj && c[e].score >= th;
+      for (int e = 0; e < 8; ++e) {
+        const int at = (e < 4 ? b : bh) + (e & 3);
+        const bool in = at < cj && c[e].score >= th;
         const uint32_t slot = agg_slot(&s_n, in);
         if (in && slot < (uint32_t)kSelList) {
           lkey[slot] = ordered_key(c[e].score);
@@ -228,20 +247,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         *u = key_at(i);
         return true;
       },
-      m, (uint32_t)K, hist, &s_digit, &s_above, &s_eq, &take, &eq);
+      m, (uint32_t)K, hist, s_res, &take, &eq);
   // Among entries equal to the K-th key, keep those with the `take` smallest
   // indices: the take-th largest complemented index is the cut.  When all of
   // them are needed there is nothing to cut.
   uint32_t cut = 0xFFFFFFFFu;
   if (take < eq) {
     uint32_t t2, e2;
+    __syncthreads();
     cut = ~radix_kth(
         [&](int i, uint32_t* u) {
           if (key_at(i) != kth) return false;
           *u = ~idx_at(i);
           return true;
         },
-        m, take, hist, &s_digit, &s_above, &s_eq, &t2, &e2);
+        m, take, hist, s_res, &t2, &e2);
   }
   auto winner = [&](int i, uint32_t* id) -> bool {
     const uint32_t u = key_at(i);
@@ -292,7 +312,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   for (int i = threadIdx.x; i < K; i += blockDim.x) o[i] = (int32_t)outv[i];
 }
 
-constexpr int kSelSmem = (2 * kSelList + (kBitmapWords > kSelOut ? kBitmapWords : kSelOut)) * 4;
+// Dynamic shared memory: the candidate key and index lists, then the bitmap
+// (one bit per key of the longest row, at most kBitmapWords words) or the sort
+// area of the long-row path (kSelOut words), whichever is larger.
+static int select_smem_bytes(int64_t max_nvis) {
+  int64_t words = (max_nvis + 31) / 32;
+  if (words > kBitmapWords) words = kBitmapWords;
+  if (words < kSelOut) words = kSelOut;
+  return (int)((2 * kSelList + words) * 4);
+}
 
 cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,
                           cudaStream_t stream) {
@@ -300,12 +328,13 @@ cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int 
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSelSmem);
+                                         select_smem_bytes((int64_t)kBitmapWords * 32));
     if (e != cudaSuccess) return e;
     attr = true;
   }
+  const int smem = select_smem_bytes(pos0 + rows);
   profile_before(DOSA_KERNEL_SELECT, stream);
-  select_kernel<<<(unsigned)rows, kSelThreads, kSelSmem, stream>>>(
+  select_kernel<<<(unsigned)rows, kSelThreads, smem, stream>>>(
       reinterpret_cast<const CandView*>(b.cand), b.seg_cap, b.cand_count, b.tau, pos0, K, out);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_SELECT, stream);

@@ -134,6 +134,34 @@ dosa_status dosa_index_topk(dosa_index_t h, const void* q, const float* q_scale,
                             int B, int K, int32_t* out_idx, void* workspace, size_t ws_bytes,
                             void* stream, dosa_stats* stats);
 
+/* Certified Top-K with the inputs and the output in HOST memory (page-locked
+ * for the copies to overlap the kernels; pageable memory works, serialised).
+ * q, q_scale, w, k, k_scale, out_idx are host pointers with the layouts of
+ * dosa_index_topk; seq_offsets as there.  The keys (and key scales) of every
+ * sequence are copied first; then the query rows stream through two device
+ * staging slots: while the kernels run on one chunk of rows, the next chunk's
+ * q, q_scale and w are copied in and the previous chunk's indices copied out,
+ * on a copy stream the handle creates on first use (per device).  The call is
+ * asynchronous on `stream` like the others: out_idx is complete when `stream`
+ * is; the host buffers must stay valid until then.  Same selection as
+ * dosa_index_topk.  Workspace (device): dosa_index_host_workspace_size.
+ * Errors as dosa_index_topk; DOSA_ERR_CUDA also when the copy stream cannot
+ * be created. */
+dosa_status dosa_index_topk_host(dosa_index_t h, const void* q, const float* q_scale,
+                                 const float* w, const void* k, const float* k_scale,
+                                 const int64_t* seq_offsets, int B, int K, int32_t* out_idx,
+                                 void* workspace, size_t ws_bytes, void* stream,
+                                 dosa_stats* stats);
+
+/* Device workspace of dosa_index_topk_host for Tq query rows, S_total keys
+ * over all sequences, at most S_max keys in one, and K; chunk_rows (0 =
+ * library choice, 16384) is the number of query rows per staging slot.  A
+ * call given less workspace than the default uses the most rows per slot
+ * that fit (at least 8). */
+dosa_status dosa_index_host_workspace_size(dosa_index_t h, int64_t Tq, int64_t S_total,
+                                           int64_t S_max, int K, int64_t chunk_rows,
+                                           size_t* bytes);
+
 /* The per-query certificate the certified path screens with (for inspection
  * and tests; the Top-K calls compute it internally).  cert_out: [Tq, 16] fp32,
  * code domain (for E4M3 the real-valued bound is q_scale[t] * k_scale[s] times

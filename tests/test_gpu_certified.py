@@ -213,3 +213,28 @@ def test_repair_pass_when_candidates_overflow(cuda_lib, screening):
     dense = to_numpy(idx.dense_topk(qd, None, wd, kd, None, so, K))
     assert np.array_equal(cert, dense)
     assert np.array_equal(cert, np.tile(np.arange(K, dtype=np.int32), (T, 1)))
+
+
+@pytest.mark.parametrize("case", [("prefill_128k_fp8", 203, 2600, 300), ("causal_1k_bf16", 300, 1900, 64)],
+                         ids=lambda c: c[0])
+def test_host_staged_call_equals_device_call(cuda_lib, case):
+    """dosa_index_topk_host: inputs and output in pinned host memory, query
+    rows streamed through two staging slots (a small workspace forces many
+    chunks, so both slots are reused); same indices as the device call."""
+    base, T, S, K = case
+    wl, x, xd = _inputs(base, T, S, K)
+    idx = binding.Index(wl.dtype, max_K=2048)
+    dev = to_numpy(idx.topk(*_args(xd, K)))
+    pin = {k: (v.contiguous().pin_memory() if torch.is_tensor(v) and k != "seq_offsets" else v)
+           for k, v in x.items()}
+    so = x["seq_offsets"]
+    ws = torch.zeros(idx.host_workspace_size(wl.T, wl.S, wl.S, K, chunk_rows=48),
+                     dtype=torch.uint8, device="cuda")
+    out, stats = idx.topk_host(*_args(pin, K), workspace=ws, stats=True)
+    assert out.device.type == "cpu"
+    assert np.array_equal(out.numpy(), dev)
+    assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
+    # again on the same workspace and stream (slots reused across calls)
+    out2 = idx.topk_host(*_args(pin, K), workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(out2.numpy(), dev)
