@@ -426,46 +426,87 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     cf[kCertOmega + j] = om;
     p.retained[i * 4 + j] = j < r ? R[j] : -1;
   }
-  // ---- F: residuals in place of the omitted heads (the coefficients are
-  // read before the barrier that precedes the Gram, which reuses their space) ----
-  for (int e = threadIdx.x; e < no * D; e += blockDim.x) {
-    const int h = O[e / D], c = e % D;
-    float x = qs[h][c];
-    for (int j = 0; j < r; ++j) x = fmaf(-(float)alpha_s[h][j], qs[R[j]][c], x);
-    qs[h][c] = x;
+  // ---- F: residuals in place of the omitted heads.  Thread c of each half
+  // of the CTA owns column c of every other omitted head; the retained heads'
+  // values of that column stay in registers (the coefficients are read before
+  // the barrier that precedes the Gram, which reuses their space). ----
+  {
+    const int c = threadIdx.x & (D - 1);
+    float qr[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) qr[j] = j < r ? qs[R[j]][c] : 0.f;
+    for (int k = threadIdx.x >> 7; k < no; k += kSetupThreads / D) {
+      const int h = O[k];
+      float x = qs[h][c];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (j < r) x = fmaf(-(float)alpha_s[h][j], qr[j], x);
+      qs[h][c] = x;
+    }
   }
   __syncthreads();
-  // ---- G: weighted residual Gram |[sqrt(w w') rho . rho']| and ||rho_h||,
-  // one pair (a >= b) per 8 threads ----
+  // ---- G: weighted residual Gram |[sqrt(w w') rho . rho']| and ||rho_h||:
+  // 4 x 4 blocks of the lower triangle, 8 threads per block (16 columns each)
+  // ----
   {
-    const int np = no * (no + 1) / 2;
+    const int nb = (no + 3) / 4, nblk = nb * (nb + 1) / 2;
     const int part = threadIdx.x & 7;
-    for (int base = 0; base < np; base += kSetupThreads / 8) {
+    for (int base = 0; base < nblk; base += kSetupThreads / 8) {
       const int task = base + (threadIdx.x >> 3);
-      int a = 0, b = 0;
-      if (task < np) {
-        a = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
-        while (a * (a + 1) / 2 > task) --a;
-        while ((a + 1) * (a + 2) / 2 <= task) ++a;
-        b = task - a * (a + 1) / 2;
-      }
-      const int ha = O[a], hb = O[b];
-      float v = 0.f;
-      if (task < np) {
+      int A = 0;
+      while ((A + 1) * (A + 2) / 2 <= task) ++A;
+      const int Bb = task - A * (A + 1) / 2;       // block (A, Bb), Bb <= A
+      float acc[4][4];
 #pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+      if (task < nblk) {
+        int ha[4], hb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ha[i] = O[min(4 * A + i, no - 1)];
+          hb[i] = O[min(4 * Bb + i, no - 1)];
+        }
+#pragma unroll 4
         for (int k = 0; k < D / 8; ++k) {
           const int c = part + 8 * k;
-          v = fmaf(qs[ha][c], qs[hb][c], v);
+          float xa[4], xb[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            xa[i] = qs[ha[i]][c];
+            xb[i] = qs[hb[i]][c];
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], xb[j], acc[i][j]);
         }
       }
-      v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-      v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-      v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-      if (part == 0 && task < np) {
-        const float g = fabsf(sqrtf(wv[ha] * wv[hb]) * v);
-        gt[a][b] = g;
-        gt[b][a] = g;
-        if (a == b) rn[ha] = sqrtf(v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float v = acc[i][j];
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+          acc[i][j] = v;
+        }
+      if (part == 0 && task < nblk) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int ra = 4 * A + i, cb = 4 * Bb + j;
+            if (ra < no && cb < no && cb <= ra) {
+              const int h1 = O[ra], h2 = O[cb];
+              const float g = fabsf(sqrtf(wv[h1] * wv[h2]) * acc[i][j]);
+              gt[ra][cb] = g;
+              gt[cb][ra] = g;
+              if (ra == cb) rn[h1] = sqrtf(acc[i][j]);
+            }
+          }
       }
     }
   }
