@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_128k_fp8", choices=sorted(WORKLOADS))
-    ap.add_argument("--path", choices=["certified", "dense"], default="certified")
+    ap.add_argument("--path", choices=["certified", "dense", "decode"], default="certified",
+                    help="decode: the decode-step call on a decode workload (decode_1m_fp8)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU baseline sample")
     ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
@@ -198,6 +199,24 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
         exact = stats["exact_pairs"] - stats.get("filtered_pairs", 0)
         work = (flops_per_pair * exact + 2 * wl.d * 8 * stats["screened_pairs"]) * steps
         name = "certified_kernel"
+    elif dom == "decode" and stats:
+        # seed + split-S scan + finish: every visible pair scored on the tensor
+        # cores, every key of the cache read once per call.  The bound is the
+        # slower of the two ideal times.
+        kbytes = wl.S * wl.d * (1 if dtype == "fp8" else 2) + (wl.S * 4 if dtype == "fp8" else 0)
+        flops = flops_per_pair * stats["exact_pairs"]
+        t_tensor = flops / (peak * 1e12)
+        t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
+        avg = ms / launches
+        if t_hbm >= t_tensor:
+            achieved = kbytes / (avg * 1e-3) / 1e9
+            return {"kernel": "decode_seed+decode_scan+decode_finish", "bound": "hbm",
+                    "achieved": round(achieved, 1), "peak": round(peaks["hbm_gbs"], 1),
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": None, "peak_source": f"{src}: hbm_gbs",
+                    "launches": launches, "avg_launch_ms": round(avg, 4)}
+        work = flops * steps
+        name = "decode_seed+decode_scan+decode_finish"
     else:
         return {"kernel": dom, "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
     achieved = work / (ms * 1e-3) / 1e12
@@ -320,14 +339,37 @@ def run_ours(args, world, rank, local):
     x = generate(rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, max_K=max(2048, wl.K), screening=args.screening)
     certified = args.path == "certified"
+    decode = args.path == "decode"
+    if decode and wl.decode_noise <= 0:
+        raise SystemExit("--path decode needs a decode workload (decode_1m_fp8)")
+    seeds = None
+    if wl.decode_noise > 0:
+        # decode workload: row 0 is the previous step, rows 1.. are timed; the
+        # previous step's selection (dense, untimed) seeds the decode call
+        from dataclasses import replace
+        m = wl.T - 1
+        one = lambda v: None if v is None else v[:1]
+        rest = lambda v: None if v is None else v[1:]
+        prev_so = [[0, 0, wl.q_pos0], [1, wl.S, 0]]
+        seeds = idx.dense_topk(one(x["q"]), one(x["q_scale"]), one(x["w"]), x["k"], x["k_scale"],
+                               prev_so, wl.K).expand(m, wl.K).contiguous()
+        x = {**x, "q": rest(x["q"]), "q_scale": rest(x["q_scale"]), "w": rest(x["w"]),
+             "positions": rest(x["positions"]), "seq_offsets": [[0, 0, wl.q_pos0 + 1], [m, wl.S, 0]]}
+        wl = replace(wl, name=f"{wl.name}[rows 1..{m}]", T=m, q_pos0=wl.q_pos0 + 1)
     so = x["seq_offsets"]
-    ws = torch.zeros(idx.workspace_size(wl.T, wl.S, wl.K, certified), dtype=torch.uint8,
-                     device="cuda")
+    if decode:
+        ws = torch.zeros(idx.decode_workspace_size(wl.T, wl.S, wl.K), dtype=torch.uint8,
+                         device="cuda")
+    else:
+        ws = torch.zeros(idx.workspace_size(wl.T, wl.S, wl.K, certified), dtype=torch.uint8,
+                         device="cuda")
     out = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
     call_args = (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], so, wl.K)
 
     def step(o=out, a=call_args):
-        if certified:
+        if decode:
+            idx.decode_topk(*a, seeds, out=o, workspace=ws)
+        elif certified:
             idx.topk(*a, out=o, workspace=ws)
         else:
             idx.dense_topk(*a, out=o, workspace=ws)
@@ -366,6 +408,8 @@ def run_ours(args, world, rank, local):
     stats = None
     if certified:
         _, stats = idx.topk(*call_args, out=out, workspace=ws, stats=True)
+    elif decode:
+        _, stats = idx.decode_topk(*call_args, seeds, out=out, workspace=ws, stats=True)
 
     # end to end through the public call with host buffers
     e2e = None
@@ -376,7 +420,25 @@ def run_ours(args, world, rank, local):
         h2d = sum(host[n].numel() * host[n].element_size() for n in names if host[n] is not None)
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         d2h = out_host.numel() * out_host.element_size()
-        if certified:
+        if decode:
+            # the step's inputs are the new rows (q, its scales, w) and the
+            # seeds; the key cache stays resident, as in serving
+            names = ["q", "q_scale", "w"]
+            h2d = sum(host[n].numel() * host[n].element_size() for n in names
+                      if host[n] is not None) + seeds.numel() * 4
+            dev_in = {n: (torch.empty_like(x[n]) if x[n] is not None else None) for n in names}
+            seeds_host = seeds.cpu().pin_memory()
+            seeds_dev = torch.empty_like(seeds)
+
+            def e2e_step():
+                for n in names:
+                    if host[n] is not None:
+                        dev_in[n].copy_(host[n], non_blocking=True)
+                seeds_dev.copy_(seeds_host, non_blocking=True)
+                idx.decode_topk(dev_in["q"], dev_in["q_scale"], dev_in["w"], x["k"], x["k_scale"],
+                                so, wl.K, seeds_dev, out=out, workspace=ws)
+                out_host.copy_(out, non_blocking=True)
+        elif certified:
             # the host-staged call: query chunks stream through two device slots,
             # copies overlapping the kernels
             sot = torch.as_tensor(so, dtype=torch.int64)

@@ -26,9 +26,10 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_index_scores", "dosa_reference_scores", "dosa_index_certificate",
            "dosa_index_dense_topk_static", "dosa_topk_rows", "dosa_check_device",
            "dosa_status_string", "dosa_profile_enable", "dosa_profile_reset",
-           "dosa_profile_read", "dosa_index_topk_host", "dosa_index_host_workspace_size")
+           "dosa_profile_read", "dosa_index_topk_host", "dosa_index_host_workspace_size",
+           "dosa_index_decode_topk", "dosa_index_decode_workspace_size")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
-           "certified": 5, "select": 6, "filter": 7}
+           "certified": 5, "select": 6, "filter": 7, "decode": 8}
 
 
 class DosaError(RuntimeError):
@@ -77,6 +78,9 @@ def load(path: str = LIB_PATH):
     lib.dosa_index_topk.argtypes = common + [ctypes.POINTER(Stats)]
     lib.dosa_index_dense_topk.argtypes = common
     lib.dosa_index_topk_host.argtypes = common + [ctypes.POINTER(Stats)]
+    lib.dosa_index_decode_topk.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ,
+                                           _P, ctypes.POINTER(Stats)]
+    lib.dosa_index_decode_workspace_size.argtypes = [_P, _I64, _I64, _I, ctypes.POINTER(_SZ)]
     lib.dosa_index_host_workspace_size.argtypes = [_P, _I64, _I64, _I64, _I, _I64,
                                                    ctypes.POINTER(_SZ)]
     lib.dosa_index_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64,
@@ -212,6 +216,28 @@ class Index:
             self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
             ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, K, _ptr(out), _ptr(workspace),
             workspace.numel(), _stream(), ctypes.byref(st) if stats else None))
+        return (out, st.as_dict()) if stats else out
+
+    def decode_workspace_size(self, Tq: int, S_max: int, K: int) -> int:
+        n = ctypes.c_size_t()
+        _check("dosa_index_decode_workspace_size",
+               self._lib.dosa_index_decode_workspace_size(self._h, Tq, S_max, K, ctypes.byref(n)))
+        return int(n.value)
+
+    def decode_topk(self, q, q_scale, w, k, k_scale, seq_offsets, K, seed_idx, out=None,
+                    workspace=None, stats: bool = False):
+        """Decode-step Top-K seeded by the previous step's selection seed_idx [Tq, K]."""
+        so, out = self._topk_args(q, q_scale, w, k, k_scale, seq_offsets, K, out)
+        if workspace is None:
+            S_max = int((so[1:, 1] - so[:-1, 1]).max())
+            workspace = torch.zeros(self.decode_workspace_size(q.shape[0], S_max, K),
+                                    dtype=torch.uint8, device=q.device)
+        seed = seed_idx.to(torch.int32).contiguous()
+        st = Stats()
+        _check("dosa_index_decode_topk", self._lib.dosa_index_decode_topk(
+            self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
+            ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, K, _ptr(seed), _ptr(out),
+            _ptr(workspace), workspace.numel(), _stream(), ctypes.byref(st) if stats else None))
         return (out, st.as_dict()) if stats else out
 
     def certificate(self, q, q_scale, w, k, k_scale, seq_offsets, workspace=None):

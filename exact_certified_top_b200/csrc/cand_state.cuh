@@ -62,27 +62,34 @@ struct Cand {
   int key;
 };
 
-// Sound lower edge of bin i: every score binned at >= i is >= the result.
-__device__ __forceinline__ float bin_edge(const QState& s, int i) {
-  const float iw = (float)i * s.w;
-  return fmaf((float)i, s.w, s.lo) - (fabsf(s.lo) + iw) * 0x1p-20f;
+// Bins of width w from lo: sound lower edge of bin i (every score binned at
+// >= i is >= the result), and the bin of a score (clamped to [0, kBins)).
+__device__ __forceinline__ float bin_edge_at(float lo, float w, int i) {
+  const float iw = (float)i * w;
+  return fmaf((float)i, w, lo) - (fabsf(lo) + iw) * 0x1p-20f;
 }
 
-__device__ __forceinline__ int bin_of(const QState& s, float score) {
-  float b = floorf((score - s.lo) * s.inv_w);
+__device__ __forceinline__ int bin_index(float lo, float inv_w, float score) {
+  float b = floorf((score - lo) * inv_w);
   b = fminf(fmaxf(b, 0.f), (float)(kBins - 1));
   return (int)b;
 }
 
-// Owner warp: highest bin whose suffix count reaches K -> its sound edge
-// (or -inf when fewer than K are counted).
-__device__ __forceinline__ float hist_threshold(const QState& s, int K, int lane) {
-  unsigned c[8], local = 0;
+__device__ __forceinline__ float bin_edge(const QState& s, int i) { return bin_edge_at(s.lo, s.w, i); }
+
+__device__ __forceinline__ int bin_of(const QState& s, float score) {
+  return bin_index(s.lo, s.inv_w, score);
+}
+
+// One warp: the highest bin whose suffix count (bins >= it) reaches K, or -1
+// when fewer than K are counted.  h points at kBins counts that other warps
+// may still be incrementing; any snapshot gives a sound answer because
+// counts only grow.
+// Counts c[0..7] are bins lane * 8 .. lane * 8 + 7.
+__device__ __forceinline__ int suffix_bin_of(const unsigned (&c)[8], int K, int lane) {
+  unsigned local = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    c[j] = *reinterpret_cast<const volatile unsigned*>(&s.hist[lane * 8 + j]);
-    local += c[j];
-  }
+  for (int j = 0; j < 8; ++j) local += c[j];
   unsigned suf = local;   // sum over lanes >= this one
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -102,9 +109,28 @@ __device__ __forceinline__ float hist_threshold(const QState& s, int K, int lane
     }
   }
   const unsigned who = __ballot_sync(0xFFFFFFFFu, best >= 0);
-  if (!who) return -INFINITY;
-  best = __shfl_sync(0xFFFFFFFFu, best, __ffs(who) - 1);
-  return bin_edge(s, best);
+  if (!who) return -1;
+  return __shfl_sync(0xFFFFFFFFu, best, __ffs(who) - 1);
+}
+
+// This lane's 8 counts of a histogram other warps may still be incrementing.
+__device__ __forceinline__ void load_bins(const unsigned* h, int lane, unsigned (&c)[8]) {
+  const volatile unsigned* v = h + lane * 8;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) c[j] = v[j];
+}
+
+__device__ __forceinline__ int suffix_bin(const unsigned* h, int K, int lane) {
+  unsigned c[8];
+  load_bins(h, lane, c);
+  return suffix_bin_of(c, K, lane);
+}
+
+// Owner warp: highest bin whose suffix count reaches K -> its sound edge
+// (or -inf when fewer than K are counted).
+__device__ __forceinline__ float hist_threshold(const QState& s, int K, int lane) {
+  const int best = suffix_bin(s.hist, K, lane);
+  return best < 0 ? -INFINITY : bin_edge(s, best);
 }
 
 // Owner warp, after a checkpoint barrier: finish warm-up (bin every candidate

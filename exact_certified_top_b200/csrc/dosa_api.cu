@@ -659,6 +659,119 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
   return DOSA_OK;
 }
 
+// ---- decode step ----------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+// Decode workspace: the header, then per query row the seed bitmap, the seed
+// bounds, counts, the shared histogram and threshold (all zeroed per call),
+// the selection inputs and the candidate list.  A row's list holds all its
+// visible keys, so it cannot overflow.
+struct DecodeLayout {
+  size_t bitmap, tau_key, smax_key, seed_count, dup, count, hist, tau_run, zero_end;
+  size_t cand_count, tau, cand, total;
+  int64_t words;
+  int64_t cap;
+};
+
+DecodeLayout decode_layout(int64_t Tq, int64_t S_max, int K) {
+  (void)K;
+  DecodeLayout L;
+  size_t off = kWsHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (size_t)round_up((int64_t)bytes, 256);
+    return at;
+  };
+  L.cap = round_up(S_max > 64 ? S_max : 64, 64);
+  L.words = (S_max + 31) / 32;
+  // zeroed per call: bitmap .. tau_run (tau_key is then set to all ones)
+  L.bitmap = take((size_t)Tq * L.words * 4);
+  L.tau_key = take((size_t)Tq * 4);
+  L.smax_key = take((size_t)Tq * 4);
+  L.seed_count = take((size_t)Tq * 4);
+  L.dup = take((size_t)Tq * 4);
+  L.count = take((size_t)Tq * 4);
+  L.hist = take((size_t)Tq * 256 * 4);
+  L.tau_run = take((size_t)Tq * 4);
+  L.zero_end = off;
+  L.cand_count = take((size_t)Tq * 16);
+  L.tau = take((size_t)Tq * 4);
+  L.cand = take((size_t)Tq * L.cap * 8);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+dosa_status dosa_index_decode_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max, int K,
+                                             size_t* bytes) {
+  const Handle* h = reinterpret_cast<const Handle*>(hh);
+  if (!h || !bytes || Tq < 0 || S_max < 0 || K < 1 || K > h->cfg.max_K)
+    return DOSA_ERR_INVALID_ARG;
+  *bytes = decode_layout(Tq, S_max, K).total;
+  return DOSA_OK;
+}
+
+dosa_status dosa_index_decode_topk(dosa_index_t hh, const void* q, const float* q_scale,
+                                   const float* w, const void* k, const float* k_scale,
+                                   const int64_t* seq_offsets, int B, int K,
+                                   const int32_t* seed_idx, int32_t* out_idx, void* workspace,
+                                   size_t ws_bytes, void* stream_, dosa_stats* stats) {
+  const Handle* h = reinterpret_cast<const Handle*>(hh);
+  dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, K, out_idx);
+  if (st != DOSA_OK) return st;
+  if (!seed_idx) return DOSA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DOSA_ERR_INVALID_ARG;
+  const int64_t Tq = seq_offsets[3 * B], S_max = max_keys(seq_offsets, B);
+  const DecodeLayout L = decode_layout(Tq, S_max, K);
+  if (ws_bytes < L.total) return DOSA_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, stream) != cudaSuccess ||
+      cudaMemsetAsync(ws + L.bitmap, 0, L.zero_end - L.bitmap, stream) != cudaSuccess ||
+      cudaMemsetAsync(ws + L.tau_key, 0xFF, (size_t)Tq * 4, stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
+  for (int b = 0; b < B; ++b) {
+    const SeqInfo s = seq_info(seq_offsets, b);
+    const SeqView v = make_view(h, q, q_scale, w, k, k_scale, s);
+    if (v.rows == 0) continue;
+    const int64_t r0 = s.q_start;
+    DecodeBuffers d;
+    d.words = L.words;
+    d.bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap) + r0 * L.words;
+    d.tau_key = reinterpret_cast<uint32_t*>(ws + L.tau_key) + r0;
+    d.smax_key = reinterpret_cast<uint32_t*>(ws + L.smax_key) + r0;
+    d.seed_count = reinterpret_cast<int*>(ws + L.seed_count) + r0;
+    d.dup = reinterpret_cast<int*>(ws + L.dup) + r0;
+    d.count = reinterpret_cast<int*>(ws + L.count) + r0;
+    d.hist = reinterpret_cast<unsigned*>(ws + L.hist) + r0 * 256;
+    d.tau_run = reinterpret_cast<uint32_t*>(ws + L.tau_run) + r0;
+    d.cand_count = reinterpret_cast<int*>(ws + L.cand_count) + r0 * 4;
+    d.tau = reinterpret_cast<float*>(ws + L.tau) + r0;
+    d.cand = ws + L.cand + (size_t)r0 * L.cap * 8;
+    d.cap = (int)L.cap;
+    d.counters = reinterpret_cast<WsHeader*>(ws)->counters;
+    d.err = &reinterpret_cast<WsHeader*>(ws)->error;
+    int32_t* out = out_idx + r0 * K;
+    if (launch_decode(*h, v, d, K, seed_idx + r0 * K, stream) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+    // selection over the candidate lists (one segment of cap entries per row)
+    CertBuffers sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.cand = d.cand;
+    sb.seg_cap = d.cap / 4;                 // rows are 4 * seg_cap apart; one segment used
+    sb.cand_count = d.cand_count;
+    sb.tau = d.tau;
+    if (launch_select(sb, v.rows, v.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+  }
+  if (stats) return read_stats(workspace, seq_offsets, B, stream, stats);
+  return DOSA_OK;
+}
+
 dosa_status dosa_index_certificate(dosa_index_t hh, const void* q, const float* q_scale,
                                    const float* w, const void* k, const float* k_scale,
                                    const int64_t* seq_offsets, int B, float* cert_out,

@@ -90,6 +90,26 @@ struct CertBuffers {
   int* err;
 };
 
+// Device buffers of a decode call (all inside the caller's workspace; per-row
+// arrays start at the sequence's first row).
+struct DecodeBuffers {
+  uint32_t* bitmap;      // [rows][words] seed de-duplication, zero on entry
+  int64_t words;
+  uint32_t* tau_key;     // [rows] ordered seed bound, 0xFFFFFFFF on entry
+  uint32_t* smax_key;    // [rows] ordered largest seed score, zero on entry
+  int* seed_count;       // [rows] zero on entry
+  int* dup;              // [rows] zero on entry
+  int* count;            // [rows] candidates appended, zero on entry
+  unsigned* hist;        // [rows][256] shared score histogram, zero on entry
+  uint32_t* tau_run;     // [rows] ordered shared threshold, zero on entry
+  int* cand_count;       // [rows][4] for the selection kernel
+  float* tau;            // [rows]
+  void* cand;            // [rows][cap] packed (score, key)
+  int cap;               // >= every row's visible keys, a multiple of 64
+  unsigned long long* counters;
+  int* err;
+};
+
 // ---- launches (each returns the cudaError_t of its launch) --------------------
 // Tensor-core scorer writing every visible score of rows [row0, row0+rows).
 cudaError_t launch_scores_tc(const Handle& h, const SeqView& v, float* scores, int64_t ld,
@@ -118,6 +138,9 @@ cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffer
 // Filter scorer (exact scores, threshold filter, no bounds) over a range.
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
                           StepRange steps, cudaStream_t stream);
+// Decode step: seed bound, split-S scan, per-row counts and repair list.
+cudaError_t launch_decode(const Handle& h, const SeqView& v, const DecodeBuffers& b, int K,
+                          const int32_t* seed, cudaStream_t stream);
 // Bytes of carried candidate state per query row.
 size_t qstate_bytes();
 cudaError_t launch_select(const CertBuffers& b, int64_t rows, int64_t pos0, int K, int32_t* out,

@@ -23,7 +23,7 @@ namespace dosa {
 constexpr int kSelThreads = 512;
 constexpr int kSelList = 4096;        // candidates >= tau held in shared memory
 constexpr int kSelOut = 4096;         // >= max K, power of two
-constexpr int kBitmapWords = 8192;    // rows of up to 262,144 keys use the bitmap
+constexpr int kBitmapWords = 32768;   // rows of up to 1,048,576 keys use the bitmap
 
 struct CandView {
   float score;
@@ -278,19 +278,49 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       if (winner(i, &id) && id < (uint32_t)nvis) atomicOr(&bm[id >> 5], 1u << (id & 31));
     }
     __syncthreads();
-    const int per = (nwords + blockDim.x - 1) / blockDim.x;
-    const int w0 = threadIdx.x * per, w1 = min(w0 + per, nwords);
+    // each warp owns a contiguous run of words, its lanes four consecutive
+    // words at a time (16-byte loads, no bank conflicts); a warp scan orders
+    // the bits within a run
+    const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int per = ((nwords + nwarps - 1) / nwarps + 127) & ~127;
+    const int w0 = (threadIdx.x >> 5) * per, w1 = min(w0 + per, nwords);
+    auto quad_at = [&](int w) -> uint4 {
+      if (w + 3 < w1) return *reinterpret_cast<const uint4*>(bm + w);
+      return make_uint4(w < w1 ? bm[w] : 0u, w + 1 < w1 ? bm[w + 1] : 0u,
+                        w + 2 < w1 ? bm[w + 2] : 0u, 0u);
+    };
     uint32_t c = 0;
-    for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
-    uint32_t at = block_exclusive_sum(c, scan);
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = bm[w];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        if (at < (uint32_t)K) o[at] = (int32_t)(w * 32 + b);
-        ++at;
+    for (int w = w0 + 4 * lane; w < w1; w += 128) {
+      const uint4 q = quad_at(w);
+      c += __popc(q.x) + __popc(q.y) + __popc(q.z) + __popc(q.w);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, off);
+    uint32_t base = block_exclusive_sum(lane == 0 ? c : 0u, scan);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    for (int wb = w0; wb < w1; wb += 128) {
+      const int w = wb + 4 * lane;
+      const uint4 q = w < w1 ? quad_at(w) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t pc = __popc(q.x) + __popc(q.y) + __popc(q.z) + __popc(q.w);
+      uint32_t inc = pc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+        if (lane >= off) inc += n;
       }
+      uint32_t at = base + inc - pc;
+      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t bits = words[e];
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (at < (uint32_t)K) o[at] = (int32_t)((w + e) * 32 + b);
+          ++at;
+        }
+      }
+      base += __shfl_sync(0xFFFFFFFFu, inc, 31);
     }
     return;
   }

@@ -44,6 +44,9 @@ class Workload:
     levels: int = 0             # 0, or 8 for integer-level quantisation
     seed: int = 0
     sink_frac: float = 0.01
+    # decode steps: rows 1.. are row 0 (the previous step) plus N(0, noise^2)
+    # per coordinate (w: plus N(0, (noise / 8)^2)), drawn before quantisation
+    decode_noise: float = 0.0
 
     @property
     def visible_pairs(self) -> int:
@@ -61,7 +64,15 @@ WORKLOADS = {
                              q_pos0=1048576 - 8192),
     "tight_64k_bf16_levels": Workload("tight_64k_bf16_levels", T=65536, S=65536, K=2048,
                                       lowrank_scale=0.1, neg_half=True, levels=8),
+    # decode step at ~1M cached keys: the last 5 rows of the sequence; row 0
+    # (position S - 5) is the previous step, whose selection seeds rows 1..4
+    # (a 4-row multi-token-prediction step)
+    "decode_1m_fp8": Workload("decode_1m_fp8", T=5, S=1048576, dtype="fp8", K=2048,
+                              q_pos0=1048576 - 5, decode_noise=0.3),
 }
+
+# Rows of a decode workload: row 0 is the previous step, rows 1.. are decoded.
+DECODE_PREV_ROWS = 1
 
 
 def small_case(base: str, T: int, S: int | None = None, **kw) -> Workload:
@@ -126,6 +137,9 @@ def generate(wl: Workload, device="cpu", chunk: int = 4096) -> dict:
         w = w.abs()
         neg = torch.argsort(torch.rand((T, H), generator=g, device=device), dim=1)[:, : H // 2]
         w.scatter_(1, neg, -w.gather(1, neg))
+    if wl.decode_noise > 0:
+        assert T <= max(1, chunk // 16), "decode workloads are a few rows"
+        w[1:] = w[0:1] + (wl.decode_noise / 8.0) * _randn(g, (T - 1, H), device)
 
     out = {"positions": torch.arange(wl.q_pos0, wl.q_pos0 + T, dtype=torch.int64, device=device),
            "seq_offsets": torch.tensor([[0, 0, wl.q_pos0], [T, S, 0]], dtype=torch.int64),
@@ -144,6 +158,8 @@ def generate(wl: Workload, device="cpu", chunk: int = 4096) -> dict:
         z = _randn(g, (n, H, 16), device)
         eps = _randn(g, (n, H, d), device)
         qf = mu_q + z @ A_q.T + 0.3 * eps
+        if wl.decode_noise > 0:
+            qf[1:] = qf[0:1] + wl.decode_noise * _randn(g, (n - 1, H, d), device)
         if wl.dtype == "fp8":
             q[t0:t0 + n], q_scale[t0:t0 + n] = _e4m3_per_token(qf)
         else:

@@ -162,6 +162,31 @@ dosa_status dosa_index_host_workspace_size(dosa_index_t h, int64_t Tq, int64_t S
                                            int64_t S_max, int K, int64_t chunk_rows,
                                            size_t* bytes);
 
+/* Decode-step Top-K: a few query rows per sequence (e.g. the next token, or a
+ * handful of multi-token-prediction rows) against the sequence's cached keys,
+ * seeded by the previous step's selection.  seed_idx: device [Tq, K] int32,
+ * indices relative to each sequence's first key (the previous step's out_idx
+ * for the same rows; -1 entries are ignored).  For each row the exact scores
+ * of its seed keys, lowered by a rounding margin, give a lower bound tau0 of
+ * its K-th largest score when the row has K distinct visible seeds; every
+ * visible key is then scored on the tensor cores with the key range split
+ * over all SMs, and only scores >= tau0 enter the selection.  Rows without K
+ * distinct visible seeds, or whose candidates exceed the list capacity
+ * (4 K, at least 4096), are rescored densely; at most 64 rows per sequence
+ * can be (more: DOSA_ERR_DEVICE_CHECK).  Returns exactly the selection of
+ * dosa_index_dense_topk.  Workspace: dosa_index_decode_workspace_size.
+ * Errors: INVALID_ARG also for a NULL seed_idx. */
+dosa_status dosa_index_decode_topk(dosa_index_t h, const void* q, const float* q_scale,
+                                   const float* w, const void* k, const float* k_scale,
+                                   const int64_t* seq_offsets, int B, int K,
+                                   const int32_t* seed_idx, int32_t* out_idx, void* workspace,
+                                   size_t ws_bytes, void* stream, dosa_stats* stats);
+
+/* Device workspace of dosa_index_decode_topk for Tq query rows (all
+ * sequences), at most S_max keys in one sequence, and K. */
+dosa_status dosa_index_decode_workspace_size(dosa_index_t h, int64_t Tq, int64_t S_max, int K,
+                                             size_t* bytes);
+
 /* The per-query certificate the certified path screens with (for inspection
  * and tests; the Top-K calls compute it internally).  cert_out: [Tq, 16] fp32,
  * code domain (for E4M3 the real-valued bound is q_scale[t] * k_scale[s] times
@@ -244,7 +269,8 @@ typedef enum {
   DOSA_KERNEL_CERTIFIED = 5,   /* seed scoring, screening, rescoring, writeback */
   DOSA_KERNEL_SELECT = 6,      /* selection over the packed candidates         */
   DOSA_KERNEL_FILTER = 7,      /* exact scoring + threshold filter, no bounds  */
-  DOSA_KERNEL_KINDS = 8
+  DOSA_KERNEL_DECODE = 8,      /* decode step: seed bound, split-S scan        */
+  DOSA_KERNEL_KINDS = 9
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

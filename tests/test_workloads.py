@@ -8,7 +8,8 @@ from oracle import decode_bf16, decode_e4m3
 
 def test_named_workloads_and_pairs():
     assert set(WORKLOADS) == {"causal_1k_bf16", "causal_16k_bf16", "prefill_128k_fp8",
-                              "chunk_1m_fp8", "tight_64k_bf16_levels"}
+                              "chunk_1m_fp8", "tight_64k_bf16_levels", "decode_1m_fp8"}
+    assert WORKLOADS["decode_1m_fp8"].visible_pairs == sum(1048576 - 5 + i + 1 for i in range(5))
     assert WORKLOADS["prefill_128k_fp8"].visible_pairs == 8_590_000_128
     assert WORKLOADS["causal_16k_bf16"].visible_pairs == 134_225_920
     assert WORKLOADS["chunk_1m_fp8"].visible_pairs == 8_556_384_256
