@@ -10,7 +10,7 @@
 // persistent CTA per SM with a TMA producer warp, an MMA warp and 8 epilogue
 // warps.  The epilogue differs: instead of storing every score it keeps the
 // candidate state of the item's 8 queries in shared memory (cand_state.cuh)
-// and appends only scores >= tau_t, refreshing tau_t every 4 key tiles.
+// and appends only scores >= tau_t, refreshing tau_t every 8 key tiles.
 //
 // A launch processes a range of steps of every item (work_items.cuh): the
 // warm-up tiles before screening starts, the rest of the items that the

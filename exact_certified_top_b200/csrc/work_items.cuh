@@ -13,7 +13,7 @@ namespace dosa {
 constexpr int kItemQueries = 8;
 // The epilogue warps meet (threshold refresh) every this many key tiles of an
 // item and at the end of the item's range.
-constexpr int kCkptTiles = 4;
+constexpr int kCkptTiles = 8;
 
 struct Geom {
   int64_t t0;        // absolute first row
