@@ -162,6 +162,9 @@ def clocks_stop(handle):
 # ---------------------------------------------------------------------------
 # roofline
 
+KERNELS_PER_RECORD = {"decode": 3}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -208,15 +211,20 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
         t_tensor = flops / (peak * 1e12)
         t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
         avg = ms / launches
+        traffic = _traffic_record("decode", wl)
+        traffic = None if traffic is None else round(traffic["dram_bytes_per_launch"])
         if t_hbm >= t_tensor:
             achieved = kbytes / (avg * 1e-3) / 1e9
             return {"kernel": "decode_seed+decode_scan+decode_finish", "bound": "hbm",
                     "achieved": round(achieved, 1), "peak": round(peaks["hbm_gbs"], 1),
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                    "traffic": None, "peak_source": f"{src}: hbm_gbs",
+                    "traffic": traffic, "peak_source": f"{src}: hbm_gbs",
                     "launches": launches, "avg_launch_ms": round(avg, 4)}
-        work = flops * steps
-        name = "decode_seed+decode_scan+decode_finish"
+        achieved = flops / (avg * 1e-3) / 1e12
+        return {"kernel": "decode_seed+decode_scan+decode_finish", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                "launches": launches, "avg_launch_ms": round(avg, 4)}
     else:
         return {"kernel": dom, "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
     achieved = work / (ms * 1e-3) / 1e12
@@ -227,9 +235,9 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
             "avg_launch_ms": round(ms / launches, 3)}
 
 
-def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
-    """DRAM bytes per launch from a committed ncu summary, scaled by pairs, or
-    None when no capture matches the current kernel source."""
+def _traffic_record(kernel: str, wl):
+    """The committed ncu DRAM-traffic record of a kernel, or None when there is
+    none or the kernel sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -237,13 +245,22 @@ def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
         rec = json.load(f).get(f"{kernel}:{wl.dtype}")
     if not rec or rec.get("source_sha") != _kernel_source_sha():
         return None
+    return rec
+
+
+def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
+    """DRAM bytes per launch from a committed ncu summary, scaled by pairs."""
+    rec = _traffic_record(kernel, wl)
+    if rec is None or "dram_bytes_per_pair" not in rec:
+        return None
     return round(rec["dram_bytes_per_pair"] * pairs_per_launch)
 
 
 def _kernel_source_sha():
     import hashlib
     h = hashlib.sha256()
-    for name in ("score_tc.cu", "certified.cu", "filter.cu", "cand_state.cuh", "work_items.cuh",
+    for name in ("score_tc.cu", "certified.cu", "filter.cu", "decode.cu", "cand_state.cuh",
+                 "work_items.cuh",
                  "score_epilogue.cuh", "dosa_device.cuh"):
         with open(os.path.join(ROOT, "exact_certified_top_b200", "csrc", name), "rb") as f:
             h.update(f.read())
@@ -403,7 +420,8 @@ def run_ours(args, world, rank, local):
 
     pairs = wl.visible_pairs
     value = job_value(pairs, world, ms)
-    launches = sum(n for n, _ in prof.values())
+    # a "decode" profile record spans three kernels (seed, scan, finish)
+    launches = sum(n * KERNELS_PER_RECORD.get(k, 1) for k, (n, _) in prof.items())
 
     stats = None
     if certified:
