@@ -354,7 +354,7 @@ def run_ours(args, world, rank, local):
     binding.load()
     wl = workload_of(args)
     x = generate(rank_workload(wl, rank), device="cuda")
-    idx = binding.Index(wl.dtype, max_K=max(2048, wl.K), screening=args.screening)
+    idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening)
     certified = args.path == "certified"
     decode = args.path == "decode"
     if decode and wl.decode_noise <= 0:

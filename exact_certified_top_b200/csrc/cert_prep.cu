@@ -202,8 +202,9 @@ __device__ __forceinline__ void decode16(const void* q, int64_t e, float* dst) {
 }
 
 struct SetupParams {
-  const void* q;          // [rows, 64, d] codes (absolute rows)
-  const float* w;         // [rows, 64]
+  const void* q;          // [rows, nh, d] codes (absolute rows)
+  const float* w;         // [rows, nh]
+  int nh;                 // heads per row: 32 or 64 (slots nh..63 are zero heads)
   const float* key_sum;   // [d] real-domain key sum of the sequence
   float inv_nkeys;        // 1 / number of keys of the sequence
   int64_t row0;           // first row of the chunk
@@ -220,7 +221,7 @@ __constant__ int8_t kPairB[10] = {0, 1, 2, 3, 1, 2, 3, 2, 3, 3};
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupParams p) {
-  constexpr int H = 64, D = kHeadDim;
+  constexpr int H = 64, D = kHeadDim;   // head slots; p.nh of them are real
   extern __shared__ float setup_dyn[];
   // code-domain heads, then residuals in place (padded rows); weighted residual Gram
   float(*qs)[kQPad] = reinterpret_cast<float(*)[kQPad]>(setup_dyn);
@@ -244,15 +245,22 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   const int64_t t = p.row0 + i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- A: decode q (16 codes per load), weights, mean key ----
+  // ---- A: decode q (16 codes per load), weights, mean key.  Slots past the
+  // row's heads hold zero heads with zero weight: neither positive nor
+  // negative, they join no list and add nothing. ----
   for (int e = threadIdx.x * 16; e < H * D; e += blockDim.x * 16) {
     float v[16];
-    decode16<kFp8>(p.q, t * H * D + e, v);
     const int h = e / D, c = e % D;
+    if (h < p.nh) {
+      decode16<kFp8>(p.q, t * p.nh * D + e, v);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = 0.f;
+    }
 #pragma unroll
     for (int k = 0; k < 16; ++k) qs[h][c + k] = v[k];
   }
-  if (threadIdx.x < H) wv[threadIdx.x] = p.w[t * H + threadIdx.x];
+  if (threadIdx.x < H) wv[threadIdx.x] = threadIdx.x < p.nh ? p.w[t * p.nh + threadIdx.x] : 0.f;
   if (threadIdx.x < D) kbar[threadIdx.x] = p.key_sum[threadIdx.x] * p.inv_nkeys;
   __syncthreads();
   // ---- B: ||q_h|| and q_h . k_mean, 4 threads per head ----
@@ -608,7 +616,7 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     __syncthreads();
   }
   // bound rows 0..3: the retained heads' own codes
-  const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (size_t)t * H * D * esz;
+  const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (size_t)t * p.nh * D * esz;
   for (int e = threadIdx.x; e < 4 * D * (int)esz; e += blockDim.x) {
     const int j = e / (D * esz), b = e % (D * esz);
     rows_out[e] = j < r ? qrow[(size_t)R[j] * D * esz + b] : 0;
@@ -671,6 +679,7 @@ cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* ke
   SetupParams p;
   p.q = v.q;
   p.w = v.w;
+  p.nh = v.H;
   p.key_sum = key_sum;
   p.inv_nkeys = 1.f / (float)v.S;
   p.row0 = v.row0;

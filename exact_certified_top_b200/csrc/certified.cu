@@ -76,7 +76,7 @@ struct CertCfg {
 };
 
 struct CertParams {
-  const float* w;          // [rows_total, 64] absolute rows
+  const float* w;          // [rows_total, H] absolute rows
   const float* q_scale;    // absolute rows (fp8)
   const float* k_scale;    // sequence base (fp8)
   const float* key_norm;   // [S] code-domain ||k||, rounded up
@@ -89,6 +89,7 @@ struct CertParams {
   int* err;
   int64_t row0, rows, pos0, S;   // chunk: absolute first row, rows, first position
   int n_items, K, seg_cap, seed_first, seed_last;
+  int H;                   // heads per query row: 32 or 64 (the MMA always sees 64)
   StepRange steps;         // what this launch processes
   int decide;              // 1: flag every item whose range ends before its last step
 };
@@ -108,7 +109,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "r"(taddr));
 }
 
-template <bool kFp8>
+// kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
+template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     certified_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap bmap,
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         mbar_arrive_expect_tx(q_full, C::kQBytes + C::kBBytes);
         for (int sub = 0; sub < C::kSub; ++sub) {
           for (int b = 0; b < C::kQRows / 256; ++b)
-            tma_load_2d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64,
-                        (int32_t)(g.t0 * C::kH + b * 256));
+            tma_load_3d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64, 0,
+                        (int32_t)(g.t0 + b * 4));
           tma_load_2d(sB + sub * C::kBSubBytes, &bmap, q_full, sub * 64,
                       (int32_t)(g.local0 * kBoundRows));
         }
@@ -451,7 +453,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             float sc = 0.f;
             if (mine) {
               const int64_t t = g.t0 + ql;
-              sc = head_reduce64_packed(x, p.w + t * C::kH);
+              sc = kHeads == 64 ? head_reduce64_packed(x, p.w + t * 64)
+                                : head_reduce32_packed(x, p.w + t * 32);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
             }
             n_exact += __popc(mk);
@@ -533,13 +536,17 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
                                     cudaStream_t stream) {
   using C = CertCfg<kFp8>;
   CUtensorMap qmap, bmap, kmap;
-  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+  if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
       !encode_rows_map(&bmap, b.bdir, kFp8, (uint64_t)v.rows * kBoundRows, C::kBRows) ||
       !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(certified_kernel<kFp8>,
+    cudaError_t e = cudaFuncSetAttribute(certified_kernel<kFp8, 64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(certified_kernel<kFp8, 32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -569,6 +576,7 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.rows = v.rows;
   p.pos0 = v.pos0;
   p.S = v.S;
+  p.H = v.H;
   p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
   p.K = K;
   p.seg_cap = b.seg_cap;
@@ -579,7 +587,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
-  certified_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
+  if (v.H == 64)
+    certified_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
+  else
+    certified_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_CERTIFIED, stream);
   return e;

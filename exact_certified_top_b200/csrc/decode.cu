@@ -79,6 +79,7 @@ struct SeedParams {
   const int32_t* seed;      // [rows, K] previous selection (sequence-relative, -1 padded)
   int64_t row0, rows, pos0, S;
   int K;
+  int H;                    // heads per query row (32: slots 32..63 are zero)
   uint32_t* bitmap;         // [rows][words], zero on entry
   int64_t words;
   uint32_t* tau_key;        // [rows] ordered keys, 0xFFFFFFFF on entry
@@ -94,7 +95,7 @@ struct SeedParams {
 // group add their head partial sums by shuffles.
 template <bool kFp8>
 __global__ void __launch_bounds__(256) decode_seed_kernel(const SeedParams p) {
-  constexpr int H = 64, D = kHeadDim, P = D + 1;
+  constexpr int H = 64, D = kHeadDim, P = D + 1;   // head slots; p.H of them are real
   extern __shared__ float seed_dyn[];
   float(*qf)[P] = reinterpret_cast<float(*)[P]>(seed_dyn);
   float(*kf)[P] = reinterpret_cast<float(*)[P]>(seed_dyn + H * P);
@@ -114,10 +115,14 @@ __global__ void __launch_bounds__(256) decode_seed_kernel(const SeedParams p) {
   constexpr int KV = kSeedKeys * KC / 256;   // 16-byte loads per thread (seed keys)
   {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                                      t * (int64_t)(H * D * EB));
+                                                      t * (int64_t)(p.H * D * EB));
+    const int nvec = p.H * D * EB / 16;
     uint4 u[QV];
 #pragma unroll
-    for (int i = 0; i < QV; ++i) u[i] = __ldg(src + threadIdx.x + i * 256);
+    for (int i = 0; i < QV; ++i) {
+      const int e16 = threadIdx.x + i * 256;
+      u[i] = e16 < nvec ? __ldg(src + e16) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
     for (int i = 0; i < QV; ++i) {
       float f[PER];
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(256) decode_seed_kernel(const SeedParams p) {
       for (int c = 0; c < PER; ++c) qf[(e + c) / D][(e + c) % D] = f[c];
     }
   }
-  if (threadIdx.x < H) wv[threadIdx.x] = p.w[t * H + threadIdx.x];
+  if (threadIdx.x < H) wv[threadIdx.x] = threadIdx.x < p.H ? p.w[t * p.H + threadIdx.x] : 0.f;
   if (threadIdx.x < kSeedKeys) {
     const int j = j0 + threadIdx.x;
     int idx = j < p.K ? p.seed[row * (int64_t)p.K + j] : -1;
@@ -268,6 +273,7 @@ struct ScanParams {
   const float* k_scale;      // the sequence's first key
   int64_t row0, rows, pos0, S;
   int n_items, parts, K;
+  int H;                     // heads per query row: 32 or 64 (the MMA always sees 64)
   const uint32_t* tau_key;   // [rows] from decode_seed
   const uint32_t* smax_key;  // [rows] from decode_seed
   const int* seed_count;
@@ -353,7 +359,8 @@ __device__ __forceinline__ Unit scan_unit(const ScanParams& p, int u) {
   return x;
 }
 
-template <bool kFp8>
+// kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
+template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
     decode_scan_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap kmap, const ScanParams p) {
@@ -423,7 +430,7 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
         if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
         mbar_arrive_expect_tx(q_full, C::kQBytes);
         for (int sub = 0; sub < C::kSub; ++sub)
-          tma_load_2d(sQ + sub * C::kQSubBytes, &qmap, q_full, sub * 64, (int32_t)(x.t0 * C::kH));
+          tma_load_3d(sQ + sub * C::kQSubBytes, &qmap, q_full, sub * 64, 0, (int32_t)x.t0);
         inflight_q = it & 1;
         ++it;
         for (int j = x.tile_lo; j < x.tile_hi; ++j, ++kc) {
@@ -502,7 +509,8 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
       const int64_t r = x.local0 + (valid ? sub : 0);
       const int64_t pos = x.pos_first + sub;
       const RowBins b = row_bins(p, r);
-      const float* wq = p.w + (x.t0 + (valid ? sub : 0)) * C::kH;
+      const float* wq = p.w + (x.t0 + (valid ? sub : 0)) * kHeads;
+      constexpr bool h64 = kHeads == 64;
       float qs = 1.f;
       if constexpr (kFp8) qs = __ldg(p.q_scale + x.t0 + (valid ? sub : 0));
       // Appends trail the scores by kHold - 1 tiles: tile j's kept scores wait
@@ -553,13 +561,15 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
         HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         tmem_ld32_async(col, v);
         tmem_wait_ld(v);
-        head_accumulate32(acc, v, wq);
-        tmem_ld32_async(col + 32, v);
-        tmem_wait_ld(v);
+        if (h64) {
+          head_accumulate32(acc, v, wq);
+          tmem_ld32_async(col + 32, v);
+          tmem_wait_ld(v);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        head_accumulate32(acc, v, wq + 32);
+        head_accumulate32(acc, v, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
         if (!valid) continue;
         float sc = head_total(acc);
         if constexpr (kFp8) sc *= qs * sk;
@@ -714,6 +724,7 @@ static cudaError_t launch_decode_impl(const Handle& h, const SeqView& v, const D
   sp.pos0 = v.pos0;
   sp.S = v.S;
   sp.K = K;
+  sp.H = v.H;
   sp.bitmap = b.bitmap;
   sp.words = b.words;
   sp.tau_key = b.tau_key;
@@ -735,12 +746,15 @@ static cudaError_t launch_decode_impl(const Handle& h, const SeqView& v, const D
   if (e != cudaSuccess) return e;
   // scan
   CUtensorMap qmap, kmap;
-  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+  if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
       !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(decode_scan_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_scan_kernel<kFp8, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_scan_kernel<kFp8, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -756,6 +770,7 @@ static cudaError_t launch_decode_impl(const Handle& h, const SeqView& v, const D
   p.rows = v.rows;
   p.pos0 = v.pos0;
   p.S = v.S;
+  p.H = v.H;
   p.n_items = (int)((v.rows + kDecRows - 1) / kDecRows);
   // about one unit per SM (the key pipeline restarts at each unit), at least
   // 16 key tiles per unit
@@ -778,7 +793,10 @@ static cudaError_t launch_decode_impl(const Handle& h, const SeqView& v, const D
   p.err = b.err;
   const int units = p.n_items * p.parts;
   const int grid = units < sms ? units : sms;
-  decode_scan_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  if (v.H == 64)
+    decode_scan_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  else
+    decode_scan_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_finish_kernel<<<(unsigned)((v.rows + 3) / 4), 128, 0, stream>>>(p, b.cand_count, b.tau);

@@ -97,6 +97,7 @@ SeqView make_view(const Handle* h, const void* q, const float* q_scale, const fl
   v.rows = s.q_end - s.q_start;
   v.pos0 = s.q_pos0;
   v.S = s.k_end - s.k_start;
+  v.H = h->cfg.H;
   return v;
 }
 
@@ -251,7 +252,7 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
       cfg->screening > 2)
     return DOSA_ERR_INVALID_ARG;
-  if (cfg->d != kHeadDim || cfg->H != 64) return DOSA_ERR_UNSUPPORTED;
+  if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
   if (!h) return DOSA_ERR_INVALID_ARG;
   h->cfg = *cfg;
@@ -478,9 +479,9 @@ HostLayout host_layout(const Handle* h, int64_t Tq, int64_t S_total, int64_t S_m
     so += (size_t)round_up((int64_t)bytes, 256);
     return at;
   };
-  H.slot_q = take_slot((size_t)rows * 64 * kHeadDim * esz);
+  H.slot_q = take_slot((size_t)rows * h->cfg.H * kHeadDim * esz);
   H.slot_qs = take_slot(fp8 ? (size_t)rows * 4 : 0);
-  H.slot_w = take_slot((size_t)rows * 64 * 4);
+  H.slot_w = take_slot((size_t)rows * h->cfg.H * 4);
   H.slot_out = take_slot((size_t)rows * K * 4);
   H.slot[0] = take(so);
   H.slot[1] = take(so);
@@ -574,7 +575,7 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
   cudaStream_t main = static_cast<cudaStream_t>(stream_), cpy = h->copy_stream;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool fp8 = h->cfg.dtype == DOSA_FP8_E4M3;
-  const size_t esz = elem_bytes(h), qrow = (size_t)64 * kHeadDim * esz;
+  const size_t esz = elem_bytes(h), qrow = (size_t)h->cfg.H * kHeadDim * esz;
   const CertBuffers buf = cert_buffers(h, H.L, ws, H.Tc);
   uint8_t* dk = ws + H.keys;
   float* dks = fp8 ? reinterpret_cast<float*>(ws + H.kscale) : nullptr;
@@ -611,7 +612,7 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
                               cudaMemcpyHostToDevice, cpy)) &&
            (!fp8 || ok(cudaMemcpyAsync(sb + H.slot_qs, q_scale + t0, (size_t)ch.rows * 4,
                                        cudaMemcpyHostToDevice, cpy))) &&
-           ok(cudaMemcpyAsync(sb + H.slot_w, w + t0 * 64, (size_t)ch.rows * 64 * 4,
+           ok(cudaMemcpyAsync(sb + H.slot_w, w + t0 * h->cfg.H, (size_t)ch.rows * h->cfg.H * 4,
                               cudaMemcpyHostToDevice, cpy)) &&
            ok(cudaEventRecord(h->ev_loaded[slot], cpy));
   };
@@ -633,6 +634,7 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
     c.rows = ch.rows;
     c.pos0 = si.q_pos0 + ch.r0;
     c.S = si.k_end - si.k_start;
+    c.H = h->cfg.H;
     int32_t* dout = reinterpret_cast<int32_t*>(sb + H.slot_out);
     if (ch.b != prev_b) {
       if (launch_key_prep(*h, c.k, c.k_scale, c.S, buf.key_norm, buf.key_sum, main) !=
@@ -806,6 +808,7 @@ static dosa_status scores_common(dosa_index_t hh, const void* q, const float* q_
   v->rows = rows;
   v->pos0 = pos0;
   v->S = S;
+  v->H = h->cfg.H;
   return DOSA_OK;
 }
 

@@ -44,6 +44,7 @@ struct SeqView {
   int64_t rows;           // number of rows
   int64_t pos0;           // position of row0 among the sequence's keys
   int64_t S;              // keys of the sequence
+  int H;                  // heads per query row: 32 or 64
 };
 
 struct Handle {
@@ -66,6 +67,10 @@ void profile_after(int kind, cudaStream_t stream);
 PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder();
 // 2-D map over `rows` rows of d = 128 elements (bf16 or fp8 codes), 128-byte
 // swizzle, boxes of one 128-byte row segment x box_rows rows (score_tc.cu).
+// Queries as a 3-D tensor [rows][H][d] read in boxes of 4 rows x 64 head
+// slots x one 128-byte row: with H = 32 the slots 32..63 lie outside the
+// tensor and arrive as zeros, so every kernel sees 64 heads per row.
+bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H);
 bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
                      uint32_t box_rows);
 

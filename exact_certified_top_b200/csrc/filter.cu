@@ -59,10 +59,12 @@ struct FilterParams {
   int* err;
   int64_t row0, rows, pos0, S;
   int n_items, K, seg_cap, seed_first, seed_last;
+  int H;                   // heads per query row: 32 or 64 (the MMA always sees 64)
   StepRange steps;         // what this launch processes
 };
 
-template <bool kFp8>
+// kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
+template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
     filter_kernel(const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap kmap, const FilterParams p) {
@@ -132,8 +134,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
         mbar_arrive_expect_tx(q_full, C::kQBytes);
         for (int sub = 0; sub < C::kSub; ++sub)
           for (int b = 0; b < C::kQRows / 256; ++b)
-            tma_load_2d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64,
-                        (int32_t)(g.t0 * C::kH + b * 256));
+            tma_load_3d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64, 0,
+                        (int32_t)(g.t0 + b * 4));
         inflight_q = it & 1;
         ++it;
         for (int ti = rg.begin; ti < rg.end; ++ti, ++kc) {
@@ -265,8 +267,9 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       const int qa = sub, qb = C::kQPerGroup + sub;
       const bool va = qa < g.nq, vb = qb < g.nq;
       const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
-      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * C::kH;
-      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * C::kH;
+      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * kHeads;
+      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * kHeads;
+      constexpr bool h64 = kHeads == 64;
       float qsa = 1.f, qsb = 1.f;
       if constexpr (kFp8) {
         qsa = __ldg(p.q_scale + g.t0 + (va ? qa : 0));
@@ -298,13 +301,15 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           tmem_ld32_async(col, x);
           tmem_wait_ld(x);
-          head_accumulate32(acc, x, wq);
-          tmem_ld32_async(col + 32, x);
-          tmem_wait_ld(x);
+          if (h64) {
+            head_accumulate32(acc, x, wq);
+            tmem_ld32_async(col + 32, x);
+            tmem_wait_ld(x);
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          head_accumulate32(acc, x, wq + 32);
+          head_accumulate32(acc, x, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
           if (grp ? vb : va) {
             QState& q = st[grp ? qb : qa];
             float sc = head_total(acc);
@@ -363,12 +368,16 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
                                       int K, StepRange steps, cudaStream_t stream) {
   using C = FilterCfg<kFp8>;
   CUtensorMap qmap, kmap;
-  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+  if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
       !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(filter_kernel<kFp8>,
+    cudaError_t e = cudaFuncSetAttribute(filter_kernel<kFp8, 64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(filter_kernel<kFp8, 32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -396,6 +405,7 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.rows = v.rows;
   p.pos0 = v.pos0;
   p.S = v.S;
+  p.H = v.H;
   p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
   p.K = K;
   p.seg_cap = b.seg_cap;
@@ -405,7 +415,10 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_FILTER, stream);
-  filter_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  if (v.H == 64)
+    filter_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  else
+    filter_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_FILTER, stream);
   return e;

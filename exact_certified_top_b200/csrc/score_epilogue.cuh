@@ -73,6 +73,12 @@ __device__ __forceinline__ float head_total(const HeadAcc2& a) {
   return 0.5f * ((a.c01.x + a.c01.y) + (a.c23.x + a.c23.y));
 }
 
+__device__ __forceinline__ float head_reduce32_packed(const float* x, const float* __restrict__ w) {
+  HeadAcc2 a = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  head_accumulate32(a, x, w);
+  return head_total(a);
+}
+
 __device__ __forceinline__ float head_reduce64_packed(const float* x, const float* __restrict__ w) {
   HeadAcc2 a = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   head_accumulate32(a, x, w);

@@ -56,6 +56,7 @@ struct ScoreParams {
   int64_t ld;
   int64_t row0, rows, pos0, S;
   int n_items;
+  int H;                 // heads per query row: 32 or 64 (the MMA always sees 64)
   int* err;
   // Row-list mode (rows repaired after a candidate-list overflow): item i scores
   // the single row row0 + row_list[i] into output row i; the number of items
@@ -94,7 +95,8 @@ __device__ __forceinline__ ItemGeom item_geom(const ScoreParams& p, int item) {
   return g;
 }
 
-template <bool kFp8>
+// kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
+template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap kmap, ScoreParams p) {
@@ -162,8 +164,8 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
         mbar_arrive_expect_tx(q_full, C::kQBytes);
         for (int sub = 0; sub < C::kSub; ++sub)
           for (int b = 0; b < C::kQRows / 256; ++b)
-            tma_load_2d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64,
-                        (int32_t)(g.t0 * C::kH + b * 256));
+            tma_load_3d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64, 0,
+                        (int32_t)(g.t0 + b * 4));
         inflight_q = it & 1;
         for (int j = 0; j < g.nkt; ++j, ++kc) {
           const int st = kc % C::kKeyStages;
@@ -247,8 +249,9 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
       const int qa = sub, qb = C::kQPerGroup + sub;
       const bool va = qa < g.nq, vb = qb < g.nq;
       const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
-      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * C::kH;
-      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * C::kH;
+      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * kHeads;
+      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * kHeads;
+      constexpr bool h64 = kHeads == 64;
       float qsa = 1.f, qsb = 1.f;
       if constexpr (kFp8) {
         qsa = __ldg(p.q_scale + g.t0 + (va ? qa : 0));
@@ -278,13 +281,15 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
           HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
           tmem_ld32_async(col, v);
           tmem_wait_ld(v);
-          head_accumulate32(acc, v, wq);
-          tmem_ld32_async(col + 32, v);
-          tmem_wait_ld(v);
+          if (h64) {
+            head_accumulate32(acc, v, wq);
+            tmem_ld32_async(col + 32, v);
+            tmem_wait_ld(v);
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          head_accumulate32(acc, v, wq + 32);
+          head_accumulate32(acc, v, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
           if (grp ? vb : va) {
             float sc = head_total(acc);
             if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
@@ -320,18 +325,37 @@ bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows
   return r == CUDA_SUCCESS;
 }
 
+bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H) {
+  auto enc = get_tensor_map_encoder();
+  if (!enc || (H != 32 && H != 64)) return false;
+  const uint64_t esz = fp8 ? 1 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * esz, (cuuint64_t)H * kHeadDim * esz};
+  const cuuint32_t box[3] = {(cuuint32_t)(fp8 ? 128 : 64), 64, 4};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         3, const_cast<void*>(q), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <bool kFp8>
 static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int* err,
                                cudaStream_t stream, const int* row_list = nullptr,
                                const int* row_count = nullptr, int list_cap = 0) {
   using C = ScoreCfg<kFp8>;
   CUtensorMap qmap, kmap;
-  if (!encode_rows_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows) * C::kH, 256) ||
+  if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
       !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<kFp8>,
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<kFp8, 64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(score_tc_kernel<kFp8, 32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -350,6 +374,7 @@ static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int*
   p.rows = v.rows;
   p.pos0 = v.pos0;
   p.S = v.S;
+  p.H = v.H;
   p.n_items = (int)((v.rows + kQueryTile - 1) / kQueryTile);
   p.err = err;
   p.row_list = row_list;
@@ -359,7 +384,10 @@ static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int*
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_SCORE, stream);
-  score_tc_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  if (v.H == 64)
+    score_tc_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  else
+    score_tc_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_SCORE, stream);
   return e;

@@ -60,6 +60,9 @@ WORKLOADS = {
     "causal_1k_bf16": Workload("causal_1k_bf16", T=1024, S=1024, K=256),
     "causal_16k_bf16": Workload("causal_16k_bf16", T=16384, S=16384, K=2048),
     "prefill_128k_fp8": Workload("prefill_128k_fp8", T=131072, S=131072, dtype="fp8", K=2048),
+    # the same prefill with a 32-head indexer (the GLM-style shape)
+    "prefill_128k_fp8_h32": Workload("prefill_128k_fp8_h32", T=131072, S=131072, H=32,
+                                     dtype="fp8", K=2048),
     "chunk_1m_fp8": Workload("chunk_1m_fp8", T=8192, S=1048576, dtype="fp8", K=2048,
                              q_pos0=1048576 - 8192),
     "tight_64k_bf16_levels": Workload("tight_64k_bf16_levels", T=65536, S=65536, K=2048,

@@ -75,7 +75,9 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
  * margin_log2 = -12, screening = 2. */
 typedef struct {
-  int H;            /* indexer heads per query (multiple of 4, <= 64)          */
+  int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
+                       read each query row into 64 head slots (the other 32
+                       arrive as zeros) and reduce only the 32 real heads.   */
   int d;            /* head dimension (128 in this build)                       */
   dosa_dtype dtype; /* storage type of q and k                                  */
   int max_K;        /* largest K the handle will be called with (<= 4096)      */
@@ -111,7 +113,7 @@ void dosa_index_config_default(dosa_index_config* cfg);
 
 /* Validate cfg and create a handle (host memory only; it holds the config and
  * per-device kernel attributes).  Errors: INVALID_ARG for NULL or out-of-range
- * fields, UNSUPPORTED for d != 128 or H not a multiple of 4 in [4, 64]. */
+ * fields, UNSUPPORTED for d != 128 or H other than 32 or 64. */
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out);
 
 /* Free a handle (NULL is accepted). */

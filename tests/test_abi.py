@@ -46,6 +46,15 @@ def test_config_default_and_create(lib):
     lib.dosa_index_destroy(None)
 
 
+def test_create_accepts_32_heads(lib):
+    cfg = binding.Config()
+    lib.dosa_index_config_default(ctypes.byref(cfg))
+    cfg.H = 32
+    h = ctypes.c_void_p()
+    assert lib.dosa_index_create(ctypes.byref(cfg), ctypes.byref(h)) == 0 and h.value
+    lib.dosa_index_destroy(h)
+
+
 @pytest.mark.parametrize("field,value,code", [("d", 64, 2), ("H", 48, 2), ("max_K", 0, 1),
                                               ("r", 5, 1), ("G", 3, 1), ("margin_log2", 0, 1),
                                               ("dtype", 7, 1), ("screening", 3, 1)])

@@ -8,7 +8,9 @@ from oracle import decode_bf16, decode_e4m3
 
 def test_named_workloads_and_pairs():
     assert set(WORKLOADS) == {"causal_1k_bf16", "causal_16k_bf16", "prefill_128k_fp8",
-                              "chunk_1m_fp8", "tight_64k_bf16_levels", "decode_1m_fp8"}
+                              "prefill_128k_fp8_h32", "chunk_1m_fp8", "tight_64k_bf16_levels",
+                              "decode_1m_fp8"}
+    assert WORKLOADS["prefill_128k_fp8_h32"].H == 32
     assert WORKLOADS["decode_1m_fp8"].visible_pairs == sum(1048576 - 5 + i + 1 for i in range(5))
     assert WORKLOADS["prefill_128k_fp8"].visible_pairs == 8_590_000_128
     assert WORKLOADS["causal_16k_bf16"].visible_pairs == 134_225_920
@@ -22,6 +24,8 @@ def test_deterministic_and_shapes():
     assert a["q"].shape == (64, 64, 128) and a["k"].shape == (64, 128) and a["w"].shape == (64, 64)
     assert torch.equal(a["q"], b["q"]) and torch.equal(a["k"], b["k"]) and torch.equal(a["w"], b["w"])
     assert a["q"].dtype == torch.bfloat16 and a["q_scale"] is None
+    h32 = generate(small_case("prefill_128k_fp8_h32", 16))
+    assert h32["q"].shape == (16, 32, 128) and h32["w"].shape == (16, 32)
 
 
 def test_fp8_codes_finite_and_scale_absmax():
