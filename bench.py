@@ -48,6 +48,9 @@ def parse_args():
                     help="budget of the oracle CPU baseline sample")
     ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
                     help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
+    ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
+                    help="certified path: packed candidates >= threshold (default), or every "
+                         "exact score into a dense matrix and its dense Top-K (ablation)")
     ap.add_argument("--tail-rows", type=int, default=0,
                     help="profile only the last N query rows of the workload (same keys)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -307,8 +310,10 @@ def oracle_sample(x, wl, budget_s: float):
 
 # ---------------------------------------------------------------------------
 
-def config_of(wl, path, world, screening=None):
+def config_of(wl, path, world, screening=None, writeback=None):
     extra = {"screening": screening} if screening is not None else {}
+    if writeback is not None:
+        extra["writeback"] = writeback
     return {"workload": wl.name, "T": wl.T, "S": wl.S, "H": wl.H, "d": wl.d, "K": wl.K,
             "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, **extra,
             "parallelism": f"rows x{world}",
@@ -354,7 +359,8 @@ def run_ours(args, world, rank, local):
     binding.load()
     wl = workload_of(args)
     x = generate(rank_workload(wl, rank), device="cuda")
-    idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening)
+    idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
+                        sparse_writeback=int(args.writeback == "sparse"))
     certified = args.path == "certified"
     decode = args.path == "decode"
     if decode and wl.decode_noise <= 0:
@@ -504,7 +510,8 @@ def run_ours(args, world, rank, local):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": wl.dtype, "data": "synthetic (seeded low-rank + sink generator)",
                 "config": config_of(wl, args.path, world,
-                                    args.screening if args.path == "certified" else None),
+                                    args.screening if args.path == "certified" else None,
+                                    args.writeback if args.path == "certified" else None),
                 "roofline": roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "kernels": {k: {"launches": n, "ms": round(t, 3)} for k, t in

@@ -29,7 +29,8 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_profile_read", "dosa_index_topk_host", "dosa_index_host_workspace_size",
            "dosa_index_decode_topk", "dosa_index_decode_workspace_size")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
-           "certified": 5, "select": 6, "filter": 7, "decode": 8}
+           "certified": 5, "select": 6, "filter": 7, "decode": 8,
+           "fill": 9}
 
 
 class DosaError(RuntimeError):
@@ -42,7 +43,8 @@ class Config(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("d", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("max_K", ctypes.c_int), ("seed_first", ctypes.c_int),
                 ("seed_last", ctypes.c_int), ("r", ctypes.c_int), ("G", ctypes.c_int),
-                ("margin_log2", ctypes.c_int), ("screening", ctypes.c_int)]
+                ("margin_log2", ctypes.c_int), ("screening", ctypes.c_int),
+                ("sparse_writeback", ctypes.c_int)]
 
 
 class Stats(ctypes.Structure):

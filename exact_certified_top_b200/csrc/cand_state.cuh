@@ -265,6 +265,7 @@ struct PublishOut {
   int* repair_list;    // rows whose list overflowed (rescored densely)
   int* repair_count;
   int repair_cap;
+  int dense;           // the selection reads a dense score matrix: no repair needed
   int* err;
 };
 
@@ -276,7 +277,7 @@ __device__ __forceinline__ void publish_query(const QState& q, const PublishOut&
 #pragma unroll
   for (int j = 0; j < kSegs; ++j) cc[j] = over ? -1 : q.seg[j];
   o.tau[q.row] = q.tau;
-  if (over) {
+  if (over && !o.dense) {
     const int r = atomicAdd(o.repair_count, 1);
     if (r < o.repair_cap) o.repair_list[r] = (int)q.row;
     else record_error(o.err, kDevBounds);

@@ -90,6 +90,8 @@ struct CertParams {
   int64_t row0, rows, pos0, S;   // chunk: absolute first row, rows, first position
   int n_items, K, seg_cap, seed_first, seed_last;
   int H;                   // heads per query row: 32 or 64 (the MMA always sees 64)
+  float* dense;            // dense writeback (ablation): [chunk rows, dense_ld], or null
+  int64_t dense_ld;
   StepRange steps;         // what this launch processes
   int decide;              // 1: flag every item whose range ends before its last step
 };
@@ -456,6 +458,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
               sc = kHeads == 64 ? head_reduce64_packed(x, p.w + t * 64)
                                 : head_reduce32_packed(x, p.w + t * 32);
               if constexpr (kFp8) sc *= __ldg(p.q_scale + t) * sk;
+              if (p.dense && s <= q.pos) p.dense[q.row * p.dense_ld + s] = sc;
             }
             n_exact += __popc(mk);
             const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
@@ -569,7 +572,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
+  p.out.dense = b.dense != nullptr;
   p.out.err = b.err;
+  p.dense = b.dense;
+  p.dense_ld = b.dense_ld;
   p.counters = b.counters;
   p.err = b.err;
   p.row0 = v.row0;

@@ -134,6 +134,7 @@ struct CertLayout {
   size_t key_norm, key_sum, repair_list, repair_count, repair_scores, fixed;
   size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
   int seg_cap;
+  int64_t dense_ld; // dense writeback: the score matrix's row length (0 when sparse)
 };
 
 CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
@@ -154,6 +155,8 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   // bound rows, record, retained, list, count, tau, carried state, item flag
   L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
               (size_t)L.seg_cap * 4 * 8 + 4 * 4 + 4 + qstate_bytes() + 1;
+  L.dense_ld = h->cfg.sparse_writeback ? 0 : round_up(S_max > 1 ? S_max : 1, 64);
+  L.per_row += (size_t)L.dense_ld * 4;
   return L;
 }
 
@@ -181,6 +184,8 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.tau = reinterpret_cast<float*>(take((size_t)Tc * 4));
   b.qstate = take((size_t)Tc * qstate_bytes());
   b.item_flag = reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4));
+  b.dense = L.dense_ld ? reinterpret_cast<float*>(take((size_t)Tc * L.dense_ld * 4)) : nullptr;
+  b.dense_ld = L.dense_ld;
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
   b.err = &reinterpret_cast<WsHeader*>(ws)->error;
   return b;
@@ -188,7 +193,7 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
 
 // Padding the per-row arrays of a chunk may need (each starts 256-aligned),
 // plus the item-flag array's extra entry.
-constexpr size_t kCertPad = 8 * 256 + 4;
+constexpr size_t kCertPad = 9 * 256 + 4;
 
 // Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
 int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
@@ -241,6 +246,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->G = 2;
   cfg->margin_log2 = -12;
   cfg->screening = 2;
+  cfg->sparse_writeback = 1;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -250,7 +256,7 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   if (cfg->max_K < 1 || cfg->max_K > 4096) return DOSA_ERR_INVALID_ARG;
   if (cfg->seed_first < 0 || cfg->seed_last < 0 || cfg->r < 0 || cfg->r > 4 || cfg->G < 0 ||
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
-      cfg->screening > 2)
+      cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -390,6 +396,9 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
                               int32_t* out, cudaStream_t stream) {
   if (cudaMemsetAsync(b.repair_count, 0, sizeof(int), stream) != cudaSuccess)
     return DOSA_ERR_CUDA;
+  // dense writeback (ablation): pairs the scorers never write (rejected) stay -inf
+  if (b.dense && launch_fill(b.dense, c.rows * b.dense_ld, -INFINITY, stream) != cudaSuccess)
+    return DOSA_ERR_CUDA;
   // screening 0: the filter scorer alone; 1: the certified scorer alone;
   // 2: warm-up by the filter scorer, a probe of kProbeSteps screened steps,
   // then each item finished by the scorer its probe chose
@@ -408,6 +417,13 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
         launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
         launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream) != cudaSuccess)
       return DOSA_ERR_CUDA;
+  }
+  if (b.dense) {
+    // the dense Top-K of every exact score; no list can need a repair
+    return launch_topk_rows(b.dense, b.dense_ld, nullptr, c.pos0 + 1, b.dense_ld, c.rows, K, out,
+                            K, stream) == cudaSuccess
+               ? DOSA_OK
+               : DOSA_ERR_CUDA;
   }
   if (launch_select(b, c.rows, c.pos0, K, out, stream) != cudaSuccess) return DOSA_ERR_CUDA;
   // rows whose candidate list overflowed: dense rescoring of just those rows

@@ -91,6 +91,8 @@ struct CertBuffers {
   int repair_cap;
   float* repair_scores;  // [repair_cap, S]
   int seg_cap;           // entries per candidate segment
+  float* dense;          // [rows, dense_ld] every exact score (dense writeback), or null
+  int64_t dense_ld;
   unsigned long long* counters;
   int* err;
 };
@@ -159,6 +161,8 @@ cudaError_t launch_scores_ref(const Handle& h, const SeqView& v, float* scores, 
                               cudaStream_t stream);
 // Per-row radix Top-K.  Row i has n_i = row_len ? row_len[i] : (len0 + i) entries
 // (clipped to max_len).
+// p[0..n) = v.
+cudaError_t launch_fill(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int64_t* row_len,
                              int64_t len0, int64_t max_len, int64_t rows, int K, int32_t* out,
                              int64_t out_ld, cudaStream_t stream);

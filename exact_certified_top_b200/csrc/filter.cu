@@ -60,6 +60,8 @@ struct FilterParams {
   int64_t row0, rows, pos0, S;
   int n_items, K, seg_cap, seed_first, seed_last;
   int H;                   // heads per query row: 32 or 64 (the MMA always sees 64)
+  float* dense;            // dense writeback (ablation): [chunk rows, dense_ld], or null
+  int64_t dense_ld;
   StepRange steps;         // what this launch processes
 };
 
@@ -318,6 +320,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             int& cnt = grp ? cnt_b : cnt_a;
             n_cand += append_candidates(q, grp ? lb : la, p.seg_cap, cnt,
                                         s <= (grp ? pos_b : pos_a) && sc >= tau, sc, s, lane);
+            if (p.dense && s <= (grp ? pos_b : pos_a))
+              p.dense[(g.local0 + (grp ? qb : qa)) * p.dense_ld + s] = sc;
           }
         }
         if (!ok) break;
@@ -398,6 +402,9 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
+  p.out.dense = b.dense != nullptr;
+  p.dense = b.dense;
+  p.dense_ld = b.dense_ld;
   p.out.err = b.err;
   p.counters = b.counters;
   p.err = b.err;

@@ -126,6 +126,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(
   }
 }
 
+__global__ void fill_kernel(float* __restrict__ p, int64_t n, float v) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+cudaError_t launch_fill(float* p, int64_t n, float v, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t blocks = (n + 255) / 256;
+  profile_before(DOSA_KERNEL_FILL, stream);
+  fill_kernel<<<(unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms), 256, 0, stream>>>(p, n, v);
+  const cudaError_t e = cudaGetLastError();
+  profile_after(DOSA_KERNEL_FILL, stream);
+  return e;
+}
+
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int64_t* row_len, int64_t len0,
                              int64_t max_len, int64_t rows, int K, int32_t* out, int64_t out_ld,
                              cudaStream_t stream) {

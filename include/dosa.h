@@ -73,7 +73,7 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
- * margin_log2 = -12, screening = 2. */
+ * margin_log2 = -12, screening = 2, sparse_writeback = 1. */
 typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
@@ -88,11 +88,17 @@ typedef struct {
   int margin_log2;  /* soundness margin 2^margin_log2 * sum|w|||q|| * ||k||     */
   int screening;    /* 1: screen every key tile with the certificate; 2: adaptive
                        (every tile of 8 queries is screened over its first key
-                       tiles; where that rejected under 1/32 of 4096 or more
+                       tiles; where that rejected under 1/32 of 2048 or more
                        screened pairs, the rest of its keys is scored exactly
                        without bounds, else screening goes on to the end);
                        0: never (ablation).  The selection is exact in every
                        mode.                                                    */
+  int sparse_writeback; /* 1 (default): only scores >= the running threshold
+                       are written, as packed (score, key) candidates, and the
+                       selection reads those; 0 (ablation): every exact score
+                       is also written into a dense [rows, keys] matrix of the
+                       chunk (rejected pairs as -inf) and the selection is the
+                       dense Top-K of that matrix.  Same result either way.   */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */
@@ -272,7 +278,8 @@ typedef enum {
   DOSA_KERNEL_SELECT = 6,      /* selection over the packed candidates         */
   DOSA_KERNEL_FILTER = 7,      /* exact scoring + threshold filter, no bounds  */
   DOSA_KERNEL_DECODE = 8,      /* decode step: seed bound, split-S scan        */
-  DOSA_KERNEL_KINDS = 9
+  DOSA_KERNEL_FILL = 9,        /* dense-writeback ablation: matrix set to -inf */
+  DOSA_KERNEL_KINDS = 10
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

@@ -238,3 +238,24 @@ def test_host_staged_call_equals_device_call(cuda_lib, case):
     out2 = idx.topk_host(*_args(pin, K), workspace=ws)
     torch.cuda.synchronize()
     assert np.array_equal(out2.numpy(), dev)
+
+
+@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
+@pytest.mark.parametrize("case", [("prefill_128k_fp8", 203, 2600, 300),
+                                  ("tight_64k_bf16_levels", 157, 2100, 512)],
+                         ids=lambda c: c[0])
+def test_dense_writeback_ablation_equals_dense(cuda_lib, case, screening):
+    """sparse_writeback = 0: every exact score also goes to a dense chunk
+    matrix (rejected pairs -inf) and the selection is its dense Top-K.  The
+    indices must equal the sparse path's and the dense path's."""
+    base, T, S, K = case
+    wl, x, xd = _inputs(base, T, S, K)
+    dense = to_numpy(binding.Index(wl.dtype, max_K=2048).dense_topk(*_args(xd, K)))
+    idx = binding.Index(wl.dtype, max_K=2048, screening=screening, sparse_writeback=0)
+    out, stats = idx.topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out), dense)
+    assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
+    # a workspace for few rows: many chunks, each with its own dense matrix
+    ws = torch.zeros(idx.workspace_size(24, wl.S, K, True), dtype=torch.uint8, device="cuda")
+    out2 = idx.topk(*_args(xd, K), workspace=ws)
+    assert np.array_equal(to_numpy(out2), dense)
