@@ -46,7 +46,7 @@ __all__ = [
     "decode_bf16", "decode_e4m3", "dequantize", "indexer_scores", "select_topk",
     "dense_topk", "nnls_retained", "Certificate", "certificate_setup", "upper_bound",
     "soundness_margin", "seed_mask", "certified_topk_row", "certified_topk",
-    "key_mean",
+    "key_mean", "key_block_stats", "block_upper_bound",
 ]
 
 # ----------------------------------------------------------------------------
@@ -281,6 +281,36 @@ def upper_bound(cert: Certificate, q_t: np.ndarray, k: np.ndarray) -> np.ndarray
         ub = ub + np.maximum(k @ q_t[cert.retained].T, 0.0) @ cert.omega
     for g in range(cert.u.shape[0]):
         ub = ub - np.maximum(k @ cert.u[g], 0.0)
+    return ub
+
+
+def key_block_stats(k_block: np.ndarray) -> tuple[np.ndarray, float, float]:
+    """A block of keys summarised by a ball: its center (the mean key), the
+    radius max_s ||k_s - center|| and the largest key norm."""
+    k_block = np.asarray(k_block, np.float64)
+    c = k_block.mean(axis=0)
+    r = float(np.max(np.linalg.norm(k_block - c, axis=1)))
+    n = float(np.max(np.linalg.norm(k_block, axis=1)))
+    return c, r, n
+
+
+def block_upper_bound(cert: Certificate, q_t: np.ndarray, center: np.ndarray, radius: float,
+                      max_norm: float) -> float:
+    """One bound for every key of a block ("DOSA: Dots Sparse Attention",
+    Daily Paper Cast transcript, future work: extending the certificate from
+    single keys to key blocks, cutting scoring and key-access costs).  Every key of
+    the block is k = center + e with ||e|| <= radius, so for any vector v
+    v.k lies in [v.center - ||v|| radius, v.center + ||v|| radius].  ReLU is
+    nondecreasing, omega_j >= 0 and ||k|| <= max_norm, hence each term of the
+    per-key bound (upper_bound) is at most its block counterpart:
+      UB_B = sum_j omega_j ReLU(q_j.c + ||q_j|| r) + beta max_norm
+             - sum_g ReLU(u_g.c - ||u_g|| r)  >=  UB(s)  for every s in B."""
+    ub = cert.beta * max_norm
+    for j, h in enumerate(cert.retained):
+        ub += cert.omega[j] * max(float(q_t[h] @ center) + float(np.linalg.norm(q_t[h])) * radius,
+                                  0.0)
+    for g in range(cert.u.shape[0]):
+        ub -= max(float(cert.u[g] @ center) - float(np.linalg.norm(cert.u[g])) * radius, 0.0)
     return ub
 
 

@@ -160,3 +160,49 @@ def test_certified_prunes_when_heads_are_redundant():
                              seed_first=8, seed_last=32)
     assert np.array_equal(res["idx"], dense_topk(q_t[None], w_t[None], k, np.array([S - 1]), K)[0])
     assert res["rejected"] > 0.8 * res["visible"]
+
+
+@pytest.mark.parametrize("r,G", [(0, 0), (2, 1), (4, 2)])
+def test_block_bound_dominates_every_key_of_the_block(r, G):
+    """UB_B >= UB(s) >= I(s) for every key of the block, including keys on the
+    ball's boundary along the head and aggregate directions (where the
+    per-key bound is largest)."""
+    from oracle import block_upper_bound, key_block_stats
+    rng = np.random.default_rng(100 + r * 10 + G)
+    for _ in range(6):
+        q_t, w_t, k = _instance(rng)
+        cert = certificate_setup(q_t, w_t, key_mean(k), r, G)
+        center = rng.standard_normal(q_t.shape[1])
+        block = center + 0.3 * rng.standard_normal((128, q_t.shape[1]))
+        dirs = np.vstack([q_t, -q_t] + ([cert.u, -cert.u] if cert.u.size else []))
+        norms = np.linalg.norm(dirs, axis=1)
+        dirs = dirs[norms > 0] / norms[norms > 0, None]       # empty groups have u = 0
+        c, rad, n = key_block_stats(block)
+        block = np.vstack([block, c + rad * dirs])       # boundary points, same ball
+        c2, rad2, n2 = key_block_stats(block)
+        ubb = block_upper_bound(cert, q_t, c2, rad2, n2)
+        ub = upper_bound(cert, q_t, block)
+        I = indexer_scores(q_t, w_t, block)
+        assert np.all(ubb >= ub - 1e-9 * (1 + np.abs(ub)))
+        assert np.all(ub >= I - 1e-9 * (1 + np.abs(I)))
+        # and it is no looser than the center's bound plus the radius terms
+        slack = rad2 * (cert.omega @ np.linalg.norm(q_t[cert.retained], axis=1)
+                        if cert.retained.size else 0.0)
+        slack += rad2 * float(np.sum(np.linalg.norm(cert.u, axis=1))) if cert.u.size else 0.0
+        slack += cert.beta * (n2 - np.linalg.norm(c2))
+        ubc = upper_bound(cert, q_t, c2[None, :])[0]
+        assert ubb <= ubc + slack + 1e-9 * (1 + abs(ubc))
+
+
+def test_block_bound_of_a_point_block_is_the_key_bound():
+    """A block whose keys all coincide has radius 0 and max norm ||k||: its
+    bound is the per-key bound of that key (closed form)."""
+    from oracle import block_upper_bound, key_block_stats
+    rng = np.random.default_rng(7)
+    q_t, w_t, k = _instance(rng)
+    cert = certificate_setup(q_t, w_t, key_mean(k), 4, 2)
+    for s in (0, 5, 37):
+        c, rad, n = key_block_stats(np.repeat(k[s:s + 1], 128, axis=0))
+        assert rad == pytest.approx(0.0, abs=1e-12)
+        assert block_upper_bound(cert, q_t, c, rad, n) == pytest.approx(
+            upper_bound(cert, q_t, k[s:s + 1])[0], rel=1e-12, abs=1e-12)
