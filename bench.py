@@ -48,6 +48,8 @@ def parse_args():
                     help="budget of the oracle CPU baseline sample")
     ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
                     help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
+    ap.add_argument("--block-bound", type=int, choices=[0, 1], default=1,
+                    help="certified path: skip key tiles whose key-block bound rules them out")
     ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
                     help="certified path: packed candidates >= threshold (default), or every "
                          "exact score into a dense matrix and its dense Top-K (ablation)")
@@ -360,7 +362,8 @@ def run_ours(args, world, rank, local):
     wl = workload_of(args)
     x = generate(rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
-                        sparse_writeback=int(args.writeback == "sparse"))
+                        sparse_writeback=int(args.writeback == "sparse"),
+                        block_bound=args.block_bound)
     certified = args.path == "certified"
     decode = args.path == "decode"
     if decode and wl.decode_noise <= 0:

@@ -92,9 +92,22 @@ struct CertParams {
   int H;                   // heads per query row: 32 or 64 (the MMA always sees 64)
   float* dense;            // dense writeback (ablation): [chunk rows, dense_ld], or null
   int64_t dense_ld;
+  const int* step_list;    // per item, the steps left by block screening, or null
+  const int* step_count;
+  int step_cap;
   StepRange steps;         // what this launch processes
   int decide;              // 1: flag every item whose range ends before its last step
 };
+
+// The steps an item processes in this launch: its range, or the list block
+// screening left of it (never empty when the range is not).
+__device__ __forceinline__ int steps_of(const CertParams& p, const Range& rg, int item) {
+  return p.step_list ? p.step_count[item] : rg.end - rg.begin;
+}
+__device__ __forceinline__ int step_at(const CertParams& p, const Range& rg, int item, int i) {
+  return p.step_list ? p.step_list[(int64_t)item * p.step_cap + i] : rg.begin + i;
+}
+
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -210,7 +223,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         }
         inflight_q = it & 1;
         ++it;
-        for (int ti = rg.begin; ti < rg.end; ++ti, ++kc) {
+        const int n_steps = steps_of(p, rg, item);
+        for (int i = 0; i < n_steps; ++i, ++kc) {
           const int s_ = kc % C::kKeyStages;
           const uint32_t rnd = kc / C::kKeyStages;
           if (!mbar_wait(&k_empty[s_], (rnd & 1) ^ 1, s_abort, p.err)) {
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&k_full[s_], C::kKeyStageBytes);
-          const int j = tile_at(ti, g.n_tiles);
+          const int j = tile_at(step_at(p, rg, item, i), g.n_tiles);
           for (int sub = 0; sub < C::kSub; ++sub)
             tma_load_2d(sK + s_ * C::kKeyStageBytes + sub * C::kKeySubBytes, &kmap, &k_full[s_],
                         sub * 64, j * kKeyTile);
@@ -248,7 +262,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         ++it;
         tc_fence_after();
         const uint32_t b_bound = smem_u32(sB);
-        const int n = rg.end - rg.begin;
+        const int n = steps_of(p, rg, item);
         // bound tiles use the same running index as key stages (kc)
         auto issue_bound = [&](int i) -> bool {
           const uint32_t c = kc + i, s_ = c % C::kKeyStages;
@@ -328,7 +342,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
       const Range rg = item_steps(p.steps, p.item_flag, g, item);
       if (rg.end <= rg.begin) continue;
-      const int n = rg.end - rg.begin;
+      const int n = steps_of(p, rg, item);
       // owner: this item's state of query slot ew (fresh, or carried over)
       {
         QState& s = st[ew];
@@ -361,7 +375,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
         cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * 2 + half].seg[quad]);
       unsigned long long it_scr = 0, it_rej = 0;   // this warp's counts, this item
       auto key_of = [&](int i) -> int64_t {
-        return (int64_t)tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        return (int64_t)tile_at(step_at(p, rg, item, i), g.n_tiles) * kKeyTile + quad * 32 + lane;
       };
       // ---- bound evaluation of step i ----
       auto bound_eval = [&](int i) -> bool {
@@ -536,7 +550,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
 template <bool kFp8>
 static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
                                     int K, StepRange steps, int decide,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, int use_list) {
   using C = CertCfg<kFp8>;
   CUtensorMap qmap, bmap, kmap;
   if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
@@ -590,6 +604,9 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.seed_last = h.cfg.seed_last;
   p.steps = steps;
   p.decide = decide;
+  p.step_list = use_list ? b.step_list : nullptr;
+  p.step_count = use_list ? b.step_count : nullptr;
+  p.step_cap = b.step_cap;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
@@ -603,10 +620,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
 }
 
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             StepRange steps, int decide, cudaStream_t stream) {
+                             StepRange steps, int decide, cudaStream_t stream, int use_list) {
   if (h.cfg.dtype == DOSA_FP8_E4M3)
-    return launch_cert_impl<true>(h, v, b, K, steps, decide, stream);
-  return launch_cert_impl<false>(h, v, b, K, steps, decide, stream);
+    return launch_cert_impl<true>(h, v, b, K, steps, decide, stream, use_list);
+  return launch_cert_impl<false>(h, v, b, K, steps, decide, stream, use_list);
 }
 
 size_t certified_smem_bytes(bool fp8) {

@@ -131,7 +131,8 @@ int seg_capacity(int K, int64_t S_max) {
 // Workspace of the certified path: a fixed part (header, key norms, key sum,
 // repair area) and Tc rows of per-query state.
 struct CertLayout {
-  size_t key_norm, key_sum, repair_list, repair_count, repair_scores, fixed;
+  size_t key_norm, key_sum, repair_list, repair_count, repair_scores, blk, fixed;
+  int step_cap;     // block screening: steps per item list (key tiles of S_max), or 0
   size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
   int seg_cap;
   int64_t dense_ld; // dense writeback: the score matrix's row length (0 when sparse)
@@ -151,12 +152,18 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.repair_list = take(kRepairRows * 4);
   L.repair_count = take(4);
   L.repair_scores = take((size_t)kRepairRows * S_max * 4);
+  // block screening covers sequences of up to 8192 key tiles (1M keys)
+  L.step_cap = h->cfg.block_bound ? (int)((S_max + kKeyTile - 1) / kKeyTile) : 0;
+  if (L.step_cap > 8192) L.step_cap = 0;
+  L.blk = take((size_t)L.step_cap * kBlkFloats * 4);
   L.fixed = off;
   // bound rows, record, retained, list, count, tau, carried state, item flag
   L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
               (size_t)L.seg_cap * 4 * 8 + 4 * 4 + 4 + qstate_bytes() + 1;
   L.dense_ld = h->cfg.sparse_writeback ? 0 : round_up(S_max > 1 ? S_max : 1, 64);
   L.per_row += (size_t)L.dense_ld * 4;
+  // step lists: one per work item of 8 rows (plus the count)
+  L.per_row += ((size_t)L.step_cap * 4 + 4 + 7) / 8;
   return L;
 }
 
@@ -186,6 +193,11 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.item_flag = reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4));
   b.dense = L.dense_ld ? reinterpret_cast<float*>(take((size_t)Tc * L.dense_ld * 4)) : nullptr;
   b.dense_ld = L.dense_ld;
+  b.blk = L.step_cap ? reinterpret_cast<float*>(ws + L.blk) : nullptr;
+  b.step_cap = L.step_cap;
+  b.step_list = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * L.step_cap * 4))
+                           : nullptr;
+  b.step_count = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
   b.err = &reinterpret_cast<WsHeader*>(ws)->error;
   return b;
@@ -193,7 +205,7 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
 
 // Padding the per-row arrays of a chunk may need (each starts 256-aligned),
 // plus the item-flag array's extra entry.
-constexpr size_t kCertPad = 9 * 256 + 4;
+constexpr size_t kCertPad = 11 * 256 + 4 + 16 * 1024 * 4;
 
 // Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
 int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
@@ -247,6 +259,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->margin_log2 = -12;
   cfg->screening = 2;
   cfg->sparse_writeback = 1;
+  cfg->block_bound = 1;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -256,7 +269,8 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   if (cfg->max_K < 1 || cfg->max_K > 4096) return DOSA_ERR_INVALID_ARG;
   if (cfg->seed_first < 0 || cfg->seed_last < 0 || cfg->r < 0 || cfg->r > 4 || cfg->G < 0 ||
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
-      cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1)
+      cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
+      cfg->block_bound < 0 || cfg->block_bound > 1)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -369,7 +383,8 @@ static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const flo
     const SeqView v = make_view(h, q, q_scale, w, k, k_scale, s);
     if (v.rows == 0) continue;
     if (launch_key_prep(*h, v.k, v.k_scale, v.S, buf.key_norm, buf.key_sum, stream) !=
-        cudaSuccess)
+            cudaSuccess ||
+        (buf.blk && launch_block_prep(*h, v.k, v.k_scale, v.S, buf.blk, stream) != cudaSuccess))
       return DOSA_ERR_CUDA;
     for (int64_t r = 0; r < v.rows; r += Tc) {
       SeqView c = v;
@@ -404,18 +419,32 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
   // then each item finished by the scorer its probe chose
   constexpr int kAll = 0x3FFFFFFF;
   const int mode = h->cfg.screening;
+  // With the key-block certificate, the certified scorer's last range is
+  // first screened tile by tile as a whole (block_screen) and then processes
+  // the steps left.
+  const bool blk = b.blk != nullptr;
+  const int W = warmup_steps(K), P = W + kProbeSteps;
   if (mode == 0) {
     if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
       return DOSA_ERR_CUDA;
   } else if (mode == 1) {
-    if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
+    if (!blk) {
+      if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
+        return DOSA_ERR_CUDA;
+    } else if (launch_certified(*h, c, b, K, StepRange{0, P, -1}, 0, stream) != cudaSuccess ||
+               launch_block_screen(*h, c, b, StepRange{P, kAll, -1}, stream) != cudaSuccess ||
+               launch_certified(*h, c, b, K, StepRange{P, kAll, -1}, 0, stream, 1) !=
+                   cudaSuccess) {
       return DOSA_ERR_CUDA;
+    }
   } else {
-    const int W = warmup_steps(K), P = W + kProbeSteps;
     if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
         launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
         launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
-        launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream) != cudaSuccess)
+        (blk && launch_block_screen(*h, c, b, StepRange{P, kAll, kItemScreen}, stream) !=
+                    cudaSuccess) ||
+        launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream, blk ? 1 : 0) !=
+            cudaSuccess)
       return DOSA_ERR_CUDA;
   }
   if (b.dense) {
@@ -451,6 +480,7 @@ static dosa_status read_stats(const void* workspace, const int64_t* seq_offsets,
   stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
   stats->candidates = (int64_t)hdr.counters[kCntCandidates];
   stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
+  stats->block_skipped_pairs = (int64_t)hdr.counters[kCntBlockSkipped];
   if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
   return DOSA_OK;
 }
@@ -654,7 +684,8 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
     int32_t* dout = reinterpret_cast<int32_t*>(sb + H.slot_out);
     if (ch.b != prev_b) {
       if (launch_key_prep(*h, c.k, c.k_scale, c.S, buf.key_norm, buf.key_sum, main) !=
-          cudaSuccess)
+              cudaSuccess ||
+          (buf.blk && launch_block_prep(*h, c.k, c.k_scale, c.S, buf.blk, main) != cudaSuccess))
         return DOSA_ERR_CUDA;
       prev_b = ch.b;
     }

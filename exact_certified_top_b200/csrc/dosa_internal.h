@@ -30,6 +30,7 @@ enum CounterId : int {
   kCntCandidates = 4,
   kCntOverflow = 5,
   kCntFiltered = 6,
+  kCntBlockSkipped = 7,
 };
 constexpr size_t kWsHeaderBytes = 256;
 
@@ -93,6 +94,10 @@ struct CertBuffers {
   int seg_cap;           // entries per candidate segment
   float* dense;          // [rows, dense_ld] every exact score (dense writeback), or null
   int64_t dense_ld;
+  float* blk;            // [key tiles][kBlkFloats] key-block balls, or null (no block bound)
+  int* step_list;        // [rows / 8 + 1][step_cap] steps left after block screening
+  int* step_count;       // [rows / 8 + 1]
+  int step_cap;
   unsigned long long* counters;
   int* err;
 };
@@ -130,6 +135,11 @@ cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale
                             float* key_norm, float* key_sum, cudaStream_t stream);
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
                               void* bdir, float* cert, int32_t* retained, cudaStream_t stream);
+// Key-block balls of a sequence: per key tile of 128 keys the real-domain
+// center, radius and largest norm (kBlkFloats floats per tile).
+constexpr int kBlkFloats = 132;
+cudaError_t launch_block_prep(const Handle& h, const void* k, const float* k_scale, int64_t S,
+                              float* blk, cudaStream_t stream);
 // The steps of every work item one launch processes: [begin, min(end,
 // n_tiles)) for the items whose probe flag equals want_flag (every item when
 // want_flag < 0).  Step 0 is key tile 0, step i >= 1 is key tile n_tiles - i.
@@ -138,10 +148,17 @@ cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* ke
 struct StepRange {
   int begin, end, want_flag;
 };
+// Key-block screening of a range: per work item, the steps of `steps` whose key
+// tile cannot hold a Top-K key of any of the item's queries (block bound +
+// margin below the carried threshold) are dropped; the rest go to
+// b.step_list / b.step_count (the range's last step is always kept).
+cudaError_t launch_block_screen(const Handle& h, const SeqView& v, const CertBuffers& b,
+                                StepRange steps, cudaStream_t stream);
 // Certified scorer over a range of steps; decide = 1 flags each item whose
-// range ends before its last step (filter or keep screening).
+// range ends before its last step (filter or keep screening).  With
+// use_list = 1 each item processes b.step_list instead of the whole range.
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             StepRange steps, int decide, cudaStream_t stream);
+                             StepRange steps, int decide, cudaStream_t stream, int use_list = 0);
 // Filter scorer (exact scores, threshold filter, no bounds) over a range.
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
                           StepRange steps, cudaStream_t stream);
@@ -159,10 +176,10 @@ size_t certified_smem_bytes(bool fp8);
 // CUDA-core reference scorer, same contract.
 cudaError_t launch_scores_ref(const Handle& h, const SeqView& v, float* scores, int64_t ld,
                               cudaStream_t stream);
-// Per-row radix Top-K.  Row i has n_i = row_len ? row_len[i] : (len0 + i) entries
-// (clipped to max_len).
 // p[0..n) = v.
 cudaError_t launch_fill(float* p, int64_t n, float v, cudaStream_t stream);
+// Per-row radix Top-K.  Row i has n_i = row_len ? row_len[i] : (len0 + i) entries
+// (clipped to max_len).
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int64_t* row_len,
                              int64_t len0, int64_t max_len, int64_t rows, int K, int32_t* out,
                              int64_t out_ld, cudaStream_t stream);

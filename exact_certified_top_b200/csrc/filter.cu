@@ -66,7 +66,8 @@ struct FilterParams {
 };
 
 // kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
-template <bool kFp8, int kHeads>
+// kDense: also write every exact score to p.dense (the dense-writeback ablation).
+template <bool kFp8, int kHeads, bool kDense>
 __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
     filter_kernel(const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap kmap, const FilterParams p) {
@@ -320,8 +321,9 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             int& cnt = grp ? cnt_b : cnt_a;
             n_cand += append_candidates(q, grp ? lb : la, p.seg_cap, cnt,
                                         s <= (grp ? pos_b : pos_a) && sc >= tau, sc, s, lane);
-            if (p.dense && s <= (grp ? pos_b : pos_a))
-              p.dense[(g.local0 + (grp ? qb : qa)) * p.dense_ld + s] = sc;
+            if constexpr (kDense)
+              if (s <= (grp ? pos_b : pos_a))
+                p.dense[(g.local0 + (grp ? qb : qa)) * p.dense_ld + s] = sc;
           }
         }
         if (!ok) break;
@@ -377,13 +379,12 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(filter_kernel<kFp8, 64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(filter_kernel<kFp8, 32>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {filter_kernel<kFp8, 64, false>, filter_kernel<kFp8, 32, false>,
+                    filter_kernel<kFp8, 64, true>, filter_kernel<kFp8, 32, true>})
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -422,10 +423,9 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_FILTER, stream);
-  if (v.H == 64)
-    filter_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
-  else
-    filter_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
+  auto fn = v.H == 64 ? (b.dense ? filter_kernel<kFp8, 64, true> : filter_kernel<kFp8, 64, false>)
+                      : (b.dense ? filter_kernel<kFp8, 32, true> : filter_kernel<kFp8, 32, false>);
+  fn<<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_FILTER, stream);
   return e;

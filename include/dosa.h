@@ -73,7 +73,7 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
- * margin_log2 = -12, screening = 2, sparse_writeback = 1. */
+ * margin_log2 = -12, screening = 2, sparse_writeback = 1, block_bound = 1. */
 typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
@@ -99,6 +99,11 @@ typedef struct {
                        is also written into a dense [rows, keys] matrix of the
                        chunk (rejected pairs as -inf) and the selection is the
                        dense Top-K of that matrix.  Same result either way.   */
+  int block_bound;  /* 1 (default): before the certified scorer resumes an item
+                       after its warm-up, every key tile is bounded as a whole
+                       (a ball around the tile's mean key) and tiles that can
+                       hold no Top-K key of the item's queries are skipped
+                       without loading their keys; 0: off (ablation).         */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */
@@ -110,6 +115,8 @@ typedef struct {
   int64_t exact_pairs;     /* pairs scored with all heads (seeds + survivors)        */
   int64_t candidates;      /* (score, index) pairs written for the final selection   */
   int64_t filtered_pairs;  /* exact pairs scored by the filter scorer (no bounds)    */
+  int64_t block_skipped_pairs; /* rejected pairs of key tiles skipped whole by the
+                                  key-block certificate (keys never loaded)      */
 } dosa_stats;
 
 typedef struct dosa_index* dosa_index_t;
@@ -279,7 +286,9 @@ typedef enum {
   DOSA_KERNEL_FILTER = 7,      /* exact scoring + threshold filter, no bounds  */
   DOSA_KERNEL_DECODE = 8,      /* decode step: seed bound, split-S scan        */
   DOSA_KERNEL_FILL = 9,        /* dense-writeback ablation: matrix set to -inf */
-  DOSA_KERNEL_KINDS = 10
+  DOSA_KERNEL_BLOCK = 10,      /* key-block certificate: block statistics and  */
+                               /* per-item block screening                      */
+  DOSA_KERNEL_KINDS = 11
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

@@ -259,3 +259,98 @@ def test_dense_writeback_ablation_equals_dense(cuda_lib, case, screening):
     ws = torch.zeros(idx.workspace_size(24, wl.S, K, True), dtype=torch.uint8, device="cuda")
     out2 = idx.topk(*_args(xd, K), workspace=ws)
     assert np.array_equal(to_numpy(out2), dense)
+
+
+def _clustered_blocks_case(T=48, n_tiles=50, seed=5, fp8=False):
+    """Keys in 128-key tiles that are tight balls: 'hot' tiles point along the
+    queries' common direction, 'cold' ones against it.  Query heads are near
+    copies (a tight certificate) with mostly positive weights, so every cold
+    tile's block bound is far below the threshold the hot keys set."""
+    g = torch.Generator().manual_seed(seed)
+    d, H = 128, 64
+    base = torch.randn(d, generator=g)
+    base = base / base.norm()
+    qdir = base + 0.2 * torch.randn((T, 1, d), generator=g)
+    q = 4.0 * qdir + 0.02 * torch.randn((T, H, d), generator=g)
+    w = torch.rand((T, H), generator=g) / 8
+    w[:, ::16] *= -0.2
+    S = n_tiles * 128
+    hot = torch.zeros(n_tiles, dtype=torch.bool)
+    hot[0] = True
+    hot[-6:] = True              # the diagonal tiles (seeds, warm-up)
+    hot[::3] = True
+    sign = torch.where(hot, 1.0, -1.0).repeat_interleave(128)[:, None]
+    k = sign * (2.0 * base + 0.05 * torch.randn((S, d), generator=g))
+    k = k + 0.3 * torch.randn((n_tiles, 1, d), generator=g).repeat_interleave(128, 0).view(S, d) * 0.1
+    pos0 = S - T
+    so = [[0, 0, pos0], [T, S, 0]]
+    if fp8:
+        from exact_certified_top_b200.workloads import _e4m3_per_token
+        q8, qs = _e4m3_per_token(q)
+        k8, ks = _e4m3_per_token(k)
+        return dict(q=q8, q_scale=qs, w=w, k=k8, k_scale=ks, seq_offsets=so,
+                    positions=torch.arange(pos0, S)), "fp8"
+    return dict(q=q.to(torch.bfloat16), q_scale=None, w=w, k=k.to(torch.bfloat16), k_scale=None,
+                seq_offsets=so, positions=torch.arange(pos0, S)), "bf16"
+
+
+@pytest.mark.parametrize("screening", [2, 1])
+@pytest.mark.parametrize("fp8", [False, True])
+def test_key_block_certificate_skips_tiles_and_stays_exact(cuda_lib, fp8, screening):
+    x, dtype = _clustered_blocks_case(fp8=fp8)
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 64
+    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
+    on = binding.Index(dtype, screening=screening, block_bound=1)
+    off = binding.Index(dtype, screening=screening, block_bound=0)
+    a, sa = on.topk(*_args(xd, K), stats=True)
+    b, sb = off.topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(a), dense) and np.array_equal(to_numpy(b), dense)
+    T, S = x["q"].shape[0], x["k"].shape[0]
+    visible = sum(S - T + t + 1 for t in range(T))
+    for st in (sa, sb):
+        assert st["exact_pairs"] + st["rejected_pairs"] == visible
+    assert sb["block_skipped_pairs"] == 0
+    assert sa["block_skipped_pairs"] > 0, sa
+    assert sa["block_skipped_pairs"] <= sa["rejected_pairs"]
+    ov = OracleView(x, dtype)
+    for t in range(0, T, 5):
+        assert_topk_matches(to_numpy(a)[t], ov.scores(t), K, t=t)
+
+
+def test_key_block_bounds_agree_with_oracle(cuda_lib):
+    """Every tile the GPU skipped has, in the fp64 oracle, a block bound below
+    the query's true K-th score for every query of the item that sees it (so
+    no Top-K key can have been skipped); checked through the selection and the
+    counters on the clustered case with one work item."""
+    from oracle import block_upper_bound, key_block_stats
+    x, dtype = _clustered_blocks_case(T=8, seed=9)
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 64
+    idx = binding.Index(dtype, screening=1, block_bound=1)
+    out, st = idx.topk(*_args(xd, K), stats=True)
+    ov = OracleView(x, dtype)
+    kb = key_mean(ov.k)
+    S = ov.k.shape[0]
+    n_tiles = S // 128
+    # tiles whose oracle block bound is below v_K for all 8 queries
+    droppable = 0
+    for j in range(1, n_tiles):
+        ok = True
+        for t in range(8):
+            p = int(ov.positions[t])
+            lo = j * 128
+            if lo > p:
+                continue
+            c = certificate_setup(ov.q[t], ov.w[t], kb, 4, 2)
+            cen, rad, nmax = key_block_stats(ov.k[lo:lo + 128])
+            vk = np.sort(ov.scores(t))[-K]
+            if not block_upper_bound(c, ov.q[t], cen, rad, nmax) < vk:
+                ok = False
+                break
+        droppable += ok
+    assert droppable > 0
+    # the GPU's skipped pairs never exceed what the ideal bound could drop
+    assert st["block_skipped_pairs"] <= droppable * 128 * 8
+    for t in range(8):
+        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
