@@ -424,27 +424,34 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
   // the steps left.
   const bool blk = b.blk != nullptr;
   const int W = warmup_steps(K), P = W + kProbeSteps;
+  // The certified scorer from step `from` on, for the items flagged `want`.
+  // With the key-block certificate the rest runs in passes [r0, 2 r0): each
+  // pass first drops the tiles that the threshold reached so far rules out.
+  auto certified_rest = [&](int from, int want) -> bool {
+    if (!blk)
+      return launch_certified(*h, c, b, K, StepRange{from, kAll, want}, 0, stream) == cudaSuccess;
+    const int max_steps = (int)((c.pos0 + c.rows - 1) / kKeyTile + 1);
+    for (int r0 = from; r0 < max_steps; r0 *= 2) {
+      const int r1 = 2 * r0 >= max_steps ? kAll : 2 * r0;
+      if (launch_block_screen(*h, c, b, StepRange{r0, r1, want}, stream) != cudaSuccess ||
+          launch_certified(*h, c, b, K, StepRange{r0, r1, want}, 0, stream, 1) != cudaSuccess)
+        return false;
+    }
+    return true;
+  };
   if (mode == 0) {
     if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
       return DOSA_ERR_CUDA;
   } else if (mode == 1) {
-    if (!blk) {
-      if (launch_certified(*h, c, b, K, StepRange{0, kAll, -1}, 0, stream) != cudaSuccess)
-        return DOSA_ERR_CUDA;
-    } else if (launch_certified(*h, c, b, K, StepRange{0, P, -1}, 0, stream) != cudaSuccess ||
-               launch_block_screen(*h, c, b, StepRange{P, kAll, -1}, stream) != cudaSuccess ||
-               launch_certified(*h, c, b, K, StepRange{P, kAll, -1}, 0, stream, 1) !=
-                   cudaSuccess) {
+    if (launch_certified(*h, c, b, K, StepRange{0, blk ? P : kAll, -1}, 0, stream) !=
+            cudaSuccess ||
+        (blk && !certified_rest(P, -1)))
       return DOSA_ERR_CUDA;
-    }
   } else {
     if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
         launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
         launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
-        (blk && launch_block_screen(*h, c, b, StepRange{P, kAll, kItemScreen}, stream) !=
-                    cudaSuccess) ||
-        launch_certified(*h, c, b, K, StepRange{P, kAll, kItemScreen}, 0, stream, blk ? 1 : 0) !=
-            cudaSuccess)
+        !certified_rest(P, kItemScreen))
       return DOSA_ERR_CUDA;
   }
   if (b.dense) {
