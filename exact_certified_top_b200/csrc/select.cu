@@ -223,14 +223,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
             c[hh * 4 + e] = bb + e < cj ? sp[bb + e] : CandView{-INFINITY, 0};
         }
       }
+      // one slot reservation per warp and pass: a warp scan of the
+      // per-thread counts, one shared atomic by the last lane
+      uint32_t mine = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int at = (e < 4 ? b : bh) + (e & 3);
-        const bool in = at < cj && c[e].score >= th;
-        const uint32_t slot = agg_slot(&s_n, in);
-        if (in && slot < (uint32_t)kSelList) {
-          lkey[slot] = ordered_key(c[e].score);
-          lidx[slot] = c[e].key;
+        if (at < cj && c[e].score >= th) mine |= 1u << e;
+      }
+      const int lane = threadIdx.x & 31;
+      const uint32_t cm = __popc(mine);
+      uint32_t incl = cm;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      uint32_t base = 0;
+      if (lane == 31 && incl) base = atomicAdd(&s_n, incl);
+      uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - cm;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if ((mine >> e) & 1u) {
+          if (slot < (uint32_t)kSelList) {
+            lkey[slot] = ordered_key(c[e].score);
+            lidx[slot] = c[e].key;
+          }
+          ++slot;
         }
       }
     }
