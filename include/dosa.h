@@ -78,7 +78,7 @@ typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
                        arrive as zeros) and reduce only the 32 real heads.   */
-  int d;            /* head dimension (128 in this build)                       */
+  int d;            /* head dimension (128 in this library)                     */
   dosa_dtype dtype; /* storage type of q and k                                  */
   int max_K;        /* largest K the handle will be called with (<= 4096)      */
   int seed_first;   /* seed subset: the first seed_first keys ...               */
