@@ -30,7 +30,7 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_index_decode_topk", "dosa_index_decode_workspace_size")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
            "certified": 5, "select": 6, "filter": 7, "decode": 8,
-           "fill": 9, "block": 10}
+           "fill": 9, "block": 10, "rescore": 11}
 
 
 class DosaError(RuntimeError):
@@ -44,14 +44,16 @@ class Config(ctypes.Structure):
                 ("max_K", ctypes.c_int), ("seed_first", ctypes.c_int),
                 ("seed_last", ctypes.c_int), ("r", ctypes.c_int), ("G", ctypes.c_int),
                 ("margin_log2", ctypes.c_int), ("screening", ctypes.c_int),
-                ("sparse_writeback", ctypes.c_int), ("block_bound", ctypes.c_int)]
+                ("sparse_writeback", ctypes.c_int), ("block_bound", ctypes.c_int),
+                ("survivor_stream", ctypes.c_int)]
 
 
 class Stats(ctypes.Structure):
     _fields_ = [("visible_pairs", ctypes.c_int64), ("seed_pairs", ctypes.c_int64),
                 ("screened_pairs", ctypes.c_int64), ("rejected_pairs", ctypes.c_int64),
                 ("exact_pairs", ctypes.c_int64), ("candidates", ctypes.c_int64),
-                ("filtered_pairs", ctypes.c_int64), ("block_skipped_pairs", ctypes.c_int64)]
+                ("filtered_pairs", ctypes.c_int64), ("block_skipped_pairs", ctypes.c_int64),
+                ("rescored_pairs", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: int(getattr(self, name)) for name, _ in self._fields_}

@@ -95,6 +95,15 @@ struct CertParams {
   const int* step_list;    // per item, the steps left by block screening, or null
   const int* step_count;
   int step_cap;
+  // Survivor mode (screening only): every survivor's key goes to its row's
+  // list, no exact score is computed, the state is saved at the range end and
+  // the item's seed/screened/rejected counts go to item_cnt (the rescoring
+  // pass credits them, or drops them when it hands the item to the filter).
+  int* surv;               // [chunk rows][surv_cap] or null
+  int* surv_count;         // [chunk rows]
+  int surv_cap;
+  unsigned long long* item_cnt;   // [items][3]
+  int stream_ok;           // the probe may choose survivor streams (kItemStream)
   StepRange steps;         // what this launch processes
   int decide;              // 1: flag every item whose range ends before its last step
 };
@@ -374,6 +383,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       for (int grp = 0; grp < C::kGroups; ++grp)
         cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * 2 + half].seg[quad]);
       unsigned long long it_scr = 0, it_rej = 0;   // this warp's counts, this item
+      const unsigned long long item_seed0 = n_seed, item_scr0 = n_screened,
+                               item_rej0 = n_rejected;
       auto key_of = [&](int i) -> int64_t {
         return (int64_t)tile_at(step_at(p, rg, item, i), g.n_tiles) * kKeyTile + quad * 32 + lane;
       };
@@ -415,6 +426,14 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           const bool surv = vis && !rej;
           const uint32_t mk = __ballot_sync(0xFFFFFFFFu, surv);
+          if (p.surv && mk) {
+            // survivor mode: the row's list gets the keys, no exact MMA
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&p.surv_count[q.row], __popc(mk));
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+            const int at = base + __popc(mk & ((1u << lane) - 1u));
+            if (surv && at < p.surv_cap) p.surv[q.row * (int64_t)p.surv_cap + at] = (int)s;
+          }
           const uint32_t scr = __popc(__ballot_sync(0xFFFFFFFFu, screen));
           const uint32_t rjm = __popc(__ballot_sync(0xFFFFFFFFu, rej));
           n_seed += __popc(__ballot_sync(0xFFFFFFFFu, vis && seed));
@@ -422,8 +441,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           n_rejected += rjm;
           it_scr += scr;
           it_rej += rjm;
-          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = mk;
-          if (mk) gbits |= 1u << (ql >> 1);
+          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = p.surv ? 0u : mk;
+          if (mk && !p.surv) gbits |= 1u << (ql >> 1);
         }
         if (lane == 0) gflag[(c % 3) * 8 + ew] = gbits;
         tc_fence_before();
@@ -517,15 +536,26 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
               tot_r += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2 + 1];
             }
             const bool pays = tot_s < kMinScreened || tot_r * kRejectRatio >= tot_s;
-            p.item_flag[item] = pays ? kItemScreen : kItemFilter;
+            // nearly everything rejected: rescore the few survivors gathered
+            const bool stream = p.stream_ok && tot_s >= kMinScreened && tot_r * 8 >= tot_s * 7;
+            p.item_flag[item] = stream ? kItemStream : pays ? kItemScreen : kItemFilter;
           }
         }
       }
       kc += n;
       // ---- range end: carry the query's state over, or publish it ----
       if (ok && ew < g.nq) {
-        if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
+        if (rg.end < g.n_tiles || p.surv) state_save(st[ew], p.qstate + st[ew].row, lane);
         else if (lane == 0) publish_query(st[ew], p.out);
+      }
+      if (p.surv && lane == 0) {
+        // this item's counts, held back until the rescoring pass decides
+        atomicAdd(&p.item_cnt[item * 3 + 0], n_seed - item_seed0);
+        atomicAdd(&p.item_cnt[item * 3 + 1], n_screened - item_scr0);
+        atomicAdd(&p.item_cnt[item * 3 + 2], n_rejected - item_rej0);
+        n_seed = item_seed0;
+        n_screened = item_scr0;
+        n_rejected = item_rej0;
       }
     }
     if (lane == 0) {
@@ -604,9 +634,14 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.seed_last = h.cfg.seed_last;
   p.steps = steps;
   p.decide = decide;
-  p.step_list = use_list ? b.step_list : nullptr;
-  p.step_count = use_list ? b.step_count : nullptr;
+  p.step_list = use_list == 1 ? b.step_list : nullptr;
+  p.step_count = use_list == 1 ? b.step_count : nullptr;
   p.step_cap = b.step_cap;
+  p.surv = use_list == 2 ? b.surv : nullptr;
+  p.surv_count = b.surv_count;
+  p.surv_cap = b.surv_cap;
+  p.item_cnt = b.item_cnt;
+  p.stream_ok = b.surv != nullptr;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);

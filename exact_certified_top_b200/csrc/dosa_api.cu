@@ -133,7 +133,9 @@ int seg_capacity(int K, int64_t S_max) {
 struct CertLayout {
   size_t key_norm, key_sum, repair_list, repair_count, repair_scores, blk, fixed;
   int step_cap;     // block screening: steps per item list (key tiles of S_max), or 0
+  int surv_cap;     // survivor streams: keys per row list (an eighth of S_max), or 0
   size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
+  size_t surv_row;  // the part of per_row taken by the survivor lists
   int seg_cap;
   int64_t dense_ld; // dense writeback: the score matrix's row length (0 when sparse)
 };
@@ -164,6 +166,12 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.per_row += (size_t)L.dense_ld * 4;
   // step lists: one per work item of 8 rows (plus the count)
   L.per_row += ((size_t)L.step_cap * 4 + 4 + 7) / 8;
+  // survivor lists: streamed items were chosen for rejecting >= 7/8 in the
+  // probe, and a pass covers at most half of the keys, so a list holds an
+  // eighth of S_max; plus held-back item counts and the overflow flag
+  L.surv_cap = h->cfg.survivor_stream ? (int)round_up(S_max / 8 + 128, 128) : 0;
+  L.surv_row = L.surv_cap ? (size_t)L.surv_cap * 4 + 4 + 4 : 0;
+  L.per_row += L.surv_row;
   return L;
 }
 
@@ -198,6 +206,13 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.step_list = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * L.step_cap * 4))
                            : nullptr;
   b.step_count = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
+  b.surv_cap = L.surv_cap;
+  b.surv = L.surv_cap ? reinterpret_cast<int*>(take((size_t)Tc * L.surv_cap * 4)) : nullptr;
+  b.surv_count = L.surv_cap ? reinterpret_cast<int*>(take((size_t)Tc * 4)) : nullptr;
+  b.item_cnt = L.surv_cap ? reinterpret_cast<unsigned long long*>(
+                                take((size_t)(Tc / 8 + 1) * 3 * 8))
+                          : nullptr;
+  b.ovf = L.surv_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
   b.err = &reinterpret_cast<WsHeader*>(ws)->error;
   return b;
@@ -205,7 +220,7 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
 
 // Padding the per-row arrays of a chunk may need (each starts 256-aligned),
 // plus the item-flag array's extra entry.
-constexpr size_t kCertPad = 11 * 256 + 4 + 16 * 1024 * 4;
+constexpr size_t kCertPad = 15 * 256 + 8 + 16 * 1024 * 4 + 3 * 8;
 
 // Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
 int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
@@ -260,6 +275,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->screening = 2;
   cfg->sparse_writeback = 1;
   cfg->block_bound = 1;
+  cfg->survivor_stream = 0;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -270,7 +286,8 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   if (cfg->seed_first < 0 || cfg->seed_last < 0 || cfg->r < 0 || cfg->r > 4 || cfg->G < 0 ||
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
       cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
-      cfg->block_bound < 0 || cfg->block_bound > 1)
+      cfg->block_bound < 0 || cfg->block_bound > 1 || cfg->survivor_stream < 0 ||
+      cfg->survivor_stream > 2)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -305,7 +322,9 @@ dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max
     const CertLayout L = cert_layout(h, S_max, K);
     int64_t rows = chunk_rows;
     if (rows == 0) {
-      rows = kDefaultCertChunkBytes / (int64_t)L.per_row;
+      // the survivor lists come on top of the budget: they do not change
+      // how many chunks a call takes
+      rows = kDefaultCertChunkBytes / (int64_t)(L.per_row - L.surv_row);
       rows = rows / 8 * 8;
       if (rows < 8) rows = 8;
     }
@@ -439,19 +458,43 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
     }
     return true;
   };
+  // Survivor streams from step `from` on, for the items flagged `want`, in
+  // passes [r0, 2 r0): screening into per-row survivor lists, rescoring of
+  // the gathered survivors (which raises the threshold the next pass screens
+  // against), and the filter scorer redoing the pass for items whose lists
+  // overflowed, from the state the screening saved.
+  auto streamed_rest = [&](int from, int want) -> bool {
+    const int max_steps = (int)((c.pos0 + c.rows - 1) / kKeyTile + 1);
+    const size_t n_items = (size_t)((c.rows + 7) / 8);
+    CertBuffers ob = b;
+    ob.item_flag = b.ovf;
+    for (int r0 = from; r0 < max_steps; r0 *= 2) {
+      const int r1 = 2 * r0 >= max_steps ? kAll : 2 * r0;
+      const StepRange sr{r0, r1, want};
+      if (cudaMemsetAsync(b.surv_count, 0, (size_t)c.rows * 4, stream) != cudaSuccess ||
+          cudaMemsetAsync(b.item_cnt, 0, n_items * 3 * 8, stream) != cudaSuccess ||
+          cudaMemsetAsync(b.ovf, 0, n_items * 4, stream) != cudaSuccess ||
+          launch_certified(*h, c, b, K, sr, 0, stream, 2) != cudaSuccess ||
+          launch_rescore(*h, c, b, K, sr, stream) != cudaSuccess ||
+          launch_filter(*h, c, ob, K, StepRange{r0, r1, 1}, stream) != cudaSuccess)
+        return false;
+    }
+    return true;
+  };
   if (mode == 0) {
     if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
       return DOSA_ERR_CUDA;
   } else if (mode == 1) {
-    if (launch_certified(*h, c, b, K, StepRange{0, blk ? P : kAll, -1}, 0, stream) !=
+    const bool streams = b.surv && h->cfg.survivor_stream == 2, split = blk || streams;
+    if (launch_certified(*h, c, b, K, StepRange{0, split ? P : kAll, -1}, 0, stream) !=
             cudaSuccess ||
-        (blk && !certified_rest(P, -1)))
+        (split && !(streams ? streamed_rest(P, -1) : certified_rest(P, -1))))
       return DOSA_ERR_CUDA;
   } else {
     if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
         launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
         launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
-        !certified_rest(P, kItemScreen))
+        !certified_rest(P, kItemScreen) || (b.surv && !streamed_rest(P, kItemStream)))
       return DOSA_ERR_CUDA;
   }
   if (b.dense) {
@@ -488,6 +531,7 @@ static dosa_status read_stats(const void* workspace, const int64_t* seq_offsets,
   stats->candidates = (int64_t)hdr.counters[kCntCandidates];
   stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
   stats->block_skipped_pairs = (int64_t)hdr.counters[kCntBlockSkipped];
+  stats->rescored_pairs = (int64_t)hdr.counters[kCntRescored];
   if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
   return DOSA_OK;
 }

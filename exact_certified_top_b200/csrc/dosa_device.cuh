@@ -110,6 +110,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Make this thread's ordinary shared-memory stores visible to the async proxy
+// (TMA, tcgen05.mma operands) before it signals them ready.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 3-D tiled load (c0 innermost), same completion mechanism as tma_load_2d.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t c0, int32_t c1, int32_t c2) {

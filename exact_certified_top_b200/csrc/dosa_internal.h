@@ -31,6 +31,7 @@ enum CounterId : int {
   kCntOverflow = 5,
   kCntFiltered = 6,
   kCntBlockSkipped = 7,
+  kCntRescored = 8,
 };
 constexpr size_t kWsHeaderBytes = 256;
 
@@ -71,7 +72,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder();
 // Queries as a 3-D tensor [rows][H][d] read in boxes of 4 rows x 64 head
 // slots x one 128-byte row: with H = 32 the slots 32..63 lie outside the
 // tensor and arrive as zeros, so every kernel sees 64 heads per row.
-bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H);
+bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H,
+                  int box_rows = 4);
 bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows,
                      uint32_t box_rows);
 
@@ -98,6 +100,11 @@ struct CertBuffers {
   int* step_list;        // [rows / 8 + 1][step_cap] steps left after block screening
   int* step_count;       // [rows / 8 + 1]
   int step_cap;
+  int* surv;             // [rows][surv_cap] survivor keys of streamed items, or null
+  int* surv_count;       // [rows], zeroed before a screening pass
+  int surv_cap;
+  unsigned long long* item_cnt;   // [rows / 8 + 1][3] held-back counts of streamed items
+  int* ovf;              // [rows / 8 + 1] survivor lists overflowed in the current pass
   unsigned long long* counters;
   int* err;
 };
@@ -155,10 +162,17 @@ struct StepRange {
 cudaError_t launch_block_screen(const Handle& h, const SeqView& v, const CertBuffers& b,
                                 StepRange steps, cudaStream_t stream);
 // Certified scorer over a range of steps; decide = 1 flags each item whose
-// range ends before its last step (filter or keep screening).  With
-// use_list = 1 each item processes b.step_list instead of the whole range.
+// range ends before its last step (filter, keep screening, or survivor
+// streams).  use_list = 1: each item processes b.step_list instead of the
+// whole range; use_list = 2: survivor mode (screening only, survivors to
+// b.surv, state saved at the range end, counts held back in b.item_cnt).
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
                              StepRange steps, int decide, cudaStream_t stream, int use_list = 0);
+// Rescoring of the survivor lists a screening pass left over `range` (gathered
+// keys on the tensor cores), publishing rows whose item ends in the range and
+// saving the others; items with an overflowed list get b.ovf[item] = 1.
+cudaError_t launch_rescore(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                           StepRange range, cudaStream_t stream);
 // Filter scorer (exact scores, threshold filter, no bounds) over a range.
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
                           StepRange steps, cudaStream_t stream);

@@ -325,13 +325,14 @@ bool encode_rows_map(CUtensorMap* map, const void* base, bool fp8, uint64_t rows
   return r == CUDA_SUCCESS;
 }
 
-bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H) {
+bool encode_q_map(CUtensorMap* map, const void* q, bool fp8, uint64_t rows, int H,
+                  int box_rows) {
   auto enc = get_tensor_map_encoder();
   if (!enc || (H != 32 && H != 64)) return false;
   const uint64_t esz = fp8 ? 1 : 2;
   const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * esz, (cuuint64_t)H * kHeadDim * esz};
-  const cuuint32_t box[3] = {(cuuint32_t)(fp8 ? 128 : 64), 64, 4};
+  const cuuint32_t box[3] = {(cuuint32_t)(fp8 ? 128 : 64), 64, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                          3, const_cast<void*>(q), dims, strides, box, estr,

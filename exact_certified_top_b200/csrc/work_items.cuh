@@ -42,7 +42,10 @@ __device__ __forceinline__ int tile_at(int ti, int n_tiles) {
 }
 
 // What the probe pass decided for an item (certified workspace flags).
-enum ItemFlag : int { kItemFilter = 1, kItemScreen = 2 };
+// Probe decisions: filter scorer, certified scorer on the resident key tile,
+// or certified screening into survivor lists then rescoring of the gathered
+// survivors (kItemStream).
+enum ItemFlag : int { kItemFilter = 1, kItemScreen = 2, kItemStream = 3 };
 
 struct Range {
   int begin, end;   // empty when end <= begin

@@ -73,7 +73,8 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
- * margin_log2 = -12, screening = 2, sparse_writeback = 1, block_bound = 1. */
+ * margin_log2 = -12, screening = 2, sparse_writeback = 1, block_bound = 1,
+ * survivor_stream = 0. */
 typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
@@ -104,6 +105,15 @@ typedef struct {
                        (a ball around the tile's mean key) and tiles that can
                        hold no Top-K key of the item's queries are skipped
                        without loading their keys; 0: off (ablation).         */
+  int survivor_stream; /* 0 (default): every screened item is rescored on the
+                       resident key tile.  1: work items whose probe rejected
+                       >= 7/8 of the screened pairs are screened into per-row
+                       survivor lists, in passes over doubling key ranges, and
+                       the survivors are gathered and rescored on dense
+                       tensor-core tiles (items whose lists overflow are
+                       rescored by the filter scorer for that pass); 2: as 1,
+                       and with screening = 1 every item streams after its
+                       probe steps.  Same result in every mode.               */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */
@@ -117,6 +127,7 @@ typedef struct {
   int64_t filtered_pairs;  /* exact pairs scored by the filter scorer (no bounds)    */
   int64_t block_skipped_pairs; /* rejected pairs of key tiles skipped whole by the
                                   key-block certificate (keys never loaded)      */
+  int64_t rescored_pairs;  /* exact pairs scored from gathered survivor streams     */
 } dosa_stats;
 
 typedef struct dosa_index* dosa_index_t;
@@ -288,7 +299,8 @@ typedef enum {
   DOSA_KERNEL_FILL = 9,        /* dense-writeback ablation: matrix set to -inf */
   DOSA_KERNEL_BLOCK = 10,      /* key-block certificate: block statistics and  */
                                /* per-item block screening                      */
-  DOSA_KERNEL_KINDS = 11
+  DOSA_KERNEL_RESCORE = 11,    /* rescoring of gathered survivors               */
+  DOSA_KERNEL_KINDS = 12
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

@@ -354,3 +354,62 @@ def test_key_block_bounds_agree_with_oracle(cuda_lib):
     assert st["block_skipped_pairs"] <= droppable * 128 * 8
     for t in range(8):
         assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_survivor_streams_rescore_gathered_keys_exactly(cuda_lib, fp8):
+    """Redundant heads and a small K: the probe rejects nearly every screened
+    pair, so the items go to survivor streams (screening into per-row lists,
+    then the gathered survivors rescored on the tensor cores).  The selection
+    must equal the dense path's, survivors must have been rescored, and the
+    counters must add up; without streams the same selection comes out."""
+    x, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=fp8)
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 32
+    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
+    on, st_on = binding.Index(dtype, survivor_stream=1).topk(*_args(xd, K), stats=True)
+    off, st_off = binding.Index(dtype, survivor_stream=0).topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(on), dense)
+    assert np.array_equal(to_numpy(off), dense)
+    T, S = x["q"].shape[0], x["k"].shape[0]
+    visible = sum(S - T + t + 1 for t in range(T))
+    for st in (st_on, st_off):
+        assert st["exact_pairs"] + st["rejected_pairs"] == visible
+    assert st_on["rescored_pairs"] > 0, st_on
+    assert st_off["rescored_pairs"] == 0
+    assert st_on["rejected_pairs"] > visible // 2
+    ov = OracleView(x, dtype)
+    for t in range(0, T, 7):
+        assert_topk_matches(to_numpy(on)[t], ov.scores(t), K, t=t)
+
+
+@pytest.mark.parametrize("redundant", [True, False], ids=["redundant", "random"])
+def test_survivor_streams_every_item(cuda_lib, redundant):
+    """screening = 1 with survivor_stream = 2: every item streams after its
+    probe steps, in passes over doubling key ranges.  On redundant heads the
+    lists hold few survivors and are rescored from the gathered keys; on the
+    random case nearly nothing is rejected, the later passes overflow their
+    lists and the filter scorer redoes those passes.  Either way the selection
+    is the dense path's and every visible pair is counted exactly once."""
+    if redundant:
+        x, dtype = _redundant_heads_case(T=64, S=20000, seed=5, fp8=True)
+        K = 32
+    else:
+        _, x, _ = _inputs("prefill_128k_fp8", 200, 9000, 300)
+        dtype = "fp8"
+        K = 300
+    xd = {k: (v.cuda() if torch.is_tensor(v) and k != "seq_offsets" else v) for k, v in x.items()}
+    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
+    out, st = binding.Index(dtype, screening=1, survivor_stream=2).topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out), dense)
+    T, S = x["q"].shape[0], x["k"].shape[0]
+    visible = sum(S - T + t + 1 for t in range(T))
+    assert st["exact_pairs"] + st["rejected_pairs"] == visible
+    assert st["rescored_pairs"] > 0, st
+    if redundant:
+        assert st["filtered_pairs"] <= visible // 4, st
+    else:
+        assert st["filtered_pairs"] > 0, st
+    ov = OracleView(x, dtype)
+    for t in range(0, T, 9):
+        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
