@@ -31,6 +31,7 @@
 #include "cert_layout.h"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
+#include "work_items.cuh"
 
 namespace dosa {
 
@@ -213,6 +214,10 @@ struct SetupParams {
   void* bdir;             // [rows, 8, d] codes (chunk-local rows)
   float* cert;            // [rows, kCertFloats]
   int32_t* retained;      // [rows, 4]
+  int sample;             // which rows (see launch_cert_setup)
+  int n_items;
+  int* item_flag;
+  const int* gate;
 };
 
 // upper-triangle pairs of the 4 retained slots
@@ -241,7 +246,19 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   __shared__ float red[8];
   __shared__ float uv[2][D], rv[2][D];
   __shared__ float s_lam;
-  const int64_t i = blockIdx.x;
+  int64_t i = blockIdx.x;
+  if (p.sample == 1) {
+    // the rows of sampled item kProbeSampleStride * (blockIdx.x / 8); items
+    // run longest rows first, so item j holds the rows of group n_items-1-j
+    const int item = kProbeSampleStride * (int)(blockIdx.x / kItemQueries);
+    i = (int64_t)(p.n_items - 1 - item) * kItemQueries + blockIdx.x % kItemQueries;
+    if (i >= p.rows) return;
+    if (threadIdx.x == 0 && blockIdx.x % kItemQueries == 0) p.item_flag[item] = kItemSample;
+  } else if (p.sample == 2) {
+    const int item = p.n_items - 1 - (int)(i / kItemQueries);
+    if (item % kProbeSampleStride == 0 || *reinterpret_cast<const volatile int*>(p.gate) == 0)
+      return;
+  }
   const int64_t t = p.row0 + i;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -673,8 +690,23 @@ cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale
   return e;
 }
 
+__global__ void probe_resolve_kernel(int* item_flag, int n_items, const int* gate) {
+  const bool probe = *gate != 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_items; i += gridDim.x * blockDim.x)
+    if (item_flag[i] == 0) item_flag[i] = probe ? kItemProbe : kItemUnprobed;
+}
+
+cudaError_t launch_probe_resolve(int* item_flag, int n_items, const int* gate,
+                                 cudaStream_t stream) {
+  if (n_items <= 0) return cudaSuccess;
+  const int grid = (n_items + 255) / 256 < 1024 ? (n_items + 255) / 256 : 1024;
+  probe_resolve_kernel<<<grid, 256, 0, stream>>>(item_flag, n_items, gate);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
-                              void* bdir, float* cert, int32_t* retained, cudaStream_t stream) {
+                              void* bdir, float* cert, int32_t* retained, cudaStream_t stream,
+                              int sample, int* item_flag, const int* gate) {
   if (v.rows <= 0) return cudaSuccess;
   SetupParams p;
   p.q = v.q;
@@ -690,6 +722,13 @@ cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* ke
   p.bdir = bdir;
   p.cert = cert;
   p.retained = retained;
+  p.sample = sample;
+  p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
+  p.item_flag = item_flag;
+  p.gate = gate;
+  unsigned grid = (unsigned)v.rows;
+  if (sample == 1)
+    grid = (unsigned)((p.n_items + kProbeSampleStride - 1) / kProbeSampleStride) * kItemQueries;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(cert_setup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -700,9 +739,9 @@ cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* ke
   }
   profile_before(DOSA_KERNEL_CERT_SETUP, stream);
   if (h.cfg.dtype == DOSA_FP8_E4M3)
-    cert_setup_kernel<true><<<(unsigned)v.rows, kSetupThreads, kSetupSmem, stream>>>(p);
+    cert_setup_kernel<true><<<grid, kSetupThreads, kSetupSmem, stream>>>(p);
   else
-    cert_setup_kernel<false><<<(unsigned)v.rows, kSetupThreads, kSetupSmem, stream>>>(p);
+    cert_setup_kernel<false><<<grid, kSetupThreads, kSetupSmem, stream>>>(p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_CERT_SETUP, stream);
   return e;

@@ -106,6 +106,7 @@ struct CertParams {
   int stream_ok;           // the probe may choose survivor streams (kItemStream)
   StepRange steps;         // what this launch processes
   int decide;              // 1: flag every item whose range ends before its last step
+  int* gate;               // set to 1 when a decision is not the filter scorer
 };
 
 // The steps an item processes in this launch: its range, or the list block
@@ -539,6 +540,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             // nearly everything rejected: rescore the few survivors gathered
             const bool stream = p.stream_ok && tot_s >= kMinScreened && tot_r * 8 >= tot_s * 7;
             p.item_flag[item] = stream ? kItemStream : pays ? kItemScreen : kItemFilter;
+            if (stream || pays) *reinterpret_cast<volatile int*>(p.gate) = 1;
           }
         }
       }
@@ -611,6 +613,7 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.cand = reinterpret_cast<Cand*>(b.cand);
   p.qstate = reinterpret_cast<QStateG*>(b.qstate);
   p.item_flag = b.item_flag;
+  p.gate = b.gate;
   p.out.cand_count = b.cand_count;
   p.out.tau = b.tau;
   p.out.repair_list = b.repair_list;

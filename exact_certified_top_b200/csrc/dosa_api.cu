@@ -213,6 +213,8 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
                                 take((size_t)(Tc / 8 + 1) * 3 * 8))
                           : nullptr;
   b.ovf = L.surv_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
+  b.gate = &reinterpret_cast<WsHeader*>(ws)->probe_gate;
+  b.probe_sample = 0;
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
   b.err = &reinterpret_cast<WsHeader*>(ws)->error;
   return b;
@@ -276,6 +278,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->sparse_writeback = 1;
   cfg->block_bound = 1;
   cfg->survivor_stream = 0;
+  cfg->probe_sample = 1;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -287,7 +290,7 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
       cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
       cfg->block_bound < 0 || cfg->block_bound > 1 || cfg->survivor_stream < 0 ||
-      cfg->survivor_stream > 2)
+      cfg->survivor_stream > 2 || cfg->probe_sample < 0 || cfg->probe_sample > 1)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -382,6 +385,31 @@ dosa_status dosa_index_dense_topk(dosa_index_t hh, const void* q, const float* q
 }  // extern "C"
 
 // Runs key prep and certificate setup for one sequence chunk by chunk, calling
+// The certificate set-up of a chunk.  With every row's record wanted (or
+// screening on every item) all rows are set up; with screening off none; in
+// the adaptive mode only the rows of the sampled items, the others after the
+// sampled probe, if it found an item worth screening (cert_chunk).
+static dosa_status setup_chunk(const Handle* h, const SeqView& c, CertBuffers& cb, bool records,
+                               cudaStream_t stream) {
+  const int mode = h->cfg.screening;
+  cb.probe_sample = 0;
+  if (!records && mode == 0) return DOSA_OK;
+  if (!records && mode == 2 && h->cfg.probe_sample) {
+    const int64_t n_items = (c.rows + 7) / 8;
+    if (cudaMemsetAsync(cb.item_flag, 0, (size_t)n_items * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(cb.gate, 0, sizeof(int), stream) != cudaSuccess ||
+        launch_cert_setup(*h, c, cb.key_sum, cb.bdir, cb.cert, cb.retained, stream, 1,
+                          cb.item_flag, cb.gate) != cudaSuccess)
+      return DOSA_ERR_CUDA;
+    cb.probe_sample = 1;
+    return DOSA_OK;
+  }
+  return launch_cert_setup(*h, c, cb.key_sum, cb.bdir, cb.cert, cb.retained, stream) ==
+                 cudaSuccess
+             ? DOSA_OK
+             : DOSA_ERR_CUDA;
+}
+
 // `body(chunk view, buffers)` after each setup.
 template <typename Body>
 static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const float* q_scale,
@@ -413,10 +441,9 @@ static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const flo
       CertBuffers cb = buf;
       if (cert_out) cb.cert = cert_out + c.row0 * kCertFloats;
       if (retained_out) cb.retained = retained_out + c.row0 * 4;
-      if (launch_cert_setup(*h, c, buf.key_sum, cb.bdir, cb.cert, cb.retained, stream) !=
-          cudaSuccess)
-        return DOSA_ERR_CUDA;
-      const dosa_status st = body(c, cb);
+      dosa_status st = setup_chunk(h, c, cb, cert_out != nullptr, stream);
+      if (st != DOSA_OK) return st;
+      st = body(c, cb);
       if (st != DOSA_OK) return st;
     }
   }
@@ -491,9 +518,26 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
         (split && !(streams ? streamed_rest(P, -1) : certified_rest(P, -1))))
       return DOSA_ERR_CUDA;
   } else {
-    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
-        launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) != cudaSuccess ||
-        launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter}, stream) != cudaSuccess ||
+    // The probe: all items, or the sampled items first and the others only
+    // when some sampled item found screening worth it (else they go to the
+    // filter scorer unprobed, from the warm-up's end).
+    const int n_items = (int)((c.rows + 7) / 8);
+    auto probe = [&]() -> bool {
+      if (!b.probe_sample)
+        return launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) == cudaSuccess;
+      return launch_certified(*h, c, b, K, StepRange{W, P, kItemSample}, 1, stream) ==
+                 cudaSuccess &&
+             launch_probe_resolve(b.item_flag, n_items, b.gate, stream) == cudaSuccess &&
+             launch_cert_setup(*h, c, b.key_sum, b.bdir, b.cert, b.retained, stream, 2,
+                               b.item_flag, b.gate) == cudaSuccess &&
+             launch_certified(*h, c, b, K, StepRange{W, P, kItemProbe}, 1, stream) ==
+                 cudaSuccess;
+    };
+    // the filter scorer finishes the items whose probe chose it, and the
+    // unprobed items from the warm-up's end, in one launch
+    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess || !probe() ||
+        launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter, kItemUnprobed, W}, stream) !=
+            cudaSuccess ||
         !certified_rest(P, kItemScreen) || (b.surv && !streamed_rest(P, kItemStream)))
       return DOSA_ERR_CUDA;
   }
@@ -740,11 +784,11 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
         return DOSA_ERR_CUDA;
       prev_b = ch.b;
     }
-    if (!ok(cudaStreamWaitEvent(main, h->ev_loaded[slot], 0)) ||
-        launch_cert_setup(*h, c, buf.key_sum, buf.bdir, buf.cert, buf.retained, main) !=
-            cudaSuccess)
-      return DOSA_ERR_CUDA;
-    st = cert_chunk(h, c, buf, K, dout, main);
+    if (!ok(cudaStreamWaitEvent(main, h->ev_loaded[slot], 0))) return DOSA_ERR_CUDA;
+    CertBuffers cb = buf;
+    st = setup_chunk(h, c, cb, false, main);
+    if (st != DOSA_OK) return st;
+    st = cert_chunk(h, c, cb, K, dout, main);
     if (st != DOSA_OK) return st;
     if (!ok(cudaEventRecord(h->ev_done[slot], main)) ||
         !ok(cudaStreamWaitEvent(cpy, h->ev_done[slot], 0)) ||

@@ -19,7 +19,7 @@ constexpr int kQueryTile = 8;     // queries resident per scorer work item
 // Workspace header: word 0 = device error word, then counters.
 struct WsHeader {
   int error;
-  int pad0;
+  int probe_gate;        // the sampled probe found an item worth screening
   unsigned long long counters[15];   // see CounterId
 };
 enum CounterId : int {
@@ -105,6 +105,8 @@ struct CertBuffers {
   int surv_cap;
   unsigned long long* item_cnt;   // [rows / 8 + 1][3] held-back counts of streamed items
   int* ovf;              // [rows / 8 + 1] survivor lists overflowed in the current pass
+  int* gate;             // set by the probe when a sampled item chose screening
+  int probe_sample;      // the chunk's set-up covered only the sampled items
   unsigned long long* counters;
   int* err;
 };
@@ -140,8 +142,17 @@ cudaError_t launch_scores_tc_rows(const Handle& h, const SeqView& v, const int* 
 // Certified pipeline pieces.
 cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale, int64_t S,
                             float* key_norm, float* key_sum, cudaStream_t stream);
+// sample 0: every row of the chunk; 1: the rows of the sampled work items
+// (every kProbeSampleStride-th), whose item_flag becomes kItemSample; 2: the
+// other rows, only when *gate is set (a no-op launch otherwise).
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
-                              void* bdir, float* cert, int32_t* retained, cudaStream_t stream);
+                              void* bdir, float* cert, int32_t* retained, cudaStream_t stream,
+                              int sample = 0, int* item_flag = nullptr,
+                              const int* gate = nullptr);
+// After the sampled probe: items still unflagged become kItemProbe when *gate
+// is set (they are set up and probed next), kItemUnprobed otherwise.
+cudaError_t launch_probe_resolve(int* item_flag, int n_items, const int* gate,
+                                 cudaStream_t stream);
 // Key-block balls of a sequence: per key tile of 128 keys the real-domain
 // center, radius and largest norm (kBlkFloats floats per tile).
 constexpr int kBlkFloats = 132;
@@ -151,9 +162,11 @@ cudaError_t launch_block_prep(const Handle& h, const void* k, const float* k_sca
 // n_tiles)) for the items whose probe flag equals want_flag (every item when
 // want_flag < 0).  Step 0 is key tile 0, step i >= 1 is key tile n_tiles - i.
 // A range that starts after step 0 resumes the state the previous launch
-// saved; a range that ends before the item's last step saves it again.
+// saved; a range that ends before the item's last step saves it again.  When
+// alt_flag > 0, the items flagged alt_flag are processed too, from alt_begin.
 struct StepRange {
   int begin, end, want_flag;
+  int alt_flag, alt_begin;
 };
 // Key-block screening of a range: per work item, the steps of `steps` whose key
 // tile cannot hold a Top-K key of any of the item's queries (block bound +

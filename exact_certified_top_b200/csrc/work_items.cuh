@@ -44,8 +44,21 @@ __device__ __forceinline__ int tile_at(int ti, int n_tiles) {
 // What the probe pass decided for an item (certified workspace flags).
 // Probe decisions: filter scorer, certified scorer on the resident key tile,
 // or certified screening into survivor lists then rescoring of the gathered
-// survivors (kItemStream).
-enum ItemFlag : int { kItemFilter = 1, kItemScreen = 2, kItemStream = 3 };
+// survivors (kItemStream).  Before the decisions: kItemSample marks the items
+// probed first (every kProbeSampleStride-th item, longest rows first), and
+// kItemProbe the others once the sample showed that screening pays somewhere;
+// otherwise they become kItemUnprobed (filter scorer from the warm-up's end).
+enum ItemFlag : int {
+  kItemFilter = 1,
+  kItemScreen = 2,
+  kItemStream = 3,
+  kItemSample = 4,
+  kItemProbe = 5,
+  kItemUnprobed = 6
+};
+// Prime, so that the sampled items spread evenly over the persistent CTAs
+// (CTA b takes items b, b + grid, ...) for any grid that is not a multiple of 7.
+constexpr int kProbeSampleStride = 7;
 
 struct Range {
   int begin, end;   // empty when end <= begin
@@ -56,7 +69,11 @@ __device__ __forceinline__ Range item_steps(const StepRange& sr, const int* item
   Range r;
   r.begin = sr.begin;
   r.end = g.n_tiles < sr.end ? g.n_tiles : sr.end;
-  if (sr.want_flag >= 0 && r.begin < r.end && item_flag[item] != sr.want_flag) r.end = r.begin;
+  if (sr.want_flag >= 0) {
+    const int f = item_flag[item];
+    if (sr.alt_flag > 0 && f == sr.alt_flag) r.begin = sr.alt_begin;
+    else if (f != sr.want_flag) r.end = r.begin;
+  }
   return r;
 }
 

@@ -74,7 +74,7 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
  * margin_log2 = -12, screening = 2, sparse_writeback = 1, block_bound = 1,
- * survivor_stream = 0. */
+ * survivor_stream = 0, probe_sample = 1. */
 typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
@@ -114,6 +114,12 @@ typedef struct {
                        rescored by the filter scorer for that pass); 2: as 1,
                        and with screening = 1 every item streams after its
                        probe steps.  Same result in every mode.               */
+  int probe_sample;  /* screening = 2 only.  1 (default): every 7th work item
+                       (longest rows first) is set up and probed first; the
+                       other items are set up and probed only if one of those
+                       chose screening, and otherwise go to the filter scorer
+                       straight after their warm-up.  0: every item is set up
+                       and probed (ablation).  Same result either way.        */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */

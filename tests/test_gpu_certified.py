@@ -166,7 +166,8 @@ def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
     rejects most keys: the probe lets screening continue) and independent
     random heads (screening rejects almost nothing: the probe hands the item to
     the filter scorer).  Both finishers run in one call; the selection stays
-    identical to the dense path and to the oracle."""
+    identical to the dense path and to the oracle.  Every item is probed
+    (probe_sample = 0); with the sampled probe the selection is the same."""
     x, dtype = _redundant_heads_case(T=160, S=7000, seed=11, fp8=fp8)
     g = torch.Generator().manual_seed(12)
     rand_rows = torch.cat([torch.arange(i, i + 8) for i in range(8, 160, 16)])
@@ -180,10 +181,13 @@ def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
     x["w"][rand_rows] = torch.randn((len(rand_rows), 64), generator=g) / 8
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 128
-    idx = binding.Index(dtype, screening=2)
+    idx = binding.Index(dtype, screening=2, probe_sample=0)
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     dense = idx.dense_topk(*_args(xd, K))
     assert torch.equal(cert, dense)
+    sampled, st_s = binding.Index(dtype, screening=2).topk(*_args(xd, K), stats=True)
+    assert torch.equal(sampled, dense)
+    assert st_s["exact_pairs"] + st_s["rejected_pairs"] == st_s["visible_pairs"]
     assert stats["exact_pairs"] + stats["rejected_pairs"] == stats["visible_pairs"]
     # about half the rows prune most of their keys, the other half hardly any
     prune = stats["rejected_pairs"] / stats["visible_pairs"]
@@ -413,3 +417,27 @@ def test_survivor_streams_every_item(cuda_lib, redundant):
     ov = OracleView(x, dtype)
     for t in range(0, T, 9):
         assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
+
+
+def test_probe_samples_items_first(cuda_lib):
+    """Adaptive screening probes every 7th work item (longest rows first)
+    before the others.  On random inputs no sampled item finds screening worth
+    it, so the other items are neither set up nor probed: only the sampled
+    items' probe steps are screened.  On redundant heads the sample finds it
+    worth it and every item is probed (most pairs end up rejected).  The
+    selection is the dense path's either way."""
+    _, x, xd = _inputs("prefill_128k_fp8", 640, 6000, 300)
+    K = 300
+    idx = binding.Index("fp8")
+    out, st = idx.topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out), to_numpy(idx.dense_topk(*_args(xd, K))))
+    n_items = 640 // 8
+    sampled = (n_items + 6) // 7
+    assert 0 < st["screened_pairs"] <= sampled * 8 * 4 * 128, st
+    assert st["exact_pairs"] + st["rejected_pairs"] == st["visible_pairs"]
+    x2, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=True)
+    xd2 = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x2.items()}
+    K2 = 32
+    out2, st2 = binding.Index(dtype).topk(*_args(xd2, K2), stats=True)
+    assert np.array_equal(to_numpy(out2), to_numpy(binding.Index(dtype).dense_topk(*_args(xd2, K2))))
+    assert st2["rejected_pairs"] > st2["visible_pairs"] // 2, st2
