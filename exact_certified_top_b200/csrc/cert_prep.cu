@@ -700,8 +700,11 @@ cudaError_t launch_probe_resolve(int* item_flag, int n_items, const int* gate,
                                  cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
   const int grid = (n_items + 255) / 256 < 1024 ? (n_items + 255) / 256 : 1024;
+  profile_before(DOSA_KERNEL_CERT_SETUP, stream);
   probe_resolve_kernel<<<grid, 256, 0, stream>>>(item_flag, n_items, gate);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  profile_after(DOSA_KERNEL_CERT_SETUP, stream);
+  return e;
 }
 
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
