@@ -58,12 +58,14 @@ struct ScoreParams {
   int n_items;
   int H;                 // heads per query row: 32 or 64 (the MMA always sees 64)
   int* err;
-  // Row-list mode (rows repaired after a candidate-list overflow): item i scores
-  // the single row row0 + row_list[i] into output row i; the number of items
-  // is min(*row_count, list_cap), read on the device.
+  // Row-list mode (rows repaired after a candidate-list overflow): item i
+  // scores part i % parts of the key tiles of the single row
+  // row0 + row_list[i / parts] into output row i / parts; the number of rows is
+  // min(*row_count, list_cap), read on the device.
   const int* row_list;
   const int* row_count;
   int list_cap;
+  int parts;
 };
 
 struct ItemGeom {
@@ -72,16 +74,17 @@ struct ItemGeom {
   int64_t pos_first;
   int64_t out0;   // output row of query t0
   int nkt;        // key tiles 0..nkt-1 cover keys 0..pos_last
+  int j0, j1;     // the key tiles this item scores (empty item when j1 <= j0)
 };
 
 __device__ __forceinline__ ItemGeom item_geom(const ScoreParams& p, int item) {
   ItemGeom g;
   if (p.row_list) {
-    const int64_t r = p.row_list[item];
+    const int64_t r = p.row_list[item / p.parts];
     g.t0 = p.row0 + r;
     g.nq = 1;
     g.pos_first = p.pos0 + r;
-    g.out0 = item;
+    g.out0 = item / p.parts;
   } else {
     const int tile = p.n_items - 1 - item;  // longest rows first
     g.t0 = p.row0 + (int64_t)tile * kQueryTile;
@@ -92,6 +95,13 @@ __device__ __forceinline__ ItemGeom item_geom(const ScoreParams& p, int item) {
   }
   const int64_t pos_last = g.pos_first + g.nq - 1;
   g.nkt = (int)(pos_last / kKeyTile) + 1;
+  g.j0 = 0;
+  g.j1 = g.nkt;
+  if (p.row_list) {
+    const int part = item % p.parts;
+    g.j0 = (int)((int64_t)g.nkt * part / p.parts);
+    g.j1 = (int)((int64_t)g.nkt * (part + 1) / p.parts);
+  }
   return g;
 }
 
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
   using C = ScoreCfg<kFp8>;
   if (p.row_list) {
     const int n = *p.row_count;
-    p.n_items = n < p.list_cap ? n : p.list_cap;
+    p.n_items = (n < p.list_cap ? n : p.list_cap) * p.parts;
     if (p.n_items <= 0) return;
   }
   extern __shared__ uint8_t smem_raw[];
@@ -158,8 +168,9 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
       int it = 0;
       uint32_t inflight_q = 0xFFFFFFFFu;   // item parity of the last Q load
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const ItemGeom g = item_geom(p, item);
+        if (g.j1 <= g.j0) continue;
         if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
         mbar_arrive_expect_tx(q_full, C::kQBytes);
         for (int sub = 0; sub < C::kSub; ++sub)
@@ -167,7 +178,8 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
             tma_load_3d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64, 0,
                         (int32_t)(g.t0 + b * 4));
         inflight_q = it & 1;
-        for (int j = 0; j < g.nkt; ++j, ++kc) {
+        ++it;
+        for (int j = g.j0; j < g.j1; ++j, ++kc) {
           const int st = kc % C::kKeyStages;
           const uint32_t rnd = kc / C::kKeyStages;
           if (!mbar_wait(&k_empty[st], (rnd & 1) ^ 1, s_abort, p.err)) {
@@ -194,11 +206,13 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
       uint32_t kc = 0, u = 0;
       int it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const ItemGeom g = item_geom(p, item);
+        if (g.j1 <= g.j0) continue;
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
+        ++it;
         tc_fence_after();
-        for (int j = 0; j < g.nkt && ok; ++j, ++kc) {
+        for (int j = g.j0; j < g.j1 && ok; ++j, ++kc) {
           const int st = kc % C::kKeyStages;
           const uint32_t rnd = kc / C::kKeyStages;
           if (!mbar_wait(&k_full[st], rnd & 1, s_abort, p.err)) {
@@ -245,6 +259,7 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const ItemGeom g = item_geom(p, item);
+      if (g.j1 <= g.j0) continue;
       // this warp's queries sub (MMA tile 0) and 4 + sub (MMA tile 1)
       const int qa = sub, qb = C::kQPerGroup + sub;
       const bool va = qa < g.nq, vb = qb < g.nq;
@@ -260,7 +275,7 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
       float* ra = p.scores + (g.out0 + (va ? qa : 0)) * p.ld;
       float* rb = p.scores + (g.out0 + (vb ? qb : 0)) * p.ld;
       const uint32_t col0 = tmem_base + lane_off + sub * 64;
-      for (int j = 0; j < g.nkt && ok; ++j) {
+      for (int j = g.j0; j < g.j1 && ok; ++j) {
         const int s = j * kKeyTile + quad * 32 + lane;
         float sk = 1.0f;
         if constexpr (kFp8) sk = (s < p.S) ? __ldg(p.k_scale + s) : 0.0f;
@@ -277,6 +292,12 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
           // 32 heads at a time (the register budget of 18 warps is 96 per thread)
           const uint32_t col = col0 + buf * C::kGroupRows;
           const float* wq = grp ? wb : wa;
+          if (!(grp ? vb : va)) {
+            // a query slot the item does not have (partial tiles, row lists)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            continue;
+          }
           float v[32];
           HeadAcc acc = {0.f, 0.f, 0.f, 0.f};
           tmem_ld32_async(col, v);
@@ -290,7 +311,7 @@ __global__ void __launch_bounds__(ScoreCfg<kFp8>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
           head_accumulate32(acc, v, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
-          if (grp ? vb : va) {
+          {
             float sc = head_total(acc);
             if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
             if (s <= (grp ? pos_b : pos_a)) (grp ? rb : ra)[s] = sc;
@@ -381,7 +402,16 @@ static cudaError_t launch_impl(const SeqView& v, float* scores, int64_t ld, int*
   p.row_list = row_list;
   p.row_count = row_count;
   p.list_cap = list_cap;
-  if (row_list) p.n_items = list_cap;
+  // row lists: each row's key tiles split into parts of at least 64 tiles,
+  // so that a few long rows still spread over every SM
+  p.parts = 1;
+  if (row_list) {
+    const int64_t nkt = (v.pos0 + v.rows - 1) / kKeyTile + 1;
+    int64_t parts = nkt / 64;
+    if (parts > 2 * sms) parts = 2 * sms;
+    p.parts = parts < 1 ? 1 : (int)parts;
+    p.n_items = list_cap * p.parts;
+  }
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_SCORE, stream);

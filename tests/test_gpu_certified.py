@@ -201,11 +201,13 @@ def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
 
 
 @pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
-def test_repair_pass_when_candidates_overflow(cuda_lib, screening):
+@pytest.mark.parametrize("S", [5200, 70000])
+def test_repair_pass_when_candidates_overflow(cuda_lib, screening, S):
     """All keys identical: every score ties, every key becomes a candidate and
     the candidate list overflows; the rows are rescored densely and the
-    selection (ties to the smaller index) is still exact."""
-    T, S, K = 40, 5200, 64
+    selection (ties to the smaller index) is still exact.  With 70,000 keys
+    each repaired row's key tiles are split over several work items."""
+    T, K = 40, 64
     g = torch.Generator().manual_seed(5)
     q = torch.randn((T, 64, 128), generator=g).to(torch.bfloat16)
     w = torch.randn((T, 64), generator=g) / 8
