@@ -53,7 +53,7 @@ class Stats(ctypes.Structure):
                 ("screened_pairs", ctypes.c_int64), ("rejected_pairs", ctypes.c_int64),
                 ("exact_pairs", ctypes.c_int64), ("candidates", ctypes.c_int64),
                 ("filtered_pairs", ctypes.c_int64), ("block_skipped_pairs", ctypes.c_int64),
-                ("rescored_pairs", ctypes.c_int64)]
+                ("rescored_pairs", ctypes.c_int64), ("repaired_rows", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: int(getattr(self, name)) for name, _ in self._fields_}

@@ -267,6 +267,7 @@ struct PublishOut {
   int repair_cap;
   int dense;           // the selection reads a dense score matrix: no repair needed
   int* err;
+  unsigned long long* n_repair;   // rows registered for the repair, all chunks
 };
 
 // Owner lane 0: publish a finished query (segment counts as of the last
@@ -278,6 +279,7 @@ __device__ __forceinline__ void publish_query(const QState& q, const PublishOut&
   for (int j = 0; j < kSegs; ++j) cc[j] = over ? -1 : q.seg[j];
   o.tau[q.row] = q.tau;
   if (over && !o.dense) {
+    atomicAdd(o.n_repair, 1ull);
     const int r = atomicAdd(o.repair_count, 1);
     if (r < o.repair_cap) o.repair_list[r] = (int)q.row;
     else record_error(o.err, kDevBounds);

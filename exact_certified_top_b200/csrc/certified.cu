@@ -619,6 +619,7 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
+  p.out.n_repair = b.counters + kCntOverflow;
   p.out.dense = b.dense != nullptr;
   p.out.err = b.err;
   p.dense = b.dense;

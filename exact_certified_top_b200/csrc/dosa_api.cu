@@ -576,6 +576,7 @@ static dosa_status read_stats(const void* workspace, const int64_t* seq_offsets,
   stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
   stats->block_skipped_pairs = (int64_t)hdr.counters[kCntBlockSkipped];
   stats->rescored_pairs = (int64_t)hdr.counters[kCntRescored];
+  stats->repaired_rows = (int64_t)hdr.counters[kCntOverflow];
   if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
   return DOSA_OK;
 }

@@ -403,6 +403,7 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
+  p.out.n_repair = b.counters + kCntOverflow;
   p.out.dense = b.dense != nullptr;
   p.dense = b.dense;
   p.dense_ld = b.dense_ld;

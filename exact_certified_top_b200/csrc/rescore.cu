@@ -373,6 +373,7 @@ static cudaError_t launch_rescore_impl(const Handle& h, const SeqView& v, const 
   p.out.repair_list = b.repair_list;
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
+  p.out.n_repair = b.counters + kCntOverflow;
   p.out.dense = 0;
   p.out.err = b.err;
   p.counters = b.counters;

@@ -134,6 +134,8 @@ typedef struct {
   int64_t block_skipped_pairs; /* rejected pairs of key tiles skipped whole by the
                                   key-block certificate (keys never loaded)      */
   int64_t rescored_pairs;  /* exact pairs scored from gathered survivor streams     */
+  int64_t repaired_rows;   /* rows whose candidate list overflowed and were scored
+                              again densely (at most 64 per chunk of rows)       */
 } dosa_stats;
 
 typedef struct dosa_index* dosa_index_t;

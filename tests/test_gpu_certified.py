@@ -215,10 +215,12 @@ def test_repair_pass_when_candidates_overflow(cuda_lib, screening, S):
     so = [[0, 0, S - T], [T, S, 0]]
     idx = binding.Index("bf16", screening=screening)
     qd, wd, kd = q.cuda(), w.cuda(), k.cuda()
-    cert = to_numpy(idx.topk(qd, None, wd, kd, None, so, K))
+    cert, stats = idx.topk(qd, None, wd, kd, None, so, K, stats=True)
+    cert = to_numpy(cert)
     dense = to_numpy(idx.dense_topk(qd, None, wd, kd, None, so, K))
     assert np.array_equal(cert, dense)
     assert np.array_equal(cert, np.tile(np.arange(K, dtype=np.int32), (T, 1)))
+    assert stats["repaired_rows"] == T
 
 
 @pytest.mark.parametrize("case", [("prefill_128k_fp8", 203, 2600, 300), ("causal_1k_bf16", 300, 1900, 64)],
