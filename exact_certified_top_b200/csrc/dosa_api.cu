@@ -384,16 +384,24 @@ dosa_status dosa_index_dense_topk(dosa_index_t hh, const void* q, const float* q
 
 }  // extern "C"
 
-// Runs key prep and certificate setup for one sequence chunk by chunk, calling
+// Whether a chunk whose longest row has max_tiles key tiles is screened at
+// all: never with screening off; in the adaptive mode only when some row
+// has key tiles past the warm-up and the probe (before them every pair is
+// scored exactly, so the chunk goes to the filter scorer alone).
+static bool screening_can_act(const Handle* h, int64_t max_tiles, int K) {
+  if (h->cfg.screening == 2) return max_tiles > warmup_steps(K) + kProbeSteps;
+  return h->cfg.screening != 0;
+}
+
 // The certificate set-up of a chunk.  With every row's record wanted (or
 // screening on every item) all rows are set up; with screening off none; in
 // the adaptive mode only the rows of the sampled items, the others after the
 // sampled probe, if it found an item worth screening (cert_chunk).
 static dosa_status setup_chunk(const Handle* h, const SeqView& c, CertBuffers& cb, bool records,
-                               cudaStream_t stream) {
+                               int K, cudaStream_t stream) {
   const int mode = h->cfg.screening;
   cb.probe_sample = 0;
-  if (!records && mode == 0) return DOSA_OK;
+  if (!records && !screening_can_act(h, (c.pos0 + c.rows - 1) / kKeyTile + 1, K)) return DOSA_OK;
   if (!records && mode == 2 && h->cfg.probe_sample) {
     const int64_t n_items = (c.rows + 7) / 8;
     if (cudaMemsetAsync(cb.item_flag, 0, (size_t)n_items * 4, stream) != cudaSuccess ||
@@ -410,6 +418,7 @@ static dosa_status setup_chunk(const Handle* h, const SeqView& c, CertBuffers& c
              : DOSA_ERR_CUDA;
 }
 
+// Runs key prep and certificate setup for one sequence chunk by chunk, calling
 // `body(chunk view, buffers)` after each setup.
 template <typename Body>
 static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const float* q_scale,
@@ -431,7 +440,8 @@ static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const flo
     if (v.rows == 0) continue;
     if (launch_key_prep(*h, v.k, v.k_scale, v.S, buf.key_norm, buf.key_sum, stream) !=
             cudaSuccess ||
-        (buf.blk && launch_block_prep(*h, v.k, v.k_scale, v.S, buf.blk, stream) != cudaSuccess))
+        (buf.blk && screening_can_act(h, (v.S + kKeyTile - 1) / kKeyTile, K) &&
+         launch_block_prep(*h, v.k, v.k_scale, v.S, buf.blk, stream) != cudaSuccess))
       return DOSA_ERR_CUDA;
     for (int64_t r = 0; r < v.rows; r += Tc) {
       SeqView c = v;
@@ -441,7 +451,7 @@ static dosa_status for_each_cert_chunk(const Handle* h, const void* q, const flo
       CertBuffers cb = buf;
       if (cert_out) cb.cert = cert_out + c.row0 * kCertFloats;
       if (retained_out) cb.retained = retained_out + c.row0 * 4;
-      dosa_status st = setup_chunk(h, c, cb, cert_out != nullptr, stream);
+      dosa_status st = setup_chunk(h, c, cb, cert_out != nullptr, K, stream);
       if (st != DOSA_OK) return st;
       st = body(c, cb);
       if (st != DOSA_OK) return st;
@@ -464,7 +474,8 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
   // 2: warm-up by the filter scorer, a probe of kProbeSteps screened steps,
   // then each item finished by the scorer its probe chose
   constexpr int kAll = 0x3FFFFFFF;
-  const int mode = h->cfg.screening;
+  const int mode =
+      screening_can_act(h, (c.pos0 + c.rows - 1) / kKeyTile + 1, K) ? h->cfg.screening : 0;
   // With the key-block certificate, the certified scorer's last range is
   // first screened tile by tile as a whole (block_screen) and then processes
   // the steps left.
@@ -781,13 +792,14 @@ dosa_status dosa_index_topk_host(dosa_index_t hh, const void* q, const float* q_
     if (ch.b != prev_b) {
       if (launch_key_prep(*h, c.k, c.k_scale, c.S, buf.key_norm, buf.key_sum, main) !=
               cudaSuccess ||
-          (buf.blk && launch_block_prep(*h, c.k, c.k_scale, c.S, buf.blk, main) != cudaSuccess))
+          (buf.blk && screening_can_act(h, (c.S + kKeyTile - 1) / kKeyTile, K) &&
+           launch_block_prep(*h, c.k, c.k_scale, c.S, buf.blk, main) != cudaSuccess))
         return DOSA_ERR_CUDA;
       prev_b = ch.b;
     }
     if (!ok(cudaStreamWaitEvent(main, h->ev_loaded[slot], 0))) return DOSA_ERR_CUDA;
     CertBuffers cb = buf;
-    st = setup_chunk(h, c, cb, false, main);
+    st = setup_chunk(h, c, cb, false, K, main);
     if (st != DOSA_OK) return st;
     st = cert_chunk(h, c, cb, K, dout, main);
     if (st != DOSA_OK) return st;
