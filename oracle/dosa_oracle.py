@@ -21,7 +21,7 @@ definition: decode the stored inputs exactly, score every visible key in fp64,
 sort, take K.  The certificate half follows the steps of [DPC] Method in order
 (seed threshold, three bound stages, tile-by-tile refinement); the pages print
 no formula, so every formula here is the plainest construction consistent with
-the wording, and each reading is listed in the design doc.
+the wording; the docstring of each function states the reading it takes.
 
 Parity status of each function (pins live in tests/test_oracle_*.py):
   decode_bf16, decode_e4m3 ...... pinned (format definitions, hand values, torch)
@@ -30,6 +30,8 @@ Parity status of each function (pins live in tests/test_oracle_*.py):
   nnls_retained ................. pinned (grid search, KKT conditions)
   certificate_setup/upper_bound . pinned (UB >= I invariant, closed-form reductions)
   certified_topk_row ............ pinned (equals dense selection; tau <= K-th)
+  key_block_stats/block_upper_bound  pinned (bound >= every key's UB in the
+                                  block, single-key blocks reduce to UB)
   prune rates ................... parity unpinned against the pages (their ~97 %
                                   is measured on trained indexers); pinned only
                                   by the ideal-rate upper limit.
