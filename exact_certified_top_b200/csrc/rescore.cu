@@ -15,7 +15,7 @@
 // with the same arithmetic as every other scorer, so the scores are bit-equal
 // to the dense path's.  Scores >= the row's running threshold are appended to
 // its candidate lists; the threshold is refreshed from the histogram every 8
-// chunks; the row is published at its end.
+// chunks and once more at the row's end.
 //
 // A launch covers one step range of the items flagged want_flag (all items
 // when want_flag < 0): rows are published when the range reaches their
