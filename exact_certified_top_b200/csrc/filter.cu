@@ -5,12 +5,16 @@
 // filtering and packed writeback; GPU kernel design: fixed-width query tiles on
 // dense tensor-core matrix operations).
 //
-// Same tile machinery as the dense scorer (score_tc.cu): A = 128 keys x d,
-// B = 4 queries x 64 heads (N = 256), two 256-column TMEM accumulators, one
-// persistent CTA per SM with a TMA producer warp, an MMA warp and 8 epilogue
-// warps.  The epilogue differs: instead of storing every score it keeps the
-// candidate state of the item's 8 queries in shared memory (cand_state.cuh)
-// and appends only scores >= tau_t, refreshing tau_t every 8 key tiles.
+// Tiles: A = 128 keys x d, B = 2 queries x 64 heads (N = 128).  Key tiles
+// are taken two at a time: each of the two 256-column TMEM accumulators holds
+// one query pair against both tiles (tile 0 in columns 0-127, tile 1 in
+// 128-255), so an epilogue thread reduces two keys of the same query per
+// accumulator wait, with the query's weights loaded once for both.  One
+// persistent CTA per SM runs a TMA producer warp, an MMA warp and 16 epilogue
+// warps in two teams of 8 (team t drains accumulator t: query pairs t and
+// t + 2).  The epilogue keeps the candidate state of the item's 8 queries in
+// shared memory (cand_state.cuh) and appends only scores >= tau_t,
+// refreshing tau_t every 8 key tiles.
 //
 // A launch processes a range of steps of every item (work_items.cuh): the
 // warm-up tiles before screening starts, the rest of the items that the
@@ -32,9 +36,9 @@ struct FilterCfg {
   static constexpr int kH = 64;
   static constexpr int kQT = kItemQueries;
   static constexpr int kQRows = kQT * kH;
-  static constexpr int kGroupRows = 256;               // MMA N: 4 queries
-  static constexpr int kGroups = kQRows / kGroupRows;
-  static constexpr int kQPerGroup = kGroupRows / kH;
+  static constexpr int kGroupRows = 128;               // MMA N: 2 queries
+  static constexpr int kGroups = kQRows / kGroupRows;  // 4 query pairs
+  static constexpr int kBufCols = 256;                 // a query pair over two key tiles
   static constexpr uint32_t kKeySubBytes = kKeyTile * 128;
   static constexpr uint32_t kKeyStageBytes = kKeySubBytes * kSub;
   static constexpr uint32_t kQSubBytes = kQRows * 128;
@@ -99,7 +103,7 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], C::kEpiWarps);
+      mbar_init(&acc_empty[i], C::kEpiWarps / 2);   // one team of 8 warps per buffer
     }
     mbar_init(tile_done, C::kEpiWarps);
     mbar_init(item_ready, C::kEpiWarps);
@@ -175,14 +179,17 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
         if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
         ++it;
         tc_fence_after();
-        for (int ti = rg.begin; ti < rg.end && ok; ++ti, ++kc) {
-          const int s_ = kc % C::kKeyStages;
-          if (!mbar_wait(&k_full[s_], (kc / C::kKeyStages) & 1, s_abort, p.err)) {
+        for (int ti = rg.begin; ti < rg.end && ok; ti += 2) {
+          const bool two = ti + 1 < rg.end;
+          const int sa = kc % C::kKeyStages, sb = (kc + 1) % C::kKeyStages;
+          if (!mbar_wait(&k_full[sa], (kc / C::kKeyStages) & 1, s_abort, p.err) ||
+              (two && !mbar_wait(&k_full[sb], ((kc + 1) / C::kKeyStages) & 1, s_abort, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
+          const uint32_t a0 = smem_u32(sK + sa * C::kKeyStageBytes);
+          const uint32_t a1 = smem_u32(sK + sb * C::kKeyStageBytes);
           for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
             const uint32_t buf = u & 1;
             if (!mbar_wait(&acc_empty[buf], ((u >> 1) & 1) ^ 1, s_abort, p.err)) {
@@ -191,17 +198,23 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             }
             tc_fence_after();
             const uint32_t b_base = smem_u32(sQ + grp * C::kGroupRows * 128);
-            const uint32_t d = tmem_base + buf * C::kGroupRows;
+            for (int t = 0; t < (two ? 2 : 1); ++t) {
+              const uint32_t a_base = t ? a1 : a0;
+              const uint32_t d = tmem_base + buf * C::kBufCols + t * C::kGroupRows;
 #pragma unroll
-            for (int step = 0; step < C::kKSteps; ++step) {
-              const uint32_t sub = step >> 2, off = (step & 3) * 32;
-              tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
-                           smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc,
-                           step > 0 ? 1u : 0u);
+              for (int step = 0; step < C::kKSteps; ++step) {
+                const uint32_t sub = step >> 2, off = (step & 3) * 32;
+                tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
+                             smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc,
+                             step > 0 ? 1u : 0u);
+              }
             }
             tc_commit(&acc_full[buf]);
           }
-          tc_commit(&k_empty[s_]);
+          if (!ok) break;
+          tc_commit(&k_empty[sa]);
+          if (two) tc_commit(&k_empty[sb]);
+          kc += two ? 2 : 1;
         }
         tc_commit(q_empty);
       }
@@ -211,15 +224,16 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
   } else {
     // ---------------- epilogue ----------------
     // 16 warps: warp (2 + ew) reads TMEM lane quadrant (warp & 3), i.e. 32
-    // keys, and query (ew >> 2) of each 4-query MMA tile.  Warps 0-7 of the
-    // epilogue also own query slot ew (state set-up, threshold refresh,
-    // publication).
+    // keys of each key tile, in team (ew >> 2) & 1, for query (ew >> 3) of
+    // each query pair.  Warps 0-7 of the epilogue also own query slot ew
+    // (state set-up, threshold refresh, publication).
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int sub = ew >> 2;
+    const int team = sub & 1, qsel = sub >> 1;   // buffer and query within the pair
     const bool owner = ew < C::kQT;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint32_t u = 0, nbar = 0;
+    uint32_t uu = 0, nbar = 0;
     int it = 0;
     unsigned long long n_seed = 0, n_exact = 0, n_cand = 0;
     bool ok = true;
@@ -265,9 +279,11 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       if (lane == 0) mbar_arrive(item_ready);
       if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
       ++it;
-      // Per item: this warp's queries sub (MMA tile 0) and 4 + sub (tile 1),
-      // their positions, weight rows, scales, list segments and counts.
-      const int qa = sub, qb = C::kQPerGroup + sub;
+      // Per item: this warp's two queries, qa (query pair `team`) and qb = qa + 4
+      // (query pair team + 2), their positions, weight rows, scales, list
+      // segments and counts.  Per pair of key tiles the warp takes 2 keys of
+      // qa, then 2 keys of qb, from buffer `team`.
+      const int qa = 2 * team + qsel, qb = qa + 4;
       const bool va = qa < g.nq, vb = qb < g.nq;
       const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
       const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * kHeads;
@@ -282,53 +298,78 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       Cand* lb = p.cand + ((g.local0 + qb) * kSegs + quad) * (int64_t)p.seg_cap;
       int cnt_a = *reinterpret_cast<volatile int*>(&st[qa].seg[quad]);
       int cnt_b = *reinterpret_cast<volatile int*>(&st[qb].seg[quad]);
-      const uint32_t col0 = tmem_base + lane_off + sub * 64;
-      for (int i = 0; i < n && ok; ++i) {
-        const int s = tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
-        float sk = 1.f;
-        if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
+      const uint32_t col0 = tmem_base + lane_off + team * C::kBufCols + qsel * C::kH;
+      for (int i = 0; i < n && ok; i += 2) {
+        const bool two = i + 1 < n;
+        const int s0 = tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        const int s1 = two ? tile_at(rg.begin + i + 1, g.n_tiles) * kKeyTile + quad * 32 + lane
+                           : 0x7FFFFFFF;
+        float sk0 = 1.f, sk1 = 1.f;
+        if constexpr (kFp8) {
+          sk0 = s0 < p.S ? __ldg(p.k_scale + s0) : 0.f;
+          sk1 = s1 < p.S ? __ldg(p.k_scale + s1) : 0.f;
+        }
 #pragma unroll
-        for (int grp = 0; grp < C::kGroups; ++grp) {
+        for (int use = 0; use < 2; ++use) {
           if (!ok) continue;
-          const uint32_t buf = u & 1;
-          if (!mbar_wait(&acc_full[buf], (u >> 1) & 1, s_abort, p.err)) {
+          if (!mbar_wait(&acc_full[team], uu & 1, s_abort, p.err)) {
             ok = false;
             continue;
           }
-          ++u;
+          ++uu;
           tc_fence_after();
-          // 32 heads at a time (the register budget of 18 warps is 96 per thread)
-          const uint32_t col = col0 + buf * C::kGroupRows;
-          const float* wq = grp ? wb : wa;
-          float x[32];
-          HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-          tmem_ld32_async(col, x);
-          tmem_wait_ld(x);
-          if (h64) {
-            head_accumulate32(acc, x, wq);
-            tmem_ld32_async(col + 32, x);
-            tmem_wait_ld(x);
+          const float* wq = use ? wb : wa;
+          HeadAcc2 acc0 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          HeadAcc2 acc1 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float x[16];
+          float4 w4[4];
+          constexpr int kQuarters = h64 ? 4 : 2;
+#pragma unroll
+          for (int hh = 0; hh < kQuarters; ++hh) {
+            load_w16(w4, wq + 16 * hh);
+            tmem_ld16_async(col0 + 16 * hh, x);
+            tmem_wait_ld16(x);
+            head_accumulate16w(acc0, x, w4);
+            if (two) {
+              tmem_ld16_async(col0 + C::kGroupRows + 16 * hh, x);
+              tmem_wait_ld16(x);
+            }
+            if (hh == kQuarters - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[team]);
+            }
+            if (two) head_accumulate16w(acc1, x, w4);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          head_accumulate32(acc, x, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
-          if (grp ? vb : va) {
-            QState& q = st[grp ? qb : qa];
-            float sc = head_total(acc);
-            if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
-            const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
-            int& cnt = grp ? cnt_b : cnt_a;
-            n_cand += append_candidates(q, grp ? lb : la, p.seg_cap, cnt,
-                                        s <= (grp ? pos_b : pos_a) && sc >= tau, sc, s, lane);
-            if constexpr (kDense)
-              if (s <= (grp ? pos_b : pos_a))
-                p.dense[(g.local0 + (grp ? qb : qa)) * p.dense_ld + s] = sc;
+          if (use ? vb : va) {
+            QState& q = st[use ? qb : qa];
+            const float qs = use ? qsb : qsa;
+            const int pos = use ? pos_b : pos_a;
+            float sc0 = head_total(acc0), sc1 = head_total(acc1);
+            if constexpr (kFp8) {
+              sc0 *= qs * sk0;
+              sc1 *= qs * sk1;
+            }
+            int& cnt = use ? cnt_b : cnt_a;
+            Cand* lst = use ? lb : la;
+            float tau = *reinterpret_cast<const volatile float*>(&q.tau);
+            n_cand += append_candidates(q, lst, p.seg_cap, cnt, s0 <= pos && sc0 >= tau, sc0, s0,
+                                        lane);
+            if (two) {
+              tau = *reinterpret_cast<const volatile float*>(&q.tau);
+              n_cand += append_candidates(q, lst, p.seg_cap, cnt, s1 <= pos && sc1 >= tau, sc1,
+                                          s1, lane);
+            }
+            if constexpr (kDense) {
+              float* drow = p.dense + (g.local0 + (use ? qb : qa)) * p.dense_ld;
+              if (s0 <= pos) drow[s0] = sc0;
+              if (two && s1 <= pos) drow[s1] = sc1;
+            }
           }
         }
         if (!ok) break;
         // ---- checkpoint: every kCkptTiles steps and at the item's last ----
-        if (((i + 1) % kCkptTiles) == 0 || i + 1 == n) {
+        if (((i + 2) % kCkptTiles) == 0 || i + 2 >= n) {
           // publish this warp's segment counts (see certified.cu)
           if (lane == 0) {
             st[qa].seg[quad] = cnt_a;
