@@ -50,6 +50,8 @@ def parse_args():
                     help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
     ap.add_argument("--block-bound", type=int, choices=[0, 1], default=1,
                     help="certified path: skip key tiles whose key-block bound rules them out")
+    ap.add_argument("--probe-sample", type=int, choices=[0, 1], default=1,
+                    help="adaptive screening: probe every 7th work item first (1) or every item (0)")
     ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
                     help="certified path: packed candidates >= threshold (default), or every "
                          "exact score into a dense matrix and its dense Top-K (ablation)")
@@ -312,10 +314,11 @@ def oracle_sample(x, wl, budget_s: float):
 
 # ---------------------------------------------------------------------------
 
-def config_of(wl, path, world, screening=None, writeback=None):
+def config_of(wl, path, world, screening=None, writeback=None, ablations=None):
     extra = {"screening": screening} if screening is not None else {}
     if writeback is not None:
         extra["writeback"] = writeback
+    extra.update(ablations or {})
     return {"workload": wl.name, "T": wl.T, "S": wl.S, "H": wl.H, "d": wl.d, "K": wl.K,
             "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, **extra,
             "parallelism": f"rows x{world}",
@@ -363,7 +366,7 @@ def run_ours(args, world, rank, local):
     x = generate(rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
                         sparse_writeback=int(args.writeback == "sparse"),
-                        block_bound=args.block_bound)
+                        block_bound=args.block_bound, probe_sample=args.probe_sample)
     certified = args.path == "certified"
     decode = args.path == "decode"
     if decode and wl.decode_noise <= 0:
@@ -514,7 +517,10 @@ def run_ours(args, world, rank, local):
                 "dtype": wl.dtype, "data": "synthetic (seeded low-rank + sink generator)",
                 "config": config_of(wl, args.path, world,
                                     args.screening if args.path == "certified" else None,
-                                    args.writeback if args.path == "certified" else None),
+                                    args.writeback if args.path == "certified" else None,
+                                    {k: v for k, v in (("block_bound", args.block_bound),
+                                                       ("probe_sample", args.probe_sample))
+                                     if args.path == "certified" and v != 1}),
                 "roofline": roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "kernels": {k: {"launches": n, "ms": round(t, 3)} for k, t in
