@@ -20,6 +20,8 @@
 // warm-up tiles before screening starts, the rest of the items that the
 // certified kernel's probe found screening does not pay for (resuming their
 // state), or every tile when screening is switched off.
+#include <type_traits>
+
 #include "cand_state.cuh"
 #include "dosa_device.cuh"
 #include "dosa_internal.h"
@@ -51,6 +53,29 @@ struct FilterCfg {
       1024 + kQBytes + kKeyStages * kKeyStageBytes + kStateBytes + 256;
 };
 
+template <bool kFp8>
+struct FilterTileCfg {
+  static constexpr int kSub = kFp8 ? 1 : 2;
+  static constexpr int kKSteps = kFp8 ? 4 : 8;
+  static constexpr int kKeyStages = kFp8 ? 4 : 2;
+  static constexpr int kH = 64;
+  static constexpr int kQT = kItemQueries;
+  static constexpr int kQRows = kQT * kH;
+  static constexpr int kGroupRows = 256;               // MMA N: 4 queries
+  static constexpr int kGroups = kQRows / kGroupRows;
+  static constexpr int kQPerGroup = kGroupRows / kH;
+  static constexpr uint32_t kKeySubBytes = kKeyTile * 128;
+  static constexpr uint32_t kKeyStageBytes = kKeySubBytes * kSub;
+  static constexpr uint32_t kQSubBytes = kQRows * 128;
+  static constexpr uint32_t kQBytes = kQSubBytes * kSub;
+  static constexpr int kEpiWarps = 16;                 // 4 per TMEM lane quadrant
+  static constexpr int kThreads = 64 + kEpiWarps * 32;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kStateBytes = sizeof(QState) * kQT;
+  static constexpr uint32_t kSmemBytes =
+      1024 + kQBytes + kKeyStages * kKeyStageBytes + kStateBytes + 256;
+};
+
 struct FilterParams {
   const float* w;          // [rows_total, 64] absolute rows
   const float* q_scale;    // absolute rows (fp8)
@@ -68,6 +93,313 @@ struct FilterParams {
   int64_t dense_ld;
   StepRange steps;         // what this launch processes
 };
+
+// One key tile per accumulator wait (B = 4 queries x 64 heads, N = 256, two
+// 256-column accumulators; 16 epilogue warps, each reducing one key of a
+// query per wait).  Used for bf16, whose two-stage key pipeline (the 8-query
+// bf16 Q tile takes 128 KB of shared memory) cannot hold a second key tile
+// ahead of a pair of tiles.
+// kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
+// kDense: also write every exact score to p.dense (the dense-writeback ablation).
+template <bool kFp8, int kHeads, bool kDense>
+__global__ void __launch_bounds__(FilterTileCfg<kFp8>::kThreads, 1)
+    filter_tile_kernel(const __grid_constant__ CUtensorMap qmap,
+                  const __grid_constant__ CUtensorMap kmap, const FilterParams p) {
+  using C = FilterTileCfg<kFp8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + C::kQBytes;
+  QState* st = reinterpret_cast<QState*>(sK + C::kKeyStages * C::kKeyStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(st + C::kQT);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* acc_full = bars + 2;     // [2]
+  uint64_t* acc_empty = bars + 4;    // [2]
+  uint64_t* tile_done = bars + 6;
+  uint64_t* item_ready = bars + 7;
+  uint64_t* done_bar = bars + 8;
+  uint64_t* k_full = bars + 9;                   // [kKeyStages]
+  uint64_t* k_empty = k_full + C::kKeyStages;    // [kKeyStages]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(k_empty + C::kKeyStages);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::kEpiWarps);
+    }
+    mbar_init(tile_done, C::kEpiWarps);
+    mbar_init(item_ready, C::kEpiWarps);
+    mbar_init(done_bar, 1);
+    for (int i = 0; i < C::kKeyStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t kc = 0;
+      int it = 0;
+      bool ok = true;
+      uint32_t inflight_q = 0xFFFFFFFFu;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
+        if (rg.end <= rg.begin) continue;
+        if (!mbar_wait(q_empty, (it & 1) ^ 1, s_abort, p.err)) break;
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        for (int sub = 0; sub < C::kSub; ++sub)
+          for (int b = 0; b < C::kQRows / 256; ++b)
+            tma_load_3d(sQ + sub * C::kQSubBytes + b * 256 * 128, &qmap, q_full, sub * 64, 0,
+                        (int32_t)(g.t0 + b * 4));
+        inflight_q = it & 1;
+        ++it;
+        for (int ti = rg.begin; ti < rg.end; ++ti, ++kc) {
+          const int s_ = kc % C::kKeyStages;
+          const uint32_t rnd = kc / C::kKeyStages;
+          if (!mbar_wait(&k_empty[s_], (rnd & 1) ^ 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[s_], C::kKeyStageBytes);
+          const int j = tile_at(ti, g.n_tiles);
+          for (int sub = 0; sub < C::kSub; ++sub)
+            tma_load_2d(sK + s_ * C::kKeyStageBytes + sub * C::kKeySubBytes, &kmap, &k_full[s_],
+                        sub * 64, j * kKeyTile);
+        }
+      }
+      if (*s_abort) {
+        if (inflight_q != 0xFFFFFFFFu) mbar_wait_drain(q_full, inflight_q);
+        for (uint32_t c = (kc > (uint32_t)C::kKeyStages ? kc - C::kKeyStages : 0); c < kc; ++c)
+          mbar_wait_drain(&k_full[c % C::kKeyStages], (c / C::kKeyStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = make_idesc<kFp8>(kKeyTile, C::kGroupRows);
+      uint32_t kc = 0, u = 0;
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+        const Range rg = item_steps(p.steps, p.item_flag, g, item);
+        if (rg.end <= rg.begin) continue;
+        if (!mbar_wait(q_full, it & 1, s_abort, p.err)) break;
+        ++it;
+        tc_fence_after();
+        for (int ti = rg.begin; ti < rg.end && ok; ++ti, ++kc) {
+          const int s_ = kc % C::kKeyStages;
+          if (!mbar_wait(&k_full[s_], (kc / C::kKeyStages) & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sK + s_ * C::kKeyStageBytes);
+          for (int grp = 0; grp < C::kGroups; ++grp, ++u) {
+            const uint32_t buf = u & 1;
+            if (!mbar_wait(&acc_empty[buf], ((u >> 1) & 1) ^ 1, s_abort, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t b_base = smem_u32(sQ + grp * C::kGroupRows * 128);
+            const uint32_t d = tmem_base + buf * C::kGroupRows;
+#pragma unroll
+            for (int step = 0; step < C::kKSteps; ++step) {
+              const uint32_t sub = step >> 2, off = (step & 3) * 32;
+              tc_mma<kFp8>(d, smem_desc_sw128(a_base + sub * C::kKeySubBytes + off),
+                           smem_desc_sw128(b_base + sub * C::kQSubBytes + off), idesc,
+                           step > 0 ? 1u : 0u);
+            }
+            tc_commit(&acc_full[buf]);
+          }
+          tc_commit(&k_empty[s_]);
+        }
+        tc_commit(q_empty);
+      }
+      tc_commit(done_bar);
+      mbar_wait_drain(done_bar, 0);
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    // 16 warps: warp (2 + ew) reads TMEM lane quadrant (warp & 3), i.e. 32
+    // keys, and query (ew >> 2) of each 4-query MMA tile.  Warps 0-7 of the
+    // epilogue also own query slot ew (state set-up, threshold refresh,
+    // publication).
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int sub = ew >> 2;
+    const bool owner = ew < C::kQT;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint32_t u = 0, nbar = 0;
+    int it = 0;
+    unsigned long long n_seed = 0, n_exact = 0, n_cand = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const Geom g = item_geometry(p.row0, p.rows, p.pos0, p.n_items, item);
+      const Range rg = item_steps(p.steps, p.item_flag, g, item);
+      if (rg.end <= rg.begin) continue;
+      const int n = rg.end - rg.begin;
+      if (owner) {
+        QState& s = st[ew];
+        const bool valid = ew < g.nq;
+        const int64_t row = g.local0 + ew;
+        if (lane == 0) {
+          s.row = row;
+          s.pos = valid ? g.pos_first + ew : -1;
+        }
+        if (valid && rg.begin > 0) state_load(s, p.qstate + row, lane);
+        else state_fresh(s, valid, lane);
+        __syncwarp();
+        __threadfence_block();
+        if (valid && lane == 0) {
+          // Visible and seed pairs of this query in the item's range: step 0
+          // is key tile 0, steps ti >= 1 are key tiles n_tiles - ti.
+          const int64_t pos = g.pos_first + ew;
+          const int64_t nonseed_lo = p.seed_first, nonseed_hi = pos - p.seed_last;
+          long long vis = 0, nonseed = 0;
+          if (rg.begin == 0) {
+            vis += overlap_count(0, kKeyTile - 1, 0, pos);
+            nonseed += overlap_count(0, (kKeyTile - 1 < pos ? kKeyTile - 1 : pos), nonseed_lo,
+                                     nonseed_hi);
+          }
+          const int t_first = rg.begin > 1 ? rg.begin : 1;
+          if (t_first < rg.end) {
+            const int64_t k_lo = (int64_t)(g.n_tiles - (rg.end - 1)) * kKeyTile;
+            const int64_t k_hi = (int64_t)(g.n_tiles - t_first) * kKeyTile + kKeyTile - 1;
+            vis += overlap_count(k_lo, k_hi, 0, pos);
+            nonseed += overlap_count(k_lo, (k_hi < pos ? k_hi : pos), nonseed_lo, nonseed_hi);
+          }
+          n_exact += vis;
+          n_seed += vis - nonseed;
+        }
+      }
+      if (lane == 0) mbar_arrive(item_ready);
+      if (!mbar_wait(item_ready, it & 1, s_abort, p.err)) break;
+      ++it;
+      // Per item: this warp's queries sub (MMA tile 0) and 4 + sub (tile 1),
+      // their positions, weight rows, scales, list segments and counts.
+      const int qa = sub, qb = C::kQPerGroup + sub;
+      const bool va = qa < g.nq, vb = qb < g.nq;
+      const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
+      const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * kHeads;
+      const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * kHeads;
+      constexpr bool h64 = kHeads == 64;
+      float qsa = 1.f, qsb = 1.f;
+      if constexpr (kFp8) {
+        qsa = __ldg(p.q_scale + g.t0 + (va ? qa : 0));
+        qsb = __ldg(p.q_scale + g.t0 + (vb ? qb : 0));
+      }
+      Cand* la = p.cand + ((g.local0 + qa) * kSegs + quad) * (int64_t)p.seg_cap;
+      Cand* lb = p.cand + ((g.local0 + qb) * kSegs + quad) * (int64_t)p.seg_cap;
+      int cnt_a = *reinterpret_cast<volatile int*>(&st[qa].seg[quad]);
+      int cnt_b = *reinterpret_cast<volatile int*>(&st[qb].seg[quad]);
+      const uint32_t col0 = tmem_base + lane_off + sub * 64;
+      for (int i = 0; i < n && ok; ++i) {
+        const int s = tile_at(rg.begin + i, g.n_tiles) * kKeyTile + quad * 32 + lane;
+        float sk = 1.f;
+        if constexpr (kFp8) sk = s < p.S ? __ldg(p.k_scale + s) : 0.f;
+#pragma unroll
+        for (int grp = 0; grp < C::kGroups; ++grp) {
+          if (!ok) continue;
+          const uint32_t buf = u & 1;
+          if (!mbar_wait(&acc_full[buf], (u >> 1) & 1, s_abort, p.err)) {
+            ok = false;
+            continue;
+          }
+          ++u;
+          tc_fence_after();
+          // 32 heads at a time (the register budget of 18 warps is 96 per thread)
+          const uint32_t col = col0 + buf * C::kGroupRows;
+          const float* wq = grp ? wb : wa;
+          float x[32];
+          HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          tmem_ld32_async(col, x);
+          tmem_wait_ld(x);
+          if (h64) {
+            head_accumulate32(acc, x, wq);
+            tmem_ld32_async(col + 32, x);
+            tmem_wait_ld(x);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          head_accumulate32(acc, x, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
+          if (grp ? vb : va) {
+            QState& q = st[grp ? qb : qa];
+            float sc = head_total(acc);
+            if constexpr (kFp8) sc *= (grp ? qsb : qsa) * sk;
+            const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
+            int& cnt = grp ? cnt_b : cnt_a;
+            n_cand += append_candidates(q, grp ? lb : la, p.seg_cap, cnt,
+                                        s <= (grp ? pos_b : pos_a) && sc >= tau, sc, s, lane);
+            if constexpr (kDense)
+              if (s <= (grp ? pos_b : pos_a))
+                p.dense[(g.local0 + (grp ? qb : qa)) * p.dense_ld + s] = sc;
+          }
+        }
+        if (!ok) break;
+        // ---- checkpoint: every kCkptTiles steps and at the item's last ----
+        if (((i + 1) % kCkptTiles) == 0 || i + 1 == n) {
+          // publish this warp's segment counts (see certified.cu)
+          if (lane == 0) {
+            st[qa].seg[quad] = cnt_a;
+            st[qb].seg[quad] = cnt_b;
+          }
+          __threadfence_block();
+          if (lane == 0) mbar_arrive(tile_done);
+          if (!mbar_wait(tile_done, nbar & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          ++nbar;
+          if (owner && ew < g.nq)
+            refresh_threshold(st[ew], p.cand + st[ew].row * kSegs * (int64_t)p.seg_cap, p.seg_cap,
+                              p.K, lane);
+        }
+      }
+      if (ok && owner && ew < g.nq) {
+        if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
+        else if (lane == 0) publish_query(st[ew], p.out);
+      }
+    }
+    if (lane == 0) {
+      atomicAdd(&p.counters[kCntSeedPairs], n_seed);
+      atomicAdd(&p.counters[kCntExact], n_exact);
+      atomicAdd(&p.counters[kCntCandidates], n_cand);
+      atomicAdd(&p.counters[kCntFiltered], n_exact);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
 
 // kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
 // kDense: also write every exact score to p.dense (the dense-writeback ablation).
@@ -410,10 +742,18 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
 
 // ---- host side ---------------------------------------------------------------------
 
+// fp8: the pair kernel (two key tiles per accumulator wait); bf16: the
+// one-tile kernel (see filter_tile_kernel).
+template <bool kFp8, int kHeads, bool kDense>
+constexpr auto filter_fn() {
+  if constexpr (kFp8) return filter_kernel<kFp8, kHeads, kDense>;
+  else return filter_tile_kernel<kFp8, kHeads, kDense>;
+}
+
 template <bool kFp8>
 static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
                                       int K, StepRange steps, cudaStream_t stream) {
-  using C = FilterCfg<kFp8>;
+  using C = std::conditional_t<kFp8, FilterCfg<kFp8>, FilterTileCfg<kFp8>>;
   CUtensorMap qmap, kmap;
   if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
       !encode_rows_map(&kmap, v.k, kFp8, (uint64_t)v.S, kKeyTile))
@@ -421,8 +761,8 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaSuccess;
-    for (auto fn : {filter_kernel<kFp8, 64, false>, filter_kernel<kFp8, 32, false>,
-                    filter_kernel<kFp8, 64, true>, filter_kernel<kFp8, 32, true>})
+    for (auto fn : {filter_fn<kFp8, 64, false>(), filter_fn<kFp8, 32, false>(),
+                    filter_fn<kFp8, 64, true>(), filter_fn<kFp8, 32, true>()})
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmemBytes);
@@ -465,8 +805,8 @@ static cudaError_t launch_filter_impl(const Handle& h, const SeqView& v, const C
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_FILTER, stream);
-  auto fn = v.H == 64 ? (b.dense ? filter_kernel<kFp8, 64, true> : filter_kernel<kFp8, 64, false>)
-                      : (b.dense ? filter_kernel<kFp8, 32, true> : filter_kernel<kFp8, 32, false>);
+  auto fn = v.H == 64 ? (b.dense ? filter_fn<kFp8, 64, true>() : filter_fn<kFp8, 64, false>())
+                      : (b.dense ? filter_fn<kFp8, 32, true>() : filter_fn<kFp8, 32, false>());
   fn<<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_FILTER, stream);
