@@ -88,6 +88,49 @@ def test_certified_varlen_batch(cuda_lib):
     assert np.array_equal(cert, dense)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_varlen_batch_with_empty_sequences(cuda_lib, dtype):
+    """A packed batch whose first and middle sequences have keys but no query
+    rows: the certified, host-staged and dense calls skip them, and every
+    other row's selection is the oracle's (indices relative to its own
+    sequence's first key)."""
+    base = "causal_1k_bf16" if dtype == "bf16" else "prefill_128k_fp8"
+    parts = [small_case(base, 0, 77, seed=4, q_pos0=77),
+             small_case(base, 130, 2300, seed=1, q_pos0=2170),
+             small_case(base, 0, 300, seed=5, q_pos0=300),
+             small_case(base, 24, 500, seed=2, q_pos0=476)]
+    xs = [generate(wl) for wl in parts]
+    cat = lambda key: torch.cat([x[key] for x in xs])
+    q, w, k = cat("q"), cat("w"), cat("k")
+    qs = cat("q_scale") if dtype == "fp8" else None
+    ks = cat("k_scale") if dtype == "fp8" else None
+    so, qr, kr = [], 0, 0
+    for wl in parts:
+        so.append([qr, kr, wl.q_pos0])
+        qr += wl.T
+        kr += wl.S
+    so.append([qr, kr, 0])
+    K = 64
+    dev = lambda t: None if t is None else t.cuda()
+    idx = binding.Index(dtype)
+    cert = to_numpy(idx.topk(dev(q), dev(qs), dev(w), dev(k), dev(ks), so, K))
+    dense = to_numpy(idx.dense_topk(dev(q), dev(qs), dev(w), dev(k), dev(ks), so, K))
+    assert cert.shape == (qr, K)
+    assert np.array_equal(cert, dense)
+    pin = lambda t: None if t is None else t.contiguous().pin_memory()
+    ws = torch.zeros(idx.host_workspace_size(qr, kr, 2300, K), dtype=torch.uint8, device="cuda")
+    host = idx.topk_host(pin(q), pin(qs), pin(w), pin(k), pin(ks), so, K, workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host.numpy(), cert)
+    r = 0
+    for wl, x in zip(parts, xs):
+        if wl.T:
+            ov = OracleView(x, dtype)
+            for t in range(0, wl.T, 5):
+                assert_topk_matches(cert[r + t], ov.scores(t), K, t=(wl.name, t))
+        r += wl.T
+
+
 def _redundant_heads_case(T=96, S=6000, seed=0, fp8=False):
     """Heads of a query are near copies of one direction and weights mostly
     positive: the certificate is tight and most keys are rejected."""
