@@ -312,6 +312,36 @@ def oracle_sample(x, wl, budget_s: float):
             "host_cores": os.cpu_count()}
 
 
+def ideal_prune_sample(x, wl, n_rows: int = 4):
+    """The certificate's ideal prune rate (the oracle's: threshold equal to
+    the true K-th score, the default certificate r = 4, G = 2) and the
+    oracle schedule's own prune rate, on n_rows rows spread over the
+    workload's positions (the longest last)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle import certified_topk_row, dequantize, key_mean
+    from exact_certified_top_b200.workloads import codes_numpy
+    kscale = None if x["k_scale"] is None else x["k_scale"].cpu().numpy()
+    k = dequantize(codes_numpy(x["k"]), kscale, wl.dtype)
+    kb = key_mean(k)
+    pos = x["positions"].cpu().numpy()
+    rows = sorted({int(r) for r in np.linspace(wl.T - 1, 0, n_rows + 1)[:n_rows]})
+    vis = ideal = rej = 0
+    t0 = time.perf_counter()
+    for t in rows:
+        qs = None if x["q_scale"] is None else x["q_scale"][t:t + 1].cpu().numpy()
+        q = dequantize(codes_numpy(x["q"][t:t + 1]), qs, wl.dtype)[0]
+        w = x["w"][t].cpu().numpy().astype(np.float64)
+        p = int(pos[t])
+        res = certified_topk_row(q, w, k[:p + 1], wl.K, k_bar=kb, r=4, G=2, margin_log2=-12)
+        vis += res["visible"]
+        ideal += res["ideal_rejected"]
+        rej += res["rejected"]
+    return {"ideal_prune_pct": round(100.0 * ideal / max(vis, 1), 4),
+            "schedule_prune_pct": round(100.0 * rej / max(vis, 1), 4), "kind": "oracle",
+            "sample": f"rows {rows} of {wl.name} ({vis} visible pairs), "
+                      f"{time.perf_counter() - t0:.1f} s"}
+
+
 # ---------------------------------------------------------------------------
 
 def config_of(wl, path, world, screening=None, writeback=None, ablations=None):
@@ -505,9 +535,11 @@ def run_ours(args, world, rank, local):
         e2e = {"value": world * pairs / (ems * 1e-3), "unit": UNIT, "ms_per_step": round(ems, 3),
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    cpu = None
+    cpu = ideal = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(x, wl, args.cpu_seconds)
+        if certified:
+            ideal = ideal_prune_sample(x, wl)
 
     if rank == 0:
         roof = roofline(prof, wl, pairs, args.steps, wl.dtype, stats)
@@ -530,6 +562,8 @@ def run_ours(args, world, rank, local):
             vis = stats["visible_pairs"]
             line["prune_pct"] = round(100.0 * stats["rejected_pairs"] / vis, 3) if vis else None
             line["stats"] = stats
+        if ideal:
+            line["ideal_prune"] = ideal
         print(json.dumps(line), flush=True)
 
 
