@@ -250,7 +250,7 @@ def _traffic_record(kernel: str, wl):
         return None
     with open(path) as f:
         rec = json.load(f).get(f"{kernel}:{wl.dtype}")
-    if not rec or rec.get("source_sha") != _kernel_source_sha():
+    if not rec or rec.get("source_sha") != _kernel_source_sha(kernel):
         return None
     return rec
 
@@ -263,12 +263,20 @@ def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
     return round(rec["dram_bytes_per_pair"] * pairs_per_launch)
 
 
-def _kernel_source_sha():
+# The sources a kernel's traffic record was taken from: its own file and the
+# headers it includes.
+KERNEL_SOURCES = {
+    "filter": ("filter.cu", "cand_state.cuh", "dosa_device.cuh", "dosa_internal.h",
+               "score_epilogue.cuh", "work_items.cuh"),
+    "decode": ("decode.cu", "cand_state.cuh", "dosa_device.cuh", "dosa_internal.h",
+               "score_epilogue.cuh", "work_items.cuh"),
+}
+
+
+def _kernel_source_sha(kernel: str):
     import hashlib
     h = hashlib.sha256()
-    for name in ("score_tc.cu", "certified.cu", "filter.cu", "decode.cu", "cand_state.cuh",
-                 "work_items.cuh",
-                 "score_epilogue.cuh", "dosa_device.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "exact_certified_top_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
