@@ -135,7 +135,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
-template <bool kFp8, int kHeads>
+// kSurv: survivor mode (p.surv set): survivors go to the row lists instead of
+// the exact MMAs.
+template <bool kFp8, int kHeads, bool kSurv>
 __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     certified_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap bmap,
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           const bool surv = vis && !rej;
           const uint32_t mk = __ballot_sync(0xFFFFFFFFu, surv);
-          if (p.surv && mk) {
+          if (kSurv && mk) {
             // survivor mode: the row's list gets the keys, no exact MMA
             int base = 0;
             if (lane == 0) base = atomicAdd(&p.surv_count[q.row], __popc(mk));
@@ -442,8 +444,8 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           n_rejected += rjm;
           it_scr += scr;
           it_rej += rjm;
-          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = p.surv ? 0u : mk;
-          if (mk && !p.surv) gbits |= 1u << (ql >> 1);
+          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = kSurv ? 0u : mk;
+          if (!kSurv && mk) gbits |= 1u << (ql >> 1);
         }
         if (lane == 0) gflag[(c % 3) * 8 + ew] = gbits;
         tc_fence_before();
@@ -547,10 +549,10 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
       kc += n;
       // ---- range end: carry the query's state over, or publish it ----
       if (ok && ew < g.nq) {
-        if (rg.end < g.n_tiles || p.surv) state_save(st[ew], p.qstate + st[ew].row, lane);
+        if (rg.end < g.n_tiles || kSurv) state_save(st[ew], p.qstate + st[ew].row, lane);
         else if (lane == 0) publish_query(st[ew], p.out);
       }
-      if (p.surv && lane == 0) {
+      if (kSurv && lane == 0) {
         // this item's counts, held back until the rescoring pass decides
         atomicAdd(&p.item_cnt[item * 3 + 0], n_seed - item_seed0);
         atomicAdd(&p.item_cnt[item * 3 + 1], n_screened - item_scr0);
@@ -591,13 +593,12 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(certified_kernel<kFp8, 64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(certified_kernel<kFp8, 32>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {certified_kernel<kFp8, 64, false>, certified_kernel<kFp8, 32, false>,
+                    certified_kernel<kFp8, 64, true>, certified_kernel<kFp8, 32, true>})
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -649,10 +650,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
-  if (v.H == 64)
-    certified_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
-  else
-    certified_kernel<kFp8, 32><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
+  const bool surv = p.surv != nullptr;
+  auto fn = v.H == 64 ? (surv ? certified_kernel<kFp8, 64, true> : certified_kernel<kFp8, 64, false>)
+                      : (surv ? certified_kernel<kFp8, 32, true> : certified_kernel<kFp8, 32, false>);
+  fn<<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_CERTIFIED, stream);
   return e;
