@@ -42,14 +42,19 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_128k_fp8", choices=sorted(WORKLOADS))
-    ap.add_argument("--path", choices=["certified", "dense", "decode"], default="certified",
-                    help="decode: the decode-step call on a decode workload (decode_1m_fp8)")
+    ap.add_argument("--path", choices=["certified", "dense", "scorer", "decode"],
+                    default="certified",
+                    help="dense: dense scorer + Top-K; scorer: the dense scorer alone (every "
+                         "visible score written, no Top-K); decode: the decode-step call on a "
+                         "decode workload (decode_1m_fp8)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU baseline sample")
     ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
                     help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
     ap.add_argument("--block-bound", type=int, choices=[0, 1], default=1,
                     help="certified path: skip key tiles whose key-block bound rules them out")
+    ap.add_argument("--survivor-stream", type=int, choices=[0, 1, 2], default=0,
+                    help="certified path: survivor streams (gathered rescoring), see dosa.h")
     ap.add_argument("--probe-sample", type=int, choices=[0, 1], default=1,
                     help="adaptive screening: probe every 7th work item first (1) or every item (0)")
     ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
@@ -352,6 +357,14 @@ def ideal_prune_sample(x, wl, n_rows: int = 4):
 
 # ---------------------------------------------------------------------------
 
+def ablations_of(args) -> dict:
+    """Certified-path switches that differ from their defaults."""
+    if args.path != "certified":
+        return {}
+    defaults = {"block_bound": 1, "probe_sample": 1, "survivor_stream": 0}
+    return {k: getattr(args, k) for k, v in defaults.items() if getattr(args, k) != v}
+
+
 def config_of(wl, path, world, screening=None, writeback=None, ablations=None):
     extra = {"screening": screening} if screening is not None else {}
     if writeback is not None:
@@ -404,9 +417,11 @@ def run_ours(args, world, rank, local):
     x = generate(rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
                         sparse_writeback=int(args.writeback == "sparse"),
-                        block_bound=args.block_bound, probe_sample=args.probe_sample)
+                        block_bound=args.block_bound, probe_sample=args.probe_sample,
+                        survivor_stream=args.survivor_stream)
     certified = args.path == "certified"
     decode = args.path == "decode"
+    scorer = args.path == "scorer"
     if decode and wl.decode_noise <= 0:
         raise SystemExit("--path decode needs a decode workload (decode_1m_fp8)")
     seeds = None
@@ -432,9 +447,20 @@ def run_ours(args, world, rank, local):
                          device="cuda")
     out = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
     call_args = (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], so, wl.K)
+    if scorer:
+        # the dense scorer alone: every visible score of a chunk of rows written
+        # into one fp32 matrix (about 4 GiB), chunk after chunk
+        sc_rows = max(8, min(wl.T, (4 << 30) // (4 * wl.S)) // 8 * 8)
+        sc_buf = torch.empty((sc_rows, wl.S), dtype=torch.float32, device="cuda")
+        sc_err = torch.zeros(16, dtype=torch.uint8, device="cuda")
 
     def step(o=out, a=call_args):
-        if decode:
+        if scorer:
+            for r0 in range(0, wl.T, sc_rows):
+                n = min(sc_rows, wl.T - r0)
+                idx.scores(a[0], a[1], a[2], a[3], a[4], r0, n, wl.q_pos0 + r0, wl.S, sc_buf,
+                           wl.S, sc_err)
+        elif decode:
             idx.decode_topk(*a, seeds, out=o, workspace=ws)
         elif certified:
             idx.topk(*a, out=o, workspace=ws)
@@ -481,7 +507,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public call with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not scorer:
         host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) and v.is_cuda else v)
                 for k, v in x.items()}
         names = ["q", "q_scale", "w", "k", "k_scale"]
@@ -544,7 +570,7 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = ideal = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not scorer:
         cpu = oracle_sample(x, wl, args.cpu_seconds)
         if certified:
             ideal = ideal_prune_sample(x, wl)
@@ -558,9 +584,7 @@ def run_ours(args, world, rank, local):
                 "config": config_of(wl, args.path, world,
                                     args.screening if args.path == "certified" else None,
                                     args.writeback if args.path == "certified" else None,
-                                    {k: v for k, v in (("block_bound", args.block_bound),
-                                                       ("probe_sample", args.probe_sample))
-                                     if args.path == "certified" and v != 1}),
+                                    ablations_of(args)),
                 "roofline": roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "kernels": {k: {"launches": n, "ms": round(t, 3)} for k, t in

@@ -1005,7 +1005,10 @@ dosa_status dosa_topk_rows(const float* scores, int64_t ld, const int64_t* row_l
 }
 
 dosa_status dosa_check_device(void* workspace, void* stream) {
-  if (!workspace) return DOSA_ERR_INVALID_ARG;
+  // NULL: the error word of dosa_index_dense_topk_static, which lives in the
+  // header of the library's fixed scratch array on the current device
+  if (!workspace) workspace = static_scratch_address();
+  if (!workspace) return DOSA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int word = 0;
   if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -61,6 +61,10 @@ struct Handle {
   std::mutex copy_mutex;
 };
 
+// Device address of the allocation-free entry point's fixed scratch array on
+// the current device (static_scratch.cu), or nullptr.
+void* static_scratch_address();
+
 // Kernel timing hooks (profile.cu): bracket one launch with events when enabled.
 void profile_before(int kind, cudaStream_t stream);
 void profile_after(int kind, cudaStream_t stream);

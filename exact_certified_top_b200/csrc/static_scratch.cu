@@ -37,6 +37,11 @@ void* scratch_address() {
 }
 
 }  // namespace
+
+// The static array's address on the current device (its header holds the
+// device error word of the static calls), or nullptr.
+void* static_scratch_address() { return scratch_address(); }
+
 }  // namespace dosa
 
 using namespace dosa;

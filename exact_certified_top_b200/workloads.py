@@ -11,6 +11,13 @@ Generator (one sequence, H heads, head dimension d):
   w[t,h] ~ N(0,1)/8 i.i.d. (mixed signs); the bound-tightness case instead
   makes a random half of each query's heads negative, w = +-|N(0,1)|/8.
   c = 1, or 0.1 for the nearly isotropic keys of the bound-tightness case.
+Redundant heads (head_noise > 0): z and eps are drawn once per query token and
+  shared by its heads, and each head adds its own N(0, head_noise^2) per
+  coordinate: q[t,h] = mu_q + A_q z_t + 0.3 eps_t + head_noise * n_{t,h}.  The
+  weights are w[t,h] = |N(0,1)|/8 with a seeded random quarter of each query's
+  heads negated.  This stands in for trained indexers, whose heads are far
+  more alike than independent draws (the pages' prune rates are measured on
+  such layers).
 Storage:
   bf16: round-to-nearest-even from fp32.
   fp8 e4m3: one fp32 scale per token = absmax / 448 (over H x d for a query
@@ -47,6 +54,8 @@ class Workload:
     # decode steps: rows 1.. are row 0 (the previous step) plus N(0, noise^2)
     # per coordinate (w: plus N(0, (noise / 8)^2)), drawn before quantisation
     decode_noise: float = 0.0
+    # redundant heads: per-head perturbation of a shared per-token query
+    head_noise: float = 0.0
 
     @property
     def visible_pairs(self) -> int:
@@ -67,6 +76,14 @@ WORKLOADS = {
                              q_pos0=1048576 - 8192),
     "tight_64k_bf16_levels": Workload("tight_64k_bf16_levels", T=65536, S=65536, K=2048,
                                       lowrank_scale=0.1, neg_half=True, levels=8),
+    # heads of a query nearly alike (trained-indexer stand-in): the certificate
+    # is tight and screening rejects most keys.  A prefill chunk of 8,192 rows
+    # at the end of a 128K context, and the whole 128K causal prefill.
+    "redundant_chunk128k_fp8": Workload("redundant_chunk128k_fp8", T=8192, S=131072,
+                                        dtype="fp8", K=2048, q_pos0=131072 - 8192,
+                                        head_noise=0.05),
+    "redundant_128k_fp8": Workload("redundant_128k_fp8", T=131072, S=131072, dtype="fp8",
+                                   K=2048, head_noise=0.05),
     # decode step at ~1M cached keys: the last 5 rows of the sequence; row 0
     # (position S - 5) is the previous step, whose selection seeds rows 1..4
     # (a 4-row multi-token-prediction step)
@@ -136,6 +153,10 @@ def generate(wl: Workload, device="cpu", chunk: int = 4096) -> dict:
 
     # head weights
     w = _randn(g, (T, H), device) / 8.0
+    if wl.head_noise > 0:
+        w = w.abs()
+        neg = torch.argsort(torch.rand((T, H), generator=g, device=device), dim=1)[:, : H // 4]
+        w.scatter_(1, neg, -w.gather(1, neg))
     if wl.neg_half:
         w = w.abs()
         neg = torch.argsort(torch.rand((T, H), generator=g, device=device), dim=1)[:, : H // 2]
@@ -158,9 +179,14 @@ def generate(wl: Workload, device="cpu", chunk: int = 4096) -> dict:
     q_step = None
     for t0 in range(0, T, max(1, chunk // 16)):
         n = min(max(1, chunk // 16), T - t0)
-        z = _randn(g, (n, H, 16), device)
-        eps = _randn(g, (n, H, d), device)
-        qf = mu_q + z @ A_q.T + 0.3 * eps
+        if wl.head_noise > 0:
+            z = _randn(g, (n, 1, 16), device)
+            eps = _randn(g, (n, 1, d), device)
+            qf = mu_q + z @ A_q.T + 0.3 * eps + wl.head_noise * _randn(g, (n, H, d), device)
+        else:
+            z = _randn(g, (n, H, 16), device)
+            eps = _randn(g, (n, H, d), device)
+            qf = mu_q + z @ A_q.T + 0.3 * eps
         if wl.decode_noise > 0:
             qf[1:] = qf[0:1] + wl.decode_noise * _randn(g, (n - 1, H, d), device)
         if wl.dtype == "fp8":

@@ -260,7 +260,11 @@ dosa_status dosa_index_dense_topk(dosa_index_t h, const void* q, const float* q_
  * whose work overlaps on the GPU race on it: serialise them.  Sizes: returns
  * DOSA_ERR_WORKSPACE when 256 + 32 * S_max bytes exceed 16 MiB (S_max = the
  * largest key count of a sequence, so up to 524280 keys), before any CUDA
- * call.  Otherwise as dosa_index_dense_topk, with identical results. */
+ * call.  Otherwise as dosa_index_dense_topk, with identical results.  A
+ * device-side failure of the call (an expired bounded wait, a bounds check)
+ * is recorded in the array's header, not returned: read it back with
+ * dosa_check_device(NULL, stream) after the call, before the next static call
+ * clears it. */
 dosa_status dosa_index_dense_topk_static(dosa_index_t h, const void* q, const float* q_scale,
                                          const float* w, const void* k, const float* k_scale,
                                          const int64_t* seq_offsets, int B, int K,
@@ -290,7 +294,11 @@ dosa_status dosa_topk_rows(const float* scores, int64_t ld, const int64_t* row_l
                            int K, int32_t* out, void* stream);
 
 /* Read back and clear the device error word of the last calls on `stream`
- * (synchronises it). */
+ * that used `workspace` (synchronises it).  workspace = NULL reads the error
+ * word of dosa_index_dense_topk_static on the current device (the header of
+ * the library's fixed scratch array).  Returns DOSA_ERR_TIMEOUT or
+ * DOSA_ERR_DEVICE_CHECK for a recorded failure, DOSA_ERR_CUDA when the copy
+ * fails, DOSA_OK otherwise. */
 dosa_status dosa_check_device(void* workspace, void* stream);
 
 /* Kernel kinds reported by the profiling counters. */

@@ -9,13 +9,16 @@ from oracle import decode_bf16, decode_e4m3
 def test_named_workloads_and_pairs():
     assert set(WORKLOADS) == {"causal_1k_bf16", "causal_16k_bf16", "prefill_128k_fp8",
                               "prefill_128k_fp8_h32", "chunk_1m_fp8", "tight_64k_bf16_levels",
-                              "decode_1m_fp8"}
+                              "decode_1m_fp8", "redundant_chunk128k_fp8", "redundant_128k_fp8"}
     assert WORKLOADS["prefill_128k_fp8_h32"].H == 32
     assert WORKLOADS["decode_1m_fp8"].visible_pairs == sum(1048576 - 5 + i + 1 for i in range(5))
     assert WORKLOADS["prefill_128k_fp8"].visible_pairs == 8_590_000_128
     assert WORKLOADS["causal_16k_bf16"].visible_pairs == 134_225_920
     assert WORKLOADS["chunk_1m_fp8"].visible_pairs == 8_556_384_256
     assert WORKLOADS["tight_64k_bf16_levels"].visible_pairs == 2_147_516_416
+    assert WORKLOADS["redundant_128k_fp8"].visible_pairs == 8_590_000_128
+    assert WORKLOADS["redundant_chunk128k_fp8"].visible_pairs == sum(
+        131072 - 8192 + i + 1 for i in range(8192))
 
 
 def test_deterministic_and_shapes():
@@ -58,3 +61,17 @@ def test_sinks_are_about_one_percent():
     x = generate(wl)
     frac = float(x["sinks"].float().mean())
     assert 0.007 < frac < 0.013
+
+
+def test_redundant_heads_share_their_direction():
+    """Heads of one query are near copies (per-head noise 0.05 per coordinate
+    on a query of norm ~11), a quarter of each query's weights is negative."""
+    wl = small_case("redundant_128k_fp8", 16)
+    x = generate(wl)
+    q = decode_e4m3(codes_numpy(x["q"])).reshape(16, 64, 128)
+    qn = q / np.linalg.norm(q, axis=2, keepdims=True)
+    cos = np.einsum("thd,tgd->thg", qn, qn)
+    assert cos.min() > 0.95
+    other = np.einsum("hd,gd->hg", qn[0], qn[1])
+    assert other.max() < 0.99
+    assert bool(torch.all((x["w"] < 0).sum(dim=1) == 16))

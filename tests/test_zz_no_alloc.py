@@ -39,6 +39,10 @@ def test_static_entry_matches_dense_topk_twice(cuda_lib, base, T, S, K):
         out = torch.full((T, K), -7, dtype=torch.int32, device="cuda")
         assert _call_static(lib, idx, x, x["seq_offsets"], K, out) == 0
         torch.cuda.synchronize()
+        # the static call's device error word (expired waits, bounds checks)
+        # sits in the fixed array's header: NULL reads it back
+        assert lib.dosa_check_device(None, ctypes.c_void_p(
+            torch.cuda.current_stream().cuda_stream)) == 0
         assert torch.equal(out, want)
 
 
