@@ -29,7 +29,10 @@ Parity status of each function (pins live in tests/test_oracle_*.py):
   select_topk ................... pinned (repeated argmax, sorted() on tuples)
   nnls_retained ................. pinned (grid search, KKT conditions)
   certificate_setup/upper_bound . pinned (UB >= I invariant, closed-form reductions)
-  certified_topk_row ............ pinned (equals dense selection; tau <= K-th)
+  certified_topk_row ............ pinned (equals dense selection; tau <= K-th;
+                                  ideal_rejected in the closed form UB = I)
+  ranked_topk_row ............... pinned (equals dense selection; every rejected
+                                  key scores below the K-th; rejected <= ideal)
   key_block_stats/block_upper_bound  pinned (bound >= every key's UB in the
                                   block, single-key blocks reduce to UB)
   prune rates ................... parity unpinned against the pages (their ~97 %
@@ -48,7 +51,7 @@ __all__ = [
     "decode_bf16", "decode_e4m3", "dequantize", "indexer_scores", "select_topk",
     "dense_topk", "nnls_retained", "Certificate", "certificate_setup", "upper_bound",
     "soundness_margin", "seed_mask", "certified_topk_row", "certified_topk",
-    "key_mean", "key_block_stats", "block_upper_bound",
+    "key_mean", "key_block_stats", "block_upper_bound", "ranked_topk_row",
 ]
 
 # ----------------------------------------------------------------------------
@@ -423,3 +426,79 @@ def certified_topk(q, w, k, positions, K, rows=None, **kw) -> tuple[np.ndarray, 
         for key in tot:
             tot[key] += res[key]
     return (np.stack(out) if out else np.zeros((0, K), np.int64)), tot
+
+
+def ranked_topk_row(q_t, w_t, k_vis, K, *, k_bar, warm_tiles, r=4, G=2, seed_first=64,
+                    seed_last=512, margin_log2=-12, tile=128, spread=2.0, growth=8) -> dict:
+    """One query through the certified pipeline with a ranked threshold
+    schedule.  The pages fix what is computed (seed threshold, certificate,
+    rejection, all-head scoring of the survivors; [DPC] Method, candidate
+    refinement) but not in which order the keys are screened; this reading
+    screens every remaining key against an estimate of the threshold and
+    checks the estimate afterwards:
+
+      1. Warm-up: key tile 0 and the warm_tiles - 1 tiles ending at the
+         diagonal are scored exactly (n_e keys).  The seed subset is scored
+         exactly wherever it lies.
+      2. Estimates U_1 > U_2 > ...: U_j = the m_j-th largest warm-up score,
+         m_1 = ceil(spread * K * n_e / n), m_{j+1} = growth * m_j, clamped to
+         [1, K].  U_1 estimates a score a little below the K-th (the warm-up
+         keys as a sample of the n visible keys); the last, m = K, is the
+         warm-up's own K-th largest score, a sound threshold.
+      3. Pass 1: every other key is a survivor when v = UB + delta >= U_1 and
+         is scored exactly.
+      4. After pass j, tau = the K-th largest exact score so far (a lower bound
+         on the true K-th, as any subset's K-th is).  If a key not scored yet
+         has v >= tau, pass j + 1 scores exactly the keys with
+         max(tau, U_{j+1}) <= v < (pass j's lower limit).  Once U_{j+1} <= tau
+         that pass leaves no key with v >= tau unscored, so the schedule ends.
+      5. Top-K over the exactly scored keys.
+    Every rejected key has I <= v < tau <= v_K, so the selection is the dense
+    one.  Returns the selection and the counts of the prune rate."""
+    n = k_vis.shape[0]
+    p = n - 1
+    w64 = w_t.astype(np.float64)
+    cert = certificate_setup(q_t, w64, k_bar, r, G)
+    full = indexer_scores(q_t, w64, k_vis)
+    v = upper_bound(cert, q_t, k_vis) + soundness_margin(q_t, w64, k_vis, margin_log2)
+    keys = np.arange(n)
+    n_tiles = p // tile + 1
+    first_diag = max(1, n_tiles - warm_tiles + 1)
+    warm = (keys < tile) | (keys >= first_diag * tile)
+    seeds = seed_mask(p, seed_first, seed_last)
+    n_e = int(warm.sum())
+    m = min(K, max(1, int(math.ceil(spread * K * n_e / n))))
+    estimates = [_kth_largest(full[warm], m)]
+    ms = [m]
+    while ms[-1] < K:
+        ms.append(min(K, ms[-1] * growth))
+        estimates.append(_kth_largest(full[warm], ms[-1]))
+    screened = ~warm & ~seeds
+    lower = estimates[0]
+    exact = warm | seeds | (screened & (v >= lower))
+    survived_1 = int((screened & exact).sum())
+    passes = 1
+    while True:
+        tau = _kth_largest(full[exact], K)
+        if not np.any(v[screened & ~exact] >= tau):
+            break
+        nxt = estimates[passes] if passes < len(estimates) else -math.inf
+        new_lower = max(tau, nxt)
+        exact = exact | (screened & (v >= new_lower) & (v < lower))
+        lower = new_lower
+        passes += 1
+    scored = np.nonzero(exact)[0]
+    vals = full[scored]
+    order = np.lexsort((scored, -vals))
+    chosen = np.sort(scored[order[: min(K, scored.size)]])
+    idx = np.full(K, -1, np.int64)
+    idx[: chosen.size] = chosen
+    vK = _kth_largest(full, K)
+    return {
+        "idx": idx, "u_hat": estimates[0], "estimates": estimates, "m": ms[0], "n_warm": n_e,
+        "tau": tau, "passes": passes, "v_K": vK, "visible": n, "seed": int(seeds.sum()),
+        "screened": int(screened.sum()), "survived_1": survived_1,
+        "rejected": int((screened & ~exact).sum()),
+        "ideal_rejected": int((screened & (v < vK)).sum()),
+        "exact": int(exact.sum()), "scores": full, "bound": v, "exact_mask": exact,
+    }
