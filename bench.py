@@ -8,8 +8,12 @@ A step is one pass of the whole indexer (every row of the workload through
 the library's Top-K call) over inputs already resident in HBM.  The headline
 workload is 128K-token causal prefill with fp8 e4m3 inputs, H = 64, d = 128,
 K = 2048.  With N > 1 (torchrun) every rank processes its own independent
-sequence of the same shape (weak scaling, no collective on the data path); the
-step time is the max over ranks.  Rank 0 prints one JSON line.
+sequence of the same shape (weak scaling, no collective on the data path), or
+with --split rows the ranks share one sequence: its query rows are cut into 2N
+blocks, rank i scores blocks i and 2N-1-i (every rank gets the same number of
+causal pairs to within a block's worth), the keys are replicated, and the
+selected indices are all-gathered (strong scaling).  The step time is the max
+over ranks.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -49,12 +53,11 @@ def parse_args():
                          "decode workload (decode_1m_fp8)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU baseline sample")
-    ap.add_argument("--screening", type=int, choices=[0, 1, 2], default=2,
-                    help="certified path: 0 no bounds, 1 screen every tile, 2 adaptive (default)")
+    ap.add_argument("--screening", type=int, choices=[0, 1, 2, 3], default=2,
+                    help="certified path: 0 no bounds, 1 streaming schedule (every tile), "
+                         "2 adaptive (default), 3 ranked schedule for every item")
     ap.add_argument("--block-bound", type=int, choices=[0, 1], default=1,
                     help="certified path: skip key tiles whose key-block bound rules them out")
-    ap.add_argument("--survivor-stream", type=int, choices=[0, 1, 2], default=0,
-                    help="certified path: survivor streams (gathered rescoring), see dosa.h")
     ap.add_argument("--probe-sample", type=int, choices=[0, 1], default=1,
                     help="adaptive screening: probe every 7th work item first (1) or every item (0)")
     ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
@@ -62,6 +65,9 @@ def parse_args():
                          "exact score into a dense matrix and its dense Top-K (ablation)")
     ap.add_argument("--tail-rows", type=int, default=0,
                     help="profile only the last N query rows of the workload (same keys)")
+    ap.add_argument("--split", choices=["sequences", "rows"], default="sequences",
+                    help="N > 1: an independent sequence per rank (default), or the rows of one "
+                         "sequence in causal-balanced zigzag blocks with the indices all-gathered")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -108,6 +114,40 @@ def rank_workload(wl, rank: int):
 def job_value(pairs_per_rank: int, world: int, ms_per_step_max: float) -> float:
     """Whole-job pairs/s: every rank's pairs over the slowest rank's step time."""
     return world * pairs_per_rank / (ms_per_step_max * 1e-3)
+
+
+def zigzag_blocks(T: int, world: int) -> list:
+    """Rows [0, T) of one causal sequence cut into 2 * world contiguous blocks;
+    rank i takes blocks i and 2 * world - 1 - i, a short block and a long one,
+    so every rank scores about the same number of causal pairs.  Returns, per
+    rank, its two (first row, end row) ranges."""
+    n = 2 * world
+    edges = [T * j // n for j in range(n + 1)]
+    return [[(edges[i], edges[i + 1]), (edges[n - 1 - i], edges[n - i])] for i in range(world)]
+
+
+def block_pairs(blocks, q_pos0: int) -> int:
+    """Visible causal pairs of a rank's row ranges (row t sits at q_pos0 + t)."""
+    return sum((r1 - r0) * (2 * q_pos0 + r0 + r1 + 1) // 2 for r0, r1 in blocks)
+
+
+def gather_rows(local: torch.Tensor, blocks_all: list, T: int) -> torch.Tensor:
+    """All-gather every rank's selected indices (its rows, in block order) into
+    the full [T, K] result on every rank."""
+    world = len(blocks_all)
+    n_max = max(sum(r1 - r0 for r0, r1 in b) for b in blocks_all)
+    K = local.shape[1]
+    pad = torch.full((n_max, K), -1, dtype=local.dtype, device=local.device)
+    pad[: local.shape[0]] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    torch.distributed.all_gather(parts, pad)
+    full = torch.empty((T, K), dtype=local.dtype, device=local.device)
+    for part, blocks in zip(parts, blocks_all):
+        at = 0
+        for r0, r1 in blocks:
+            full[r0:r1] = part[at: at + r1 - r0]
+            at += r1 - r0
+    return full
 
 
 # ---------------------------------------------------------------------------
@@ -361,7 +401,7 @@ def ablations_of(args) -> dict:
     """Certified-path switches that differ from their defaults."""
     if args.path != "certified":
         return {}
-    defaults = {"block_bound": 1, "probe_sample": 1, "survivor_stream": 0}
+    defaults = {"block_bound": 1, "probe_sample": 1}
     return {k: getattr(args, k) for k, v in defaults.items() if getattr(args, k) != v}
 
 
@@ -370,9 +410,11 @@ def config_of(wl, path, world, screening=None, writeback=None, ablations=None):
     if writeback is not None:
         extra["writeback"] = writeback
     extra.update(ablations or {})
+    # world < 0: the rows of one sequence split over -world ranks (zigzag)
+    par = f"rows zigzag x{-world}, indices all-gathered" if world < 0 else f"rows x{world}"
     return {"workload": wl.name, "T": wl.T, "S": wl.S, "H": wl.H, "d": wl.d, "K": wl.K,
             "dtype": wl.dtype, "q_pos0": wl.q_pos0, "path": path, **extra,
-            "parallelism": f"rows x{world}",
+            "parallelism": par,
             "l2": "flushed between timed steps (256 MiB write, outside the timed windows)",
             "visible_pairs_per_gpu": wl.visible_pairs}
 
@@ -414,11 +456,14 @@ def run_ours(args, world, rank, local):
     from exact_certified_top_b200 import binding
     binding.load()
     wl = workload_of(args)
-    x = generate(rank_workload(wl, rank), device="cuda")
+    split_rows = world > 1 and args.split == "rows"
+    if split_rows and args.path not in ("certified", "dense"):
+        raise SystemExit("--split rows runs the certified or the dense path")
+    # one shared sequence (same seed on every rank) or one per rank
+    x = generate(wl if split_rows else rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
                         sparse_writeback=int(args.writeback == "sparse"),
-                        block_bound=args.block_bound, probe_sample=args.probe_sample,
-                        survivor_stream=args.survivor_stream)
+                        block_bound=args.block_bound, probe_sample=args.probe_sample)
     certified = args.path == "certified"
     decode = args.path == "decode"
     scorer = args.path == "scorer"
@@ -439,13 +484,16 @@ def run_ours(args, world, rank, local):
              "positions": rest(x["positions"]), "seq_offsets": [[0, 0, wl.q_pos0 + 1], [m, wl.S, 0]]}
         wl = replace(wl, name=f"{wl.name}[rows 1..{m}]", T=m, q_pos0=wl.q_pos0 + 1)
     so = x["seq_offsets"]
+    blocks_all = zigzag_blocks(wl.T, world) if split_rows else None
+    my_rows = (sum(r1 - r0 for r0, r1 in blocks_all[rank]) if split_rows else wl.T)
     if decode:
         ws = torch.zeros(idx.decode_workspace_size(wl.T, wl.S, wl.K), dtype=torch.uint8,
                          device="cuda")
     else:
-        ws = torch.zeros(idx.workspace_size(wl.T, wl.S, wl.K, certified), dtype=torch.uint8,
+        ws = torch.zeros(idx.workspace_size(my_rows, wl.S, wl.K, certified), dtype=torch.uint8,
                          device="cuda")
     out = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    out_local = torch.empty((my_rows, wl.K), dtype=torch.int32, device="cuda")
     call_args = (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], so, wl.K)
     if scorer:
         # the dense scorer alone: every visible score of a chunk of rows written
@@ -454,8 +502,25 @@ def run_ours(args, world, rank, local):
         sc_buf = torch.empty((sc_rows, wl.S), dtype=torch.float32, device="cuda")
         sc_err = torch.zeros(16, dtype=torch.uint8, device="cuda")
 
+    def step_rows():
+        # this rank's two row blocks of the shared sequence, then the exchange
+        at = 0
+        for r0, r1 in blocks_all[rank]:
+            n = r1 - r0
+            sl = lambda v: None if v is None else v[r0:r1]
+            a = (sl(x["q"]), sl(x["q_scale"]), sl(x["w"]), x["k"], x["k_scale"],
+                 [[0, 0, wl.q_pos0 + r0], [n, wl.S, 0]], wl.K)
+            if certified:
+                idx.topk(*a, out=out_local[at:at + n], workspace=ws)
+            else:
+                idx.dense_topk(*a, out=out_local[at:at + n], workspace=ws)
+            at += n
+        out.copy_(gather_rows(out_local, blocks_all, wl.T))
+
     def step(o=out, a=call_args):
-        if scorer:
+        if split_rows:
+            step_rows()
+        elif scorer:
             for r0 in range(0, wl.T, sc_rows):
                 n = min(sc_rows, wl.T - r0)
                 idx.scores(a[0], a[1], a[2], a[3], a[4], r0, n, wl.q_pos0 + r0, wl.S, sc_buf,
@@ -495,19 +560,20 @@ def run_ours(args, world, rank, local):
     binding.check_device(ws)
 
     pairs = wl.visible_pairs
-    value = job_value(pairs, world, ms)
+    # split rows: the ranks share one sequence; otherwise each has its own
+    value = job_value(pairs, 1 if split_rows else world, ms)
     # a "decode" profile record spans three kernels (seed, scan, finish)
     launches = sum(n * KERNELS_PER_RECORD.get(k, 1) for k, (n, _) in prof.items())
 
     stats = None
-    if certified:
+    if certified and not split_rows:
         _, stats = idx.topk(*call_args, out=out, workspace=ws, stats=True)
     elif decode:
         _, stats = idx.decode_topk(*call_args, seeds, out=out, workspace=ws, stats=True)
 
     # end to end through the public call with host buffers
     e2e = None
-    if not args.no_e2e and not scorer:
+    if not args.no_e2e and not scorer and not split_rows:
         host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) and v.is_cuda else v)
                 for k, v in x.items()}
         names = ["q", "q_scale", "w", "k", "k_scale"]
@@ -579,9 +645,10 @@ def run_ours(args, world, rank, local):
         roof = roofline(prof, wl, pairs, args.steps, wl.dtype, stats)
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "higher_is_better": True, "scaling": "strong" if split_rows else "weak",
+                "vs_baseline": None,
                 "dtype": wl.dtype, "data": "synthetic (seeded low-rank + sink generator)",
-                "config": config_of(wl, args.path, world,
+                "config": config_of(wl, args.path, world if not split_rows else -world,
                                     args.screening if args.path == "certified" else None,
                                     args.writeback if args.path == "certified" else None,
                                     ablations_of(args)),

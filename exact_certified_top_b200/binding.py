@@ -30,7 +30,7 @@ EXPORTS = ("dosa_index_config_default", "dosa_index_create", "dosa_index_destroy
            "dosa_index_decode_topk", "dosa_index_decode_workspace_size")
 KERNELS = {"score": 0, "topk": 1, "reference": 2, "key_prep": 3, "cert_setup": 4,
            "certified": 5, "select": 6, "filter": 7, "decode": 8,
-           "fill": 9, "block": 10, "rescore": 11}
+           "fill": 9, "block": 10, "rescore": 11, "rank": 12}
 
 
 class DosaError(RuntimeError):
@@ -45,7 +45,7 @@ class Config(ctypes.Structure):
                 ("seed_last", ctypes.c_int), ("r", ctypes.c_int), ("G", ctypes.c_int),
                 ("margin_log2", ctypes.c_int), ("screening", ctypes.c_int),
                 ("sparse_writeback", ctypes.c_int), ("block_bound", ctypes.c_int),
-                ("survivor_stream", ctypes.c_int), ("probe_sample", ctypes.c_int)]
+                ("probe_sample", ctypes.c_int)]
 
 
 class Stats(ctypes.Structure):
@@ -53,7 +53,8 @@ class Stats(ctypes.Structure):
                 ("screened_pairs", ctypes.c_int64), ("rejected_pairs", ctypes.c_int64),
                 ("exact_pairs", ctypes.c_int64), ("candidates", ctypes.c_int64),
                 ("filtered_pairs", ctypes.c_int64), ("block_skipped_pairs", ctypes.c_int64),
-                ("rescored_pairs", ctypes.c_int64), ("repaired_rows", ctypes.c_int64)]
+                ("rescored_pairs", ctypes.c_int64), ("repaired_rows", ctypes.c_int64),
+                ("rescreened_pairs", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: int(getattr(self, name)) for name, _ in self._fields_}
@@ -92,7 +93,8 @@ def load(path: str = LIB_PATH):
     lib.dosa_reference_scores.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P,
                                           _I64, _P]
     lib.dosa_index_dense_topk_static.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P]
-    lib.dosa_index_certificate.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]
+    lib.dosa_index_certificate.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _SZ,
+                                           _P]
     lib.dosa_topk_rows.argtypes = [_P, _I64, _P, _I64, _I, _P, _P]
     lib.dosa_check_device.argtypes = [_P, _P]
     lib.dosa_profile_enable.argtypes = [_I]
@@ -244,17 +246,21 @@ class Index:
             _ptr(workspace), workspace.numel(), _stream(), ctypes.byref(st) if stats else None))
         return (out, st.as_dict()) if stats else out
 
-    def certificate(self, q, q_scale, w, k, k_scale, seq_offsets, workspace=None):
-        """Per-query certificate records [Tq, 16] (code domain) and retained heads [Tq, 4]."""
+    def certificate(self, q, q_scale, w, k, k_scale, seq_offsets, workspace=None,
+                    bound_rows: bool = False):
+        """Per-query certificate records [Tq, 16] (code domain), retained heads
+        [Tq, 4] and, when asked, the bound rows [Tq, 8, d] (codes, q's dtype)."""
         so = _seq_offsets(seq_offsets)
         cert = torch.empty((q.shape[0], 16), dtype=torch.float32, device=q.device)
         ret = torch.empty((q.shape[0], 4), dtype=torch.int32, device=q.device)
+        rows = (torch.empty((q.shape[0], 8, q.shape[2]), dtype=q.dtype, device=q.device)
+                if bound_rows else None)
         ws = self._workspace(q, so, 1, True, workspace)
         _check("dosa_index_certificate", self._lib.dosa_index_certificate(
             self._h, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k), _ptr(k_scale),
-            ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, _ptr(cert), _ptr(ret), _ptr(ws),
-            ws.numel(), _stream()))
-        return cert, ret
+            ctypes.c_void_p(so.data_ptr()), so.shape[0] - 1, _ptr(cert), _ptr(ret), _ptr(rows),
+            _ptr(ws), ws.numel(), _stream()))
+        return (cert, ret, rows) if bound_rows else (cert, ret)
 
     def scores(self, q, q_scale, w, k, k_scale, row0, rows, pos0, S, out, ld, scratch):
         _check("dosa_index_scores", self._lib.dosa_index_scores(

@@ -25,13 +25,10 @@
 // end of a range, the epilogue warps meet and each query's owner warp
 // refreshes its threshold.
 //
-// A launch processes a range of steps of every item (work_items.cuh).  With
-// adaptive screening, the filter scorer (filter.cu) scores the warm-up tiles,
-// where nothing can be rejected yet; this kernel then probes the next 4 tiles
-// of each item with screening and decides from the item's own counts whether
-// screening pays there: an item that rejected fewer than 1 in 32 screened
-// pairs is finished by the filter scorer without bounds, any other by this
-// kernel, screening every remaining tile.
+// A launch processes a range of steps of every item (work_items.cuh).  This
+// kernel runs the pages' own schedule (screening = 1: every tile after the
+// warm-up is screened, the threshold rising as tiles are scored); the ranked
+// schedule of the other screening modes is rank_screen.cu + rescore.cu.
 #include "cand_state.cuh"
 #include "cert_layout.h"
 #include "dosa_device.cuh"
@@ -40,11 +37,6 @@
 #include "work_items.cuh"
 
 namespace dosa {
-
-// Items whose probe screened at least this many pairs and rejected fewer than
-// 1 in kRejectRatio of them are handed to the filter scorer.
-constexpr unsigned long long kMinScreened = 2048;
-constexpr unsigned long long kRejectRatio = 32;
 
 template <bool kFp8>
 struct CertCfg {
@@ -95,18 +87,7 @@ struct CertParams {
   const int* step_list;    // per item, the steps left by block screening, or null
   const int* step_count;
   int step_cap;
-  // Survivor mode (screening only): every survivor's key goes to its row's
-  // list, no exact score is computed, the state is saved at the range end and
-  // the item's seed/screened/rejected counts go to item_cnt (the rescoring
-  // pass credits them, or drops them when it hands the item to the filter).
-  int* surv;               // [chunk rows][surv_cap] or null
-  int* surv_count;         // [chunk rows]
-  int surv_cap;
-  unsigned long long* item_cnt;   // [items][3]
-  int stream_ok;           // the probe may choose survivor streams (kItemStream)
   StepRange steps;         // what this launch processes
-  int decide;              // 1: flag every item whose range ends before its last step
-  int* gate;               // set to 1 when a decision is not the filter scorer
 };
 
 // The steps an item processes in this launch: its range, or the list block
@@ -135,9 +116,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // kHeads: heads per query row (32 or 64); the MMA always sees 64 head slots.
-// kSurv: survivor mode (p.surv set): survivors go to the row lists instead of
-// the exact MMAs.
-template <bool kFp8, int kHeads, bool kSurv>
+template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
     certified_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap bmap,
@@ -174,7 +153,6 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
   uint32_t* gflag = masks + 3 * 8 * 4;                                      // [3][8]
   uint32_t* s_tmem = gflag + 3 * 8;
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  unsigned long long* snap = reinterpret_cast<unsigned long long*>(s_tmem + 4);  // [2][8][2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -385,9 +363,6 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
 #pragma unroll
       for (int grp = 0; grp < C::kGroups; ++grp)
         cnt[grp] = *reinterpret_cast<volatile int*>(&st[grp * 2 + half].seg[quad]);
-      unsigned long long it_scr = 0, it_rej = 0;   // this warp's counts, this item
-      const unsigned long long item_seed0 = n_seed, item_scr0 = n_screened,
-                               item_rej0 = n_rejected;
       auto key_of = [&](int i) -> int64_t {
         return (int64_t)tile_at(step_at(p, rg, item, i), g.n_tiles) * kKeyTile + quad * 32 + lane;
       };
@@ -429,23 +404,11 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           }
           const bool surv = vis && !rej;
           const uint32_t mk = __ballot_sync(0xFFFFFFFFu, surv);
-          if (kSurv && mk) {
-            // survivor mode: the row's list gets the keys, no exact MMA
-            int base = 0;
-            if (lane == 0) base = atomicAdd(&p.surv_count[q.row], __popc(mk));
-            base = __shfl_sync(0xFFFFFFFFu, base, 0);
-            const int at = base + __popc(mk & ((1u << lane) - 1u));
-            if (surv && at < p.surv_cap) p.surv[q.row * (int64_t)p.surv_cap + at] = (int)s;
-          }
-          const uint32_t scr = __popc(__ballot_sync(0xFFFFFFFFu, screen));
-          const uint32_t rjm = __popc(__ballot_sync(0xFFFFFFFFu, rej));
           n_seed += __popc(__ballot_sync(0xFFFFFFFFu, vis && seed));
-          n_screened += scr;
-          n_rejected += rjm;
-          it_scr += scr;
-          it_rej += rjm;
-          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = kSurv ? 0u : mk;
-          if (!kSurv && mk) gbits |= 1u << (ql >> 1);
+          n_screened += __popc(__ballot_sync(0xFFFFFFFFu, screen));
+          n_rejected += __popc(__ballot_sync(0xFFFFFFFFu, rej));
+          if (lane == 0) masks[((c % 3) * 8 + ql) * 4 + quad] = mk;
+          if (mk) gbits |= 1u << (ql >> 1);
         }
         if (lane == 0) gflag[(c % 3) * 8 + ew] = gbits;
         tc_fence_before();
@@ -517,8 +480,6 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
           if (lane == 0) {
 #pragma unroll
             for (int grp = 0; grp < C::kGroups; ++grp) st[grp * 2 + half].seg[quad] = cnt[grp];
-            snap[(nbar & 1) * 16 + ew * 2 + 0] = it_scr;
-            snap[(nbar & 1) * 16 + ew * 2 + 1] = it_rej;
           }
           __threadfence_block();
           if (lane == 0) mbar_arrive(tile_done);
@@ -526,40 +487,17 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t slot = nbar & 1;
           ++nbar;
           if (ew < g.nq)
             refresh_threshold(st[ew], p.cand + st[ew].row * kSegs * (int64_t)p.seg_cap, p.seg_cap,
                               p.K, lane);
-          if (last && p.decide && rg.end < g.n_tiles && ew == 0 && lane == 0) {
-            // the probe's decision, from the counts every warp left at this barrier
-            unsigned long long tot_s = 0, tot_r = 0;
-            for (int w = 0; w < C::kEpiWarps; ++w) {
-              tot_s += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2];
-              tot_r += reinterpret_cast<volatile unsigned long long*>(snap)[slot * 16 + w * 2 + 1];
-            }
-            const bool pays = tot_s < kMinScreened || tot_r * kRejectRatio >= tot_s;
-            // nearly everything rejected: rescore the few survivors gathered
-            const bool stream = p.stream_ok && tot_s >= kMinScreened && tot_r * 8 >= tot_s * 7;
-            p.item_flag[item] = stream ? kItemStream : pays ? kItemScreen : kItemFilter;
-            if (stream || pays) *reinterpret_cast<volatile int*>(p.gate) = 1;
-          }
         }
       }
       kc += n;
       // ---- range end: carry the query's state over, or publish it ----
       if (ok && ew < g.nq) {
-        if (rg.end < g.n_tiles || kSurv) state_save(st[ew], p.qstate + st[ew].row, lane);
+        if (rg.end < g.n_tiles) state_save(st[ew], p.qstate + st[ew].row, lane);
         else if (lane == 0) publish_query(st[ew], p.out);
-      }
-      if (kSurv && lane == 0) {
-        // this item's counts, held back until the rescoring pass decides
-        atomicAdd(&p.item_cnt[item * 3 + 0], n_seed - item_seed0);
-        atomicAdd(&p.item_cnt[item * 3 + 1], n_screened - item_scr0);
-        atomicAdd(&p.item_cnt[item * 3 + 2], n_rejected - item_rej0);
-        n_seed = item_seed0;
-        n_screened = item_scr0;
-        n_rejected = item_rej0;
       }
     }
     if (lane == 0) {
@@ -583,8 +521,7 @@ __global__ void __launch_bounds__(CertCfg<kFp8>::kThreads, 1)
 
 template <bool kFp8>
 static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const CertBuffers& b,
-                                    int K, StepRange steps, int decide,
-                                    cudaStream_t stream, int use_list) {
+                                    int K, StepRange steps, cudaStream_t stream, int use_list) {
   using C = CertCfg<kFp8>;
   CUtensorMap qmap, bmap, kmap;
   if (!encode_q_map(&qmap, v.q, kFp8, (uint64_t)(v.row0 + v.rows), v.H) ||
@@ -594,8 +531,7 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaSuccess;
-    for (auto fn : {certified_kernel<kFp8, 64, false>, certified_kernel<kFp8, 32, false>,
-                    certified_kernel<kFp8, 64, true>, certified_kernel<kFp8, 32, true>})
+    for (auto fn : {certified_kernel<kFp8, 64>, certified_kernel<kFp8, 32>})
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmemBytes);
@@ -614,7 +550,6 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.cand = reinterpret_cast<Cand*>(b.cand);
   p.qstate = reinterpret_cast<QStateG*>(b.qstate);
   p.item_flag = b.item_flag;
-  p.gate = b.gate;
   p.out.cand_count = b.cand_count;
   p.out.tau = b.tau;
   p.out.repair_list = b.repair_list;
@@ -638,21 +573,13 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
   p.seed_first = h.cfg.seed_first;
   p.seed_last = h.cfg.seed_last;
   p.steps = steps;
-  p.decide = decide;
   p.step_list = use_list == 1 ? b.step_list : nullptr;
   p.step_count = use_list == 1 ? b.step_count : nullptr;
   p.step_cap = b.step_cap;
-  p.surv = use_list == 2 ? b.surv : nullptr;
-  p.surv_count = b.surv_count;
-  p.surv_cap = b.surv_cap;
-  p.item_cnt = b.item_cnt;
-  p.stream_ok = b.surv != nullptr;
   if (p.n_items == 0) return cudaSuccess;
   const int grid = p.n_items < sms ? p.n_items : sms;
   profile_before(DOSA_KERNEL_CERTIFIED, stream);
-  const bool surv = p.surv != nullptr;
-  auto fn = v.H == 64 ? (surv ? certified_kernel<kFp8, 64, true> : certified_kernel<kFp8, 64, false>)
-                      : (surv ? certified_kernel<kFp8, 32, true> : certified_kernel<kFp8, 32, false>);
+  auto fn = v.H == 64 ? certified_kernel<kFp8, 64> : certified_kernel<kFp8, 32>;
   fn<<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, bmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_CERTIFIED, stream);
@@ -660,10 +587,10 @@ static cudaError_t launch_cert_impl(const Handle& h, const SeqView& v, const Cer
 }
 
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             StepRange steps, int decide, cudaStream_t stream, int use_list) {
+                             StepRange steps, cudaStream_t stream, int use_list) {
   if (h.cfg.dtype == DOSA_FP8_E4M3)
-    return launch_cert_impl<true>(h, v, b, K, steps, decide, stream, use_list);
-  return launch_cert_impl<false>(h, v, b, K, steps, decide, stream, use_list);
+    return launch_cert_impl<true>(h, v, b, K, steps, stream, use_list);
+  return launch_cert_impl<false>(h, v, b, K, steps, stream, use_list);
 }
 
 size_t certified_smem_bytes(bool fp8) {

@@ -103,7 +103,14 @@ SeqView make_view(const Handle* h, const void* q, const float* q_scale, const fl
 
 constexpr int64_t kDefaultChunkBytes = (int64_t)4 << 30;   // dense score chunk budget
 constexpr int64_t kDefaultCertChunkBytes = (int64_t)8 << 30;   // certified per-row arrays
-constexpr int kRepairRows = 64;                             // overflowed rows per chunk
+// Rows per chunk whose candidate list may overflow and be rescored densely:
+// as many fp32 score rows of S_max keys as fit in 1 GiB, at least 64 and at
+// most 512 (a row overflows when a tie at its K-th score spans more keys than
+// its list holds).
+int64_t repair_rows(int64_t S_max) {
+  const int64_t n = ((int64_t)1 << 30) / (4 * (S_max > 1 ? S_max : 1));
+  return n < 64 ? 64 : n > 512 ? 512 : n;
+}
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
@@ -131,11 +138,11 @@ int seg_capacity(int K, int64_t S_max) {
 // Workspace of the certified path: a fixed part (header, key norms, key sum,
 // repair area) and Tc rows of per-query state.
 struct CertLayout {
-  size_t key_norm, key_sum, repair_list, repair_count, repair_scores, blk, fixed;
+  size_t key_norm, key_sum, repair_list, repair_count, repair_scores, blk, pass_any, fixed;
+  int64_t repair_rows;
   int step_cap;     // block screening: steps per item list (key tiles of S_max), or 0
-  int surv_cap;     // survivor streams: keys per row list (an eighth of S_max), or 0
+  int64_t words;    // ranked screening: survivor words per row (4 per key tile), or 0
   size_t per_row;   // bytes per chunk row (bound rows, record, retained, list, count, tau)
-  size_t surv_row;  // the part of per_row taken by the survivor lists
   int seg_cap;
   int64_t dense_ld; // dense writeback: the score matrix's row length (0 when sparse)
 };
@@ -151,13 +158,15 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.seg_cap = seg_capacity(K, S_max);
   L.key_norm = take((size_t)S_max * 4);
   L.key_sum = take(kHeadDim * 4);
-  L.repair_list = take(kRepairRows * 4);
+  L.repair_rows = repair_rows(S_max);
+  L.repair_list = take((size_t)L.repair_rows * 4);
   L.repair_count = take(4);
-  L.repair_scores = take((size_t)kRepairRows * S_max * 4);
+  L.repair_scores = take((size_t)L.repair_rows * S_max * 4);
   // block screening covers sequences of up to 8192 key tiles (1M keys)
   L.step_cap = h->cfg.block_bound ? (int)((S_max + kKeyTile - 1) / kKeyTile) : 0;
   if (L.step_cap > 8192) L.step_cap = 0;
   L.blk = take((size_t)L.step_cap * kBlkFloats * 4);
+  L.pass_any = take((kRankEst + 2) * 4);
   L.fixed = off;
   // bound rows, record, retained, list, count, tau, carried state, item flag
   L.per_row = (size_t)kBoundRows * kHeadDim * elem_bytes(h) + kCertFloats * 4 + 4 * 4 +
@@ -166,12 +175,11 @@ CertLayout cert_layout(const Handle* h, int64_t S_max, int K) {
   L.per_row += (size_t)L.dense_ld * 4;
   // step lists: one per work item of 8 rows (plus the count)
   L.per_row += ((size_t)L.step_cap * 4 + 4 + 7) / 8;
-  // survivor lists: streamed items were chosen for rejecting >= 7/8 in the
-  // probe, and a pass covers at most half of the keys, so a list holds an
-  // eighth of S_max; plus held-back item counts and the overflow flag
-  L.surv_cap = h->cfg.survivor_stream ? (int)round_up(S_max / 8 + 128, 128) : 0;
-  L.surv_row = L.surv_cap ? (size_t)L.surv_cap * 4 + 4 + 4 : 0;
-  L.per_row += L.surv_row;
+  // ranked screening: survivor bits, threshold estimates, band, largest
+  // rejected bound and pass of each row, probe counts of each item
+  const bool ranked = h->cfg.screening >= 2;
+  L.words = ranked ? (S_max + kKeyTile - 1) / kKeyTile * 4 : 0;
+  if (ranked) L.per_row += (size_t)L.words * 4 + kRankEst * 4 + 4 * 4 + 2;
   return L;
 }
 
@@ -189,7 +197,7 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.repair_list = reinterpret_cast<int*>(ws + L.repair_list);
   b.repair_count = reinterpret_cast<int*>(ws + L.repair_count);
   b.repair_scores = reinterpret_cast<float*>(ws + L.repair_scores);
-  b.repair_cap = kRepairRows;
+  b.repair_cap = (int)L.repair_rows;
   b.seg_cap = L.seg_cap;
   b.bdir = take((size_t)Tc * kBoundRows * kHeadDim * elem_bytes(h));
   b.cert = reinterpret_cast<float*>(take((size_t)Tc * kCertFloats * 4));
@@ -206,13 +214,17 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
   b.step_list = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * L.step_cap * 4))
                            : nullptr;
   b.step_count = L.step_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
-  b.surv_cap = L.surv_cap;
-  b.surv = L.surv_cap ? reinterpret_cast<int*>(take((size_t)Tc * L.surv_cap * 4)) : nullptr;
-  b.surv_count = L.surv_cap ? reinterpret_cast<int*>(take((size_t)Tc * 4)) : nullptr;
-  b.item_cnt = L.surv_cap ? reinterpret_cast<unsigned long long*>(
-                                take((size_t)(Tc / 8 + 1) * 3 * 8))
-                          : nullptr;
-  b.ovf = L.surv_cap ? reinterpret_cast<int*>(take((size_t)(Tc / 8 + 1) * 4)) : nullptr;
+  b.words = L.words;
+  const bool ranked = L.words > 0;
+  b.bits = ranked ? reinterpret_cast<uint32_t*>(take((size_t)Tc * L.words * 4)) : nullptr;
+  b.est = ranked ? reinterpret_cast<float*>(take((size_t)Tc * kRankEst * 4)) : nullptr;
+  b.band_lo = ranked ? reinterpret_cast<float*>(take((size_t)Tc * 4)) : nullptr;
+  b.band_hi = ranked ? reinterpret_cast<float*>(take((size_t)Tc * 4)) : nullptr;
+  b.maxrej = ranked ? reinterpret_cast<uint32_t*>(take((size_t)Tc * 4)) : nullptr;
+  b.row_next = ranked ? reinterpret_cast<int*>(take((size_t)Tc * 4)) : nullptr;
+  b.rank_cnt = ranked ? reinterpret_cast<unsigned long long*>(take((size_t)(Tc / 8 + 1) * 16))
+                      : nullptr;
+  b.pass_any = reinterpret_cast<int*>(ws + L.pass_any);
   b.gate = &reinterpret_cast<WsHeader*>(ws)->probe_gate;
   b.probe_sample = 0;
   b.counters = reinterpret_cast<WsHeader*>(ws)->counters;
@@ -222,7 +234,7 @@ CertBuffers cert_buffers(const Handle* h, const CertLayout& L, uint8_t* ws, int6
 
 // Padding the per-row arrays of a chunk may need (each starts 256-aligned),
 // plus the item-flag array's extra entry.
-constexpr size_t kCertPad = 15 * 256 + 8 + 16 * 1024 * 4 + 3 * 8;
+constexpr size_t kCertPad = 20 * 256 + 16 + 16 * 1024 * 4;
 
 // Rows per certified chunk that fit in ws_bytes (a multiple of 8, or 0).
 int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
@@ -235,6 +247,8 @@ int64_t cert_chunk_rows(const CertLayout& L, size_t ws_bytes) {
 // is partial), rounded up to the threshold checkpoint interval, and the
 // steps the probe screens after it.
 int warmup_steps(int K) { return ((K + kKeyTile - 1) / kKeyTile + 1 + 3) / 4 * 4; }
+// Screening every tile with the key-block certificate: the certified scorer
+// runs this many steps after the warm-up before the first block pass.
 constexpr int kProbeSteps = 4;
 
 int64_t total_visible(const int64_t* so, int B) {
@@ -277,7 +291,6 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->screening = 2;
   cfg->sparse_writeback = 1;
   cfg->block_bound = 1;
-  cfg->survivor_stream = 0;
   cfg->probe_sample = 1;
 }
 
@@ -288,9 +301,9 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
   if (cfg->max_K < 1 || cfg->max_K > 4096) return DOSA_ERR_INVALID_ARG;
   if (cfg->seed_first < 0 || cfg->seed_last < 0 || cfg->r < 0 || cfg->r > 4 || cfg->G < 0 ||
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
-      cfg->screening > 2 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
-      cfg->block_bound < 0 || cfg->block_bound > 1 || cfg->survivor_stream < 0 ||
-      cfg->survivor_stream > 2 || cfg->probe_sample < 0 || cfg->probe_sample > 1)
+      cfg->screening > 3 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
+      cfg->block_bound < 0 || cfg->block_bound > 1 || cfg->probe_sample < 0 ||
+      cfg->probe_sample > 1)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -325,9 +338,7 @@ dosa_status dosa_index_workspace_size(dosa_index_t hh, int64_t Tq, int64_t S_max
     const CertLayout L = cert_layout(h, S_max, K);
     int64_t rows = chunk_rows;
     if (rows == 0) {
-      // the survivor lists come on top of the budget: they do not change
-      // how many chunks a call takes
-      rows = kDefaultCertChunkBytes / (int64_t)(L.per_row - L.surv_row);
+      rows = kDefaultCertChunkBytes / (int64_t)L.per_row;
       rows = rows / 8 * 8;
       if (rows < 8) rows = 8;
     }
@@ -385,11 +396,13 @@ dosa_status dosa_index_dense_topk(dosa_index_t hh, const void* q, const float* q
 }  // extern "C"
 
 // Whether a chunk whose longest row has max_tiles key tiles is screened at
-// all: never with screening off; in the adaptive mode only when some row
-// has key tiles past the warm-up and the probe (before them every pair is
-// scored exactly, so the chunk goes to the filter scorer alone).
+// all: never with screening off; with ranked screening only when some row
+// has key tiles past the warm-up (past the probe too, in the adaptive mode):
+// before them every pair is scored exactly, so the chunk goes to the filter
+// scorer alone.
 static bool screening_can_act(const Handle* h, int64_t max_tiles, int K) {
-  if (h->cfg.screening == 2) return max_tiles > warmup_steps(K) + kProbeSteps;
+  if (h->cfg.screening == 2) return max_tiles > warmup_steps(K) + kRankProbeTiles;
+  if (h->cfg.screening == 3) return max_tiles > warmup_steps(K);
   return h->cfg.screening != 0;
 }
 
@@ -470,9 +483,11 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
   // dense writeback (ablation): pairs the scorers never write (rejected) stay -inf
   if (b.dense && launch_fill(b.dense, c.rows * b.dense_ld, -INFINITY, stream) != cudaSuccess)
     return DOSA_ERR_CUDA;
-  // screening 0: the filter scorer alone; 1: the certified scorer alone;
-  // 2: warm-up by the filter scorer, a probe of kProbeSteps screened steps,
-  // then each item finished by the scorer its probe chose
+  // screening 0: the filter scorer alone; 1: the certified scorer alone (the
+  // pages' streaming schedule); 3: warm-up by the filter scorer, then ranked
+  // screening of every item; 2: warm-up, a ranked probe of kRankProbeTiles
+  // key tiles per item, then each item finished by ranked screening or by the
+  // filter scorer, as its probe chose
   constexpr int kAll = 0x3FFFFFFF;
   const int mode =
       screening_can_act(h, (c.pos0 + c.rows - 1) / kKeyTile + 1, K) ? h->cfg.screening : 0;
@@ -481,75 +496,80 @@ static dosa_status cert_chunk(const Handle* h, const SeqView& c, const CertBuffe
   // the steps left.
   const bool blk = b.blk != nullptr;
   const int W = warmup_steps(K), P = W + kProbeSteps;
-  // The certified scorer from step `from` on, for the items flagged `want`.
-  // With the key-block certificate the rest runs in passes [r0, 2 r0): each
-  // pass first drops the tiles that the threshold reached so far rules out.
-  auto certified_rest = [&](int from, int want) -> bool {
+  const int n_items = (int)((c.rows + 7) / 8);
+  // The certified scorer from step `from` on.  With the key-block certificate
+  // the rest runs in passes [r0, 2 r0): each pass first drops the tiles that
+  // the threshold reached so far rules out.
+  auto certified_rest = [&](int from) -> bool {
     if (!blk)
-      return launch_certified(*h, c, b, K, StepRange{from, kAll, want}, 0, stream) == cudaSuccess;
+      return launch_certified(*h, c, b, K, StepRange{from, kAll, -1}, stream) == cudaSuccess;
     const int max_steps = (int)((c.pos0 + c.rows - 1) / kKeyTile + 1);
     for (int r0 = from; r0 < max_steps; r0 *= 2) {
       const int r1 = 2 * r0 >= max_steps ? kAll : 2 * r0;
-      if (launch_block_screen(*h, c, b, StepRange{r0, r1, want}, stream) != cudaSuccess ||
-          launch_certified(*h, c, b, K, StepRange{r0, r1, want}, 0, stream, 1) != cudaSuccess)
+      if (launch_block_screen(*h, c, b, StepRange{r0, r1, -1}, stream) != cudaSuccess ||
+          launch_certified(*h, c, b, K, StepRange{r0, r1, -1}, stream, 1) != cudaSuccess)
         return false;
     }
     return true;
   };
-  // Survivor streams from step `from` on, for the items flagged `want`, in
-  // passes [r0, 2 r0): screening into per-row survivor lists, rescoring of
-  // the gathered survivors (which raises the threshold the next pass screens
-  // against), and the filter scorer redoing the pass for items whose lists
-  // overflowed, from the state the screening saved.
-  auto streamed_rest = [&](int from, int want) -> bool {
-    const int max_steps = (int)((c.pos0 + c.rows - 1) / kKeyTile + 1);
-    const size_t n_items = (size_t)((c.rows + 7) / 8);
-    CertBuffers ob = b;
-    ob.item_flag = b.ovf;
-    for (int r0 = from; r0 < max_steps; r0 *= 2) {
-      const int r1 = 2 * r0 >= max_steps ? kAll : 2 * r0;
-      const StepRange sr{r0, r1, want};
-      if (cudaMemsetAsync(b.surv_count, 0, (size_t)c.rows * 4, stream) != cudaSuccess ||
-          cudaMemsetAsync(b.item_cnt, 0, n_items * 3 * 8, stream) != cudaSuccess ||
-          cudaMemsetAsync(b.ovf, 0, n_items * 4, stream) != cudaSuccess ||
-          launch_certified(*h, c, b, K, sr, 0, stream, 2) != cudaSuccess ||
-          launch_rescore(*h, c, b, K, sr, stream) != cudaSuccess ||
-          launch_filter(*h, c, ob, K, StepRange{r0, r1, 1}, stream) != cudaSuccess)
+  // Ranked passes of the rows waiting for pass 1 (of the items flagged `want`
+  // when sel is set): pass 1 screens the tiles the probe left (lo_off), every
+  // later pass the whole range for the rows the rescoring sent back.
+  auto ranked = [&](const int* sel, int want, int lo_off) -> bool {
+    for (int pass = 1; pass <= kRankEst; ++pass) {
+      const RankPass rp{pass, pass == 1 ? lo_off : 0, 0, pass == 1 ? sel : nullptr, want,
+                        nullptr};
+      if (launch_rank_screen(*h, c, b, K, W, rp, stream) != cudaSuccess ||
+          launch_rescore(*h, c, b, K, W, rp, stream) != cudaSuccess)
         return false;
     }
     return true;
   };
+  // The probe of the items flagged `want`: estimates, kRankProbeTiles screened
+  // tiles per item, and the decision (kItemRank or kItemFilter).
+  auto probe = [&](int want) -> bool {
+    const RankPass rp{1, 0, kRankProbeTiles, b.item_flag, want, b.rank_cnt};
+    return cudaMemsetAsync(b.rank_cnt, 0, (size_t)n_items * 16, stream) == cudaSuccess &&
+           launch_rank_prep(*h, c, b, K, W, b.item_flag, want, stream) == cudaSuccess &&
+           launch_rank_screen(*h, c, b, K, W, rp, stream) == cudaSuccess &&
+           launch_rank_decide(b.item_flag, b.rank_cnt, n_items, want, b.gate, b.counters,
+                              stream) == cudaSuccess;
+  };
+  if (mode >= 2 && (cudaMemsetAsync(b.row_next, 0, (size_t)c.rows * 4, stream) != cudaSuccess ||
+                    cudaMemsetAsync(b.pass_any, 0, (kRankEst + 2) * 4, stream) != cudaSuccess))
+    return DOSA_ERR_CUDA;
   if (mode == 0) {
     if (launch_filter(*h, c, b, K, StepRange{0, kAll, -1}, stream) != cudaSuccess)
       return DOSA_ERR_CUDA;
   } else if (mode == 1) {
-    const bool streams = b.surv && h->cfg.survivor_stream == 2, split = blk || streams;
-    if (launch_certified(*h, c, b, K, StepRange{0, split ? P : kAll, -1}, 0, stream) !=
-            cudaSuccess ||
-        (split && !(streams ? streamed_rest(P, -1) : certified_rest(P, -1))))
+    if (launch_certified(*h, c, b, K, StepRange{0, blk ? P : kAll, -1}, stream) != cudaSuccess ||
+        (blk && !certified_rest(P)))
+      return DOSA_ERR_CUDA;
+  } else if (mode == 3) {
+    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess ||
+        launch_rank_prep(*h, c, b, K, W, nullptr, 0, stream) != cudaSuccess ||
+        !ranked(nullptr, 0, 0))
       return DOSA_ERR_CUDA;
   } else {
     // The probe: all items, or the sampled items first and the others only
-    // when some sampled item found screening worth it (else they go to the
+    // when some sampled item chose ranked screening (else they go to the
     // filter scorer unprobed, from the warm-up's end).
-    const int n_items = (int)((c.rows + 7) / 8);
-    auto probe = [&]() -> bool {
+    auto probes = [&]() -> bool {
       if (!b.probe_sample)
-        return launch_certified(*h, c, b, K, StepRange{W, P, -1}, 1, stream) == cudaSuccess;
-      return launch_certified(*h, c, b, K, StepRange{W, P, kItemSample}, 1, stream) ==
-                 cudaSuccess &&
+        return cudaMemsetAsync(b.item_flag, 0, (size_t)n_items * 4, stream) == cudaSuccess &&
+               probe(0);
+      return probe(kItemSample) &&
              launch_probe_resolve(b.item_flag, n_items, b.gate, stream) == cudaSuccess &&
              launch_cert_setup(*h, c, b.key_sum, b.bdir, b.cert, b.retained, stream, 2,
                                b.item_flag, b.gate) == cudaSuccess &&
-             launch_certified(*h, c, b, K, StepRange{W, P, kItemProbe}, 1, stream) ==
-                 cudaSuccess;
+             probe(kItemProbe);
     };
     // the filter scorer finishes the items whose probe chose it, and the
-    // unprobed items from the warm-up's end, in one launch
-    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess || !probe() ||
-        launch_filter(*h, c, b, K, StepRange{P, kAll, kItemFilter, kItemUnprobed, W}, stream) !=
+    // unprobed items, from the warm-up's end, in one launch
+    if (launch_filter(*h, c, b, K, StepRange{0, W, -1}, stream) != cudaSuccess || !probes() ||
+        launch_filter(*h, c, b, K, StepRange{W, kAll, kItemFilter, kItemUnprobed, W}, stream) !=
             cudaSuccess ||
-        !certified_rest(P, kItemScreen) || (b.surv && !streamed_rest(P, kItemStream)))
+        !ranked(b.item_flag, kItemRank, kRankProbeTiles))
       return DOSA_ERR_CUDA;
   }
   if (b.dense) {
@@ -581,13 +601,17 @@ static dosa_status read_stats(const void* workspace, const int64_t* seq_offsets,
   stats->visible_pairs = total_visible(seq_offsets, B);
   stats->seed_pairs = (int64_t)hdr.counters[kCntSeedPairs];
   stats->screened_pairs = (int64_t)hdr.counters[kCntScreened];
-  stats->rejected_pairs = (int64_t)hdr.counters[kCntRejected];
+  // pairs rejected by the first ranked pass and scored by a later one are not
+  // rejected in the end
+  stats->rejected_pairs =
+      (int64_t)hdr.counters[kCntRejected] - (int64_t)hdr.counters[kCntBandPairs];
   stats->exact_pairs = (int64_t)hdr.counters[kCntExact];
   stats->candidates = (int64_t)hdr.counters[kCntCandidates];
   stats->filtered_pairs = (int64_t)hdr.counters[kCntFiltered];
   stats->block_skipped_pairs = (int64_t)hdr.counters[kCntBlockSkipped];
   stats->rescored_pairs = (int64_t)hdr.counters[kCntRescored];
   stats->repaired_rows = (int64_t)hdr.counters[kCntOverflow];
+  stats->rescreened_pairs = (int64_t)hdr.counters[kCntBandPairs];
   if (hdr.error) return hdr.error == kDevTimeout ? DOSA_ERR_TIMEOUT : DOSA_ERR_DEVICE_CHECK;
   return DOSA_OK;
 }
@@ -932,15 +956,24 @@ dosa_status dosa_index_decode_topk(dosa_index_t hh, const void* q, const float* 
 dosa_status dosa_index_certificate(dosa_index_t hh, const void* q, const float* q_scale,
                                    const float* w, const void* k, const float* k_scale,
                                    const int64_t* seq_offsets, int B, float* cert_out,
-                                   int32_t* retained_out, void* workspace, size_t ws_bytes,
-                                   void* stream_) {
+                                   int32_t* retained_out, void* bound_out, void* workspace,
+                                   size_t ws_bytes, void* stream_) {
   const Handle* h = reinterpret_cast<const Handle*>(hh);
   if (!cert_out || !retained_out) return DOSA_ERR_INVALID_ARG;
   dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, 1, retained_out);
   if (st != DOSA_OK) return st;
-  return for_each_cert_chunk(h, q, q_scale, w, k, k_scale, seq_offsets, B, 1, workspace, ws_bytes,
-                             static_cast<cudaStream_t>(stream_), cert_out, retained_out,
-                             [](const SeqView&, const CertBuffers&) { return DOSA_OK; });
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const size_t row_bytes = (size_t)kBoundRows * kHeadDim * elem_bytes(h);
+  return for_each_cert_chunk(
+      h, q, q_scale, w, k, k_scale, seq_offsets, B, 1, workspace, ws_bytes, stream, cert_out,
+      retained_out, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {
+        if (!bound_out || c.rows == 0) return DOSA_OK;
+        return cudaMemcpyAsync(static_cast<uint8_t*>(bound_out) + (size_t)c.row0 * row_bytes,
+                               b.bdir, (size_t)c.rows * row_bytes, cudaMemcpyDeviceToDevice,
+                               stream) == cudaSuccess
+                   ? DOSA_OK
+                   : DOSA_ERR_CUDA;
+      });
 }
 
 static dosa_status scores_common(dosa_index_t hh, const void* q, const float* q_scale,

@@ -32,6 +32,7 @@ enum CounterId : int {
   kCntFiltered = 6,
   kCntBlockSkipped = 7,
   kCntRescored = 8,
+  kCntBandPairs = 9,       // survivors of the later ranked passes (rejected by pass 1)
 };
 constexpr size_t kWsHeaderBytes = 256;
 
@@ -104,11 +105,16 @@ struct CertBuffers {
   int* step_list;        // [rows / 8 + 1][step_cap] steps left after block screening
   int* step_count;       // [rows / 8 + 1]
   int step_cap;
-  int* surv;             // [rows][surv_cap] survivor keys of streamed items, or null
-  int* surv_count;       // [rows], zeroed before a screening pass
-  int surv_cap;
-  unsigned long long* item_cnt;   // [rows / 8 + 1][3] held-back counts of streamed items
-  int* ovf;              // [rows / 8 + 1] survivor lists overflowed in the current pass
+  // ranked screening (rank_screen.cu, rescore.cu)
+  uint32_t* bits;        // [rows][words] survivor bits of the current pass
+  int64_t words;         // 32-bit words per row: 4 per key tile of S_max
+  float* est;            // [rows][kRankEst] descending threshold estimates
+  float* band_lo;        // [rows] the current pass keeps lo <= v < hi
+  float* band_hi;
+  uint32_t* maxrej;      // [rows] ordered largest bound the current pass rejected
+  int* row_next;         // [rows] the pass a row waits for (0: done or not ranked)
+  int* pass_any;         // [kRankEst + 2] some row waits for pass j
+  unsigned long long* rank_cnt;   // [rows / 8 + 1][2] probe: screened, kept pairs per item
   int* gate;             // set by the probe when a sampled item chose screening
   int probe_sample;      // the chunk's set-up covered only the sampled items
   unsigned long long* counters;
@@ -178,18 +184,49 @@ struct StepRange {
 // b.step_list / b.step_count (the range's last step is always kept).
 cudaError_t launch_block_screen(const Handle& h, const SeqView& v, const CertBuffers& b,
                                 StepRange steps, cudaStream_t stream);
-// Certified scorer over a range of steps; decide = 1 flags each item whose
-// range ends before its last step (filter, keep screening, or survivor
-// streams).  use_list = 1: each item processes b.step_list instead of the
-// whole range; use_list = 2: survivor mode (screening only, survivors to
-// b.surv, state saved at the range end, counts held back in b.item_cnt).
+// Certified scorer (the streaming schedule) over a range of steps.  use_list
+// = 1: each item processes b.step_list instead of the whole range.
 cudaError_t launch_certified(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                             StepRange steps, int decide, cudaStream_t stream, int use_list = 0);
-// Rescoring of the survivor lists a screening pass left over `range` (gathered
-// keys on the tensor cores), publishing rows whose item ends in the range and
-// saving the others; items with an overflowed list get b.ovf[item] = 1.
+                             StepRange steps, cudaStream_t stream, int use_list = 0);
+
+// ---- ranked screening (rank_screen.cu, rescore.cu) ----------------------------
+constexpr int kRankRows = 32;          // query rows per bound unit (N = 32 x 8 = 256)
+constexpr int kRankUnitTiles = 64;     // key tiles per bound unit, at most
+constexpr int kRankEst = 5;            // threshold estimates per row (m, 8m, ..., K)
+constexpr int kRankProbeTiles = 4;     // key tiles per item the probe screens
+// The probe keeps an item on ranked screening when it screened at least
+// kRankMinScreened pairs and kept at most 1 in kRankKeepRatio of them.
+constexpr unsigned long long kRankMinScreened = 1024;
+constexpr unsigned long long kRankKeepRatio = 4;
+// One pass of ranked screening: pass 1 keeps v >= the row's first estimate,
+// pass j > 1 the band the previous rescoring chose.  Key tiles [jlo, jhi) of
+// an item with L = n_tiles - W + 1 screened tiles [1, L): jhi = L - lo_off,
+// jlo = hi_off > 0 ? L - hi_off : 1 (the probe: hi_off = kRankProbeTiles; the
+// rest after it: lo_off = kRankProbeTiles).  Rows: those with
+// row_next == pass, of the items whose flag equals `want` (all when
+// item_sel is null).
+struct RankPass {
+  int pass;
+  int lo_off, hi_off;
+  const int* item_sel;
+  int want;
+  unsigned long long* item_cnt;   // probe counts per item, or null
+};
+// Threshold estimates from each selected row's warm-up histogram; the rows
+// then wait for pass 1.
+cudaError_t launch_rank_prep(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                             int W, const int* item_sel, int want, cudaStream_t stream);
+// The bound pass: survivor bits, per-row largest rejected bound, counters.
+cudaError_t launch_rank_screen(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
+                               int W, const RankPass& rp, cudaStream_t stream);
+// Rescoring of the pass's survivors; rows are published or given the next band.
 cudaError_t launch_rescore(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
-                           StepRange range, cudaStream_t stream);
+                           int W, const RankPass& rp, cudaStream_t stream);
+// After the probe: items flagged `want` become kItemRank (raising *gate and
+// adding their probe counts to the call's counters) or kItemFilter.
+cudaError_t launch_rank_decide(int* item_flag, const unsigned long long* item_cnt, int n_items,
+                               int want, int* gate, unsigned long long* counters,
+                               cudaStream_t stream);
 // Filter scorer (exact scores, threshold filter, no bounds) over a range.
 cudaError_t launch_filter(const Handle& h, const SeqView& v, const CertBuffers& b, int K,
                           StepRange steps, cudaStream_t stream);

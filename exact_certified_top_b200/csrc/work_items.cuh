@@ -41,17 +41,15 @@ __device__ __forceinline__ int tile_at(int ti, int n_tiles) {
   return ti == 0 ? 0 : n_tiles - ti;
 }
 
-// What the probe pass decided for an item (certified workspace flags).
-// Probe decisions: filter scorer, certified scorer on the resident key tile,
-// or certified screening into survivor lists then rescoring of the gathered
-// survivors (kItemStream).  Before the decisions: kItemSample marks the items
-// probed first (every kProbeSampleStride-th item, longest rows first), and
-// kItemProbe the others once the sample showed that screening pays somewhere;
-// otherwise they become kItemUnprobed (filter scorer from the warm-up's end).
+// What the probe pass decided for an item (certified workspace flags): the
+// filter scorer finishes it, or ranked screening does (rank_screen.cu,
+// rescore.cu).  Before the decisions: kItemSample marks the items probed first
+// (every kProbeSampleStride-th, longest rows first), and kItemProbe the others
+// once the sample showed that screening pays somewhere; otherwise they become
+// kItemUnprobed (filter scorer from the warm-up's end).
 enum ItemFlag : int {
   kItemFilter = 1,
-  kItemScreen = 2,
-  kItemStream = 3,
+  kItemRank = 2,
   kItemSample = 4,
   kItemProbe = 5,
   kItemUnprobed = 6

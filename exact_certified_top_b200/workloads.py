@@ -133,14 +133,23 @@ def generate(wl: Workload, device="cpu", chunk: int = 4096) -> dict:
     int64, seq_offsets [[0, 0, q_pos0], [T, S, 0]] int64 (host), sinks [S] bool.
     The same seed on the same device gives the same bytes."""
     device = torch.device(device)
-    g = torch.Generator(device=device)
-    g.manual_seed(int(wl.seed) * 1000003 + 17)
+    # The workload's own constants (means, low-rank maps, sink positions) come
+    # from a host generator, so every device draws the same workload; the
+    # per-token draws use the device's generator (same seed).
+    seed = int(wl.seed) * 1000003 + 17
+    gh = torch.Generator(device="cpu")
+    gh.manual_seed(seed)
     H, d, T, S = wl.H, wl.d, wl.T, wl.S
-    mu_k = _randn(g, (d,), device)
-    A_k = _randn(g, (d, 16), device) / 4.0
-    mu_q = _randn(g, (d,), device)
-    A_q = _randn(g, (d, 16), device) / 4.0
-    sinks = torch.rand((S,), generator=g, device=device) < wl.sink_frac
+    mu_k = _randn(gh, (d,), "cpu").to(device)
+    A_k = (_randn(gh, (d, 16), "cpu") / 4.0).to(device)
+    mu_q = _randn(gh, (d,), "cpu").to(device)
+    A_q = (_randn(gh, (d, 16), "cpu") / 4.0).to(device)
+    sinks = (torch.rand((S,), generator=gh) < wl.sink_frac).to(device)
+    if device.type == "cpu":
+        g = gh
+    else:
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
 
     # keys, chunked over tokens
     kf = torch.empty((S, d), dtype=torch.float32, device=device)

@@ -74,7 +74,7 @@ typedef enum { DOSA_BF16 = 0, DOSA_FP8_E4M3 = 1 } dosa_dtype;
 /* Fixed at create time.  Defaults (dosa_index_config_default): H = 64, d = 128,
  * bf16, max_K = 2048, seed_first = 64, seed_last = 512, r = 4, G = 2,
  * margin_log2 = -12, screening = 2, sparse_writeback = 1, block_bound = 1,
- * survivor_stream = 0, probe_sample = 1. */
+ * probe_sample = 1. */
 typedef struct {
   int H;            /* indexer heads per query: 64 or 32.  With 32 the kernels
                        read each query row into 64 head slots (the other 32
@@ -87,33 +87,36 @@ typedef struct {
   int r;            /* retained positive heads evaluated exactly (0..4)         */
   int G;            /* negative-head groups (0 = no negative aggregate, 1, 2)   */
   int margin_log2;  /* soundness margin 2^margin_log2 * sum|w|||q|| * ||k||     */
-  int screening;    /* 1: screen every key tile with the certificate; 2: adaptive
-                       (every tile of 8 queries is screened over its first key
-                       tiles; where that rejected under 1/32 of 2048 or more
-                       screened pairs, the rest of its keys is scored exactly
-                       without bounds, else screening goes on to the end);
-                       0: never (ablation).  The selection is exact in every
-                       mode.                                                    */
+  int screening;    /* How keys are screened after the warm-up (key tile 0 and
+                       the tiles at the diagonal, scored exactly until K exact
+                       scores exist).  3: ranked -- every remaining key of a
+                       row is screened once against an estimate of a score a
+                       little below its K-th (from the warm-up scores); the
+                       survivors are gathered and scored with all heads, and
+                       the estimate is then checked against the K-th reached:
+                       a row where a rejected key's bound is not below it is
+                       screened again over the band of bounds between them
+                       (lower estimates, down to the warm-up threshold).
+                       2 (default): adaptive -- each work item of 8 queries
+                       is screened over 4 key tiles first and goes on with
+                       ranked screening where that kept at most 1 in 4 of
+                       1024 or more screened pairs; the others are scored
+                       exactly without bounds.  1: the streaming schedule --
+                       every tile is screened against the threshold reached
+                       so far, tile after tile.  0: never (ablation).  The
+                       selection is exact in every mode.                      */
   int sparse_writeback; /* 1 (default): only scores >= the running threshold
                        are written, as packed (score, key) candidates, and the
                        selection reads those; 0 (ablation): every exact score
                        is also written into a dense [rows, keys] matrix of the
                        chunk (rejected pairs as -inf) and the selection is the
                        dense Top-K of that matrix.  Same result either way.   */
-  int block_bound;  /* 1 (default): before the certified scorer resumes an item
-                       after its warm-up, every key tile is bounded as a whole
-                       (a ball around the tile's mean key) and tiles that can
-                       hold no Top-K key of the item's queries are skipped
-                       without loading their keys; 0: off (ablation).         */
-  int survivor_stream; /* 0 (default): every screened item is rescored on the
-                       resident key tile.  1: work items whose probe rejected
-                       >= 7/8 of the screened pairs are screened into per-row
-                       survivor lists, in passes over doubling key ranges, and
-                       the survivors are gathered and rescored on dense
-                       tensor-core tiles (items whose lists overflow are
-                       rescored by the filter scorer for that pass); 2: as 1,
-                       and with screening = 1 every item streams after its
-                       probe steps.  Same result in every mode.               */
+  int block_bound;  /* screening = 1 only.  1 (default): before the certified
+                       scorer resumes an item after its warm-up, every key
+                       tile is bounded as a whole (a ball around the tile's
+                       mean key) and tiles that can hold no Top-K key of the
+                       item's queries are skipped without loading their keys;
+                       0: off (ablation).                                     */
   int probe_sample;  /* screening = 2 only.  1 (default): every 7th work item
                        (longest rows first) is set up and probed first; the
                        other items are set up and probed only if one of those
@@ -133,9 +136,13 @@ typedef struct {
   int64_t filtered_pairs;  /* exact pairs scored by the filter scorer (no bounds)    */
   int64_t block_skipped_pairs; /* rejected pairs of key tiles skipped whole by the
                                   key-block certificate (keys never loaded)      */
-  int64_t rescored_pairs;  /* exact pairs scored from gathered survivor streams     */
+  int64_t rescored_pairs;  /* exact pairs scored from gathered survivors (ranked)   */
   int64_t repaired_rows;   /* rows whose candidate list overflowed and were scored
-                              again densely (at most 64 per chunk of rows)       */
+                              again densely (a tie at the K-th score spanning
+                              more keys than the list holds; at most 64 to 512
+                              rows per chunk of rows, depending on S_max)       */
+  int64_t rescreened_pairs; /* ranked screening: pairs the first pass rejected and
+                               a later pass (a lower band of bounds) scored      */
 } dosa_stats;
 
 typedef struct dosa_index* dosa_index_t;
@@ -231,12 +238,19 @@ dosa_status dosa_index_decode_workspace_size(dosa_index_t h, int64_t Tq, int64_t
  * [10] the per-head residual sum, [11] the joint (spectral) residual bound,
  * [12] |A_1|, [13] |A_2|, [14] number of omitted positive heads, [15] unused.
  * retained_out: [Tq, 4] int32 retained head indices, ascending, -1 padded.
+ * bound_out (nullable): [Tq, 8, d] codes in the input type, the bound rows the
+ * screening multiplies with the keys: rows 0..3 the retained heads' query codes
+ * (zero rows when fewer are retained), rows 4..7 the negative aggregates u_1
+ * and u_2, each as a hi row and a lo row (u_g = scale[6+2g] * hi + scale[7+2g]
+ * * lo, code domain).  With them and cert_out, the bound of every pair can be
+ * rebuilt: UB = sum_j omega_j ReLU(row_j . k) + (beta + c) ||k|| -
+ * sum_g ReLU(scale_hi row_hi . k + scale_lo row_lo . k).
  * Workspace: as dosa_index_topk (certified = 1, K = 1 is enough). */
 dosa_status dosa_index_certificate(dosa_index_t h, const void* q, const float* q_scale,
                                    const float* w, const void* k, const float* k_scale,
                                    const int64_t* seq_offsets, int B, float* cert_out,
-                                   int32_t* retained_out, void* workspace, size_t ws_bytes,
-                                   void* stream);
+                                   int32_t* retained_out, void* bound_out, void* workspace,
+                                   size_t ws_bytes, void* stream);
 
 /* Dense Top-K: every visible key is scored with all heads (tensor-core scorer),
  * score rows are materialised chunk by chunk in the workspace, then a per-row
@@ -316,7 +330,8 @@ typedef enum {
   DOSA_KERNEL_BLOCK = 10,      /* key-block certificate: block statistics and  */
                                /* per-item block screening                      */
   DOSA_KERNEL_RESCORE = 11,    /* rescoring of gathered survivors               */
-  DOSA_KERNEL_KINDS = 12
+  DOSA_KERNEL_RANK = 12,       /* ranked screening: estimates and bound passes  */
+  DOSA_KERNEL_KINDS = 13
 } dosa_kernel;
 
 /* Kernel timing.  While enabled, every kernel a call launches is bracketed by

@@ -174,10 +174,16 @@ def nnls_retained(Q_R: np.ndarray, v: np.ndarray) -> np.ndarray:
     "Positive-weight heads are retained, while projections minimize their
     residual norm" ([DPC] Method) with nonnegative coefficients ("nonnegative
     head projections", [DPC] Conclusion; [ZICQ] point 2).  Solved exactly for
-    small r by trying every support: the NNLS optimum is the unconstrained
+    r <= 4 by trying every support: the NNLS optimum is the unconstrained
     least-squares solution on its own support, so the best feasible candidate
-    over all supports is the optimum."""
+    over all supports is the optimum.  For more retained heads (the head-budget
+    study) scipy's NNLS routine (Lawson and Hanson's active-set method) serves
+    as the step."""
     r = Q_R.shape[0]
+    if r > 4:
+        from scipy.optimize import nnls
+        alpha, _ = nnls(Q_R.T, v)
+        return alpha
     best_alpha = np.zeros(r)
     best_res = float(v @ v)
     for size in range(1, r + 1):

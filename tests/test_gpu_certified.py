@@ -33,7 +33,10 @@ def _args(x, K):
     return (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], x["seq_offsets"], K)
 
 
-@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
+MODES = dict(argvalues=[3, 2, 1, 0], ids=["ranked", "adaptive", "streaming", "off"])
+
+
+@pytest.mark.parametrize("screening", **MODES)
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
 def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     base, T, S, K = case
@@ -45,7 +48,7 @@ def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     assert np.array_equal(cert, dense), "certified selection differs from the dense selection"
     ov = OracleView(x, wl.dtype)
     for t in range(0, wl.T, max(1, wl.T // 120)):
-        assert_topk_matches(cert[t], ov.scores(t), K, t=t, exact=wl.levels > 0)
+        assert_topk_matches(cert[t], ov.scores(t), K, mag=ov.magnitude(t), t=t, exact=wl.levels > 0)
     assert stats["visible_pairs"] == wl.visible_pairs
     assert 0 <= stats["rejected_pairs"] <= stats["screened_pairs"]
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
@@ -55,6 +58,8 @@ def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
         assert stats["filtered_pairs"] == wl.visible_pairs
     if screening == 1:
         assert stats["filtered_pairs"] == 0
+    if screening >= 2:
+        assert stats["rescreened_pairs"] <= stats["exact_pairs"]
 
 
 def test_certified_small_workspace_many_chunks(cuda_lib):
@@ -127,7 +132,7 @@ def test_varlen_batch_with_empty_sequences(cuda_lib, dtype):
         if wl.T:
             ov = OracleView(x, dtype)
             for t in range(0, wl.T, 5):
-                assert_topk_matches(cert[r + t], ov.scores(t), K, t=(wl.name, t))
+                assert_topk_matches(cert[r + t], ov.scores(t), K, mag=ov.magnitude(t), t=(wl.name, t))
         r += wl.T
 
 
@@ -153,7 +158,7 @@ def _redundant_heads_case(T=96, S=6000, seed=0, fp8=False):
                 seq_offsets=so, positions=torch.arange(pos0, S)), "bf16"
 
 
-@pytest.mark.parametrize("screening", [2, 1])
+@pytest.mark.parametrize("screening", [3, 2, 1], ids=["ranked", "adaptive", "streaming"])
 @pytest.mark.parametrize("fp8", [False, True])
 def test_certified_prunes_and_stays_exact_when_heads_are_redundant(cuda_lib, fp8, screening):
     x, dtype = _redundant_heads_case(fp8=fp8)
@@ -240,10 +245,10 @@ def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
     ov = OracleView(x, dtype)
     cert = to_numpy(cert)
     for t in range(0, 160, 7):
-        assert_topk_matches(cert[t], ov.scores(t), K, t=t, exact=False)
+        assert_topk_matches(cert[t], ov.scores(t), K, mag=ov.magnitude(t), t=t, exact=False)
 
 
-@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
+@pytest.mark.parametrize("screening", **MODES)
 @pytest.mark.parametrize("S", [5200, 70000])
 def test_repair_pass_when_candidates_overflow(cuda_lib, screening, S):
     """All keys identical: every score ties, every key becomes a candidate and
@@ -291,7 +296,7 @@ def test_host_staged_call_equals_device_call(cuda_lib, case):
     assert np.array_equal(out2.numpy(), dev)
 
 
-@pytest.mark.parametrize("screening", [2, 1, 0], ids=["adaptive", "always", "off"])
+@pytest.mark.parametrize("screening", **MODES)
 @pytest.mark.parametrize("case", [("prefill_128k_fp8", 203, 2600, 300),
                                   ("tight_64k_bf16_levels", 157, 2100, 512)],
                          ids=lambda c: c[0])
@@ -345,9 +350,11 @@ def _clustered_blocks_case(T=48, n_tiles=50, seed=5, fp8=False):
                 seq_offsets=so, positions=torch.arange(pos0, S)), "bf16"
 
 
-@pytest.mark.parametrize("screening", [2, 1])
+@pytest.mark.parametrize("screening", [1])
 @pytest.mark.parametrize("fp8", [False, True])
 def test_key_block_certificate_skips_tiles_and_stays_exact(cuda_lib, fp8, screening):
+    """The key-block certificate acts in the streaming schedule (screening =
+    1): whole tiles whose block bound rules them out are skipped."""
     x, dtype = _clustered_blocks_case(fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
@@ -366,7 +373,7 @@ def test_key_block_certificate_skips_tiles_and_stays_exact(cuda_lib, fp8, screen
     assert sa["block_skipped_pairs"] <= sa["rejected_pairs"]
     ov = OracleView(x, dtype)
     for t in range(0, T, 5):
-        assert_topk_matches(to_numpy(a)[t], ov.scores(t), K, t=t)
+        assert_topk_matches(to_numpy(a)[t], ov.scores(t), K, mag=ov.magnitude(t), t=t)
 
 
 def test_key_block_bounds_agree_with_oracle(cuda_lib):
@@ -404,87 +411,118 @@ def test_key_block_bounds_agree_with_oracle(cuda_lib):
     # the GPU's skipped pairs never exceed what the ideal bound could drop
     assert st["block_skipped_pairs"] <= droppable * 128 * 8
     for t in range(8):
-        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
+        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, mag=ov.magnitude(t), t=t)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
-def test_survivor_streams_rescore_gathered_keys_exactly(cuda_lib, fp8):
-    """Redundant heads and a small K: the probe rejects nearly every screened
-    pair, so the items go to survivor streams (screening into per-row lists,
-    then the gathered survivors rescored on the tensor cores).  The selection
-    must equal the dense path's, survivors must have been rescored, and the
-    counters must add up; without streams the same selection comes out."""
+def test_ranked_screening_rescores_gathered_survivors_exactly(cuda_lib, fp8):
+    """Redundant heads and a small K, ranked screening of every item: one bound
+    pass keeps the keys above each row's estimate, the gathered survivors are
+    scored on the tensor cores.  The selection equals the dense path's, the
+    counters add up, most pairs are rejected, and no more than the oracle's
+    ideal screening (threshold = the true K-th) would reject."""
     x, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 32
     dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
-    on, st_on = binding.Index(dtype, survivor_stream=1).topk(*_args(xd, K), stats=True)
-    off, st_off = binding.Index(dtype, survivor_stream=0).topk(*_args(xd, K), stats=True)
-    assert np.array_equal(to_numpy(on), dense)
-    assert np.array_equal(to_numpy(off), dense)
-    T, S = x["q"].shape[0], x["k"].shape[0]
-    visible = sum(S - T + t + 1 for t in range(T))
-    for st in (st_on, st_off):
-        assert st["exact_pairs"] + st["rejected_pairs"] == visible
-    assert st_on["rescored_pairs"] > 0, st_on
-    assert st_off["rescored_pairs"] == 0
-    assert st_on["rejected_pairs"] > visible // 2
-    ov = OracleView(x, dtype)
-    for t in range(0, T, 7):
-        assert_topk_matches(to_numpy(on)[t], ov.scores(t), K, t=t)
-
-
-@pytest.mark.parametrize("redundant", [True, False], ids=["redundant", "random"])
-def test_survivor_streams_every_item(cuda_lib, redundant):
-    """screening = 1 with survivor_stream = 2: every item streams after its
-    probe steps, in passes over doubling key ranges.  On redundant heads the
-    lists hold few survivors and are rescored from the gathered keys; on the
-    random case nearly nothing is rejected, the later passes overflow their
-    lists and the filter scorer redoes those passes.  Either way the selection
-    is the dense path's and every visible pair is counted exactly once."""
-    if redundant:
-        x, dtype = _redundant_heads_case(T=64, S=20000, seed=5, fp8=True)
-        K = 32
-    else:
-        _, x, _ = _inputs("prefill_128k_fp8", 200, 9000, 300)
-        dtype = "fp8"
-        K = 300
-    xd = {k: (v.cuda() if torch.is_tensor(v) and k != "seq_offsets" else v) for k, v in x.items()}
-    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
-    out, st = binding.Index(dtype, screening=1, survivor_stream=2).topk(*_args(xd, K), stats=True)
+    out, st = binding.Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), dense)
     T, S = x["q"].shape[0], x["k"].shape[0]
     visible = sum(S - T + t + 1 for t in range(T))
     assert st["exact_pairs"] + st["rejected_pairs"] == visible
     assert st["rescored_pairs"] > 0, st
-    if redundant:
-        assert st["filtered_pairs"] <= visible // 4, st
-    else:
-        assert st["filtered_pairs"] > 0, st
+    assert st["rejected_pairs"] > 0.8 * visible, st
     ov = OracleView(x, dtype)
-    for t in range(0, T, 9):
-        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, t=t)
+    kb = key_mean(ov.k)
+    ideal = 0
+    for t in range(T):
+        p = int(ov.positions[t])
+        res = certified_topk_row(ov.q[t], ov.w[t], ov.k[: p + 1], K, k_bar=kb, r=4, G=2,
+                                 margin_log2=-12)
+        ideal += res["ideal_rejected"]
+        if t % 7 == 0:
+            assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, mag=ov.magnitude(t), t=t)
+    assert st["rejected_pairs"] <= ideal * 1.002 + 16, (st, ideal)
+
+
+def _overshoot_case(fp8):
+    """Redundant heads along one direction b; random keys, plus a few keys
+    along b in the warm-up region (very high scores) and a few hundred keys
+    along b in the middle of the sequence (high, but below those).  The
+    warm-up sample then puts the first estimate above the K-th score, pass 1
+    keeps too few keys, and later passes over lower bands must find the
+    middle keys."""
+    g = torch.Generator().manual_seed(17)
+    d, H, T, S = 128, 64, 16, 20000
+    b = torch.randn(d, generator=g)
+    b = b / b.norm()
+    q = 3.0 * b + 0.02 * torch.randn((T, H, d), generator=g)
+    w = torch.rand((T, H), generator=g) / 8
+    k = torch.randn((S, d), generator=g)
+    k[:6] += 8.0 * b                                  # tile 0: very high
+    k[S - 200:S - 194] += 8.0 * b                     # diagonal tiles: very high
+    mid = torch.randperm(S - 4000, generator=g)[:300] + 2000
+    k[mid] += 4.0 * b                                 # the rest of the Top-K
+    so = [[0, 0, S - T], [T, S, 0]]
+    if fp8:
+        from exact_certified_top_b200.workloads import _e4m3_per_token
+        q8, qs = _e4m3_per_token(q)
+        k8, ks = _e4m3_per_token(k)
+        return dict(q=q8, q_scale=qs, w=w, k=k8, k_scale=ks, seq_offsets=so,
+                    positions=torch.arange(S - T, S)), "fp8"
+    return dict(q=q.to(torch.bfloat16), q_scale=None, w=w, k=k.to(torch.bfloat16),
+                k_scale=None, seq_offsets=so, positions=torch.arange(S - T, S)), "bf16"
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_ranked_later_passes_recover_an_estimate_set_too_high(cuda_lib, fp8):
+    x, dtype = _overshoot_case(fp8)
+    xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    K = 64
+    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
+    out, st = binding.Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out), dense)
+    assert st["rescreened_pairs"] > 0, st
+    assert st["exact_pairs"] + st["rejected_pairs"] == st["visible_pairs"]
+    assert st["rejected_pairs"] > 0.5 * st["visible_pairs"], st
+    ov = OracleView(x, dtype)
+    for t in range(0, 16, 3):
+        assert_topk_matches(to_numpy(out)[t], ov.scores(t), K, mag=ov.magnitude(t), t=t)
+
+
+def test_ranked_screening_on_a_loose_bound_keeps_every_key(cuda_lib):
+    """Independent random heads (the bound is loose): ranked screening keeps
+    nearly every key, gathers and scores them all, and still returns the
+    dense selection; the adaptive mode hands the same rows to the filter
+    scorer after its probe."""
+    _, x, xd = _inputs("prefill_128k_fp8", 200, 9000, 300)
+    K = 300
+    dense = to_numpy(binding.Index("fp8").dense_topk(*_args(xd, K)))
+    out, st = binding.Index("fp8", screening=3).topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out), dense)
+    assert st["rescored_pairs"] > 0.5 * st["visible_pairs"], st
+    out2, st2 = binding.Index("fp8", screening=2, probe_sample=0).topk(*_args(xd, K), stats=True)
+    assert np.array_equal(to_numpy(out2), dense)
+    assert st2["rescored_pairs"] == 0 and st2["filtered_pairs"] == st2["visible_pairs"], st2
 
 
 def test_probe_samples_items_first(cuda_lib):
     """Adaptive screening probes every 7th work item (longest rows first)
-    before the others.  On random inputs no sampled item finds screening worth
-    it, so the other items are neither set up nor probed: only the sampled
-    items' probe steps are screened.  On redundant heads the sample finds it
-    worth it and every item is probed (most pairs end up rejected).  The
-    selection is the dense path's either way."""
+    before the others.  On random inputs no sampled item finds ranked
+    screening worth it, so no item is screened past its probe (no screened
+    pairs are counted) and the filter scorer scores every pair.  On redundant
+    heads the sample finds it worth it, every item is probed, and most pairs
+    are rejected.  The selection is the dense path's either way."""
     _, x, xd = _inputs("prefill_128k_fp8", 640, 6000, 300)
     K = 300
     idx = binding.Index("fp8")
     out, st = idx.topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), to_numpy(idx.dense_topk(*_args(xd, K))))
-    n_items = 640 // 8
-    sampled = (n_items + 6) // 7
-    assert 0 < st["screened_pairs"] <= sampled * 8 * 4 * 128, st
-    assert st["exact_pairs"] + st["rejected_pairs"] == st["visible_pairs"]
+    assert st["screened_pairs"] == 0 and st["filtered_pairs"] == st["visible_pairs"], st
     x2, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=True)
     xd2 = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x2.items()}
     K2 = 32
     out2, st2 = binding.Index(dtype).topk(*_args(xd2, K2), stats=True)
     assert np.array_equal(to_numpy(out2), to_numpy(binding.Index(dtype).dense_topk(*_args(xd2, K2))))
     assert st2["rejected_pairs"] > st2["visible_pairs"] // 2, st2
+    assert st2["rescored_pairs"] > 0, st2

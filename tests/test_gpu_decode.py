@@ -52,7 +52,8 @@ def test_decode_seeded_by_previous_step_equals_dense(cuda_lib, case):
     assert np.array_equal(out, dense)
     ov = OracleView(x, wl.dtype)
     for r in range(m):
-        assert_topk_matches(out[r], ov.scores(r + 1), K, t=r + 1, exact=False)
+        assert_topk_matches(out[r], ov.scores(r + 1), K, t=r + 1, exact=False,
+                            mag=ov.magnitude(r + 1))
     assert stats["exact_pairs"] == sum(S - m + r + 1 for r in range(m))
     # the candidates are the keys at or above the seed threshold: at least K
     # per row, and no more than the keys the oracle puts above the lowest

@@ -76,7 +76,7 @@ def test_dense_topk_matches_oracle(cuda_lib, case, K):
     out = to_numpy(idx.dense_topk(x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"],
                                   x["seq_offsets"], K))
     for t in range(wl.T):
-        assert_topk_matches(out[t], ov.scores(t), K, t=t, exact=wl.levels > 0)
+        assert_topk_matches(out[t], ov.scores(t), K, mag=ov.magnitude(t), t=t, exact=wl.levels > 0)
 
 
 def test_dense_topk_small_workspace_many_chunks(cuda_lib):
@@ -88,7 +88,7 @@ def test_dense_topk_small_workspace_many_chunks(cuda_lib):
                                   x["seq_offsets"], 32, workspace=ws))
     binding.check_device(ws)
     for t in range(wl.T):
-        assert_topk_matches(out[t], ov.scores(t), 32, t=t)
+        assert_topk_matches(out[t], ov.scores(t), 32, mag=ov.magnitude(t), t=t)
 
 
 def test_dense_topk_varlen_batch(cuda_lib):
@@ -112,7 +112,7 @@ def test_dense_topk_varlen_batch(cuda_lib):
     for wl, x in zip(parts, xs):
         ov = OracleView(x, "bf16")
         for t in range(wl.T):
-            assert_topk_matches(out[r + t], ov.scores(t), 50, t=(wl.name, t))
+            assert_topk_matches(out[r + t], ov.scores(t), 50, mag=ov.magnitude(t), t=(wl.name, t))
         r += wl.T
 
 

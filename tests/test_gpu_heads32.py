@@ -62,7 +62,7 @@ def test_h32_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     assert np.array_equal(to_numpy(cert), dense)
     ov = OracleView(x, wl.dtype)
     for t in range(0, wl.T, 5):
-        assert_topk_matches(dense[t], ov.scores(t), K, t=t, exact=wl.levels > 0)
+        assert_topk_matches(dense[t], ov.scores(t), K, mag=ov.magnitude(t), t=t, exact=wl.levels > 0)
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
 
 

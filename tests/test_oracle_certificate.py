@@ -41,6 +41,26 @@ def test_nnls_kkt_r4(seed):
             assert g[j] <= 1e-8        # no descent direction off the support
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_nnls_library_solver_agrees_with_exhaustive_supports(seed):
+    """The r > 4 path (scipy's active-set NNLS) against the exhaustive-support
+    solver on r <= 4, and the KKT conditions at r = 8 and 16."""
+    from scipy.optimize import nnls
+    rng = np.random.default_rng(40 + seed)
+    for r in (2, 3, 4):
+        Q = rng.standard_normal((r, 10)) + 0.5
+        v = rng.standard_normal(10) + 0.5
+        a_lib, _ = nnls(Q.T, v)
+        np.testing.assert_allclose(nnls_retained(Q, v), a_lib, atol=1e-9)
+    for r in (8, 16):
+        Q = rng.standard_normal((r, 32)) + 0.3
+        v = rng.standard_normal(32) + 0.3
+        a = nnls_retained(Q, v)
+        g = Q @ (v - a @ Q)
+        assert np.all(a >= 0)
+        assert np.all(np.abs(g[a > 1e-10]) < 1e-8) and np.all(g[a <= 1e-10] <= 1e-8)
+
+
 def test_nnls_exact_member_and_negative_target():
     Q = np.array([[1.0, 0.0, 0.0], [0.0, 1.0, 0.0]])
     assert np.allclose(nnls_retained(Q, np.array([2.0, 3.0, 5.0])), [2.0, 3.0])

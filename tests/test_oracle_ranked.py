@@ -116,3 +116,39 @@ def test_ideal_rejected_in_the_closed_form_where_the_bound_is_the_score():
                              seed_last=32, tile=16)
     assert res["ideal_rejected"] == want
     assert want > n // 2
+
+
+def test_stored_prune_study_matches_a_fresh_oracle_run():
+    """tests/golden/prune_study.json is written by tests/prune_study.py from
+    the oracle alone (64 rows per workload).  A fresh run of the same code on
+    one row per workload must agree with its conclusions: at the library's
+    head budget (r = 4) the mandated generator leaves nothing to prune, even
+    every positive head retained leaves the negative aggregate loose, and
+    redundant heads prune most pairs."""
+    import json
+    import os
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path.insert(0, here)
+    import prune_study
+    with open(os.path.join(here, "golden", "prune_study.json")) as f:
+        stored = {r["workload"]: r for r in json.load(f)["results"]}
+    assert stored["prefill_128k_fp8"]["ideal_prune_pct"]["r=4,G=2"] < 0.01
+    assert stored["tight_64k_bf16_levels"]["ideal_prune_pct"]["r=4,G=2"] < 0.01
+    assert stored["redundant_chunk128k_fp8"]["ideal_prune_pct"]["r=4,G=2"] > 90.0
+    assert len(stored["prefill_128k_fp8"]["rows"]) == 64
+    from dataclasses import replace
+    from exact_certified_top_b200.workloads import WORKLOADS, generate, small_case, codes_numpy
+    from oracle import dequantize, key_mean
+    for name, lo, hi in (("prefill_128k_fp8", 0.0, 0.01), ("redundant_chunk128k_fp8", 50.0, 100.0)):
+        wl = small_case(name, 2, 16384, q_pos0=16382)
+        x = generate(wl)
+        ks = None if x["k_scale"] is None else x["k_scale"].numpy()
+        k = dequantize(codes_numpy(x["k"]), ks, wl.dtype)
+        qs = None if x["q_scale"] is None else x["q_scale"][1:2].numpy()
+        q = dequantize(codes_numpy(x["q"][1:2]), qs, wl.dtype)[0]
+        res = prune_study.row_study(q, x["w"][1].numpy().astype(np.float64),
+                                    k[: wl.q_pos0 + 2], key_mean(k), wl.K)
+        pct = 100.0 * res["ideal"]["r=4,G=2"] / res["visible"]
+        assert lo <= pct <= hi, (name, pct)
+        assert res["ranked_rejected"] <= res["ideal"]["r=4,G=2"]
