@@ -254,6 +254,23 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
         exact = stats["exact_pairs"] - stats.get("filtered_pairs", 0)
         work = (flops_per_pair * exact + 2 * wl.d * 8 * stats["screened_pairs"]) * steps
         name = "certified_kernel"
+    elif dom == "rescore" and stats:
+        work = flops_per_pair * stats["rescored_pairs"] * steps
+        name = "rescore_kernel"
+    elif dom == "rank" and stats:
+        # the bound pass is bound by its epilogue's fp32 ALU work: 18 operations
+        # per screened pair (4 ReLU + 4 multiply-adds of the retained heads, the
+        # norm term, 2 x (2 multiply-adds, a ReLU, a subtraction) of the negative
+        # aggregates, the scale product), one operation per FP32 lane per clock
+        clk = (measured_peaks()[0].get("sm_max_mhz") or 1965.0) * 1e6
+        alu_peak = 148 * 128 * clk / 1e12              # T ops/s
+        ops = 18 * (stats["screened_pairs"] + stats.get("rescreened_pairs", 0)) * steps
+        achieved = ops / (ms * 1e-3) / 1e12
+        return {"kernel": "rank_screen_kernel (+ rank_prep)", "bound": "alu",
+                "achieved": round(achieved, 2), "peak": round(alu_peak, 2), "unit": "Tops/s",
+                "frac": round(achieved / alu_peak, 4), "traffic": None,
+                "peak_source": "148 SMs x 128 FP32 lanes x sm_max_mhz (one op per lane per clock)",
+                "launches": launches, "avg_launch_ms": round(ms / launches, 3)}
     elif dom == "decode" and stats:
         # seed + split-S scan + finish: every visible pair scored on the tensor
         # cores, every key of the cache read once per call.  The bound is the

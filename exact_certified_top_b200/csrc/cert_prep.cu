@@ -526,7 +526,9 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
             const int ra = 4 * A + i, cb = 4 * Bb + j;
             if (ra < no && cb < no && cb <= ra) {
               const int h1 = O[ra], h2 = O[cb];
-              const float g = fabsf(sqrtf(wv[h1] * wv[h2]) * acc[i][j]);
+              // sqrt(w) sqrt(w'), not sqrt(w w'): the product of two small
+              // weights can underflow fp32 where each root does not
+              const float g = fabsf(sqrtf(wv[h1]) * sqrtf(wv[h2]) * acc[i][j]);
               gt[ra][cb] = g;
               gt[cb][ra] = g;
               if (ra == cb) rn[h1] = sqrtf(acc[i][j]);
@@ -567,7 +569,9 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
       if (row && q == 0) vec[a] = mm > 0.f ? sa / mm : 1.f;
       __syncthreads();
     }
-    lam = row ? sa / fmaxf(vec[a], 1e-30f) : 0.f;
+    // Collatz-Wielandt needs v_a > 0; an entry that underflowed makes the
+    // joint bound unusable (beta falls back to the per-head sum)
+    lam = row ? (vec[a] > 0x1p-100f ? sa / vec[a] : INFINITY) : 0.f;
     lam = warp_max(lam);
     __syncthreads();
     if (lane == 0) red[warp] = lam;
@@ -654,7 +658,7 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
     if (lane == 0) {
       // lambda bound: CW value with rounding headroom plus the Gram entry errors
       const float lam_b = s_lam * (1.f + 0x1p-16f) + 0x1p-16f * z2;
-      const float bjoint = sqrtf(wO * lam_b) * (1.f + 0x1p-20f);
+      const float bjoint = sqrtf(wO) * sqrtf(lam_b) * (1.f + 0x1p-20f);
       const float bs = bsum * (1.f + 0x1p-20f);
       float beta = no > 0 ? fminf(bs, bjoint) : 0.f;
       beta += 0x1p-16f * scale + beta_add;

@@ -76,7 +76,7 @@ struct RankRow {
   float lo, hi;       // band of v that survives
   int jlo;            // screened key tiles [jlo, jhi)
   int jhi;
-  int pad;
+  int jplain;         // tiles below it hold no seed key and only visible keys
   long long pos;      // position of the row among the keys
 };
 static_assert(sizeof(RankRow) == 64, "RankRow is four 16-byte vectors");
@@ -293,13 +293,18 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
         R.hi = sel ? p.band_hi[r] : INFINITY;
         R.jlo = sel ? jlo : 0;
         R.jhi = sel ? jhi : 0;
-        R.pad = 0;
+        // seed-free, fully visible tiles: past the first seed keys and ending
+        // before the last seed_last keys (which end at the row's position)
+        const long long last_free = p.pos0 + r - p.seed_last;   // keys <= it are not seeds
+        const int jp = last_free >= kKeyTile - 1 ? (int)((last_free + 1) / kKeyTile) : 0;
+        R.jplain = (p.seed_first <= jlo * kKeyTile || jlo == 0) ? jp : 0;
         R.pos = p.pos0 + r;
         prm[lane] = R;
       }
       __syncwarp();
       const int item = rank_item_of_row(p, row_base);
-      unsigned long long it_scr = 0, it_surv = 0;
+      // this unit's counts (32 bits suffice: at most 64 tiles x 32 keys x 8 rows)
+      uint32_t u_seed = 0, u_scr = 0, u_kept = 0, u_band = 0;
       float mr[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mr[i] = -INFINITY;
@@ -343,27 +348,38 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
             ub -= fmaxf(fmaf(R.sc[0], x[4], R.sc[1] * x[5]), 0.f);
             ub -= fmaxf(fmaf(R.sc[2], x[6], R.sc[3] * x[7]), 0.f);
             const float v = ub * sk;
-            const bool vis = key_ok && s <= R.pos;
-            const bool seed = s < p.seed_first || s > R.pos - p.seed_last;
-            bool surv;
-            if (p.pass == 1) surv = vis && (seed || v >= R.lo);
-            else surv = vis && !seed && v >= R.lo && v < R.hi;
-            const bool rej = vis && !seed && v < R.lo;
-            mr[i] = fmaxf(mr[i], rej ? v : -INFINITY);
-            const uint32_t mask = __ballot_sync(0xFFFFFFFFu, surv);
-            if (lane == i) word = mask;
-            if (p.pass == 1) {
-              const uint32_t sm = __ballot_sync(0xFFFFFFFFu, vis && seed);
-              const uint32_t vm = __ballot_sync(0xFFFFFFFFu, vis);
-              const unsigned ns = __popc(vm & ~sm), nv = __popc(mask & ~sm);
-              n_seed += __popc(sm);
-              n_scr += ns;
-              n_rej += ns - nv;
-              it_scr += ns;
-              it_surv += nv;
+            uint32_t mask;
+            if (j < R.jplain) {
+              // no seed, every key visible: the common case
+              const bool rej = v < R.lo;
+              mr[i] = fmaxf(mr[i], rej ? v : -INFINITY);
+              mask = __ballot_sync(0xFFFFFFFFu, p.pass == 1 ? !rej : (!rej && v < R.hi));
+              if (p.pass == 1) {
+                u_scr += 32;
+                u_kept += __popc(mask);
+              } else {
+                u_band += __popc(mask);
+              }
             } else {
-              n_band += __popc(mask);
+              const bool vis = key_ok && s <= R.pos;
+              const bool seed = s < p.seed_first || s > R.pos - p.seed_last;
+              bool surv;
+              if (p.pass == 1) surv = vis && (seed || v >= R.lo);
+              else surv = vis && !seed && v >= R.lo && v < R.hi;
+              const bool rej = vis && !seed && v < R.lo;
+              mr[i] = fmaxf(mr[i], rej ? v : -INFINITY);
+              mask = __ballot_sync(0xFFFFFFFFu, surv);
+              if (p.pass == 1) {
+                const uint32_t sm = __ballot_sync(0xFFFFFFFFu, vis && seed);
+                const uint32_t vm = __ballot_sync(0xFFFFFFFFu, vis);
+                u_seed += __popc(sm);
+                u_scr += __popc(vm & ~sm);
+                u_kept += __popc(mask & ~sm);
+              } else {
+                u_band += __popc(mask);
+              }
             }
+            if (lane == i) word = mask;
           }
         }
         if (lane < 8 && j >= prm[lane].jlo && j < prm[lane].jhi)
@@ -378,10 +394,14 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
         if (lane == 0 && m > -INFINITY && prm[i].jhi > prm[i].jlo)
           atomicMax(p.maxrej + row_base + i, ordered_key(m));
       }
-      if (lane == 0 && p.item_cnt && it_scr) {
-        atomicAdd(&p.item_cnt[item * 2 + 0], it_scr);
-        atomicAdd(&p.item_cnt[item * 2 + 1], it_surv);
+      if (lane == 0 && p.item_cnt && u_scr) {
+        atomicAdd(&p.item_cnt[item * 2 + 0], (unsigned long long)u_scr);
+        atomicAdd(&p.item_cnt[item * 2 + 1], (unsigned long long)u_kept);
       }
+      n_seed += u_seed;
+      n_scr += u_scr;
+      n_rej += u_scr - u_kept;
+      n_band += u_band;
       __syncwarp();
     }
     if (lane == 0 && !p.item_cnt) {     // a probe's counts go through rank_decide
@@ -406,7 +426,7 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
 // ---- per-row estimates of the threshold ---------------------------------------
 
 // One warp per chunk row of the selected items: the descending estimates U_j
-// (the m_j-th largest warm-up score, m_1 = ceil(2 K n_e / n), m_{j+1} = 8 m_j,
+// (the m_j-th largest warm-up score, m_1 = ceil(1.5 K n_e / n), m_{j+1} = 8 m_j,
 // the last with m = K) from the row's warm-up histogram, the pass-1 band
 // [U_1, inf), and the row's pass bookkeeping.  A histogram lower edge is at or
 // below the score it stands for, so every estimate is at or below the exact
@@ -426,7 +446,7 @@ __global__ void rank_prep_kernel(const RankParams p, const QStateG* qstate, floa
   const int64_t n_e = (n < kKeyTile ? n : kKeyTile) + (n > first ? n - first : 0);
   const QStateG& q = qstate[r];
   const bool have = q.phase == 2;
-  int64_t m = (2 * (int64_t)p.K * n_e + n - 1) / n;
+  int64_t m = (3 * (int64_t)p.K * n_e + 2 * n - 1) / (2 * n);   // ceil(1.5 K n_e / n)
   if (m < 1) m = 1;
   if (m > p.K) m = p.K;
   float prev = INFINITY;

@@ -31,12 +31,15 @@ template <bool kFp8>
 struct RsCfg {
   static constexpr int kSub = kFp8 ? 1 : 2;
   static constexpr int kKSteps = kFp8 ? 4 : 8;
-  static constexpr int kStages = kFp8 ? 6 : 4;             // gathered key tiles
+  static constexpr int kStages = kFp8 ? 4 : 3;             // gathered key tiles
   static constexpr int kInFlight = 2;                      // cp.async groups left pending
   static constexpr int kBufs = 4;                          // TMEM accumulators of 64 columns
   static constexpr int kChunk = 128;                       // keys per MMA tile
   static constexpr int kHeadsN = 64;                       // MMA N: one row's head slots
-  static constexpr int kRing = 2048;                       // survivor keys staged by warp 0
+  static constexpr int kBatchWords = 64;                   // survivor words per scan step
+  static constexpr int kRing = 4096;                       // survivor keys staged by warp 0
+  static_assert(kRing >= kBatchWords * 32 + kChunk, "a scan step must fit in the ring");
+  static constexpr int kCtasPerSm = kFp8 ? 2 : 1;
   static constexpr uint32_t kASubBytes = kChunk * 128;
   static constexpr uint32_t kAStageBytes = kASubBytes * kSub;
   static constexpr uint32_t kBSubBytes = kHeadsN * 128;
@@ -70,6 +73,8 @@ struct RescoreParams {
   int* pass_any;             // this pass has rows
   int* pass_any_next;        // set when a row needs the next pass
   PublishOut out;
+  float* dense;              // dense writeback (ablation): [chunk rows, dense_ld], or null
+  int64_t dense_ld;
   unsigned long long* counters;
   int* err;
   int64_t row0, rows, pos0, S;
@@ -105,7 +110,7 @@ __device__ __forceinline__ int64_t rescore_row_at(const RescoreParams& p, int f)
 }
 
 template <bool kFp8, int kHeads>
-__global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, 1)
+__global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm)
     rescore_kernel(const __grid_constant__ CUtensorMap qmap, const RescoreParams p) {
   using C = RsCfg<kFp8>;
   if (*p.pass_any == 0) return;
@@ -199,15 +204,25 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, 1)
                                    p.n_items - 1 - (int)(r / kItemQueries));
       const int64_t L = g.n_tiles - p.W + 1;                   // screened tiles [1, L)
       const int64_t wlo = 4, whi = L > 1 ? 4 * L : 4;
-      const uint32_t* words = p.bits + r * p.words;
+      // the row's survivor words, two per lane per scan step (64-bit loads;
+      // word counts and limits are multiples of 4), the next step's words
+      // loaded while this step's are expanded
+      const uint2* words = reinterpret_cast<const uint2*>(p.bits + r * p.words);
+      auto load_step = [&](int64_t w0) -> uint2 {
+        const int64_t wi = w0 + 2 * lane;
+        return wi < whi ? __ldcs(words + wi / 2) : make_uint2(0u, 0u);
+      };
       int64_t wpos = wlo;
+      uint2 next = load_step(wpos);
       uint32_t n_avail = 0, rd = 0;
       while (ok) {
         // refill the ring until a full tile of survivors is staged
         while (n_avail - rd < (uint32_t)C::kChunk && wpos < whi) {
-          const int64_t wi = wpos + lane;
-          uint32_t word = wi < whi ? words[wi] : 0u;
-          const uint32_t cnt = __popc(word);
+          const uint2 cur = next;
+          const int64_t wi = wpos + 2 * lane;
+          wpos += C::kBatchWords;
+          if (wpos < whi) next = load_step(wpos);
+          const uint32_t cnt = __popc(cur.x) + __popc(cur.y);
           uint32_t incl = cnt;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -215,14 +230,17 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, 1)
             if (lane >= o) incl += y;
           }
           uint32_t at = n_avail + incl - cnt;
-          const int key0 = (int)(wi * 32);
-          while (word) {
-            ring[at % C::kRing] = key0 + __ffs(word) - 1;
-            ++at;
-            word &= word - 1;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t word = h ? cur.y : cur.x;
+            const int key0 = (int)((wi + h) * 32);
+            while (word) {
+              ring[at % C::kRing] = key0 + __ffs(word) - 1;
+              ++at;
+              word &= word - 1;
+            }
           }
           n_avail += __shfl_sync(0xFFFFFFFFu, incl, 31);
-          wpos += 32;
           __syncwarp();
         }
         const uint32_t left = n_avail - rd;
@@ -388,6 +406,7 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, 1)
         head_accumulate32(acc, x, wq + (kHeads == 64 ? 32 : 0));
         float sc = head_total(acc);
         if constexpr (kFp8) sc *= qs * sk;
+        if (p.dense && valid) p.dense[r * p.dense_ld + key] = sc;
         n_exact += __popc(__ballot_sync(0xFFFFFFFFu, valid));
         const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
         n_cand += append_candidates(q, seg, p.seg_cap, cnt, valid && sc >= tau, sc, key, lane);
@@ -461,7 +480,7 @@ static cudaError_t launch_rescore_impl(const SeqView& v, const RescoreParams& p,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rows8 = p.n_items * kItemQueries;
-  const int grid = rows8 < sms ? rows8 : sms;
+  const int grid = rows8 < C::kCtasPerSm * sms ? rows8 : C::kCtasPerSm * sms;
   profile_before(DOSA_KERNEL_RESCORE, stream);
   if (v.H == 64)
     rescore_kernel<kFp8, 64><<<grid, C::kThreads, C::kSmemBytes, stream>>>(qmap, p);
@@ -500,8 +519,10 @@ cudaError_t launch_rescore(const Handle& h, const SeqView& v, const CertBuffers&
   p.out.repair_count = b.repair_count;
   p.out.repair_cap = b.repair_cap;
   p.out.n_repair = b.counters + kCntOverflow;
-  p.out.dense = 0;
+  p.out.dense = b.dense != nullptr;
   p.out.err = b.err;
+  p.dense = b.dense;
+  p.dense_ld = b.dense_ld;
   p.counters = b.counters;
   p.err = b.err;
   p.row0 = v.row0;

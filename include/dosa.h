@@ -9,8 +9,9 @@
  * index).  Source: "DOSA: Dots Sparse Attention", Daily Paper Cast transcript,
  * Method section (problem formulation: one query with several indexer heads,
  * each with its own query vector and weight, scored against shared keys; the
- * top K keys by score) and Experiments section (the dense baseline is "dense
- * scoring with Top-K selection", K = 2048).  The certified entry point returns
+ * top K keys by score) and Experiments section (the dense baseline scores
+ * every visible key and then selects the Top-K, K = 2048).  The certified
+ * entry point returns
  * the same selection while scoring only the keys a certificate cannot reject
  * (same transcript, Method section: seed threshold, three bound stages,
  * candidate refinement per key tile; "Xiaohongshu DoSA sparse attention cuts
@@ -28,6 +29,17 @@
  *    device-side bounded wait that expires, or a device bounds check that
  *    fires, is reported as DOSA_ERR_TIMEOUT / DOSA_ERR_DEVICE_CHECK by the
  *    call that reads it back (any call given `stats`, or dosa_check_device).
+ *
+ * Bit-identical selections.  Every scorer computes a score with the same
+ * tensor-core dot products and the same fp32 head sum in the same order.  The
+ * dense scorer sums w * ReLU(x) head by head; the other scorers sum
+ * w * (x + |x|), which is exactly twice as much at every step, and halve the
+ * total.  Doubling commutes with fp32 rounding as long as no partial sum is
+ * subnormal (below 2^-126 in magnitude, zero excepted) or overflows, so the
+ * certified, decode and dense selections are identical for weights and keys
+ * of ordinary magnitude; a head sum whose partial sums reach the subnormal
+ * range (for instance weights below about 2^-100) can round differently by
+ * one unit in the last place and flip an exact tie at the K-th score.
  *
  * Layouts
  *  - q:       [Tq, H, d] row-major codes: bf16 (2 bytes) or OCP FP8 E4M3

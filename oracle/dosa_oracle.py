@@ -435,7 +435,7 @@ def certified_topk(q, w, k, positions, K, rows=None, **kw) -> tuple[np.ndarray, 
 
 
 def ranked_topk_row(q_t, w_t, k_vis, K, *, k_bar, warm_tiles, r=4, G=2, seed_first=64,
-                    seed_last=512, margin_log2=-12, tile=128, spread=2.0, growth=8) -> dict:
+                    seed_last=512, margin_log2=-12, tile=128, spread=1.5, growth=8) -> dict:
     """One query through the certified pipeline with a ranked threshold
     schedule.  The pages fix what is computed (seed threshold, certificate,
     rejection, all-head scoring of the survivors; [DPC] Method, candidate

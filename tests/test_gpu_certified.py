@@ -526,3 +526,17 @@ def test_probe_samples_items_first(cuda_lib):
     assert np.array_equal(to_numpy(out2), to_numpy(binding.Index(dtype).dense_topk(*_args(xd2, K2))))
     assert st2["rejected_pairs"] > st2["visible_pairs"] // 2, st2
     assert st2["rescored_pairs"] > 0, st2
+
+
+@pytest.mark.parametrize("scale_log2", [-90, 60])
+def test_certified_equals_dense_at_extreme_weight_magnitudes(cuda_lib, scale_log2):
+    """Weights scaled by a power of two (every score scales exactly with
+    them): the head sums stay in the normal fp32 range, where the doubled head
+    sum of the certified and filter scorers rounds like the dense scorer's, so
+    the selections are identical in every screening mode."""
+    wl, x, xd = _inputs("causal_1k_bf16", 301, 2500, 100)
+    xd["w"] = (xd["w"].double() * 2.0 ** scale_log2).float()
+    dense = to_numpy(binding.Index("bf16").dense_topk(*_args(xd, 100)))
+    for screening in (3, 2, 1, 0):
+        idx = binding.Index("bf16", screening=screening)
+        assert np.array_equal(to_numpy(idx.topk(*_args(xd, 100))), dense), screening
