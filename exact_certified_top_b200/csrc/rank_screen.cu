@@ -65,21 +65,22 @@ struct RankCfg {
   static constexpr int kThreads = 64 + kEpiWarps * 32;
   static constexpr uint32_t kTmemCols = 512;           // two 256-column accumulators
   static constexpr uint32_t kSmemBytes =
-      1024 + kBBytes + kKeyStages * kKeyStageBytes + kEpiWarps * 8 * 64 + 256;
+      1024 + kBBytes + kKeyStages * kKeyStageBytes + kEpiWarps * 8 * 80 + 256;
 };
 
-// One row of a unit, as an epilogue warp reads it (64 bytes).
+// One row of a unit, as an epilogue warp reads it (five 16-byte vectors).
 struct RankRow {
-  float om[4];        // folded retained-head weights x q_scale
-  float sc[4];        // negative-aggregate row scales x q_scale
-  float bm;           // (beta + margin) x q_scale: coefficient of ||k||
-  float lo, hi;       // band of v that survives
+  float4 om;          // folded retained-head weights x q_scale
+  float4 sc;          // negative-aggregate row scales x q_scale
+  float4 blh;         // (beta + margin) x q_scale (coefficient of ||k||), band lo, hi
   int jlo;            // screened key tiles [jlo, jhi)
   int jhi;
   int jplain;         // tiles below it hold no seed key and only visible keys
+  int pad;
   long long pos;      // position of the row among the keys
+  long long pad2;
 };
-static_assert(sizeof(RankRow) == 64, "RankRow is four 16-byte vectors");
+static_assert(sizeof(RankRow) == 80, "RankRow is five 16-byte vectors");
 
 // Units: groups of 32 chunk rows (longest first) x `parts` key-tile ranges.
 struct RankUnit {
@@ -136,7 +137,9 @@ __device__ __forceinline__ RankUnit rank_unit(const RankParams& p, int u) {
   return U;
 }
 
-template <bool kFp8>
+// kFirst: pass 1 (keep v >= lo; count screened and kept pairs), or a later
+// pass (keep lo <= v < hi; count the band's pairs).
+template <bool kFp8, bool kFirst>
 __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
     rank_screen_kernel(const __grid_constant__ CUtensorMap bmap,
                        const __grid_constant__ CUtensorMap kmap, const RankParams p) {
@@ -148,6 +151,7 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
   uint8_t* sB = smem;
   uint8_t* sK = sB + C::kBBytes;
   RankRow* prm_all = reinterpret_cast<RankRow*>(sK + C::kKeyStages * C::kKeyStageBytes);
+  static_assert((RankCfg<kFp8>::kKeyStages * RankCfg<kFp8>::kKeyStageBytes) % 16 == 0, "");
   uint64_t* bars = reinterpret_cast<uint64_t*>(prm_all + C::kEpiWarps * 8);
   uint64_t* b_full = bars + 0;
   uint64_t* b_empty = bars + 1;
@@ -284,24 +288,37 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
         if (sel) rank_tiles_of_row(p, r, jlo, jhi);
         const float* cf = p.cert + (sel ? r : 0) * kCertFloats;
         const float sq = (kFp8 && sel) ? __ldg(p.q_scale + p.row0 + r) : 1.f;
-        for (int j = 0; j < 4; ++j) {
-          R.om[j] = sel ? cf[kCertOmega + j] * sq : 0.f;
-          R.sc[j] = sel ? cf[kCertScale + j] * sq : 0.f;
-        }
-        R.bm = sel ? (cf[kCertBeta] + cf[kCertMargin]) * sq : 0.f;
-        R.lo = sel ? p.band_lo[r] : INFINITY;
-        R.hi = sel ? p.band_hi[r] : INFINITY;
+        auto f = [&](int at) { return sel ? cf[at] * sq : 0.f; };
+        R.om = make_float4(f(kCertOmega), f(kCertOmega + 1), f(kCertOmega + 2), f(kCertOmega + 3));
+        R.sc = make_float4(f(kCertScale), f(kCertScale + 1), f(kCertScale + 2), f(kCertScale + 3));
+        R.blh = make_float4(sel ? (cf[kCertBeta] + cf[kCertMargin]) * sq : 0.f,
+                            sel ? p.band_lo[r] : INFINITY, sel ? p.band_hi[r] : INFINITY, 0.f);
         R.jlo = sel ? jlo : 0;
         R.jhi = sel ? jhi : 0;
         // seed-free, fully visible tiles: past the first seed keys and ending
         // before the last seed_last keys (which end at the row's position)
         const long long last_free = p.pos0 + r - p.seed_last;   // keys <= it are not seeds
         const int jp = last_free >= kKeyTile - 1 ? (int)((last_free + 1) / kKeyTile) : 0;
-        R.jplain = (p.seed_first <= jlo * kKeyTile || jlo == 0) ? jp : 0;
+        R.jplain = p.seed_first <= jlo * kKeyTile ? jp : 0;
+        R.pad = 0;
         R.pos = p.pos0 + r;
+        R.pad2 = 0;
         prm[lane] = R;
       }
       __syncwarp();
+      // rows of this warp that take part, and whether every one of them is
+      // seed-free and fully visible over the whole unit (the fast loop)
+      uint32_t live = 0;
+      bool fast = true;
+      if (lane < 8) {
+        const RankRow& R = prm[lane];
+        const bool in = R.jhi > R.jlo && U.j0 < R.jhi && U.j1 > R.jlo;
+        const bool whole = R.jlo <= U.j0 && U.j1 <= R.jhi && U.j1 <= R.jplain;
+        live = in ? 1u : 0u;
+        fast = !in || whole;
+      }
+      live = __ballot_sync(0xFFFFFFFFu, live != 0) & 0xFFu;
+      fast = __all_sync(0xFFFFFFFFu, fast);
       const int item = rank_item_of_row(p, row_base);
       // this unit's counts (32 bits suffice: at most 64 tiles x 32 keys x 8 rows)
       uint32_t u_seed = 0, u_scr = 0, u_kept = 0, u_band = 0;
@@ -334,42 +351,81 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
+          if (fast && ((live >> (half * 4)) & 0xFu) == 0xFu) {
+            // four seed-free, fully visible rows: four independent chains
+            float v[4], lo[4], hi[4];
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float4* R4 = reinterpret_cast<const float4*>(prm + half * 4 + qq);
+              const float4 om = R4[0], sc = R4[1], blh = R4[2];
+              const float* x = x32 + qq * 8;
+              float ub = om.x * fmaxf(x[0], 0.f);
+              ub = fmaf(om.y, fmaxf(x[1], 0.f), ub);
+              ub = fmaf(om.z, fmaxf(x[2], 0.f), ub);
+              ub = fmaf(om.w, fmaxf(x[3], 0.f), ub);
+              ub = fmaf(blh.x, nk, ub);
+              ub -= fmaxf(fmaf(sc.x, x[4], sc.y * x[5]), 0.f);
+              ub -= fmaxf(fmaf(sc.z, x[6], sc.w * x[7]), 0.f);
+              v[qq] = ub * sk;
+              lo[qq] = blh.y;
+              hi[qq] = blh.z;
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const int i = half * 4 + qq;
+              const bool rej = v[qq] < lo[qq];
+              mr[i] = fmaxf(mr[i], rej ? v[qq] : -INFINITY);
+              const uint32_t mask =
+                  __ballot_sync(0xFFFFFFFFu, kFirst ? !rej : (!rej && v[qq] < hi[qq]));
+              if constexpr (kFirst) {
+                u_scr += 32;
+                u_kept += __popc(mask);
+              } else {
+                u_band += __popc(mask);
+              }
+              if (lane == i) word = mask;
+            }
+            continue;
+          }
 #pragma unroll
           for (int qq = 0; qq < 4; ++qq) {
             const int i = half * 4 + qq;
-            const RankRow& R = prm[i];
-            if (j < R.jlo || j >= R.jhi) continue;          // uniform over the warp
+            if (!(live >> i & 1)) continue;                   // uniform over the warp
+            const float4* R4 = reinterpret_cast<const float4*>(prm + i);
+            const float4 om = R4[0], sc = R4[1], blh = R4[2];
             const float* x = x32 + qq * 8;
-            float ub = R.om[0] * fmaxf(x[0], 0.f);
-            ub = fmaf(R.om[1], fmaxf(x[1], 0.f), ub);
-            ub = fmaf(R.om[2], fmaxf(x[2], 0.f), ub);
-            ub = fmaf(R.om[3], fmaxf(x[3], 0.f), ub);
-            ub = fmaf(R.bm, nk, ub);
-            ub -= fmaxf(fmaf(R.sc[0], x[4], R.sc[1] * x[5]), 0.f);
-            ub -= fmaxf(fmaf(R.sc[2], x[6], R.sc[3] * x[7]), 0.f);
+            float ub = om.x * fmaxf(x[0], 0.f);
+            ub = fmaf(om.y, fmaxf(x[1], 0.f), ub);
+            ub = fmaf(om.z, fmaxf(x[2], 0.f), ub);
+            ub = fmaf(om.w, fmaxf(x[3], 0.f), ub);
+            ub = fmaf(blh.x, nk, ub);
+            ub -= fmaxf(fmaf(sc.x, x[4], sc.y * x[5]), 0.f);
+            ub -= fmaxf(fmaf(sc.z, x[6], sc.w * x[7]), 0.f);
             const float v = ub * sk;
             uint32_t mask;
-            if (j < R.jplain) {
-              // no seed, every key visible: the common case
-              const bool rej = v < R.lo;
+            if (fast || (j >= prm[i].jlo && j < prm[i].jhi && j < prm[i].jplain)) {
+              // no seed, every key visible
+              const bool rej = v < blh.y;
               mr[i] = fmaxf(mr[i], rej ? v : -INFINITY);
-              mask = __ballot_sync(0xFFFFFFFFu, p.pass == 1 ? !rej : (!rej && v < R.hi));
-              if (p.pass == 1) {
+              mask = __ballot_sync(0xFFFFFFFFu, kFirst ? !rej : (!rej && v < blh.z));
+              if constexpr (kFirst) {
                 u_scr += 32;
                 u_kept += __popc(mask);
               } else {
                 u_band += __popc(mask);
               }
             } else {
-              const bool vis = key_ok && s <= R.pos;
-              const bool seed = s < p.seed_first || s > R.pos - p.seed_last;
+              if (j < prm[i].jlo || j >= prm[i].jhi) continue;   // uniform over the warp
+              const long long pos = prm[i].pos;
+              const bool vis = key_ok && s <= pos;
+              const bool seed = s < p.seed_first || s > pos - p.seed_last;
               bool surv;
-              if (p.pass == 1) surv = vis && (seed || v >= R.lo);
-              else surv = vis && !seed && v >= R.lo && v < R.hi;
-              const bool rej = vis && !seed && v < R.lo;
+              if constexpr (kFirst) surv = vis && (seed || v >= blh.y);
+              else surv = vis && !seed && v >= blh.y && v < blh.z;
+              const bool rej = vis && !seed && v < blh.y;
               mr[i] = fmaxf(mr[i], rej ? v : -INFINITY);
               mask = __ballot_sync(0xFFFFFFFFu, surv);
-              if (p.pass == 1) {
+              if constexpr (kFirst) {
                 const uint32_t sm = __ballot_sync(0xFFFFFFFFu, vis && seed);
                 const uint32_t vm = __ballot_sync(0xFFFFFFFFu, vis);
                 u_seed += __popc(sm);
@@ -405,7 +461,7 @@ __global__ void __launch_bounds__(RankCfg<kFp8>::kThreads, 1)
       __syncwarp();
     }
     if (lane == 0 && !p.item_cnt) {     // a probe's counts go through rank_decide
-      if (p.pass == 1) {
+      if (kFirst) {
         atomicAdd(&p.counters[kCntSeedPairs], n_seed);
         atomicAdd(&p.counters[kCntScreened], n_scr);
         atomicAdd(&p.counters[kCntRejected], n_rej);
@@ -541,8 +597,12 @@ static cudaError_t launch_rank_impl(const SeqView& v, const RankParams& p, const
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        rank_screen_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(rank_screen_kernel<kFp8, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(rank_screen_kernel<kFp8, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -552,7 +612,10 @@ static cudaError_t launch_rank_impl(const SeqView& v, const RankParams& p, const
   const int units = p.n_groups * p.parts;
   const int grid = units < sms ? units : sms;
   profile_before(DOSA_KERNEL_RANK, stream);
-  rank_screen_kernel<kFp8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(bmap, kmap, p);
+  if (p.pass == 1)
+    rank_screen_kernel<kFp8, true><<<grid, C::kThreads, C::kSmemBytes, stream>>>(bmap, kmap, p);
+  else
+    rank_screen_kernel<kFp8, false><<<grid, C::kThreads, C::kSmemBytes, stream>>>(bmap, kmap, p);
   const cudaError_t e = cudaGetLastError();
   profile_after(DOSA_KERNEL_RANK, stream);
   return e;

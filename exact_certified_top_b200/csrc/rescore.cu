@@ -36,8 +36,10 @@ struct RsCfg {
   static constexpr int kBufs = 4;                          // TMEM accumulators of 64 columns
   static constexpr int kChunk = 128;                       // keys per MMA tile
   static constexpr int kHeadsN = 64;                       // MMA N: one row's head slots
-  static constexpr int kBatchWords = 64;                   // survivor words per scan step
-  static constexpr int kRing = 4096;                       // survivor keys staged by warp 0
+  static constexpr int kKeySlots = 8;                      // tiles' key lists (epilogue side)
+  static constexpr int kBatchWords = 32;                   // survivor words per scan step
+  static constexpr int kRing = 1280;                       // survivor keys staged by warp 0
+  static constexpr int kBitsWords = 1024;                  // survivor words per bulk copy
   static_assert(kRing >= kBatchWords * 32 + kChunk, "a scan step must fit in the ring");
   static constexpr int kCtasPerSm = kFp8 ? 2 : 1;
   static constexpr uint32_t kASubBytes = kChunk * 128;
@@ -49,8 +51,8 @@ struct RsCfg {
   static constexpr uint32_t kTmemCols = kBufs * kHeadsN;
   static constexpr int kCkptChunks = 8;
   static constexpr uint32_t kSmemBytes = 1024 + 2 * kBBytes + kStages * kAStageBytes +
-                                         kStages * (kChunk * 4 + 16) + kRing * 4 +
-                                         (uint32_t)sizeof(QState) + 512;
+                                         kKeySlots * (kChunk * 8 + 16) + kRing * 4 +
+                                         2 * kBitsWords * 4 + (uint32_t)sizeof(QState) + 512;
 };
 
 struct RescoreParams {
@@ -90,6 +92,9 @@ struct StageMeta {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -119,10 +124,12 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                            // [2] query head tiles
   uint8_t* sA = sQ + 2 * C::kBBytes;                             // [kStages] key tiles
-  int* skeys = reinterpret_cast<int*>(sA + C::kStages * C::kAStageBytes);   // [kStages][128]
-  StageMeta* meta = reinterpret_cast<StageMeta*>(skeys + C::kStages * C::kChunk);
-  int* ring = reinterpret_cast<int*>(meta + C::kStages);
-  QState* st = reinterpret_cast<QState*>(ring + C::kRing);
+  int* skeys = reinterpret_cast<int*>(sA + C::kStages * C::kAStageBytes);   // [kKeySlots][128]
+  float* sscale = reinterpret_cast<float*>(skeys + C::kKeySlots * C::kChunk);  // [kKeySlots][128]
+  StageMeta* meta = reinterpret_cast<StageMeta*>(sscale + C::kKeySlots * C::kChunk);
+  int* ring = reinterpret_cast<int*>(meta + C::kKeySlots);
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(ring + C::kRing);     // [2][kBitsWords]
+  QState* st = reinterpret_cast<QState*>(sbits + 2 * C::kBitsWords);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(st + 1) + 7) & ~uintptr_t(7));
   uint64_t* q_full = bars;                          // [2]
@@ -131,7 +138,10 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
   uint64_t* a_empty = a_full + C::kStages;          // [kStages]
   uint64_t* acc_full = a_empty + C::kStages;        // [kBufs]
   uint64_t* acc_empty = acc_full + C::kBufs;        // [kBufs]
-  uint64_t* done_bar = acc_empty + C::kBufs;
+  uint64_t* ks_full = acc_empty + C::kBufs;         // [kKeySlots] a tile's keys and scales landed
+  uint64_t* ks_empty = ks_full + C::kKeySlots;      // [kKeySlots] ... and read by the epilogue
+  uint64_t* bits_full = ks_empty + C::kKeySlots;    // [2] a piece of survivor words landed
+  uint64_t* done_bar = bits_full + 2;
   uint64_t* ep_bar = done_bar + 1;                  // epilogue meeting point
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ep_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
@@ -145,8 +155,14 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
     }
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 1 + C::kEpiWarps);   // the MMA commit and the epilogue warps
+      mbar_init(&a_empty[i], 1);                  // the MMA's commit
     }
+    for (int i = 0; i < C::kKeySlots; ++i) {
+      mbar_init(&ks_full[i], 1);
+      mbar_init(&ks_empty[i], C::kEpiWarps);
+    }
+    mbar_init(&bits_full[0], 1);
+    mbar_init(&bits_full[1], 1);
     for (int i = 0; i < C::kBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], C::kEpiWarps);
@@ -168,7 +184,8 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
 
   if (warp == 0) {
     // ---------------- compaction + gather ----------------
-    uint32_t ac = 0, done = 0, qc = 0;
+    uint32_t ac = 0, done = 0, qc = 0, bc = 0;   // bc: survivor-word pieces of earlier rows
+    int fetched = 0, waited = 0;                 // pieces of the current row in flight / landed
     bool ok = true;
     const char* kbase = static_cast<const char*>(p.k);
     for (int f = blockIdx.x; f < n_flat && ok; f += gridDim.x) {
@@ -185,7 +202,10 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0)
-          for (; done < ac; ++done) mbar_arrive(&a_full[done % C::kStages]);
+          for (; done < ac; ++done) {
+            mbar_arrive(&a_full[done % C::kStages]);
+            mbar_arrive(&ks_full[done % C::kKeySlots]);
+          }
         done = ac;
       }
       if (lane == 0) {
@@ -204,25 +224,50 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
                                    p.n_items - 1 - (int)(r / kItemQueries));
       const int64_t L = g.n_tiles - p.W + 1;                   // screened tiles [1, L)
       const int64_t wlo = 4, whi = L > 1 ? 4 * L : 4;
-      // the row's survivor words, two per lane per scan step (64-bit loads;
-      // word counts and limits are multiples of 4), the next step's words
-      // loaded while this step's are expanded
-      const uint2* words = reinterpret_cast<const uint2*>(p.bits + r * p.words);
-      auto load_step = [&](int64_t w0) -> uint2 {
-        const int64_t wi = w0 + 2 * lane;
-        return wi < whi ? __ldcs(words + wi / 2) : make_uint2(0u, 0u);
+      // the row's survivor words come into shared memory in pieces of
+      // kBitsWords (bulk copies, double-buffered: the next piece is in flight
+      // while this one is scanned); a scan step takes one word per lane
+      const uint32_t* gwords = p.bits + r * p.words;
+      const int64_t n_words = whi - wlo;
+      const int n_pieces = (int)((n_words + C::kBitsWords - 1) / C::kBitsWords);
+      auto fetch_piece = [&](int piece) {
+        if (lane == 0 && piece < n_pieces) {
+          const int64_t w0 = wlo + (int64_t)piece * C::kBitsWords;
+          const int64_t nw = whi - w0 < C::kBitsWords ? whi - w0 : C::kBitsWords;
+          const uint32_t b = (bc + piece) & 1;
+          fetched = piece + 1;
+          mbar_arrive_expect_tx(&bits_full[b], (uint32_t)nw * 4);
+          bulk_copy_g2s(sbits + b * C::kBitsWords, gwords + w0, (uint32_t)nw * 4, &bits_full[b]);
+        }
       };
+      fetch_piece(0);
+      fetch_piece(1);
+      fetched = n_pieces < 2 ? n_pieces : 2;
+      int piece = 0;                   // piece being scanned
+      int pw = 0;                      // next word of it
+      bool have = false;               // the piece has landed
       int64_t wpos = wlo;
-      uint2 next = load_step(wpos);
       uint32_t n_avail = 0, rd = 0;
       while (ok) {
         // refill the ring until a full tile of survivors is staged
         while (n_avail - rd < (uint32_t)C::kChunk && wpos < whi) {
-          const uint2 cur = next;
-          const int64_t wi = wpos + 2 * lane;
+          const uint32_t b = (bc + piece) & 1;
+          if (!have) {
+            bool w_ok = true;
+            if (lane == 0) w_ok = mbar_wait(&bits_full[b], ((bc + piece) >> 1) & 1, s_abort, p.err);
+            if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) {
+              ok = false;
+              break;
+            }
+            have = true;
+            waited = piece + 1;
+          }
+          const int64_t wi = wpos + lane;
+          uint32_t word = (wi < whi && pw + lane < C::kBitsWords) ? sbits[b * C::kBitsWords + pw + lane]
+                                                                  : 0u;
           wpos += C::kBatchWords;
-          if (wpos < whi) next = load_step(wpos);
-          const uint32_t cnt = __popc(cur.x) + __popc(cur.y);
+          pw += C::kBatchWords;
+          const uint32_t cnt = __popc(word);
           uint32_t incl = cnt;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -230,26 +275,33 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
             if (lane >= o) incl += y;
           }
           uint32_t at = n_avail + incl - cnt;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t word = h ? cur.y : cur.x;
-            const int key0 = (int)((wi + h) * 32);
-            while (word) {
-              ring[at % C::kRing] = key0 + __ffs(word) - 1;
-              ++at;
-              word &= word - 1;
-            }
+          const int key0 = (int)(wi * 32);
+          while (word) {
+            ring[at % C::kRing] = key0 + __ffs(word) - 1;
+            ++at;
+            word &= word - 1;
           }
           n_avail += __shfl_sync(0xFFFFFFFFu, incl, 31);
           __syncwarp();
+          if (pw >= C::kBitsWords) {
+            // piece done (every lane has used its word): its buffer takes the
+            // piece after next
+            fence_proxy_async_smem();
+            __syncwarp();
+            fetch_piece(piece + 2);
+            ++piece;
+            pw = 0;
+            have = false;
+          }
         }
         const uint32_t left = n_avail - rd;
         const int cnt = (int)(left < (uint32_t)C::kChunk ? left : (uint32_t)C::kChunk);
         const int end = (wpos >= whi && left <= (uint32_t)C::kChunk) ? 1 : 0;
-        const int s_ = (int)(ac % C::kStages);
+        const int s_ = (int)(ac % C::kStages), ks = (int)(ac % C::kKeySlots);
         bool w_ok = true;
         if (lane == 0)
-          w_ok = mbar_wait(&a_empty[s_], ((ac / C::kStages) & 1) ^ 1, s_abort, p.err);
+          w_ok = mbar_wait(&a_empty[s_], ((ac / C::kStages) & 1) ^ 1, s_abort, p.err) &&
+                 mbar_wait(&ks_empty[ks], ((ac / C::kKeySlots) & 1) ^ 1, s_abort, p.err);
         if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) {
           ok = false;
           break;
@@ -261,7 +313,10 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
           const int row = lane + 32 * i;
           const bool valid = row < cnt;
           const int key = valid ? ring[(rd + row) % C::kRing] : pad_key;
-          skeys[s_ * C::kChunk + row] = valid ? key : -1;
+          skeys[ks * C::kChunk + row] = valid ? key : -1;
+          // the key's scale travels with its codes (the epilogue would
+          // otherwise wait for it at every tile)
+          if constexpr (kFp8) cp_async4(smem_u32(sscale + ks * C::kChunk + row), p.k_scale + key);
           const char* src = kbase + (int64_t)key * kHeadDim * (kFp8 ? 1 : 2);
           const uint32_t dst = smem_u32(stage + row * 128);
 #pragma unroll
@@ -272,9 +327,10 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
                          src + sub * 128 + c * 16);
         }
         if (lane == 0) {
-          meta[s_].count = cnt;
-          meta[s_].end = end;
+          meta[ks].count = cnt;
+          meta[ks].end = end;
         }
+        __syncwarp();
         cp_async_commit();
         rd += (uint32_t)cnt;
         ++ac;
@@ -284,18 +340,34 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0)
-            for (; done < ac - C::kInFlight; ++done) mbar_arrive(&a_full[done % C::kStages]);
+            for (; done < ac - C::kInFlight; ++done) {
+              mbar_arrive(&a_full[done % C::kStages]);
+              mbar_arrive(&ks_full[done % C::kKeySlots]);
+            }
           done = ac - C::kInFlight;
         }
         if (end) break;
+      }
+      // every piece of the row was fetched and waited for (a row's scan reads
+      // all of its words before its last tile), so the buffers are free
+      if (ok) {
+        bc += (uint32_t)n_pieces;
+        fetched = waited = 0;
       }
     }
     cp_async_wait<0>();
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0)
-      for (; done < ac; ++done) mbar_arrive(&a_full[done % C::kStages]);
+      for (; done < ac; ++done) {
+        mbar_arrive(&a_full[done % C::kStages]);
+        mbar_arrive(&ks_full[done % C::kKeySlots]);
+      }
     if (lane == 0 && *s_abort && qc > 0) mbar_wait_drain(&q_full[(qc - 1) & 1], ((qc - 1) >> 1) & 1);
+    // survivor-word copies still in flight after an abort
+    if (lane == 0 && *s_abort)
+      for (int k = waited; k < fetched; ++k)
+        mbar_wait_drain(&bits_full[(bc + k) & 1], ((bc + k) >> 1) & 1);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -317,7 +389,7 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
             ok = false;
             break;
           }
-          const int end = reinterpret_cast<volatile int*>(&meta[s_].end)[0];
+          const int end = reinterpret_cast<volatile int*>(&meta[ac % C::kKeySlots].end)[0];
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + s_ * C::kAStageBytes);
           const uint32_t d = tmem_base + buf * C::kHeadsN;
@@ -373,19 +445,19 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
       float qs = 1.f;
       if constexpr (kFp8) qs = __ldg(p.q_scale + p.row0 + r);
       for (int nc = 0; ok; ++nc) {
-        const uint32_t s_ = ac % C::kStages, buf = ac % C::kBufs;
-        if (!mbar_wait(&a_full[s_], (ac / C::kStages) & 1, s_abort, p.err) ||
+        const uint32_t ks = ac % C::kKeySlots, buf = ac % C::kBufs;
+        if (!mbar_wait(&ks_full[ks], (ac / C::kKeySlots) & 1, s_abort, p.err) ||
             !mbar_wait(&acc_full[buf], (ac / C::kBufs) & 1, s_abort, p.err)) {
           ok = false;
           break;
         }
-        const int end = reinterpret_cast<volatile int*>(&meta[s_].end)[0];
-        const int tile_cnt = reinterpret_cast<volatile int*>(&meta[s_].count)[0];
+        const int end = reinterpret_cast<volatile int*>(&meta[ks].end)[0];
+        const int tile_cnt = reinterpret_cast<volatile int*>(&meta[ks].count)[0];
         const int at = quad * 32 + lane;
         const bool valid = at < tile_cnt;
-        const int key = valid ? skeys[s_ * C::kChunk + at] : 0;
+        const int key = valid ? skeys[ks * C::kChunk + at] : 0;
         float sk = 1.f;
-        if constexpr (kFp8) sk = valid ? __ldg(p.k_scale + key) : 0.f;
+        if constexpr (kFp8) sk = valid ? sscale[ks * C::kChunk + at] : 0.f;
         tc_fence_after();
         const uint32_t col = tmem_base + lane_off + buf * C::kHeadsN;
         float x[32];
@@ -401,7 +473,7 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&acc_empty[buf]);
-          mbar_arrive(&a_empty[s_]);
+          mbar_arrive(&ks_empty[ks]);
         }
         head_accumulate32(acc, x, wq + (kHeads == 64 ? 32 : 0));
         float sc = head_total(acc);
