@@ -5,16 +5,20 @@
 //
 // A pass of rank_screen leaves, per query row, one survivor bit per screened
 // key.  One CTA takes a row at a time:
-//   warp 0      compaction and gather: reads the row's survivor words 32 at a
-//               time (ballot-free prefix sums over popcounts) into a ring of
-//               key indices, then gathers 128 survivors per tile with 16-byte
-//               cp.async into the 128-byte swizzled layout the MMA reads, a
-//               few tiles in flight; it also TMA-loads the row's 64 head slots
+//   warp 0      compaction: reads the row's survivor words (bulk copies into
+//               shared memory, 64 words per step, prefix sums of the popcounts
+//               from bit-sliced ballots) into a ring of key indices and cuts
+//               it into tiles of 128 keys; it also TMA-loads the row's 64
+//               head slots
 //   warp 1      MMA: M = 128 gathered keys x N = 64 heads, fp32 in TMEM
 //   warps 2-5   epilogue, one TMEM lane quadrant each: the head reduction
 //               shared with every other scorer (bit-identical scores), the
 //               threshold filter and the packed append; the threshold is
-//               refreshed from the histogram every 8 tiles and at the row end.
+//               refreshed from the histogram every 8 tiles and at the row end
+//   warps 6-7   gather, alternate tiles: 16-byte cp.async into the 128-byte
+//               swizzled layout the MMA reads, eight lanes per key row so
+//               that one instruction moves four whole rows; a tile is handed
+//               to the MMA once it has landed
 // At the row end the owner warp checks the pass: if a key the pass rejected
 // has a bound at or above the threshold now reached, the row gets the next
 // band [max(tau, next estimate), this pass's lower limit) and its state is
@@ -31,28 +35,32 @@ template <bool kFp8>
 struct RsCfg {
   static constexpr int kSub = kFp8 ? 1 : 2;
   static constexpr int kKSteps = kFp8 ? 4 : 8;
-  static constexpr int kStages = kFp8 ? 4 : 3;             // gathered key tiles
-  static constexpr int kInFlight = 2;                      // cp.async groups left pending
+  static constexpr int kStages = 4;                        // gathered key tiles
+  static constexpr int kGatherWarps = 2;                   // copy issuers, alternate tiles
   static constexpr int kBufs = 4;                          // TMEM accumulators of 64 columns
   static constexpr int kChunk = 128;                       // keys per MMA tile
   static constexpr int kHeadsN = 64;                       // MMA N: one row's head slots
-  static constexpr int kKeySlots = 8;                      // tiles' key lists (epilogue side)
-  static constexpr int kBatchWords = 32;                   // survivor words per scan step
-  static constexpr int kRing = 1280;                       // survivor keys staged by warp 0
-  static constexpr int kBitsWords = 1024;                  // survivor words per bulk copy
-  static_assert(kRing >= kBatchWords * 32 + kChunk, "a scan step must fit in the ring");
+  static constexpr int kKeySlots = 8;                      // tiles' key lists
+  static constexpr int kScanWords = 64;                    // survivor words per scan step
+  static constexpr int kRing = 4096;                       // survivor keys staged by warp 0
+  static constexpr int kBitsWords = 512;                   // survivor words per bulk copy
+  static_assert(kRing >= kScanWords * 32 + kChunk, "a scan step must fit in the ring");
+  static_assert((kRing & (kRing - 1)) == 0, "ring positions wrap by mask");
+  static_assert(kBitsWords % kScanWords == 0, "a scan step stays inside one piece");
+  static_assert(kKeySlots % kGatherWarps == 0, "a gather warp keeps its key slots");
   static constexpr int kCtasPerSm = kFp8 ? 2 : 1;
   static constexpr uint32_t kASubBytes = kChunk * 128;
   static constexpr uint32_t kAStageBytes = kASubBytes * kSub;
   static constexpr uint32_t kBSubBytes = kHeadsN * 128;
   static constexpr uint32_t kBBytes = kBSubBytes * kSub;
   static constexpr int kEpiWarps = 4;
-  static constexpr int kThreads = 64 + kEpiWarps * 32;
+  static constexpr int kGatherWarp0 = 2 + kEpiWarps;
+  static constexpr int kThreads = 32 * (kGatherWarp0 + kGatherWarps);
   static constexpr uint32_t kTmemCols = kBufs * kHeadsN;
   static constexpr int kCkptChunks = 8;
   static constexpr uint32_t kSmemBytes = 1024 + 2 * kBBytes + kStages * kAStageBytes +
                                          kKeySlots * (kChunk * 8 + 16) + kRing * 4 +
-                                         2 * kBitsWords * 4 + (uint32_t)sizeof(QState) + 512;
+                                         2 * kBitsWords * 4 + 256 + (uint32_t)sizeof(QState) + 1024;
 };
 
 struct RescoreParams {
@@ -84,7 +92,7 @@ struct RescoreParams {
 };
 
 struct StageMeta {
-  int count;    // valid keys in the tile
+  int count;    // valid keys in the tile; -1: no more tiles (gather warps stop)
   int end;      // last tile of its row
   int pad[2];
 };
@@ -114,6 +122,22 @@ __device__ __forceinline__ int64_t rescore_row_at(const RescoreParams& p, int f)
   return r;
 }
 
+// Warp-wide exclusive prefix sum and total of per-lane counts below 128, from
+// one ballot per bit of the count (independent ballots instead of a chain of
+// dependent shuffles).
+__device__ __forceinline__ uint32_t warp_excl_sum7(uint32_t cnt, int lane, uint32_t& total) {
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t excl = 0, tot = 0;
+#pragma unroll
+  for (int b = 0; b < 7; ++b) {
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, (cnt >> b) & 1u);
+    excl += (uint32_t)__popc(m & lt) << b;
+    tot += (uint32_t)__popc(m) << b;
+  }
+  total = tot;
+  return excl;
+}
+
 template <bool kFp8, int kHeads>
 __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm)
     rescore_kernel(const __grid_constant__ CUtensorMap qmap, const RescoreParams p) {
@@ -129,17 +153,19 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
   StageMeta* meta = reinterpret_cast<StageMeta*>(sscale + C::kKeySlots * C::kChunk);
   int* ring = reinterpret_cast<int*>(meta + C::kKeySlots);
   uint32_t* sbits = reinterpret_cast<uint32_t*>(ring + C::kRing);     // [2][kBitsWords]
-  QState* st = reinterpret_cast<QState*>(sbits + 2 * C::kBitsWords);
+  float* sw = reinterpret_cast<float*>(sbits + 2 * C::kBitsWords);   // [64] the row's weights
+  QState* st = reinterpret_cast<QState*>(sw + 64);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(st + 1) + 7) & ~uintptr_t(7));
   uint64_t* q_full = bars;                          // [2]
   uint64_t* q_empty = bars + 2;                     // [2]
-  uint64_t* a_full = bars + 4;                      // [kStages]
-  uint64_t* a_empty = a_full + C::kStages;          // [kStages]
+  uint64_t* a_full = bars + 4;                      // [kStages] a tile's codes landed
+  uint64_t* a_empty = a_full + C::kStages;          // [kStages] ... and were read by the MMA
   uint64_t* acc_full = a_empty + C::kStages;        // [kBufs]
   uint64_t* acc_empty = acc_full + C::kBufs;        // [kBufs]
-  uint64_t* ks_full = acc_empty + C::kBufs;         // [kKeySlots] a tile's keys and scales landed
-  uint64_t* ks_empty = ks_full + C::kKeySlots;      // [kKeySlots] ... and read by the epilogue
+  uint64_t* k_full = acc_empty + C::kBufs;          // [kKeySlots] a tile's key list is cut
+  uint64_t* sc_full = k_full + C::kKeySlots;        // [kKeySlots] ... its scales landed
+  uint64_t* ks_empty = sc_full + C::kKeySlots;      // [kKeySlots] ... read by the epilogue
   uint64_t* bits_full = ks_empty + C::kKeySlots;    // [2] a piece of survivor words landed
   uint64_t* done_bar = bits_full + 2;
   uint64_t* ep_bar = done_bar + 1;                  // epilogue meeting point
@@ -158,7 +184,8 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
       mbar_init(&a_empty[i], 1);                  // the MMA's commit
     }
     for (int i = 0; i < C::kKeySlots; ++i) {
-      mbar_init(&ks_full[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&sc_full[i], 1);
       mbar_init(&ks_empty[i], C::kEpiWarps);
     }
     mbar_init(&bits_full[0], 1);
@@ -183,33 +210,17 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
   const uint32_t tmem_base = *s_tmem;
 
   if (warp == 0) {
-    // ---------------- compaction + gather ----------------
-    uint32_t ac = 0, done = 0, qc = 0, bc = 0;   // bc: survivor-word pieces of earlier rows
+    // ---------------- compaction: survivor words -> key tiles ----------------
+    uint32_t ac = 0, qc = 0, bc = 0;             // bc: survivor-word pieces of earlier rows
     int fetched = 0, waited = 0;                 // pieces of the current row in flight / landed
     bool ok = true;
-    const char* kbase = static_cast<const char*>(p.k);
     for (int f = blockIdx.x; f < n_flat && ok; f += gridDim.x) {
       const int64_t r = rescore_row_at(p, f);
       if (r < 0) continue;
       // the head tile buffer is free once the MMA finished the row before the
-      // last one; if that row's last tiles are still held back here, hand them
-      // over first (the MMA cannot finish the row without them)
-      const uint32_t qfree = (((qc >> 1) & 1) ^ 1);
-      bool ready = true;
-      if (lane == 0) ready = mbar_try_wait(smem_u32(&q_empty[qc & 1]), qfree);
-      if (!__shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) && done < ac) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0)
-          for (; done < ac; ++done) {
-            mbar_arrive(&a_full[done % C::kStages]);
-            mbar_arrive(&ks_full[done % C::kKeySlots]);
-          }
-        done = ac;
-      }
+      // last one (the gather warps hand every tile over without waiting here)
       if (lane == 0) {
-        if (!mbar_wait(&q_empty[qc & 1], qfree, s_abort, p.err)) ok = false;
+        if (!mbar_wait(&q_empty[qc & 1], ((qc >> 1) & 1) ^ 1, s_abort, p.err)) ok = false;
         if (ok) {
           mbar_arrive_expect_tx(&q_full[qc & 1], C::kBBytes);
           for (int sub = 0; sub < C::kSub; ++sub)
@@ -226,7 +237,7 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
       const int64_t wlo = 4, whi = L > 1 ? 4 * L : 4;
       // the row's survivor words come into shared memory in pieces of
       // kBitsWords (bulk copies, double-buffered: the next piece is in flight
-      // while this one is scanned); a scan step takes one word per lane
+      // while this one is scanned)
       const uint32_t* gwords = p.bits + r * p.words;
       const int64_t n_words = whi - wlo;
       const int n_pieces = (int)((n_words + C::kBitsWords - 1) / C::kBitsWords);
@@ -235,7 +246,6 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
           const int64_t w0 = wlo + (int64_t)piece * C::kBitsWords;
           const int64_t nw = whi - w0 < C::kBitsWords ? whi - w0 : C::kBitsWords;
           const uint32_t b = (bc + piece) & 1;
-          fetched = piece + 1;
           mbar_arrive_expect_tx(&bits_full[b], (uint32_t)nw * 4);
           bulk_copy_g2s(sbits + b * C::kBitsWords, gwords + w0, (uint32_t)nw * 4, &bits_full[b]);
         }
@@ -249,7 +259,9 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
       int64_t wpos = wlo;
       uint32_t n_avail = 0, rd = 0;
       while (ok) {
-        // refill the ring until a full tile of survivors is staged
+        // refill the ring until a full tile of survivors is staged; a step
+        // takes two words per lane (keys in any order: the selection orders
+        // candidates by score and index)
         while (n_avail - rd < (uint32_t)C::kChunk && wpos < whi) {
           const uint32_t b = (bc + piece) & 1;
           if (!have) {
@@ -261,91 +273,68 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
             }
             have = true;
             waited = piece + 1;
+            __syncwarp();
           }
-          const int64_t wi = wpos + lane;
-          uint32_t word = (wi < whi && pw + lane < C::kBitsWords) ? sbits[b * C::kBitsWords + pw + lane]
-                                                                  : 0u;
-          wpos += C::kBatchWords;
-          pw += C::kBatchWords;
-          const uint32_t cnt = __popc(word);
-          uint32_t incl = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          uint32_t at = n_avail + incl - cnt;
-          const int key0 = (int)(wi * 32);
-          while (word) {
-            ring[at % C::kRing] = key0 + __ffs(word) - 1;
+          const int64_t wi0 = wpos + lane, wi1 = wpos + 32 + lane;
+          const uint32_t* sb = sbits + b * C::kBitsWords + pw;
+          uint32_t w0 = wi0 < whi ? sb[lane] : 0u;
+          uint32_t w1 = wi1 < whi ? sb[32 + lane] : 0u;
+          wpos += C::kScanWords;
+          pw += C::kScanWords;
+          uint32_t total;
+          const uint32_t excl = warp_excl_sum7((uint32_t)(__popc(w0) + __popc(w1)), lane, total);
+          uint32_t at = n_avail + excl;
+          const int key0 = (int)(wi0 * 32), key1 = (int)(wi1 * 32);
+          while (w0) {
+            ring[at & (C::kRing - 1)] = key0 + __ffs(w0) - 1;
             ++at;
-            word &= word - 1;
+            w0 &= w0 - 1;
           }
-          n_avail += __shfl_sync(0xFFFFFFFFu, incl, 31);
-          __syncwarp();
+          while (w1) {
+            ring[at & (C::kRing - 1)] = key1 + __ffs(w1) - 1;
+            ++at;
+            w1 &= w1 - 1;
+          }
+          n_avail += total;
           if (pw >= C::kBitsWords) {
-            // piece done (every lane has used its word): its buffer takes the
-            // piece after next
+            // piece done (every lane has used its words): its buffer takes
+            // the piece after next
             fence_proxy_async_smem();
             __syncwarp();
             fetch_piece(piece + 2);
+            if (piece + 2 < n_pieces) fetched = piece + 3;
             ++piece;
             pw = 0;
             have = false;
           }
         }
+        if (!ok) break;
+        __syncwarp();
         const uint32_t left = n_avail - rd;
         const int cnt = (int)(left < (uint32_t)C::kChunk ? left : (uint32_t)C::kChunk);
         const int end = (wpos >= whi && left <= (uint32_t)C::kChunk) ? 1 : 0;
-        const int s_ = (int)(ac % C::kStages), ks = (int)(ac % C::kKeySlots);
+        const int ks = (int)(ac % C::kKeySlots);
         bool w_ok = true;
         if (lane == 0)
-          w_ok = mbar_wait(&a_empty[s_], ((ac / C::kStages) & 1) ^ 1, s_abort, p.err) &&
-                 mbar_wait(&ks_empty[ks], ((ac / C::kKeySlots) & 1) ^ 1, s_abort, p.err);
+          w_ok = mbar_wait(&ks_empty[ks], ((ac / C::kKeySlots) & 1) ^ 1, s_abort, p.err);
         if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) {
           ok = false;
           break;
         }
-        uint8_t* stage = sA + s_ * C::kAStageBytes;
-        const int pad_key = cnt > 0 ? ring[rd % C::kRing] : 0;
 #pragma unroll
         for (int i = 0; i < C::kChunk / 32; ++i) {
           const int row = lane + 32 * i;
-          const bool valid = row < cnt;
-          const int key = valid ? ring[(rd + row) % C::kRing] : pad_key;
-          skeys[ks * C::kChunk + row] = valid ? key : -1;
-          // the key's scale travels with its codes (the epilogue would
-          // otherwise wait for it at every tile)
-          if constexpr (kFp8) cp_async4(smem_u32(sscale + ks * C::kChunk + row), p.k_scale + key);
-          const char* src = kbase + (int64_t)key * kHeadDim * (kFp8 ? 1 : 2);
-          const uint32_t dst = smem_u32(stage + row * 128);
-#pragma unroll
-          for (int sub = 0; sub < C::kSub; ++sub)
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              cp_async16(dst + sub * C::kASubBytes + ((c ^ (row & 7)) << 4),
-                         src + sub * 128 + c * 16);
+          skeys[ks * C::kChunk + row] = row < cnt ? ring[(rd + row) & (C::kRing - 1)] : -1;
         }
         if (lane == 0) {
           meta[ks].count = cnt;
           meta[ks].end = end;
         }
+        __threadfence_block();
         __syncwarp();
-        cp_async_commit();
+        if (lane == 0) mbar_arrive(&k_full[ks]);
         rd += (uint32_t)cnt;
         ++ac;
-        // tiles older than the newest kInFlight have landed: hand them over
-        if (ac - done > (uint32_t)C::kInFlight) {
-          cp_async_wait<C::kInFlight>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0)
-            for (; done < ac - C::kInFlight; ++done) {
-              mbar_arrive(&a_full[done % C::kStages]);
-              mbar_arrive(&ks_full[done % C::kKeySlots]);
-            }
-          done = ac - C::kInFlight;
-        }
         if (end) break;
       }
       // every piece of the row was fetched and waited for (a row's scan reads
@@ -355,19 +344,99 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
         fetched = waited = 0;
       }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0)
-      for (; done < ac; ++done) {
-        mbar_arrive(&a_full[done % C::kStages]);
-        mbar_arrive(&ks_full[done % C::kKeySlots]);
+    // one stop mark per gather warp, in the key slots they would read next
+    for (int g = 0; g < C::kGatherWarps && ok; ++g, ++ac) {
+      const int ks = (int)(ac % C::kKeySlots);
+      bool w_ok = true;
+      if (lane == 0) {
+        w_ok = mbar_wait(&ks_empty[ks], ((ac / C::kKeySlots) & 1) ^ 1, s_abort, p.err);
+        if (w_ok) {
+          meta[ks].count = -1;
+          meta[ks].end = 1;
+          __threadfence_block();
+          mbar_arrive(&k_full[ks]);
+        }
       }
+      ok = __shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0) != 0;
+    }
     if (lane == 0 && *s_abort && qc > 0) mbar_wait_drain(&q_full[(qc - 1) & 1], ((qc - 1) >> 1) & 1);
     // survivor-word copies still in flight after an abort
     if (lane == 0 && *s_abort)
       for (int k = waited; k < fetched; ++k)
         mbar_wait_drain(&bits_full[(bc + k) & 1], ((bc + k) >> 1) & 1);
+  } else if (warp >= C::kGatherWarp0) {
+    // ---------------- gather: key codes into the swizzled tiles ----------------
+    const int g = warp - C::kGatherWarp0;
+    const int piece = lane & 7;        // 16-byte piece of a 128-byte row
+    const int r4 = lane >> 3;          // row within each group of four
+    // swizzled offsets of this lane's piece in rows r4 + 8m and r4 + 4 + 8m
+    const uint32_t off0 = (uint32_t)(r4 * 128 + ((piece ^ r4) << 4));
+    const uint32_t off1 = (uint32_t)((r4 + 4) * 128 + ((piece ^ (r4 + 4)) << 4));
+    const char* kbase = static_cast<const char*>(p.k);
+    constexpr int kRowBytes = kHeadDim * (kFp8 ? 1 : 2);
+    bool held = false;                 // a tile issued and not yet handed over
+    uint32_t held_c = 0;
+    auto hand_over = [&]() {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&a_full[held_c % C::kStages]);
+        mbar_arrive(&sc_full[held_c % C::kKeySlots]);
+      }
+      held = false;
+    };
+    for (uint32_t c = (uint32_t)g;; c += C::kGatherWarps) {
+      const int ks = (int)(c % C::kKeySlots), s_ = (int)(c % C::kStages);
+      // never block with a tile held back: the MMA (and through it the
+      // compaction warp) may be waiting for it
+      bool ready = true;
+      if (lane == 0) ready = mbar_try_wait(smem_u32(&k_full[ks]), (c / C::kKeySlots) & 1);
+      if (!__shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) && held) {
+        cp_async_wait<0>();
+        hand_over();
+      }
+      bool w_ok = true;
+      if (lane == 0) w_ok = mbar_wait(&k_full[ks], (c / C::kKeySlots) & 1, s_abort, p.err);
+      if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) break;
+      __syncwarp();                    // lane 0's acquire covers the whole warp
+      const int count = reinterpret_cast<volatile int*>(&meta[ks].count)[0];
+      if (count < 0) break;
+      if (lane == 0) w_ok = mbar_wait(&a_empty[s_], ((c / C::kStages) & 1) ^ 1, s_abort, p.err);
+      if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) break;
+      const uint32_t stage = smem_u32(sA + s_ * C::kAStageBytes);
+      const int* keys = skeys + ks * C::kChunk;
+#pragma unroll 4
+      for (int i = 0; i < C::kChunk / 4; ++i) {
+        const int row = r4 + 4 * i;
+        if (row < count) {
+          const char* src = kbase + (int64_t)keys[row] * kRowBytes + piece * 16;
+          const uint32_t dst = stage + (uint32_t)(i >> 1) * 1024u + ((i & 1) ? off1 : off0);
+#pragma unroll
+          for (int sub = 0; sub < C::kSub; ++sub)
+            cp_async16(dst + sub * C::kASubBytes, src + sub * 128);
+        }
+      }
+      if constexpr (kFp8) {
+#pragma unroll
+        for (int i = 0; i < C::kChunk / 32; ++i) {
+          const int row = lane + 32 * i;
+          if (row < count)
+            cp_async4(smem_u32(sscale + ks * C::kChunk + row), p.k_scale + keys[row]);
+        }
+      }
+      cp_async_commit();
+      // the previous tile of this warp has landed once only the newest group
+      // is pending
+      if (held) {
+        cp_async_wait<1>();
+        hand_over();
+      }
+      held = true;
+      held_c = c;
+    }
+    cp_async_wait<0>();
+    if (held && !*s_abort) hand_over();
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -437,16 +506,22 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
           q.pos = p.pos0 + r;
         }
         state_load(q, p.qstate + r, lane);
+        // the row's head weights, read by every key of every tile
+        const float* wq = p.w + (p.row0 + r) * kHeads;
+        for (int h = lane; h < kHeads; h += 32) sw[h] = __ldg(wq + h);
       }
       meet();
       int cnt = *reinterpret_cast<volatile int*>(&q.seg[quad]);
+      // a row whose threshold comes from the histogram alone (past warm-up)
+      // refreshes it without meeting: counts only grow, so any snapshot of
+      // the histogram gives a sound threshold
+      const bool settled = *reinterpret_cast<volatile int*>(&q.phase) == 2;
       Cand* seg = p.cand + (r * kSegs + quad) * (int64_t)p.seg_cap;
-      const float* wq = p.w + (p.row0 + r) * kHeads;
       float qs = 1.f;
       if constexpr (kFp8) qs = __ldg(p.q_scale + p.row0 + r);
       for (int nc = 0; ok; ++nc) {
         const uint32_t ks = ac % C::kKeySlots, buf = ac % C::kBufs;
-        if (!mbar_wait(&ks_full[ks], (ac / C::kKeySlots) & 1, s_abort, p.err) ||
+        if (!mbar_wait(&sc_full[ks], (ac / C::kKeySlots) & 1, s_abort, p.err) ||
             !mbar_wait(&acc_full[buf], (ac / C::kBufs) & 1, s_abort, p.err)) {
           ok = false;
           break;
@@ -460,35 +535,37 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
         if constexpr (kFp8) sk = valid ? sscale[ks * C::kChunk + at] : 0.f;
         tc_fence_after();
         const uint32_t col = tmem_base + lane_off + buf * C::kHeadsN;
-        float x[32];
-        HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        tmem_ld32_async(col, x);
-        tmem_wait_ld(x);
-        if constexpr (kHeads == 64) {
-          head_accumulate32(acc, x, wq);
-          tmem_ld32_async(col + 32, x);
-          tmem_wait_ld(x);
-        }
+        float x0[32], x1[32];
+        tmem_ld32_async(col, x0);
+        if constexpr (kHeads == 64) tmem_ld32_async(col + 32, x1);
+        const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
+        tmem_wait_ld(x0);
+        if constexpr (kHeads == 64) tmem_wait_ld(x1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&acc_empty[buf]);
           mbar_arrive(&ks_empty[ks]);
         }
-        head_accumulate32(acc, x, wq + (kHeads == 64 ? 32 : 0));
+        HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        head_accumulate32_smem(acc, x0, sw);
+        if constexpr (kHeads == 64) head_accumulate32_smem(acc, x1, sw + 32);
         float sc = head_total(acc);
         if constexpr (kFp8) sc *= qs * sk;
         if (p.dense && valid) p.dense[r * p.dense_ld + key] = sc;
         n_exact += __popc(__ballot_sync(0xFFFFFFFFu, valid));
-        const float tau = *reinterpret_cast<const volatile float*>(&q.tau);
         n_cand += append_candidates(q, seg, p.seg_cap, cnt, valid && sc >= tau, sc, key, lane);
         ++ac;
-        if ((nc + 1) % C::kCkptChunks == 0 || end) {
+        if (end || (!settled && (nc + 1) % C::kCkptChunks == 0)) {
           if (lane == 0) q.seg[quad] = cnt;
           meet();
           if (ew == 0 && ok)
             refresh_threshold(q, p.cand + r * kSegs * (int64_t)p.seg_cap, p.seg_cap, p.K, lane);
           meet();
+        } else if (settled && ew == 0 && (nc + 1) % C::kCkptChunks == 0) {
+          const float tn = hist_threshold(q, p.K, lane);
+          if (lane == 0 && tn > q.tau) *reinterpret_cast<volatile float*>(&q.tau) = tn;
+          __syncwarp();
         }
         if (end) break;
       }

@@ -69,6 +69,23 @@ __device__ __forceinline__ void head_accumulate32(HeadAcc2& a, const float* x,
   }
 }
 
+// The same packed reduction with the weights in shared memory (broadcast
+// reads; identical FMA sequence).
+__device__ __forceinline__ void head_accumulate32_smem(HeadAcc2& a, const float* x,
+                                                       const float* w) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 ww = w4[i];
+    const float2 y01 = __fadd2_rn(make_float2(x[4 * i + 0], x[4 * i + 1]),
+                                  make_float2(fabsf(x[4 * i + 0]), fabsf(x[4 * i + 1])));
+    const float2 y23 = __fadd2_rn(make_float2(x[4 * i + 2], x[4 * i + 3]),
+                                  make_float2(fabsf(x[4 * i + 2]), fabsf(x[4 * i + 3])));
+    a.c01 = __ffma2_rn(make_float2(ww.x, ww.y), y01, a.c01);
+    a.c23 = __ffma2_rn(make_float2(ww.z, ww.w), y23, a.c23);
+  }
+}
+
 // The packed reduction over 16 heads with their weights already in
 // registers (same FMA sequence, chain by chain, as head_accumulate32 above).
 __device__ __forceinline__ void load_w16(float4 (&w4)[4], const float* __restrict__ w) {
