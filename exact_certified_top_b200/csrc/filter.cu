@@ -617,7 +617,8 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
       // qa, then 2 keys of qb, from buffer `team`.
       const int qa = 2 * team + qsel, qb = qa + 4;
       const bool va = qa < g.nq, vb = qb < g.nq;
-      const int pos_a = (int)(g.pos_first + qa), pos_b = (int)(g.pos_first + qb);
+      const int pos_a = va ? (int)(g.pos_first + qa) : -1;
+      const int pos_b = vb ? (int)(g.pos_first + qb) : -1;
       const float* wa = p.w + (g.t0 + (va ? qa : g.nq - 1)) * kHeads;
       const float* wb = p.w + (g.t0 + (vb ? qb : g.nq - 1)) * kHeads;
       constexpr bool h64 = kHeads == 64;
@@ -641,39 +642,44 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
           sk0 = s0 < p.S ? __ldg(p.k_scale + s0) : 0.f;
           sk1 = s1 < p.S ? __ldg(p.k_scale + s1) : 0.f;
         }
+        // the body specialised on whether the second key tile exists (every
+        // pair but an odd item's last tile): no per-quarter branch on it
+        auto uses = [&](auto two_c) {
+          constexpr bool two = decltype(two_c)::value;
 #pragma unroll
-        for (int use = 0; use < 2; ++use) {
-          if (!ok) continue;
-          if (!mbar_wait(&acc_full[team], uu & 1, s_abort, p.err)) {
-            ok = false;
-            continue;
-          }
-          ++uu;
-          tc_fence_after();
-          const float* wq = use ? wb : wa;
-          HeadAcc2 acc0 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-          HeadAcc2 acc1 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-          float x[16];
-          float4 w4[4];
-          constexpr int kQuarters = h64 ? 4 : 2;
+          for (int use = 0; use < 2; ++use) {
+            if (!ok) continue;
+            if (!mbar_wait(&acc_full[team], uu & 1, s_abort, p.err)) {
+              ok = false;
+              continue;
+            }
+            ++uu;
+            tc_fence_after();
+            const float* wq = use ? wb : wa;
+            HeadAcc2 acc0 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            HeadAcc2 acc1 = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            float x[16];
+            float4 w4[4];
+            constexpr int kQuarters = h64 ? 4 : 2;
 #pragma unroll
-          for (int hh = 0; hh < kQuarters; ++hh) {
-            load_w16(w4, wq + 16 * hh);
-            tmem_ld16_async(col0 + 16 * hh, x);
-            tmem_wait_ld16(x);
-            head_accumulate16w(acc0, x, w4);
-            if (two) {
-              tmem_ld16_async(col0 + C::kGroupRows + 16 * hh, x);
+            for (int hh = 0; hh < kQuarters; ++hh) {
+              load_w16(w4, wq + 16 * hh);
+              tmem_ld16_async(col0 + 16 * hh, x);
               tmem_wait_ld16(x);
+              head_accumulate16w(acc0, x, w4);
+              if constexpr (two) {
+                tmem_ld16_async(col0 + C::kGroupRows + 16 * hh, x);
+                tmem_wait_ld16(x);
+              }
+              if (hh == kQuarters - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[team]);
+              }
+              if constexpr (two) head_accumulate16w(acc1, x, w4);
             }
-            if (hh == kQuarters - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[team]);
-            }
-            if (two) head_accumulate16w(acc1, x, w4);
-          }
-          if (use ? vb : va) {
+            // an invalid query slot (past the item's last row) never appends:
+            // its position is -1
             QState& q = st[use ? qb : qa];
             const float qs = use ? qsb : qsa;
             const int pos = use ? pos_b : pos_a;
@@ -687,18 +693,22 @@ __global__ void __launch_bounds__(FilterCfg<kFp8>::kThreads, 1)
             float tau = *reinterpret_cast<const volatile float*>(&q.tau);
             n_cand += append_candidates(q, lst, p.seg_cap, cnt, s0 <= pos && sc0 >= tau, sc0, s0,
                                         lane);
-            if (two) {
+            if constexpr (two) {
               tau = *reinterpret_cast<const volatile float*>(&q.tau);
               n_cand += append_candidates(q, lst, p.seg_cap, cnt, s1 <= pos && sc1 >= tau, sc1,
                                           s1, lane);
             }
             if constexpr (kDense) {
-              float* drow = p.dense + (g.local0 + (use ? qb : qa)) * p.dense_ld;
-              if (s0 <= pos) drow[s0] = sc0;
-              if (two && s1 <= pos) drow[s1] = sc1;
+              if (use ? vb : va) {
+                float* drow = p.dense + (g.local0 + (use ? qb : qa)) * p.dense_ld;
+                if (s0 <= pos) drow[s0] = sc0;
+                if (two && s1 <= pos) drow[s1] = sc1;
+              }
             }
           }
-        }
+        };
+        if (two) uses(std::true_type{});
+        else uses(std::false_type{});
         if (!ok) break;
         // ---- checkpoint: every kCkptTiles steps and at the item's last ----
         if (((i + 2) % kCkptTiles) == 0 || i + 2 >= n) {
