@@ -41,10 +41,10 @@ struct RsCfg {
   static constexpr int kChunk = 128;                       // keys per MMA tile
   static constexpr int kHeadsN = 64;                       // MMA N: one row's head slots
   static constexpr int kKeySlots = 8;                      // tiles' key lists
-  static constexpr int kScanWords = 64;                    // survivor words per scan step
+  static constexpr int kScanWords = 64;                    // survivor words per scan half-step
   static constexpr int kRing = 4096;                       // survivor keys staged by warp 0
   static constexpr int kBitsWords = 512;                   // survivor words per bulk copy
-  static_assert(kRing >= kScanWords * 32 + kChunk, "a scan step must fit in the ring");
+  static_assert(kRing >= kScanWords * 32 + kChunk, "a half-step must fit in the ring");
   static_assert((kRing & (kRing - 1)) == 0, "ring positions wrap by mask");
   static_assert(kBitsWords % kScanWords == 0, "a scan step stays inside one piece");
   static_assert(kKeySlots % kGatherWarps == 0, "a gather warp keeps its key slots");
@@ -275,27 +275,47 @@ __global__ void __launch_bounds__(RsCfg<kFp8>::kThreads, RsCfg<kFp8>::kCtasPerSm
             waited = piece + 1;
             __syncwarp();
           }
-          const int64_t wi0 = wpos + lane, wi1 = wpos + 32 + lane;
+          // two independent halves of 64 words (A, then B when the piece has
+          // room for it), two adjacent words per lane in each: their prefix
+          // sums and expansions interleave, so one step's dependency chain
+          // covers 128 words.  B waits for the next step when both halves
+          // together could overrun the ring (only at survivor densities
+          // near one).
           const uint32_t* sb = sbits + b * C::kBitsWords + pw;
-          uint32_t w0 = wi0 < whi ? sb[lane] : 0u;
-          uint32_t w1 = wi1 < whi ? sb[32 + lane] : 0u;
-          wpos += C::kScanWords;
-          pw += C::kScanWords;
-          uint32_t total;
-          const uint32_t excl = warp_excl_sum7((uint32_t)(__popc(w0) + __popc(w1)), lane, total);
-          uint32_t at = n_avail + excl;
-          const int key0 = (int)(wi0 * 32), key1 = (int)(wi1 * 32);
-          while (w0) {
-            ring[at & (C::kRing - 1)] = key0 + __ffs(w0) - 1;
-            ++at;
-            w0 &= w0 - 1;
+          const int64_t wa = wpos + 2 * lane, wb = wa + C::kScanWords;
+          uint64_t ma = 0, mb = 0;
+          if (wa < whi) {
+            const uint2 v = *reinterpret_cast<const uint2*>(sb + 2 * lane);
+            ma = ((uint64_t)v.y << 32) | v.x;
           }
-          while (w1) {
-            ring[at & (C::kRing - 1)] = key1 + __ffs(w1) - 1;
-            ++at;
-            w1 &= w1 - 1;
+          const bool half_b = pw + 2 * C::kScanWords <= C::kBitsWords;
+          if (half_b && wb < whi) {
+            const uint2 v = *reinterpret_cast<const uint2*>(sb + C::kScanWords + 2 * lane);
+            mb = ((uint64_t)v.y << 32) | v.x;
           }
-          n_avail += total;
+          uint32_t tot_a, tot_b;
+          const uint32_t ex_a = warp_excl_sum7((uint32_t)__popcll(ma), lane, tot_a);
+          const uint32_t ex_b = warp_excl_sum7((uint32_t)__popcll(mb), lane, tot_b);
+          const bool take_b = half_b && (n_avail - rd) + tot_a + tot_b <= (uint32_t)C::kRing;
+          if (!take_b) mb = 0;
+          uint32_t at_a = n_avail + ex_a, at_b = n_avail + tot_a + ex_b;
+          const int kb_a = (int)(wa * 32), kb_b = (int)(wb * 32);
+          while (ma | mb) {
+            if (ma) {
+              ring[at_a & (C::kRing - 1)] = kb_a + __ffsll(ma) - 1;
+              ++at_a;
+              ma &= ma - 1;
+            }
+            if (mb) {
+              ring[at_b & (C::kRing - 1)] = kb_b + __ffsll(mb) - 1;
+              ++at_b;
+              mb &= mb - 1;
+            }
+          }
+          n_avail += tot_a + (take_b ? tot_b : 0u);
+          const int adv = take_b ? 2 * C::kScanWords : C::kScanWords;
+          wpos += adv;
+          pw += adv;
           if (pw >= C::kBitsWords) {
             // piece done (every lane has used its words): its buffer takes
             // the piece after next
