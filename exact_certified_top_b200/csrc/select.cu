@@ -7,8 +7,12 @@
 // time, and the row's final threshold tau is <= its K-th score, so the Top-K
 // are exactly the K best candidates with score >= tau.  Those are gathered
 // into shared memory (when they fit; otherwise the passes read the whole list
-// from global memory), the K-th score is found by 4 radix passes over
-// order-preserving keys, and when more entries tie with it than are needed, a
+// from global memory).  The K-th (score, index) is found in one pass when
+// the list fits: a 2048-bin histogram of the order-preserving keys above tau,
+// a suffix scan for the bin of the K-th key, and a direct rank of that bin's
+// few entries (score descending, index ascending).  Otherwise (the list is in
+// global memory, or the bin holds more than 1024 entries) 4 radix passes
+// find the K-th score, and when more entries tie with it than are needed, a
 // second radix select over the complemented key indices of the tied entries
 // finds the smallest indices (skipped when every tied entry is needed).  The
 // K indices are put in ascending order through a bitmap over the row's keys
@@ -159,6 +163,97 @@ __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t* sc
   return scratch[warp] + incl - v;
 }
 
+constexpr int kFineBins = 2048;       // one histogram pass over keys above tau
+constexpr int kBoundaryCap = 1024;    // entries of the K-th key's bin ranked directly
+
+// The K-th largest (key, index) pair of the n entries lkey/lidx (key
+// descending, index ascending), as the pair (*kth, *cut): the winners are the
+// entries with key > kth, or key == kth and index <= cut.  Every key is >=
+// lo.  scratch: kFineBins + 2 kBoundaryCap words; red: 32 words.  Returns
+// false (and leaves *kth, *cut alone) when the bin of the K-th key holds more
+// than kBoundaryCap entries; the caller then runs the radix passes.  Called by
+// the whole CTA; n >= K.
+__device__ bool fine_bin_kth(const uint32_t* lkey, const int32_t* lidx, int n, uint32_t K,
+                             uint32_t lo, uint32_t* scratch, uint32_t* red, uint32_t* kth,
+                             uint32_t* cut) {
+  __shared__ uint32_t s_shift, s_bin, s_need, s_cnt, s_kth, s_cut, s_nb;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* h = scratch;                                   // [kFineBins]
+  uint32_t* bk = scratch + kFineBins;                      // [kBoundaryCap] keys
+  uint32_t* bi = bk + kBoundaryCap;                        // [kBoundaryCap] indices
+  if (n < (int)K) return false;
+  // the largest key, then the shift that maps [lo, max] into kFineBins bins
+  uint32_t mx = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) mx = max(mx, lkey[i]);
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  for (int j = threadIdx.x; j < kFineBins; j += blockDim.x) h[j] = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t m2 = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m2 = max(m2, red[w]);
+    const uint32_t range = m2 - lo;
+    uint32_t sh = 0;
+    while ((range >> sh) >= (uint32_t)kFineBins) ++sh;
+    s_shift = sh;
+    s_nb = 0;
+  }
+  __syncthreads();
+  const uint32_t sh = s_shift;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&h[(lkey[i] - lo) >> sh], 1u);
+  __syncthreads();
+  // bins in descending order: thread t holds bins kFineBins-1-4t .. -4t-3
+  uint32_t c[4], local = 0;
+  const int per = kFineBins / kSelThreads;
+#pragma unroll
+  for (int j = 0; j < per; ++j) {
+    c[j] = h[kFineBins - 1 - per * threadIdx.x - j];
+    local += c[j];
+  }
+  const uint32_t above = block_exclusive_sum(local, red);
+  if (above < K && K <= above + local) {
+    uint32_t acc = above;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      if (acc < K && K <= acc + c[j]) {
+        s_bin = kFineBins - 1 - per * threadIdx.x - j;
+        s_need = K - acc;                 // entries of the bin that win
+        s_cnt = c[j];
+      }
+      acc += c[j];
+    }
+  }
+  __syncthreads();
+  const uint32_t bin = s_bin, need = s_need, cnt = s_cnt;
+  if (cnt > (uint32_t)kBoundaryCap) return false;
+  // the bin's entries, then each one's rank among them
+  for (int i = threadIdx.x; i < ((n + 31) & ~31); i += blockDim.x) {
+    const bool in = i < n && ((lkey[i] - lo) >> sh) == bin;
+    const uint32_t slot = agg_slot(&s_nb, in);
+    if (in) {
+      bk[slot] = lkey[i];
+      bi[slot] = (uint32_t)lidx[i];
+    }
+  }
+  __syncthreads();
+  for (uint32_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+    const uint32_t ke = bk[e], ie = bi[e];
+    uint32_t rank = 0;
+    for (uint32_t f = 0; f < cnt; ++f) {
+      const uint32_t kf = bk[f];
+      rank += (kf > ke || (kf == ke && bi[f] < ie)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {
+      s_kth = ke;
+      s_cut = ie;
+    }
+  }
+  __syncthreads();
+  *kth = s_kth;
+  *cut = s_cut;
+  return true;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const CandView* __restrict__ cand, int seg_cap, const int* __restrict__ cand_count,
     const float* __restrict__ tau, int64_t pos0, int K, int32_t* __restrict__ out) {
@@ -260,27 +355,37 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int m = in_smem ? n : cnt;            // the global path scans every candidate
   auto key_at = [&](int i) -> uint32_t { return in_smem ? lkey[i] : ordered_key(entry(i).score); };
   auto idx_at = [&](int i) -> uint32_t { return (uint32_t)(in_smem ? lidx[i] : entry(i).key); };
-  uint32_t take = 0, eq = 0;
-  const uint32_t kth = radix_kth(
-      [&](int i, uint32_t* u) {
-        *u = key_at(i);
-        return true;
-      },
-      m, (uint32_t)K, hist, s_res, &take, &eq);
-  // Among entries equal to the K-th key, keep those with the `take` smallest
-  // indices: the take-th largest complemented index is the cut.  When all of
-  // them are needed there is nothing to cut.
-  uint32_t cut = 0xFFFFFFFFu;
-  if (take < eq) {
-    uint32_t t2, e2;
-    __syncthreads();
-    cut = ~radix_kth(
+  uint32_t kth = 0, cut = 0xFFFFFFFFu;
+  // Fast path (the list is in shared memory): one histogram of the keys above
+  // the threshold in kFineBins bins, the bin that holds the K-th key from a
+  // block suffix scan, and the exact rank (key descending, index ascending)
+  // of the few entries of that bin.  Falls back to the radix passes when that
+  // bin holds more than kBoundaryCap entries (heavy ties).
+  bool done = false;
+  if (in_smem) done = fine_bin_kth(lkey, lidx, n, (uint32_t)K, ordered_key(th), bm, scan, &kth, &cut);
+  __syncthreads();
+  if (!done) {
+    uint32_t take = 0, eq = 0;
+    kth = radix_kth(
         [&](int i, uint32_t* u) {
-          if (key_at(i) != kth) return false;
-          *u = ~idx_at(i);
+          *u = key_at(i);
           return true;
         },
-        m, take, hist, s_res, &t2, &e2);
+        m, (uint32_t)K, hist, s_res, &take, &eq);
+    // Among entries equal to the K-th key, keep those with the `take` smallest
+    // indices: the take-th largest complemented index is the cut.  When all of
+    // them are needed there is nothing to cut.
+    if (take < eq) {
+      uint32_t t2, e2;
+      __syncthreads();
+      cut = ~radix_kth(
+          [&](int i, uint32_t* u) {
+            if (key_at(i) != kth) return false;
+            *u = ~idx_at(i);
+            return true;
+          },
+          m, take, hist, s_res, &t2, &e2);
+    }
   }
   auto winner = [&](int i, uint32_t* id) -> bool {
     const uint32_t u = key_at(i);
