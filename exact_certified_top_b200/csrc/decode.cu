@@ -15,9 +15,10 @@
 //                 score is kept too: it spans the row's histogram.
 //   decode_scan   every visible key, split over all SMs by key range: the
 //                 tensor-core scorer of the filter kernel (one MMA tile per 4
-//                 query rows), scores >= tau counted in the row's 256-bin
-//                 histogram over [tau0, max seed score] and appended to the
-//                 row's list two tiles later.  Each CTA counts into shared
+//                 query rows; two epilogue teams drain the two accumulators,
+//                 alternate key tiles), scores >= tau counted in the row's
+//                 256-bin histogram over [tau0, max seed score] and appended
+//                 to the row's list eight tiles later.  Each CTA counts into shared
 //                 memory; a threshold warp per CTA keeps moving those counts
 //                 into the row's global histogram (shared by all CTAs) and
 //                 raises the CTA's threshold to the lower edge of the highest
@@ -261,10 +262,11 @@ struct ScanCfg {
   static constexpr int kUnitThreads = (kEpiWarps + 1) * 32;   // named barrier: epilogue + threshold
   static constexpr uint32_t kTmemCols = 512;           // two accumulators of 256 columns
   static constexpr uint32_t kSmemBytes = 1024 + kQBytes + kKeyStages * kKeyStageBytes + 256;
-  // appends trail the scores by kHold - 1 tiles: long enough for the counts
-  // of a tile to reach the global histogram from every CTA and come back as
-  // a higher threshold (a few passes of the threshold warps)
-  static constexpr int kHold = 9;
+  // appends trail the scores by 2 kHoldT - 2 tiles (kHoldT - 1 of a team's
+  // tiles): long enough for the counts of a tile to reach the global
+  // histogram from every CTA and come back as a higher threshold (a few
+  // passes of the threshold warps)
+  static constexpr int kHoldT = 5;
 };
 
 struct ScanParams {
@@ -383,7 +385,7 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_units = p.n_items * p.parts;
-  __shared__ float s_hold[C::kEpiWarps][C::kHold][32];   // [warp][tile mod kHold][lane]
+  __shared__ float s_hold[C::kEpiWarps][2][C::kHoldT][32];   // [warp][row][team tile mod kHoldT][lane]
   __shared__ unsigned s_hist[kDecRows][kBins];            // this CTA's counts not yet moved
   __shared__ float s_tau[kDecRows];                       // the CTA's view of the shared threshold
   __shared__ unsigned s_done;                             // epilogue warps done, over all units
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], C::kEpiWarps);
+      mbar_init(&acc_empty[i], C::kEpiWarps / 2);   // one team per accumulator
     }
     mbar_init(done_bar, 1);
     for (int i = 0; i < C::kKeyStages; ++i) {
@@ -492,109 +494,144 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
       mbar_wait_drain(done_bar, 0);
     }
   } else if (warp < C::kTauWarp) {
-    // ---------------- epilogue: 16 warps = (TMEM lane quadrant, row of the item) ----------------
+    // ---------------- epilogue: two teams of 8 warps ----------------
+    // Team t drains accumulator t, i.e. the key tiles the CTA takes at even
+    // or odd counts, so the two teams' TMEM loads and arithmetic interleave.
+    // Warp (2 + ew) reads TMEM lane quadrant (warp & 3) for rows 2 rp and
+    // 2 rp + 1 of the item (rp = ew >> 3): two reductions per wait.
     const int ew = warp - 2;
     const int quad = warp & 3;
-    const int sub = ew >> 2;
+    const int team = (ew >> 2) & 1;
+    const int rp = ew >> 3;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     uint32_t kc = 0;
     unsigned long long n_exact = 0, n_cand = 0;
     bool ok = true;
-    float(*hold)[32] = s_hold[ew];
+    float(*hold)[C::kHoldT][32] = s_hold[ew];
     const volatile float* vtau = s_tau;
+    constexpr bool h64 = kHeads == 64;
+    constexpr int D = C::kHoldT - 1;          // team tiles an append trails by
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const Unit x = scan_unit(p, u);
-      if (x.tile_hi <= x.tile_lo) continue;
-      const bool valid = sub < x.nq;
-      const int64_t r = x.local0 + (valid ? sub : 0);
-      const int64_t pos = x.pos_first + sub;
-      const RowBins b = row_bins(p, r);
-      const float* wq = p.w + (x.t0 + (valid ? sub : 0)) * kHeads;
-      constexpr bool h64 = kHeads == 64;
-      float qs = 1.f;
-      if constexpr (kFp8) qs = __ldg(p.q_scale + x.t0 + (valid ? sub : 0));
-      // Appends trail the scores by kHold - 1 tiles: tile j's kept scores wait
-      // in shared memory until tile j + kHold - 1, by which time the
-      // threshold reflects the counts of tile j from every CTA, so the first
-      // tiles are filtered by the K-th largest of everything scored so far
-      // rather than by the seed bound alone.
-      auto append_held = [&](int slot, int key0, float tau) {
-        const float sc = hold[slot][lane];
+      if (x.tile_hi <= x.tile_lo) {
+        continue;
+      }
+      bool valid[2];
+      int64_t rr[2], pos[2];
+      RowBins bins[2];
+      const float* wq[2];
+      float qs[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int sub = 2 * rp + k;
+        valid[k] = sub < x.nq;
+        rr[k] = x.local0 + (valid[k] ? sub : 0);
+        pos[k] = x.pos_first + sub;
+        bins[k] = row_bins(p, rr[k]);
+        wq[k] = p.w + (x.t0 + (valid[k] ? sub : 0)) * kHeads;
+        qs[k] = 1.f;
+        if constexpr (kFp8) qs[k] = __ldg(p.q_scale + x.t0 + (valid[k] ? sub : 0));
+      }
+      // Appends trail the scores by D of this team's tiles (2 D tiles): a
+      // tile's kept scores wait in shared memory until then, by which time
+      // the threshold reflects the counts of that tile from every CTA, so the
+      // first tiles are filtered by the K-th largest of everything scored so
+      // far rather than by the seed bound alone.
+      auto append_held = [&](int k, int slot, int key0, float tau) {
+        const float sc = hold[k][slot][lane];
         const bool app = sc >= tau;
         const unsigned am = __ballot_sync(0xFFFFFFFFu, app);
         if (am) {
           int base = 0;
-          if (lane == 0) base = atomicAdd(&p.count[r], __popc(am));
+          if (lane == 0) base = atomicAdd(&p.count[rr[k]], __popc(am));
           base = __shfl_sync(0xFFFFFFFFu, base, 0);
           const int at = base + __popc(am & ((1u << lane) - 1u));
           if (app && at < p.cap) {
             Cand cd;
             cd.score = sc;
             cd.key = key0 + lane;
-            p.cand[r * p.cap + at] = cd;
+            p.cand[rr[k] * p.cap + at] = cd;
           }
           n_cand += __popc(am);
         }
       };
-      // the key scales come from DRAM: loaded a tile ahead
+      // this team's first tile of the unit (tiles alternate between teams)
+      const int j_first = x.tile_lo + (int)(((uint32_t)team - kc) & 1u);
       float sk_next = 1.f;
       if constexpr (kFp8) {
-        const int s0 = x.tile_lo * kKeyTile + quad * 32 + lane;
-        sk_next = s0 < p.S ? __ldg(p.k_scale + s0) : 0.f;
+        const int s0 = j_first * kKeyTile + quad * 32 + lane;
+        sk_next = (j_first < x.tile_hi && s0 < p.S) ? __ldg(p.k_scale + s0) : 0.f;
       }
-      for (int j = x.tile_lo; j < x.tile_hi && ok; ++j, ++kc) {
+      int m = 0;                                  // this team's tiles of the unit so far
+      int j_last = -1;
+      for (int j = j_first; j < x.tile_hi && ok; j += 2, ++m) {
+        const uint32_t kt = kc + (uint32_t)(j - x.tile_lo);   // the CTA's count of this tile
         const int s = j * kKeyTile + quad * 32 + lane;
-        const int nth = j - x.tile_lo;
         const float sk = sk_next;
         if constexpr (kFp8) {
-          const int sn = s + kKeyTile;
-          sk_next = (j + 1 < x.tile_hi && sn < p.S) ? __ldg(p.k_scale + sn) : 0.f;
+          const int sn = s + 2 * kKeyTile;
+          sk_next = (j + 2 < x.tile_hi && sn < p.S) ? __ldg(p.k_scale + sn) : 0.f;
         }
-        const uint32_t buf = kc & 1;
-        if (!mbar_wait(&acc_full[buf], (kc >> 1) & 1, s_abort, p.err)) {
+        if (!mbar_wait(&acc_full[team], (kt >> 1) & 1, s_abort, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t col = tmem_base + lane_off + buf * C::kQRows + sub * 64;
-        float v[32];
-        HeadAcc2 acc = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        tmem_ld32_async(col, v);
-        tmem_wait_ld(v);
-        if (h64) {
-          head_accumulate32(acc, v, wq);
-          tmem_ld32_async(col + 32, v);
-          tmem_wait_ld(v);
+        const uint32_t col = tmem_base + lane_off + team * C::kQRows + (2 * rp) * 64;
+        HeadAcc2 acc[2] = {{make_float2(0.f, 0.f), make_float2(0.f, 0.f)},
+                           {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}};
+        constexpr int kQuarters = h64 ? 4 : 2;
+#pragma unroll
+        for (int hq = 0; hq < kQuarters; ++hq) {
+          float xa[16], xb[16];
+          float4 w4[4];
+          tmem_ld16_async(col + 16 * hq, xa);
+          tmem_ld16_async(col + 64 + 16 * hq, xb);
+          tmem_wait_ld16(xa);
+          tmem_wait_ld16(xb);
+          if (hq == kQuarters - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[team]);
+          }
+          load_w16(w4, wq[0] + 16 * hq);
+          head_accumulate16w(acc[0], xa, w4);
+          load_w16(w4, wq[1] + 16 * hq);
+          head_accumulate16w(acc[1], xb, w4);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        head_accumulate32(acc, v, wq + (h64 ? 32 : 0));   // H = 32: heads 0-31 only
-        if (!valid) continue;
-        float sc = head_total(acc);
-        if constexpr (kFp8) sc *= qs * sk;
-        const float tau = fmaxf(b.t0, vtau[sub]);
-        const bool vis = s <= pos;
-        n_exact += __popc(__ballot_sync(0xFFFFFFFFu, vis));
-        const bool keep = vis && sc >= tau;
-        if (b.on && __any_sync(0xFFFFFFFFu, keep)) {
-          // count the kept scores in the CTA's histogram, one shared-memory
-          // atomic per distinct bin of the warp
-          const int bin = keep ? bin_index(b.lo, b.inv_w, sc) : -1;
-          const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
-          if (keep && lane == __ffs(peers) - 1) atomicAdd(&s_hist[sub][bin], (unsigned)__popc(peers));
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          if (!valid[k]) continue;
+          float sc = head_total(acc[k]);
+          if constexpr (kFp8) sc *= qs[k] * sk;
+          const int sub = 2 * rp + k;
+          const float tau = fmaxf(bins[k].t0, vtau[sub]);
+          const bool vis = s <= pos[k];
+          n_exact += __popc(__ballot_sync(0xFFFFFFFFu, vis));
+          const bool keep = vis && sc >= tau;
+          if (bins[k].on && __any_sync(0xFFFFFFFFu, keep)) {
+            // count the kept scores in the CTA's histogram, one shared-memory
+            // atomic per distinct bin of the warp
+            const int bin = keep ? bin_index(bins[k].lo, bins[k].inv_w, sc) : -1;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (keep && lane == __ffs(peers) - 1)
+              atomicAdd(&s_hist[sub][bin], (unsigned)__popc(peers));
+          }
+          hold[k][m % C::kHoldT][lane] = keep ? sc : -INFINITY;
+          if (m >= D) append_held(k, (m - D) % C::kHoldT, s - 2 * D * kKeyTile - lane, tau);
         }
-        hold[nth % C::kHold][lane] = keep ? sc : -INFINITY;
-        constexpr int D = C::kHold - 1;
-        if (nth >= D) append_held((nth - D) % C::kHold, s - D * kKeyTile - lane, tau);
+        j_last = j;
       }
-      // the unit's last kHold - 1 tiles
-      if (ok && valid) {
-        const int n = x.tile_hi - x.tile_lo;
-        const float tau = fmaxf(b.t0, vtau[sub]);
-        for (int nth = (n > C::kHold - 1 ? n - (C::kHold - 1) : 0); nth < n; ++nth)
-          append_held(nth % C::kHold, (x.tile_lo + nth) * kKeyTile + quad * 32, tau);
+      // this team's last D tiles of the unit
+      if (ok && m > 0) {
+        for (int k = 0; k < 2; ++k) {
+          if (!valid[k]) continue;
+          const float tau = fmaxf(bins[k].t0, vtau[2 * rp + k]);
+          for (int mm = (m > D ? m - D : 0); mm < m; ++mm)
+            append_held(k, mm % C::kHoldT, (j_last - 2 * (m - 1 - mm)) * kKeyTile + quad * 32, tau);
+        }
       }
+      kc += (uint32_t)(x.tile_hi - x.tile_lo);
       __syncwarp();
       __threadfence_block();
       if (lane == 0) atomicAdd(&s_done, 1u);
