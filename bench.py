@@ -60,6 +60,9 @@ def parse_args():
                     help="certified path: skip key tiles whose key-block bound rules them out")
     ap.add_argument("--probe-sample", type=int, choices=[0, 1], default=1,
                     help="adaptive screening: probe every 7th work item first (1) or every item (0)")
+    ap.add_argument("--short-dense-keys", type=int, default=16384,
+                    help="adaptive screening: calls whose sequences all have at most this many "
+                         "keys take the dense scorer and Top-K (0: never)")
     ap.add_argument("--writeback", choices=["sparse", "dense"], default="sparse",
                     help="certified path: packed candidates >= threshold (default), or every "
                          "exact score into a dense matrix and its dense Top-K (ablation)")
@@ -418,7 +421,7 @@ def ablations_of(args) -> dict:
     """Certified-path switches that differ from their defaults."""
     if args.path != "certified":
         return {}
-    defaults = {"block_bound": 1, "probe_sample": 1}
+    defaults = {"block_bound": 1, "probe_sample": 1, "short_dense_keys": 16384}
     return {k: getattr(args, k) for k, v in defaults.items() if getattr(args, k) != v}
 
 
@@ -480,7 +483,8 @@ def run_ours(args, world, rank, local):
     x = generate(wl if split_rows else rank_workload(wl, rank), device="cuda")
     idx = binding.Index(wl.dtype, H=wl.H, max_K=max(2048, wl.K), screening=args.screening,
                         sparse_writeback=int(args.writeback == "sparse"),
-                        block_bound=args.block_bound, probe_sample=args.probe_sample)
+                        block_bound=args.block_bound, probe_sample=args.probe_sample,
+                        short_dense_keys=args.short_dense_keys)
     certified = args.path == "certified"
     decode = args.path == "decode"
     scorer = args.path == "scorer"

@@ -45,7 +45,7 @@ class Config(ctypes.Structure):
                 ("seed_last", ctypes.c_int), ("r", ctypes.c_int), ("G", ctypes.c_int),
                 ("margin_log2", ctypes.c_int), ("screening", ctypes.c_int),
                 ("sparse_writeback", ctypes.c_int), ("block_bound", ctypes.c_int),
-                ("probe_sample", ctypes.c_int)]
+                ("probe_sample", ctypes.c_int), ("short_dense_keys", ctypes.c_int)]
 
 
 class Stats(ctypes.Structure):

@@ -292,6 +292,7 @@ void dosa_index_config_default(dosa_index_config* cfg) {
   cfg->sparse_writeback = 1;
   cfg->block_bound = 1;
   cfg->probe_sample = 1;
+  cfg->short_dense_keys = 16384;
 }
 
 dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
@@ -303,7 +304,7 @@ dosa_status dosa_index_create(const dosa_index_config* cfg, dosa_index_t* out) {
       cfg->G > 2 || cfg->margin_log2 > -4 || cfg->margin_log2 < -24 || cfg->screening < 0 ||
       cfg->screening > 3 || cfg->sparse_writeback < 0 || cfg->sparse_writeback > 1 ||
       cfg->block_bound < 0 || cfg->block_bound > 1 || cfg->probe_sample < 0 ||
-      cfg->probe_sample > 1)
+      cfg->probe_sample > 1 || cfg->short_dense_keys < 0)
     return DOSA_ERR_INVALID_ARG;
   if (cfg->d != kHeadDim || (cfg->H != 32 && cfg->H != 64)) return DOSA_ERR_UNSUPPORTED;
   Handle* h = new (std::nothrow) Handle;
@@ -693,6 +694,16 @@ dosa_status ensure_copy_stream(Handle* h) {
 
 }  // namespace
 
+// Whether a certified call takes the dense path: the adaptive mode, every
+// sequence within short_dense_keys keys, and room in the workspace for at
+// least one query tile of scores.
+static bool short_dense(const Handle* h, const int64_t* seq_offsets, int B, size_t ws_bytes) {
+  if (h->cfg.screening != 2 || h->cfg.short_dense_keys <= 0) return false;
+  const int64_t S_max = max_keys(seq_offsets, B);
+  if (S_max > h->cfg.short_dense_keys) return false;
+  return ws_bytes >= kWsHeaderBytes + (size_t)kQueryTile * (size_t)(S_max > 0 ? S_max : 1) * 4;
+}
+
 extern "C" {
 
 dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale, const float* w,
@@ -703,6 +714,19 @@ dosa_status dosa_index_topk(dosa_index_t hh, const void* q, const float* q_scale
   dosa_status st = check_common(h, q, q_scale, w, k, k_scale, seq_offsets, B, K, out_idx);
   if (st != DOSA_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (short_dense(h, seq_offsets, B, ws_bytes)) {
+    // short rows: the dense scorer and radix Top-K, the same selection
+    if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, stream) != cudaSuccess) return DOSA_ERR_CUDA;
+    st = dosa_index_dense_topk(hh, q, q_scale, w, k, k_scale, seq_offsets, B, K, out_idx,
+                               workspace, ws_bytes, stream_);
+    if (st != DOSA_OK) return st;
+    if (stats) {
+      st = read_stats(workspace, seq_offsets, B, stream, stats);
+      stats->exact_pairs = stats->visible_pairs;
+      return st;
+    }
+    return DOSA_OK;
+  }
   st = for_each_cert_chunk(
       h, q, q_scale, w, k, k_scale, seq_offsets, B, K, workspace, ws_bytes, stream, nullptr,
       nullptr, [&](const SeqView& c, const CertBuffers& b) -> dosa_status {

@@ -135,6 +135,14 @@ typedef struct {
                        chose screening, and otherwise go to the filter scorer
                        straight after their warm-up.  0: every item is set up
                        and probed (ablation).  Same result either way.        */
+  int short_dense_keys; /* screening = 2 only.  A dosa_index_topk call whose
+                       sequences all have at most this many keys runs the dense
+                       scorer and radix Top-K instead (the same selection:
+                       every pair scored exactly, ties to the smaller index;
+                       on short rows the certified path's set-up, warm-up and
+                       probe launches cost more than they save).  Default
+                       16384; 0: never.  Its stats count every visible pair as
+                       exact and nothing as screened or filtered.               */
 } dosa_index_config;
 
 /* Counters of the last certified call (filled when `stats` is non-NULL). */

@@ -40,7 +40,8 @@ def test_config_default_and_create(lib):
     lib.dosa_index_config_default(ctypes.byref(cfg))
     assert (cfg.H, cfg.d, cfg.max_K, cfg.seed_first, cfg.seed_last, cfg.r, cfg.G,
             cfg.margin_log2, cfg.screening, cfg.sparse_writeback, cfg.block_bound,
-            cfg.probe_sample) == (64, 128, 2048, 64, 512, 4, 2, -12, 2, 1, 1, 1)
+            cfg.probe_sample, cfg.short_dense_keys) == (64, 128, 2048, 64, 512, 4, 2, -12, 2, 1, 1,
+                                                        1, 16384)
     h = ctypes.c_void_p()
     assert lib.dosa_index_create(ctypes.byref(cfg), ctypes.byref(h)) == 0 and h.value
     lib.dosa_index_destroy(h)
@@ -60,7 +61,7 @@ def test_create_accepts_32_heads(lib):
                                               ("r", 5, 1), ("G", 3, 1), ("margin_log2", 0, 1),
                                               ("dtype", 7, 1), ("screening", 4, 1),
                                               ("sparse_writeback", 2, 1), ("block_bound", -1, 1),
-                                              ("probe_sample", 2, 1)])
+                                              ("probe_sample", 2, 1), ("short_dense_keys", -1, 1)])
 def test_create_rejects_bad_config(lib, field, value, code):
     cfg = binding.Config()
     lib.dosa_index_config_default(ctypes.byref(cfg))

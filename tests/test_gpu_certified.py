@@ -33,6 +33,14 @@ def _args(x, K):
     return (x["q"], x["q_scale"], x["w"], x["k"], x["k_scale"], x["seq_offsets"], K)
 
 
+def Index(*a, **kw):
+    """A handle that runs the certified machinery at every size: these tests
+    look inside it on small shapes, which the adaptive mode would otherwise
+    hand to the dense path (short_dense_keys)."""
+    kw.setdefault("short_dense_keys", 0)
+    return binding.Index(*a, **kw)
+
+
 MODES = dict(argvalues=[3, 2, 1, 0], ids=["ranked", "adaptive", "streaming", "off"])
 
 
@@ -41,7 +49,7 @@ MODES = dict(argvalues=[3, 2, 1, 0], ids=["ranked", "adaptive", "streaming", "of
 def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     base, T, S, K = case
     wl, x, xd = _inputs(base, T, S, K)
-    idx = binding.Index(wl.dtype, max_K=2048, screening=screening)
+    idx = Index(wl.dtype, max_K=2048, screening=screening)
     dense = to_numpy(idx.dense_topk(*_args(xd, K)))
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     cert = to_numpy(cert)
@@ -64,7 +72,7 @@ def test_certified_equals_dense_and_oracle(cuda_lib, case, screening):
 
 def test_certified_small_workspace_many_chunks(cuda_lib):
     wl, x, xd = _inputs("causal_1k_bf16", 301, 2500, 100, q_pos0=2199)
-    idx = binding.Index("bf16")
+    idx = Index("bf16")
     ws = torch.zeros(idx.workspace_size(wl.T, wl.S, 100, True, chunk_rows=16), dtype=torch.uint8,
                      device="cuda")
     cert = to_numpy(idx.topk(*_args(xd, 100), workspace=ws))
@@ -87,7 +95,7 @@ def test_certified_varlen_batch(cuda_lib):
         qr += wl.T
         kr += wl.S
     so.append([qr, kr, 0])
-    idx = binding.Index("bf16")
+    idx = Index("bf16")
     cert = to_numpy(idx.topk(q, None, w, k, None, so, 70))
     dense = to_numpy(idx.dense_topk(q, None, w, k, None, so, 70))
     assert np.array_equal(cert, dense)
@@ -117,7 +125,7 @@ def test_varlen_batch_with_empty_sequences(cuda_lib, dtype):
     so.append([qr, kr, 0])
     K = 64
     dev = lambda t: None if t is None else t.cuda()
-    idx = binding.Index(dtype)
+    idx = Index(dtype)
     cert = to_numpy(idx.topk(dev(q), dev(qs), dev(w), dev(k), dev(ks), so, K))
     dense = to_numpy(idx.dense_topk(dev(q), dev(qs), dev(w), dev(k), dev(ks), so, K))
     assert cert.shape == (qr, K)
@@ -164,7 +172,7 @@ def test_certified_prunes_and_stays_exact_when_heads_are_redundant(cuda_lib, fp8
     x, dtype = _redundant_heads_case(fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
-    idx = binding.Index(dtype, screening=screening)
+    idx = Index(dtype, screening=screening)
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     dense = idx.dense_topk(*_args(xd, K))
     assert torch.equal(cert, dense)
@@ -189,7 +197,7 @@ def test_certificate_matches_oracle(cuda_lib):
         x, dtype = _redundant_heads_case(T=24, S=700, seed=3, fp8=fp8)
         # make heads less redundant so the residual bounds are non-trivial
         xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
-        idx = binding.Index(dtype)
+        idx = Index(dtype)
         cert, ret = idx.certificate(xd["q"], xd["q_scale"], xd["w"], xd["k"], xd["k_scale"],
                                     x["seq_offsets"])
         cert, ret = to_numpy(cert), to_numpy(ret)
@@ -229,11 +237,11 @@ def test_certified_mixed_items_hand_over_and_continue(cuda_lib, fp8):
     x["w"][rand_rows] = torch.randn((len(rand_rows), 64), generator=g) / 8
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 128
-    idx = binding.Index(dtype, screening=2, probe_sample=0)
+    idx = Index(dtype, screening=2, probe_sample=0)
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     dense = idx.dense_topk(*_args(xd, K))
     assert torch.equal(cert, dense)
-    sampled, st_s = binding.Index(dtype, screening=2).topk(*_args(xd, K), stats=True)
+    sampled, st_s = Index(dtype, screening=2).topk(*_args(xd, K), stats=True)
     assert torch.equal(sampled, dense)
     assert st_s["exact_pairs"] + st_s["rejected_pairs"] == st_s["visible_pairs"]
     assert stats["exact_pairs"] + stats["rejected_pairs"] == stats["visible_pairs"]
@@ -261,7 +269,7 @@ def test_repair_pass_when_candidates_overflow(cuda_lib, screening, S):
     w = torch.randn((T, 64), generator=g) / 8
     k = torch.randn((1, 128), generator=g).expand(S, 128).contiguous().to(torch.bfloat16)
     so = [[0, 0, S - T], [T, S, 0]]
-    idx = binding.Index("bf16", screening=screening)
+    idx = Index("bf16", screening=screening)
     qd, wd, kd = q.cuda(), w.cuda(), k.cuda()
     cert, stats = idx.topk(qd, None, wd, kd, None, so, K, stats=True)
     cert = to_numpy(cert)
@@ -279,7 +287,7 @@ def test_host_staged_call_equals_device_call(cuda_lib, case):
     chunks, so both slots are reused); same indices as the device call."""
     base, T, S, K = case
     wl, x, xd = _inputs(base, T, S, K)
-    idx = binding.Index(wl.dtype, max_K=2048)
+    idx = Index(wl.dtype, max_K=2048)
     dev = to_numpy(idx.topk(*_args(xd, K)))
     pin = {k: (v.contiguous().pin_memory() if torch.is_tensor(v) and k != "seq_offsets" else v)
            for k, v in x.items()}
@@ -306,8 +314,8 @@ def test_dense_writeback_ablation_equals_dense(cuda_lib, case, screening):
     indices must equal the sparse path's and the dense path's."""
     base, T, S, K = case
     wl, x, xd = _inputs(base, T, S, K)
-    dense = to_numpy(binding.Index(wl.dtype, max_K=2048).dense_topk(*_args(xd, K)))
-    idx = binding.Index(wl.dtype, max_K=2048, screening=screening, sparse_writeback=0)
+    dense = to_numpy(Index(wl.dtype, max_K=2048).dense_topk(*_args(xd, K)))
+    idx = Index(wl.dtype, max_K=2048, screening=screening, sparse_writeback=0)
     out, stats = idx.topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), dense)
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
@@ -358,9 +366,9 @@ def test_key_block_certificate_skips_tiles_and_stays_exact(cuda_lib, fp8, screen
     x, dtype = _clustered_blocks_case(fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
-    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
-    on = binding.Index(dtype, screening=screening, block_bound=1)
-    off = binding.Index(dtype, screening=screening, block_bound=0)
+    dense = to_numpy(Index(dtype).dense_topk(*_args(xd, K)))
+    on = Index(dtype, screening=screening, block_bound=1)
+    off = Index(dtype, screening=screening, block_bound=0)
     a, sa = on.topk(*_args(xd, K), stats=True)
     b, sb = off.topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(a), dense) and np.array_equal(to_numpy(b), dense)
@@ -385,7 +393,7 @@ def test_key_block_bounds_agree_with_oracle(cuda_lib):
     x, dtype = _clustered_blocks_case(T=8, seed=9)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
-    idx = binding.Index(dtype, screening=1, block_bound=1)
+    idx = Index(dtype, screening=1, block_bound=1)
     out, st = idx.topk(*_args(xd, K), stats=True)
     ov = OracleView(x, dtype)
     kb = key_mean(ov.k)
@@ -424,8 +432,8 @@ def test_ranked_screening_rescores_gathered_survivors_exactly(cuda_lib, fp8):
     x, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 32
-    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
-    out, st = binding.Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
+    dense = to_numpy(Index(dtype).dense_topk(*_args(xd, K)))
+    out, st = Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), dense)
     T, S = x["q"].shape[0], x["k"].shape[0]
     visible = sum(S - T + t + 1 for t in range(T))
@@ -479,8 +487,8 @@ def test_ranked_later_passes_recover_an_estimate_set_too_high(cuda_lib, fp8):
     x, dtype = _overshoot_case(fp8)
     xd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     K = 64
-    dense = to_numpy(binding.Index(dtype).dense_topk(*_args(xd, K)))
-    out, st = binding.Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
+    dense = to_numpy(Index(dtype).dense_topk(*_args(xd, K)))
+    out, st = Index(dtype, screening=3).topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), dense)
     assert st["rescreened_pairs"] > 0, st
     assert st["exact_pairs"] + st["rejected_pairs"] == st["visible_pairs"]
@@ -497,11 +505,11 @@ def test_ranked_screening_on_a_loose_bound_keeps_every_key(cuda_lib):
     scorer after its probe."""
     _, x, xd = _inputs("prefill_128k_fp8", 200, 9000, 300)
     K = 300
-    dense = to_numpy(binding.Index("fp8").dense_topk(*_args(xd, K)))
-    out, st = binding.Index("fp8", screening=3).topk(*_args(xd, K), stats=True)
+    dense = to_numpy(Index("fp8").dense_topk(*_args(xd, K)))
+    out, st = Index("fp8", screening=3).topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), dense)
     assert st["rescored_pairs"] > 0.5 * st["visible_pairs"], st
-    out2, st2 = binding.Index("fp8", screening=2, probe_sample=0).topk(*_args(xd, K), stats=True)
+    out2, st2 = Index("fp8", screening=2, probe_sample=0).topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out2), dense)
     assert st2["rescored_pairs"] == 0 and st2["filtered_pairs"] == st2["visible_pairs"], st2
 
@@ -515,15 +523,15 @@ def test_probe_samples_items_first(cuda_lib):
     are rejected.  The selection is the dense path's either way."""
     _, x, xd = _inputs("prefill_128k_fp8", 640, 6000, 300)
     K = 300
-    idx = binding.Index("fp8")
+    idx = Index("fp8")
     out, st = idx.topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(out), to_numpy(idx.dense_topk(*_args(xd, K))))
     assert st["screened_pairs"] == 0 and st["filtered_pairs"] == st["visible_pairs"], st
     x2, dtype = _redundant_heads_case(T=64, S=20000, seed=11, fp8=True)
     xd2 = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x2.items()}
     K2 = 32
-    out2, st2 = binding.Index(dtype).topk(*_args(xd2, K2), stats=True)
-    assert np.array_equal(to_numpy(out2), to_numpy(binding.Index(dtype).dense_topk(*_args(xd2, K2))))
+    out2, st2 = Index(dtype).topk(*_args(xd2, K2), stats=True)
+    assert np.array_equal(to_numpy(out2), to_numpy(Index(dtype).dense_topk(*_args(xd2, K2))))
     assert st2["rejected_pairs"] > st2["visible_pairs"] // 2, st2
     assert st2["rescored_pairs"] > 0, st2
 
@@ -536,7 +544,27 @@ def test_certified_equals_dense_at_extreme_weight_magnitudes(cuda_lib, scale_log
     the selections are identical in every screening mode."""
     wl, x, xd = _inputs("causal_1k_bf16", 301, 2500, 100)
     xd["w"] = (xd["w"].double() * 2.0 ** scale_log2).float()
-    dense = to_numpy(binding.Index("bf16").dense_topk(*_args(xd, 100)))
+    dense = to_numpy(Index("bf16").dense_topk(*_args(xd, 100)))
     for screening in (3, 2, 1, 0):
-        idx = binding.Index("bf16", screening=screening)
+        idx = Index("bf16", screening=screening)
         assert np.array_equal(to_numpy(idx.topk(*_args(xd, 100))), dense), screening
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_short_rows_take_the_dense_path_with_the_same_selection(cuda_lib, dtype):
+    """The adaptive mode hands a call whose sequences all have at most
+    short_dense_keys keys to the dense scorer and radix Top-K: the selection is
+    the certified machinery's, the stats count every pair as exact."""
+    base = "causal_1k_bf16" if dtype == "bf16" else "prefill_128k_fp8"
+    wl, x, xd = _inputs(base, 300, 3000, 256)
+    K = 256
+    short, st = binding.Index(wl.dtype, short_dense_keys=4096).topk(*_args(xd, K), stats=True)
+    full, st_full = Index(wl.dtype).topk(*_args(xd, K), stats=True)
+    dense = binding.Index(wl.dtype).dense_topk(*_args(xd, K))
+    assert torch.equal(short, dense) and torch.equal(full, dense)
+    assert st["visible_pairs"] == st["exact_pairs"] == wl.visible_pairs
+    assert st["screened_pairs"] == st["filtered_pairs"] == st["candidates"] == 0, st
+    assert st_full["filtered_pairs"] > 0, st_full
+    # above the limit the certified machinery runs
+    _, st_long = binding.Index(wl.dtype, short_dense_keys=2999).topk(*_args(xd, K), stats=True)
+    assert st_long["filtered_pairs"] > 0, st_long

@@ -70,6 +70,11 @@ def test_full_size_certified_equals_dense_and_oracle(cuda_lib, name):
     cert, stats = idx.topk(*args, stats=True)
     torch.cuda.synchronize()
     assert torch.equal(cert, dense), "certified selection differs from the dense selection"
+    if wl.S <= idx.cfg.short_dense_keys:
+        # the default call took the dense path: run the certified machinery too
+        machinery = binding.Index(wl.dtype, max_K=max(2048, wl.K), short_dense_keys=0)
+        cert, stats = machinery.topk(*args, stats=True)
+        assert torch.equal(cert, dense), "certified selection differs from the dense selection"
     assert stats["visible_pairs"] == wl.visible_pairs
     assert stats["exact_pairs"] + stats["rejected_pairs"] == wl.visible_pairs
     del x["sinks"]

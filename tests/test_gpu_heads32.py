@@ -56,7 +56,7 @@ def test_h32_scores_match_oracle(cuda_lib, case):
 def test_h32_certified_equals_dense_and_oracle(cuda_lib, case, screening):
     base, T, S, K = case
     wl, x, xd = _inputs(base, T, S, K)
-    idx = binding.Index(wl.dtype, H=32, max_K=2048, screening=screening)
+    idx = binding.Index(wl.dtype, H=32, max_K=2048, screening=screening, short_dense_keys=0)
     dense = to_numpy(idx.dense_topk(*_args(xd, K)))
     cert, stats = idx.topk(*_args(xd, K), stats=True)
     assert np.array_equal(to_numpy(cert), dense)
