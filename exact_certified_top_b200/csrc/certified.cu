@@ -1,11 +1,11 @@
 // Certified indexer scorer for sm_100a: screening, rescoring and sparse
 // writeback fused in one persistent tcgen05 kernel ("DOSA: Dots Sparse
-// Attention", Daily Paper Cast transcript, Method section: candidate
-// refinement = screening dot products, bound evaluation, pruning and score
-// compaction, repeated for every tile of visible keys and query tiles; GPU
-// kernel design: fixed-width query tiles on tensor cores, survivor masks
-// compacted into shared streams so key loads are not repeated, full-score
-// computation fused with threshold filtering and packed writeback).
+// Attention", Daily Paper Cast transcript, Method section: every tile of
+// visible keys goes through the screening products, the bound, the pruning
+// and the compaction of what survives; GPU kernel design: query tiles of a
+// fixed width on the tensor cores, the survivors of a key tile packed so the
+// tile is loaded once, exact scoring fused with the threshold test and the
+// packed writeback).
 //
 // Work item = 8 consecutive query rows (work_items.cuh).  Resident in shared
 // memory: their 8 x 64 head rows and their 8 x 8 bound rows (4 retained heads,

@@ -1,9 +1,9 @@
 // Filter scorer of the certified indexer for sm_100a: exact scores of every
 // visible pair of a work item, filtered against the running threshold and
 // written back packed ("DOSA: Dots Sparse Attention", Daily Paper Cast
-// transcript, Method section: full-score computation fused with threshold
-// filtering and packed writeback; GPU kernel design: fixed-width query tiles on
-// dense tensor-core matrix operations).
+// transcript, Method section: exact scoring fused with the threshold test and
+// the packed writeback; GPU kernel design: query tiles of a fixed width as
+// dense tensor-core products).
 //
 // Tiles: A = 128 keys x d, B = 2 queries x 64 heads (N = 128).  Key tiles
 // are taken two at a time: each of the two 256-column TMEM accumulators holds

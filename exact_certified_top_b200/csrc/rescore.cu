@@ -1,7 +1,8 @@
 // Survivor rescoring of the certified indexer for sm_100a ("DOSA: Dots Sparse
-// Attention", Daily Paper Cast transcript, Method section: survivor masks
-// compacted into per-query refinement streams, every survivor scored with all
-// heads, scores at or above the threshold written back packed).
+// Attention", Daily Paper Cast transcript, Method section, GPU kernel design:
+// the keys that survive screening are packed into a separate stream per
+// query and scored exactly with every head; only scores at or above the
+// threshold are written back, packed).
 //
 // A pass of rank_screen leaves, per query row, one survivor bit per screened
 // key.  One CTA takes a row at a time:

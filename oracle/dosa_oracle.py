@@ -15,8 +15,8 @@ Sources (all web pages on DoSA):
 
 What the method computes.  The pages state that DoSA keeps the original scoring
 function and returns exactly the Top-K the dense indexer returns ([PICX] 02,
-[ZICQ] point 2 "exact token selection", [DPC] Introduction "rejected tokens
-could not have made it into the Top-K").  So the dense oracle below is the plain
+[ZICQ] point 2: the token selection is exact; [DPC] Introduction: a rejected
+key could never have been among the Top-K).  So the dense oracle below is the plain
 definition: decode the stored inputs exactly, score every visible key in fp64,
 sort, take K.  The certificate half follows the steps of [DPC] Method in order
 (seed threshold, three bound stages, tile-by-tile refinement); the pages print
@@ -139,7 +139,7 @@ def select_topk(scores: np.ndarray, K: int) -> np.ndarray:
     """Indices of the K largest scores, ties to the smaller index, returned in
     ascending index order and padded with -1 when fewer than K keys exist.
 
-    The dense baseline is "dense scoring with Top-K selection" ([DPC]
+    The dense baseline scores every key and then takes the Top-K ([DPC]
     Experiments, baselines).  Tie rule: smaller key index wins."""
     n = int(scores.shape[0])
     order = np.lexsort((np.arange(n), -scores))     # -score ascending, then index
@@ -171,9 +171,10 @@ def dense_topk(q: np.ndarray, w: np.ndarray, k: np.ndarray, positions: np.ndarra
 def nnls_retained(Q_R: np.ndarray, v: np.ndarray) -> np.ndarray:
     """alpha = argmin_{alpha >= 0} || v - alpha @ Q_R ||  (Q_R: [r, d], v: [d]).
 
-    "Positive-weight heads are retained, while projections minimize their
-    residual norm" ([DPC] Method) with nonnegative coefficients ("nonnegative
-    head projections", [DPC] Conclusion; [ZICQ] point 2).  Solved exactly for
+    The pages keep some positive-weight heads and project the others onto
+    them so that the projection residual is as small as possible ([DPC]
+    Method), with coefficients that are nonnegative ([DPC] Conclusion;
+    [ZICQ] point 2).  Solved exactly for
     r <= 4 by trying every support: the NNLS optimum is the unconstrained
     least-squares solution on its own support, so the best feasible candidate
     over all supports is the optimum.  For more retained heads (the head-budget
@@ -217,25 +218,25 @@ def certificate_setup(q_t: np.ndarray, w_t: np.ndarray, k_bar: np.ndarray,
                       r: int, G: int) -> Certificate:
     """Build the certificate of one query (real-valued q_t [H, d], w_t [H]).
 
-    Stage 1, positive heads ([DPC] Method, "upper-bounding omitted positive
-    heads"; [ZICQ] 2 "nonnegative head projections and joint residual bounds to
-    limit positive contributions"):
+    Stage 1, positive heads ([DPC] Method: the positive heads left out are
+    bounded from above; [ZICQ] 2: nonnegative projections and one joint bound
+    on the residuals cap what the positive heads can add):
       P = {h : w_h > 0}; R = the r heads of P with the largest w_h ||q_h||
       (ties to the smaller head).  For each omitted h in O = P \\ R,
       alpha_h = NNLS projection onto the retained heads, rho_h its residual.
       ReLU is positively homogeneous and subadditive, and alpha >= 0, so
         ReLU(q_h.k) <= sum_j alpha_hj ReLU(q_j.k) + |rho_h.k|.
-      The retained heads reuse their computed dot products ([DPC] Method:
-      "retained positive heads reuse computed dot products"):
+      The retained heads' dot products are computed once and reused ([DPC]
+      Method):
         omega_j = w_j + sum_{h in O} w_h alpha_hj.
       Joint residual bound: sum_h w_h |rho_h.k| <= beta ||k|| with
         beta = min( sum_h w_h ||rho_h|| ,  sqrt( W_O * lambda_max(M) ) ),
         W_O = sum_{h in O} w_h,  M = sum_{h in O} w_h rho_h rho_h^T
       (the second is Cauchy-Schwarz with weights w_h, then the spectral norm:
       it bounds all residual heads jointly).
-    Stage 2, negative heads ([DPC] Method: "negative heads are aggregated based
-    on support derived from activation patterns"; [ZICQ] 2 "activation-informed
-    aggregation to bound the magnitude subtracted by negative heads"):
+    Stage 2, negative heads ([DPC] Method: the negative heads are summed over
+    supports chosen from which heads are active; [ZICQ] 2: that aggregate
+    bounds how much the negative heads can subtract):
       for a >= 0, sum_{h in A} a_h ReLU(x_h) >= ReLU(sum_{h in A} a_h x_h).
       N = {h : w_h < 0}.  A_1 = {h in N : q_h.k_bar > 0} (heads active on the
       mean key), A_2 = N \\ A_1 when G >= 2.  u_g = sum_{h in A_g} |w_h| q_h.
@@ -283,8 +284,8 @@ def certificate_setup(q_t: np.ndarray, w_t: np.ndarray, k_bar: np.ndarray,
 
 
 def upper_bound(cert: Certificate, q_t: np.ndarray, k: np.ndarray) -> np.ndarray:
-    """Stage 3, the combined bound ([DPC] Method: "a unified score certificate
-    that combines these retained and bounded contributions"):
+    """Stage 3, the combined bound ([DPC] Method: one certificate per key adds
+    the retained heads' exact terms and the bounds of the other heads):
       UB(s) = sum_j omega_j ReLU(q_j.k_s) + beta ||k_s|| - sum_g ReLU(u_g.k_s).
     k: [n, d] real values.  UB(s) >= I(t,s) for every key (tests pin this)."""
     ub = cert.beta * np.linalg.norm(k, axis=1)
@@ -338,9 +339,8 @@ def soundness_margin(q_t: np.ndarray, w_t: np.ndarray, k: np.ndarray,
 
 def seed_mask(p: int, seed_first: int, seed_last: int) -> np.ndarray:
     """Seed subset of the visible keys 0..p: the first ``seed_first`` keys and the
-    last ``seed_last`` keys ending at p ([DPC] Method: "choosing a subset of
-    visible keys ... and setting a threshold based on the K-th largest score
-    within this subset")."""
+    last ``seed_last`` keys ending at p ([DPC] Method: the threshold starts as
+    the K-th largest exact score over a subset of the visible keys)."""
     s = np.arange(p + 1)
     return (s < seed_first) | (s > p - seed_last)
 
@@ -373,8 +373,8 @@ def certified_topk_row(q_t, w_t, k_vis, K, *, k_bar, r=4, G=2, seed_first=64,
       3. Top-K over the exactly scored keys.
 
     k_vis: [p+1, d] real values of the visible keys.  Returns the selection and
-    the counts used for the prune rate ([DPC] Experiments: "percentage of
-    query-key pairs removed during certificate screening")."""
+    the counts used for the prune rate ([DPC] Experiments: the share of
+    query-key pairs that screening removes)."""
     n = k_vis.shape[0]
     p = n - 1
     w64 = w_t.astype(np.float64)
