@@ -10,11 +10,13 @@
 // from global memory).  The K-th (score, index) is found in one pass when
 // the list fits: a 2048-bin histogram of the order-preserving keys above tau,
 // a suffix scan for the bin of the K-th key, and a direct rank of that bin's
-// few entries (score descending, index ascending).  Otherwise (the list is in
-// global memory, or the bin holds more than 1024 entries) 4 radix passes
-// find the K-th score, and when more entries tie with it than are needed, a
-// second radix select over the complemented key indices of the tied entries
-// finds the smallest indices (skipped when every tied entry is needed).  The
+// few entries (score descending, index ascending).  A bin of more than 128
+// entries that all hold one score is a tie at the K-th score: only the index
+// cut among them is left.  Otherwise (the list is in global memory, or a
+// crowded bin holds several scores) 4 radix passes find the K-th score, and
+// when more entries tie with it than are needed, a second radix select over
+// the complemented key indices of the tied entries finds the smallest
+// indices (skipped when every tied entry is needed).  The
 // K indices are put in ascending order through a bitmap over the row's keys
 // (one bit per key, then a block-wide prefix count), or by a bitonic sort for
 // rows longer than the bitmap.  Every step is a parallel pass; nothing is
@@ -164,24 +166,29 @@ __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t* sc
 }
 
 constexpr int kFineBins = 2048;       // one histogram pass over keys above tau
-constexpr int kBoundaryCap = 1024;    // entries of the K-th key's bin ranked directly
+constexpr int kBoundaryCap = 128;     // entries of the K-th key's bin ranked directly
+                                      // (quadratic: larger bins take the tie or radix path)
 
 // The K-th largest (key, index) pair of the n entries lkey/lidx (key
 // descending, index ascending), as the pair (*kth, *cut): the winners are the
 // entries with key > kth, or key == kth and index <= cut.  Every key is >=
 // lo.  scratch: kFineBins + 2 kBoundaryCap words; red: 32 words.  Returns
-// false (and leaves *kth, *cut alone) when the bin of the K-th key holds more
-// than kBoundaryCap entries; the caller then runs the radix passes.  Called by
-// the whole CTA; n >= K.
-__device__ bool fine_bin_kth(const uint32_t* lkey, const int32_t* lidx, int n, uint32_t K,
-                             uint32_t lo, uint32_t* scratch, uint32_t* red, uint32_t* kth,
-                             uint32_t* cut) {
-  __shared__ uint32_t s_shift, s_bin, s_need, s_cnt, s_kth, s_cut, s_nb;
+//   kFineDone   *kth and *cut set;
+//   kFineTies   the bin of the K-th key holds more than kBoundaryCap entries,
+//               all with one key: *kth set, and the winners among them are
+//               the *take with the smallest indices (the caller cuts them);
+//   kFineRadix  neither: the caller runs the radix passes.
+// Called by the whole CTA.
+constexpr int kFineRadix = 0, kFineDone = 1, kFineTies = 2;
+__device__ int fine_bin_kth(const uint32_t* lkey, const int32_t* lidx, int n, uint32_t K,
+                            uint32_t lo, uint32_t* scratch, uint32_t* red, uint32_t* kth,
+                            uint32_t* cut, uint32_t* take) {
+  __shared__ uint32_t s_shift, s_bin, s_need, s_cnt, s_kth, s_cut, s_nb, s_kmin, s_kmax;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t* h = scratch;                                   // [kFineBins]
   uint32_t* bk = scratch + kFineBins;                      // [kBoundaryCap] keys
   uint32_t* bi = bk + kBoundaryCap;                        // [kBoundaryCap] indices
-  if (n < (int)K) return false;
+  if (n < (int)K) return kFineRadix;
   // the largest key, then the shift that maps [lo, max] into kFineBins bins
   uint32_t mx = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) mx = max(mx, lkey[i]);
@@ -225,7 +232,36 @@ __device__ bool fine_bin_kth(const uint32_t* lkey, const int32_t* lidx, int n, u
   }
   __syncthreads();
   const uint32_t bin = s_bin, need = s_need, cnt = s_cnt;
-  if (cnt > (uint32_t)kBoundaryCap) return false;
+  if (cnt > (uint32_t)kBoundaryCap) {
+    // a crowded bin: when it holds a single key (a tie at the K-th score)
+    // only the index cut among the tied entries is left
+    if (threadIdx.x == 0) {
+      s_kmin = 0xFFFFFFFFu;
+      s_kmax = 0u;
+    }
+    __syncthreads();
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t u = lkey[i];
+      if (((u - lo) >> sh) == bin) {
+        kmin = min(kmin, u);
+        kmax = max(kmax, u);
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+    }
+    if (lane == 0) {
+      atomicMin(&s_kmin, kmin);
+      atomicMax(&s_kmax, kmax);
+    }
+    __syncthreads();
+    if (s_kmin != s_kmax) return kFineRadix;
+    *kth = s_kmin;
+    *take = need;
+    return kFineTies;
+  }
   // the bin's entries, then each one's rank among them
   for (int i = threadIdx.x; i < ((n + 31) & ~31); i += blockDim.x) {
     const bool in = i < n && ((lkey[i] - lo) >> sh) == bin;
@@ -251,7 +287,7 @@ __device__ bool fine_bin_kth(const uint32_t* lkey, const int32_t* lidx, int n, u
   __syncthreads();
   *kth = s_kth;
   *cut = s_cut;
-  return true;
+  return kFineDone;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
@@ -361,10 +397,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   // block suffix scan, and the exact rank (key descending, index ascending)
   // of the few entries of that bin.  Falls back to the radix passes when that
   // bin holds more than kBoundaryCap entries (heavy ties).
-  bool done = false;
-  if (in_smem) done = fine_bin_kth(lkey, lidx, n, (uint32_t)K, ordered_key(th), bm, scan, &kth, &cut);
+  uint32_t tie_take = 0;
+  const int fine = in_smem ? fine_bin_kth(lkey, lidx, n, (uint32_t)K, ordered_key(th), bm, scan,
+                                          &kth, &cut, &tie_take)
+                           : kFineRadix;
   __syncthreads();
-  if (!done) {
+  if (fine == kFineTies) {
+    // the K-th key is known; keep the tie_take smallest indices among its
+    // entries (the tie_take-th largest complemented index is the cut)
+    uint32_t t2, e2;
+    cut = ~radix_kth(
+        [&](int i, uint32_t* u) {
+          if (key_at(i) != kth) return false;
+          *u = ~idx_at(i);
+          return true;
+        },
+        m, tie_take, hist, s_res, &t2, &e2);
+  } else if (fine == kFineRadix) {
     uint32_t take = 0, eq = 0;
     kth = radix_kth(
         [&](int i, uint32_t* u) {
