@@ -302,7 +302,9 @@ def roofline(prof: dict, wl, pairs_per_step: int, steps: int, dtype: str, stats=
     achieved = work / (ms * 1e-3) / 1e12
     return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1),
             "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "traffic": _traffic_per_launch(dom, wl, pairs_per_step * steps / launches),
+            "traffic": _traffic_per_launch(
+                dom, wl, pairs_per_step * steps / launches,
+                stats["candidates"] * steps / launches if stats else None),
             "peak_source": peak_src, "launches": launches,
             "avg_launch_ms": round(ms / launches, 3)}
 
@@ -320,10 +322,18 @@ def _traffic_record(kernel: str, wl):
     return rec
 
 
-def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float):
-    """DRAM bytes per launch from a committed ncu summary, scaled by pairs."""
+def _traffic_per_launch(kernel: str, wl, pairs_per_launch: float, cands_per_launch=None):
+    """DRAM bytes per launch from a committed ncu summary: the reads scaled by
+    the launch's visible pairs (queries, keys, scales), the writes by its
+    appended candidates (8-byte packed entries), each from the capture's own
+    ratio; or, for an older record, all bytes scaled by pairs."""
     rec = _traffic_record(kernel, wl)
-    if rec is None or "dram_bytes_per_pair" not in rec:
+    if rec is None:
+        return None
+    if "dram_read_bytes_per_pair" in rec and cands_per_launch is not None:
+        return round(rec["dram_read_bytes_per_pair"] * pairs_per_launch
+                     + rec["dram_write_bytes_per_candidate"] * cands_per_launch)
+    if "dram_bytes_per_pair" not in rec:
         return None
     return round(rec["dram_bytes_per_pair"] * pairs_per_launch)
 
