@@ -215,6 +215,7 @@ struct SetupParams {
   float* cert;            // [rows, kCertFloats]
   int32_t* retained;      // [rows, 4]
   int sample;             // which rows (see launch_cert_setup)
+  int stride;             // every stride-th item is sampled (probe_stride)
   int n_items;
   int* item_flag;
   const int* gate;
@@ -248,15 +249,15 @@ __global__ void __launch_bounds__(kSetupThreads) cert_setup_kernel(const SetupPa
   __shared__ float s_lam;
   int64_t i = blockIdx.x;
   if (p.sample == 1) {
-    // the rows of sampled item kProbeSampleStride * (blockIdx.x / 8); items
-    // run longest rows first, so item j holds the rows of group n_items-1-j
-    const int item = kProbeSampleStride * (int)(blockIdx.x / kItemQueries);
+    // the rows of sampled item stride * (blockIdx.x / 8); items run longest
+    // rows first, so item j holds the rows of group n_items-1-j
+    const int item = p.stride * (int)(blockIdx.x / kItemQueries);
     i = (int64_t)(p.n_items - 1 - item) * kItemQueries + blockIdx.x % kItemQueries;
     if (i >= p.rows) return;
     if (threadIdx.x == 0 && blockIdx.x % kItemQueries == 0) p.item_flag[item] = kItemSample;
   } else if (p.sample == 2) {
     const int item = p.n_items - 1 - (int)(i / kItemQueries);
-    if (item % kProbeSampleStride == 0 || *reinterpret_cast<const volatile int*>(p.gate) == 0)
+    if (item % p.stride == 0 || *reinterpret_cast<const volatile int*>(p.gate) == 0)
       return;
   }
   const int64_t t = p.row0 + i;
@@ -731,11 +732,11 @@ cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* ke
   p.retained = retained;
   p.sample = sample;
   p.n_items = (int)((v.rows + kItemQueries - 1) / kItemQueries);
+  p.stride = probe_stride(p.n_items);
   p.item_flag = item_flag;
   p.gate = gate;
   unsigned grid = (unsigned)v.rows;
-  if (sample == 1)
-    grid = (unsigned)((p.n_items + kProbeSampleStride - 1) / kProbeSampleStride) * kItemQueries;
+  if (sample == 1) grid = (unsigned)((p.n_items + p.stride - 1) / p.stride) * kItemQueries;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(cert_setup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -153,7 +153,7 @@ cudaError_t launch_scores_tc_rows(const Handle& h, const SeqView& v, const int* 
 cudaError_t launch_key_prep(const Handle& h, const void* k, const float* k_scale, int64_t S,
                             float* key_norm, float* key_sum, cudaStream_t stream);
 // sample 0: every row of the chunk; 1: the rows of the sampled work items
-// (every kProbeSampleStride-th), whose item_flag becomes kItemSample; 2: the
+// (every probe_stride(n_items)-th), whose item_flag becomes kItemSample; 2: the
 // other rows, only when *gate is set (a no-op launch otherwise).
 cudaError_t launch_cert_setup(const Handle& h, const SeqView& v, const float* key_sum,
                               void* bdir, float* cert, int32_t* retained, cudaStream_t stream,

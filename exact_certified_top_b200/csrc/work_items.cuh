@@ -54,9 +54,24 @@ enum ItemFlag : int {
   kItemProbe = 5,
   kItemUnprobed = 6
 };
-// Prime, so that the sampled items spread evenly over the persistent CTAs
-// (CTA b takes items b, b + grid, ...) for any grid that is not a multiple of 7.
+// Every kProbeSampleStride-th item is sampled; on a chunk of more items than
+// kProbeSampleStride * kProbeSampleItems the stride grows so that about
+// kProbeSampleItems are (enough for the decision, and the sample's set-up and
+// probe cost stops growing with the chunk).  The stride is prime and not 37,
+// so that the sampled items spread evenly over the persistent CTAs (CTA b
+// takes items b, b + grid, ...) for a grid of 148 or any other grid that is
+// not a multiple of it.
 constexpr int kProbeSampleStride = 7;
+constexpr int kProbeSampleItems = 256;
+
+inline int probe_stride(int n_items) {
+  static const int kPrimes[] = {7, 11, 13, 17, 19, 23, 29, 31, 41, 43, 47, 53, 59, 61,
+                                67, 71, 73, 79, 83, 89, 97, 101, 103, 107, 109, 113};
+  const int want = (n_items + kProbeSampleItems - 1) / kProbeSampleItems;
+  for (int pr : kPrimes)
+    if (pr >= want) return pr;
+  return 127;
+}
 
 struct Range {
   int begin, end;   // empty when end <= begin

@@ -130,7 +130,9 @@ typedef struct {
                        item's queries are skipped without loading their keys;
                        0: off (ablation).                                     */
   int probe_sample;  /* screening = 2 only.  1 (default): every 7th work item
-                       (longest rows first) is set up and probed first; the
+                       (on chunks of more than 1,792 items a larger prime
+                       stride, about 256 items; longest rows first) is set
+                       up and probed first; the
                        other items are set up and probed only if one of those
                        chose screening, and otherwise go to the filter scorer
                        straight after their warm-up.  0: every item is set up
