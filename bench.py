@@ -395,11 +395,16 @@ def oracle_sample(x, wl, budget_s: float):
             "host_cores": os.cpu_count()}
 
 
-def ideal_prune_sample(x, wl, n_rows: int = 4):
+def ideal_prune_sample(x, wl, n_rows: int = 64):
     """The certificate's ideal prune rate (the oracle's: threshold equal to
     the true K-th score, the default certificate r = 4, G = 2) and the
     oracle schedule's own prune rate, on n_rows rows spread over the
-    workload's positions (the longest last)."""
+    workload's positions (the longest first), one row per host core at a
+    time; plus the committed oracle prune study's figure for the workload
+    (tests/golden/prune_study.json, written by tests/prune_study.py) when it
+    has one."""
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from oracle import certified_topk_row, dequantize, key_mean
     from exact_certified_top_b200.workloads import codes_numpy
@@ -407,22 +412,38 @@ def ideal_prune_sample(x, wl, n_rows: int = 4):
     k = dequantize(codes_numpy(x["k"]), kscale, wl.dtype)
     kb = key_mean(k)
     pos = x["positions"].cpu().numpy()
-    rows = sorted({int(r) for r in np.linspace(wl.T - 1, 0, n_rows + 1)[:n_rows]})
-    vis = ideal = rej = 0
+    rows = sorted({int(r) for r in np.linspace(wl.T - 1, 0, n_rows + 1)[:n_rows]}, reverse=True)
+    qc = codes_numpy(x["q"])
+    qsc = None if x["q_scale"] is None else x["q_scale"].cpu().numpy()
+    wv = x["w"].cpu().numpy().astype(np.float64)
     t0 = time.perf_counter()
-    for t in rows:
-        qs = None if x["q_scale"] is None else x["q_scale"][t:t + 1].cpu().numpy()
-        q = dequantize(codes_numpy(x["q"][t:t + 1]), qs, wl.dtype)[0]
-        w = x["w"][t].cpu().numpy().astype(np.float64)
-        p = int(pos[t])
-        res = certified_topk_row(q, w, k[:p + 1], wl.K, k_bar=kb, r=4, G=2, margin_log2=-12)
-        vis += res["visible"]
-        ideal += res["ideal_rejected"]
-        rej += res["rejected"]
-    return {"ideal_prune_pct": round(100.0 * ideal / max(vis, 1), 4),
-            "schedule_prune_pct": round(100.0 * rej / max(vis, 1), 4), "kind": "oracle",
-            "sample": f"rows {rows} of {wl.name} ({vis} visible pairs), "
-                      f"{time.perf_counter() - t0:.1f} s"}
+
+    def one(t):
+        q = dequantize(qc[t:t + 1], None if qsc is None else qsc[t:t + 1], wl.dtype)[0]
+        res = certified_topk_row(q, wv[t], k[:int(pos[t]) + 1], wl.K, k_bar=kb, r=4, G=2,
+                                 margin_log2=-12)
+        return res["visible"], res["ideal_rejected"], res["rejected"]
+
+    with threadpool_limits(1):
+        with ThreadPoolExecutor(max(1, os.cpu_count() or 1)) as ex:
+            out = list(ex.map(one, rows))
+    vis = sum(o[0] for o in out)
+    ideal = sum(o[1] for o in out)
+    rej = sum(o[2] for o in out)
+    res = {"ideal_prune_pct": round(100.0 * ideal / max(vis, 1), 4),
+           "schedule_prune_pct": round(100.0 * rej / max(vis, 1), 4), "kind": "oracle",
+           "sample": f"{len(rows)} rows of {wl.name} spread over its positions ({vis} visible "
+                     f"pairs), {time.perf_counter() - t0:.1f} s"}
+    study = os.path.join(ROOT, "tests", "golden", "prune_study.json")
+    if os.path.exists(study):
+        with open(study) as f:
+            for r in json.load(f)["results"]:
+                if r["workload"] == wl.name:
+                    res["study"] = {"file": "tests/golden/prune_study.json",
+                                    "rows": len(r["rows"]),
+                                    "ideal_prune_pct": r["ideal_prune_pct"],
+                                    "ranked_prune_pct": r.get("ranked_prune_pct")}
+    return res
 
 
 # ---------------------------------------------------------------------------
