@@ -389,6 +389,7 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
   __shared__ unsigned s_hist[kDecRows][kBins];            // this CTA's counts not yet moved
   __shared__ float s_tau[kDecRows];                       // the CTA's view of the shared threshold
   __shared__ unsigned s_done;                             // epilogue warps done, over all units
+  __shared__ float4 s_w[kDecRows][16];                    // the unit's head weights (64 per row)
   for (int i = threadIdx.x; i < kDecRows * kBins; i += blockDim.x) (&s_hist[0][0])[i] = 0u;
   if (threadIdx.x < kDecRows) s_tau[threadIdx.x] = -INFINITY;
   if (threadIdx.x == 0) s_done = 0u;
@@ -555,6 +556,16 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
           n_cand += __popc(am);
         }
       };
+      // the unit's weights into shared memory, once per unit (warps 0 and 8
+      // of the epilogue write their two rows; the previous unit's readers are
+      // past the barrier that ended it)
+      if ((ew & 7) == 0) {
+        float* sw = reinterpret_cast<float*>(s_w[2 * rp]);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          for (int hh = lane; hh < 64; hh += 32) sw[k * 64 + hh] = hh < kHeads ? __ldg(wq[k] + hh) : 0.f;
+      }
+      asm volatile("bar.sync 2, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
       // this team's first tile of the unit (tiles alternate between teams)
       const int j_first = x.tile_lo + (int)(((uint32_t)team - kc) & 1u);
       float sk_next = 1.f;
@@ -594,9 +605,11 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[team]);
           }
-          load_w16(w4, wq[0] + 16 * hq);
+#pragma unroll
+          for (int m4 = 0; m4 < 4; ++m4) w4[m4] = s_w[2 * rp][4 * hq + m4];
           head_accumulate16w(acc[0], xa, w4);
-          load_w16(w4, wq[1] + 16 * hq);
+#pragma unroll
+          for (int m4 = 0; m4 < 4; ++m4) w4[m4] = s_w[2 * rp + 1][4 * hq + m4];
           head_accumulate16w(acc[1], xb, w4);
         }
 #pragma unroll
