@@ -48,3 +48,19 @@ def test_ablation_flags_parse(flag, monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", flag, "0"])
     args = bench.parse_args()
     assert getattr(args, flag.lstrip("-").replace("-", "_")) == 0
+
+
+def test_traffic_scales_reads_by_pairs_and_writes_by_candidates(monkeypatch):
+    """A split traffic record: reads per visible pair, writes per appended
+    candidate, each scaled by the launch's own counts; an older record scales
+    everything by pairs; a record of other sources gives none."""
+    wl = small_case("prefill_128k_fp8", 8, 64)
+    split = {"dram_read_bytes_per_pair": 0.25, "dram_write_bytes_per_candidate": 6.0}
+    monkeypatch.setattr(bench, "_traffic_record", lambda kernel, w: split)
+    assert bench._traffic_per_launch("filter", wl, 1000.0, 100.0) == 250 + 600
+    assert bench._traffic_per_launch("filter", wl, 1000.0) is None      # no candidate count
+    monkeypatch.setattr(bench, "_traffic_record", lambda kernel, w: {"dram_bytes_per_pair": 0.5})
+    assert bench._traffic_per_launch("filter", wl, 1000.0, 100.0) == 500
+    monkeypatch.setattr(bench, "_traffic_record", lambda kernel, w: None)
+    assert bench._traffic_per_launch("filter", wl, 1000.0, 100.0) is None
+
