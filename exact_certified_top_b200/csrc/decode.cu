@@ -538,22 +538,43 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
       // the threshold reflects the counts of that tile from every CTA, so the
       // first tiles are filtered by the K-th largest of everything scored so
       // far rather than by the seed bound alone.
+      // Appends are staged in registers, one pending entry per lane and row
+      // (lanes 0 .. pend - 1), and written 32 at a time: one reservation on
+      // the row's shared count per 32 entries instead of one per append (all
+      // CTAs update the same few counts), and an exact one at the unit's end.
+      float ps[2] = {0.f, 0.f};
+      int pk[2] = {0, 0}, pend[2] = {0, 0};
+      auto flush = [&](int k, int cnt) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&p.count[rr[k]], cnt);
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        if (lane < cnt && base + lane < p.cap) p.cand[rr[k] * p.cap + base + lane] = Cand{ps[k], pk[k]};
+        n_cand += cnt;
+      };
+      // new entries (lanes of am, in lane order) into the pending lanes from
+      // `first`: entry j goes to lane first + j, for j < count
+      auto stage = [&](int k, unsigned am, float sc, int key0, int first, int from, int count) {
+        const int j = lane - first;
+        const bool mine = j >= 0 && j < count;
+        const int src = mine ? (int)__fns(am, 0, from + j + 1) : 0;
+        const float v = __shfl_sync(0xFFFFFFFFu, sc, src);
+        if (mine) {
+          ps[k] = v;
+          pk[k] = key0 + src;
+        }
+      };
       auto append_held = [&](int k, int slot, int key0, float tau) {
         const float sc = hold[k][slot][lane];
-        const bool app = sc >= tau;
-        const unsigned am = __ballot_sync(0xFFFFFFFFu, app);
-        if (am) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&p.count[rr[k]], __popc(am));
-          base = __shfl_sync(0xFFFFFFFFu, base, 0);
-          const int at = base + __popc(am & ((1u << lane) - 1u));
-          if (app && at < p.cap) {
-            Cand cd;
-            cd.score = sc;
-            cd.key = key0 + lane;
-            p.cand[rr[k] * p.cap + at] = cd;
-          }
-          n_cand += __popc(am);
+        const unsigned am = __ballot_sync(0xFFFFFFFFu, sc >= tau);
+        if (!am) return;
+        const int n = __popc(am);
+        const int fill = n < 32 - pend[k] ? n : 32 - pend[k];
+        stage(k, am, sc, key0, pend[k], 0, fill);
+        pend[k] += fill;
+        if (pend[k] == 32) {
+          flush(k, 32);
+          pend[k] = n - fill;
+          if (pend[k] > 0) stage(k, am, sc, key0, 0, fill, pend[k]);
         }
       };
       // the unit's weights into shared memory, once per unit (warps 0 and 8
@@ -635,7 +656,7 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
         }
         j_last = j;
       }
-      // this team's last D tiles of the unit
+      // this team's last D tiles of the unit, then what is still pending
       if (ok && m > 0) {
         for (int k = 0; k < 2; ++k) {
           if (!valid[k]) continue;
@@ -644,6 +665,9 @@ __global__ void __launch_bounds__(ScanCfg<kFp8>::kThreads, 1)
             append_held(k, mm % C::kHoldT, (j_last - 2 * (m - 1 - mm)) * kKeyTile + quad * 32, tau);
         }
       }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (pend[k] > 0) flush(k, pend[k]);
       kc += (uint32_t)(x.tile_hi - x.tile_lo);
       __syncwarp();
       __threadfence_block();
