@@ -13,6 +13,9 @@ possible (at least 4K visible keys), it computes with the fp64 oracle:
     and the joint spectral one) and which is smaller.
 
     python tests/prune_study.py [--rows 64] [--out tests/golden/prune_study.json]
+                                [--workloads A,B] [--merge]
+
+--merge keeps the stored results of the workloads not listed.
 
 Every number comes from oracle/ (the certificate, the bound, the exact scores);
 the seeded generator only draws the inputs.
@@ -35,7 +38,8 @@ from exact_certified_top_b200.workloads import WORKLOADS, codes_numpy, generate 
 from oracle import (certificate_setup, dequantize, indexer_scores, key_mean,  # noqa: E402
                     ranked_topk_row, seed_mask, soundness_margin, upper_bound)
 
-STUDY_WORKLOADS = ["prefill_128k_fp8", "tight_64k_bf16_levels", "redundant_chunk128k_fp8"]
+STUDY_WORKLOADS = ["prefill_128k_fp8", "tight_64k_bf16_levels", "redundant_chunk128k_fp8",
+                   "redundant_128k_fp8"]
 BUDGETS = [4, 8, 16, "P"]
 GROUPS = [0, 1, 2]
 MARGIN_LOG2 = -12
@@ -117,8 +121,18 @@ def main():
     ap.add_argument("--rows", type=int, default=64)
     ap.add_argument("--out", default=os.path.join(HERE, "golden", "prune_study.json"))
     ap.add_argument("--workloads", default=",".join(STUDY_WORKLOADS))
+    ap.add_argument("--merge", action="store_true",
+                    help="keep the stored results of the workloads not listed")
     args = ap.parse_args()
     results = [study(name, args.rows) for name in args.workloads.split(",")]
+    if args.merge and os.path.exists(args.out):
+        with open(args.out) as f:
+            stored = json.load(f)
+        assert stored["rows_per_workload"] == args.rows and stored["margin_log2"] == MARGIN_LOG2
+        done = {r["workload"] for r in results}
+        order = {name: i for i, name in enumerate(STUDY_WORKLOADS)}
+        results = sorted([r for r in stored["results"] if r["workload"] not in done] + results,
+                         key=lambda r: order.get(r["workload"], len(order)))
     with open(args.out, "w") as f:
         json.dump({"margin_log2": MARGIN_LOG2, "rows_per_workload": args.rows,
                    "results": results}, f, indent=1)
